@@ -1,0 +1,274 @@
+"""Plain fp64 CPU oracle of the FlashBlock block-diffusion attention step.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+benchmark's CPU-baseline leg may import this module.  The product path (the
+CUDA library and its Python binding) never calls it, and this module imports
+nothing from the product.  It is slow on purpose: every function is the
+textbook definition written out in float64 numpy, with matrix products as the
+only library primitive, so a reader can check it against the pages by eye.
+
+Source: "FlashBlock: Attention Caching for Efficient Long-Context Block
+Diffusion" (gist.science technical summary, section "Mécanisme Central" and
+"Stratégies de Réutilisation Adaptatives"; fugumt abstract page, "Abstract").
+
+What the pages define, and how it is written here
+-------------------------------------------------
+* Attention over a key set J, for one query q (section "Mécanisme Central"):
+  s_j = scale * q.k_j, Z = sum_j exp(s_j), A = sum_j exp(s_j) v_j / Z and the
+  log-normaliser L = log Z.  ``attention_part``.
+* The split into block-internal keys J_in (the current block) and
+  block-external keys J_out (everything outside the block: the prefix KV
+  cache), giving (A_in, L_in) and (A_out, L_out).  ``inblock``, ``outblock``.
+* The log-space merge: m = max(L_out, L_in),
+  A = (e^{L_out-m} A_out + e^{L_in-m} A_in) / (e^{L_out-m} + e^{L_in-m}).
+  The merged normaliser L = m + log(e^{L_out-m} + e^{L_in-m}) follows from
+  L = log Z (Z adds over disjoint key sets).  ``merge`` (N-way).
+* Reuse of the cached (A_out, L_out) of an earlier diffusion step when the
+  updated-token count M < tau (discrete diffusion), and only in heads whose
+  similarity exceeds gamma (video) (section "Stratégies de Réutilisation
+  Adaptatives").  ``FlashBlockOracle.step``.
+* Sparse attention compatibility: the keys a sparse method did not select
+  are treated as the block-external set and their residual contribution is
+  cached (same section, third bullet).  ``outblock_selected``.
+
+Readings where the pages are silent (each one is listed in the design notes):
+scale = 1/sqrt(D); natural log; bidirectional attention inside the block;
+query head h uses KV head floor(h / G); M is the per-step count supplied by
+the caller, compared strictly (M == tau recomputes); the cached A_out is the
+most recently computed one; the similarity is the cosine of the flattened
+[Nb, D] block-external output of a head between the fresh and the cached
+value, defined from step 1 on, compared strictly, and a head that reuses keeps
+its cache and similarity until the block ends; an empty key set gives
+(A, L) = (0, -inf).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+from typing import List, Optional, Sequence, Tuple
+
+import numpy as np
+
+NEG_INF = -np.inf
+
+
+def default_scale(D: int) -> float:
+    """Softmax scale when the caller gives none: 1/sqrt(D) (pages silent)."""
+    return 1.0 / math.sqrt(D)
+
+
+def attention_part(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):
+    """Softmax attention of queries q [n, D] over keys k, values v [m, D].
+
+    Returns (A [n, D], L [n]) with L = log sum_j exp(scale q.k_j) (natural log)
+    and A = sum_j softmax_j v_j ("Mécanisme Central": A with L = log Z).
+    An empty key set (m = 0) gives A = 0 and L = -inf.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    n, D = q.shape
+    if k.shape[0] == 0:
+        return np.zeros((n, v.shape[1])), np.full(n, NEG_INF)
+    s = scale * (q @ k.T)                       # [n, m]
+    mx = s.max(axis=1, keepdims=True)           # shift for exp range only
+    e = np.exp(s - mx)
+    z = e.sum(axis=1, keepdims=True)
+    A = (e @ v) / z
+    L = (mx + np.log(z))[:, 0]
+    return A, L
+
+
+def merge(parts: Sequence[Tuple[np.ndarray, np.ndarray]]):
+    """N-way log-space merge of attention parts over disjoint key sets.
+
+    With m = max_p L_p and w_p = exp(L_p - m):
+        A = sum_p w_p A_p / sum_p w_p,   L = m + log sum_p w_p
+    which for two parts is the merge formula of "Mécanisme Central".  Rows
+    whose parts all have L = -inf give (0, -inf) (no key at all); a part with
+    L = -inf has weight exactly 0, so merging with it is the identity.
+    """
+    As = [np.asarray(a, dtype=np.float64) for a, _ in parts]
+    Ls = [np.asarray(l, dtype=np.float64) for _, l in parts]
+    Lstack = np.stack(Ls)                                   # [P, ...]
+    m = Lstack.max(axis=0)
+    empty = np.isneginf(m)
+    m_safe = np.where(empty, 0.0, m)
+    w = [np.where(np.isneginf(l), 0.0, np.exp(l - m_safe)) for l in Ls]
+    wsum = np.sum(w, axis=0)
+    num = np.zeros_like(As[0])
+    for wp, ap in zip(w, As):
+        num = num + wp[..., None] * ap
+    den = np.where(empty, 1.0, wsum)
+    A = np.where(empty[..., None], 0.0, num / den[..., None])
+    L = np.where(empty, NEG_INF, m_safe + np.log(den))
+    return A, L
+
+
+def kv_head(h: int, Hq: int, Hkv: int) -> int:
+    """KV head of query head h under grouped-query attention (contiguous groups)."""
+    return h // (Hq // Hkv)
+
+
+def outblock(Q, Kp, Vp, prefix_len: int, scale: float):
+    """Block-external attention over the prefix KV cache J_out.
+
+    Q [B, Hq, Nb, D]; Kp, Vp [B, Hkv, >=prefix_len, D].
+    Returns A_out [B, Hq, Nb, D], L_out [B, Hq, Nb].
+    """
+    B, Hq, Nb, D = Q.shape
+    Hkv = Kp.shape[1]
+    A = np.zeros((B, Hq, Nb, D))
+    L = np.zeros((B, Hq, Nb))
+    for b in range(B):
+        for h in range(Hq):
+            g = kv_head(h, Hq, Hkv)
+            A[b, h], L[b, h] = attention_part(
+                Q[b, h], Kp[b, g, :prefix_len], Vp[b, g, :prefix_len], scale)
+    return A, L
+
+
+def inblock(Q, Kin, Vin, scale: float):
+    """Block-internal attention over the block's own keys J_in (bidirectional)."""
+    B, Hq, Nb, D = Q.shape
+    Hkv = Kin.shape[1]
+    A = np.zeros((B, Hq, Nb, D))
+    L = np.zeros((B, Hq, Nb))
+    for b in range(B):
+        for h in range(Hq):
+            g = kv_head(h, Hq, Hkv)
+            A[b, h], L[b, h] = attention_part(Q[b, h], Kin[b, g], Vin[b, g], scale)
+    return A, L
+
+
+def outblock_selected(Q, Kp, Vp, prefix_len: int, scale: float, sel, residual: bool):
+    """Sparse split of the prefix (section "Stratégies de Réutilisation
+    Adaptatives", sparse bullet): each query head h keeps the prefix positions
+    sel[b, h] (set S); the rest U = prefix minus S is the block-external set
+    whose contribution FlashBlock caches.
+
+    Returns (A_S, L_S) over S, or with ``residual`` (A_U, L_U) over U;
+    each [B, Hq, Nb, D] / [B, Hq, Nb].
+    """
+    B, Hq, Nb, D = Q.shape
+    Hkv = Kp.shape[1]
+    A = np.zeros((B, Hq, Nb, D)); L = np.zeros((B, Hq, Nb))
+    for b in range(B):
+        for h in range(Hq):
+            g = kv_head(h, Hq, Hkv)
+            chosen = np.zeros(prefix_len, dtype=bool)
+            chosen[np.asarray(sel[b, h], dtype=np.int64)] = True
+            keep = ~chosen if residual else chosen
+            K = Kp[b, g, :prefix_len]; V = Vp[b, g, :prefix_len]
+            A[b, h], L[b, h] = attention_part(Q[b, h], K[keep], V[keep], scale)
+    return A, L
+
+
+def full_attention(Q, Kin, Vin, Kp, Vp, prefix_len: int, scale: float):
+    """Plain attention of the block's queries over prefix and block keys together."""
+    B, Hq, Nb, D = Q.shape
+    Hkv = Kp.shape[1]
+    A = np.zeros((B, Hq, Nb, D)); L = np.zeros((B, Hq, Nb))
+    for b in range(B):
+        for h in range(Hq):
+            g = kv_head(h, Hq, Hkv)
+            K = np.concatenate([Kp[b, g, :prefix_len], Kin[b, g]])
+            V = np.concatenate([Vp[b, g, :prefix_len], Vin[b, g]])
+            A[b, h], L[b, h] = attention_part(Q[b, h], K, V, scale)
+    return A, L
+
+
+def cosine_similarity(a: np.ndarray, c: np.ndarray) -> float:
+    """cos(a, c) of two flattened vectors; 0 when either has zero norm."""
+    a = np.asarray(a, dtype=np.float64).ravel()
+    c = np.asarray(c, dtype=np.float64).ravel()
+    na = math.sqrt(float(a @ a)); nc = math.sqrt(float(c @ c))
+    if na == 0.0 or nc == 0.0:
+        return 0.0
+    return float(a @ c) / (na * nc)
+
+
+def kv_append(Kp, Vp, prefix_len: int, Kin, Vin):
+    """Write the finished block's K/V at prefix positions [prefix_len, prefix_len + Nb)."""
+    Nb = Kin.shape[2]
+    Kp = np.array(Kp, copy=True); Vp = np.array(Vp, copy=True)
+    Kp[:, :, prefix_len:prefix_len + Nb] = Kin
+    Vp[:, :, prefix_len:prefix_len + Nb] = Vin
+    return Kp, Vp, prefix_len + Nb
+
+
+@dataclass
+class StepResult:
+    o: np.ndarray             # [B, Hq, Nb, D] merged attention output
+    lse: np.ndarray           # [B, Hq, Nb] natural-log normaliser of o
+    recompute: bool           # tau decision: False = cached block-external part allowed
+    head_reuse: np.ndarray    # bool [B, Hq]: this step used the cached part
+    sim: np.ndarray           # [B, Hq] last computed similarity (nan: undefined)
+
+
+class FlashBlockOracle:
+    """The FlashBlock step policy, one attention layer, run step by step.
+
+    State: the cached block-external part (A, L) per (b, h) (the prefix part,
+    or for sparse attention the residual over the non-selected keys), its
+    validity, and for the gamma gate each head's last similarity.
+    """
+
+    def __init__(self, B, Hq, Hkv, D, Nb, scale: Optional[float] = None,
+                 gamma: Optional[Sequence[float]] = None):
+        self.B, self.Hq, self.Hkv, self.D, self.Nb = B, Hq, Hkv, D, Nb
+        self.scale = default_scale(D) if not scale else float(scale)
+        self.gamma = None if gamma is None else np.asarray(gamma, dtype=np.float64)
+        self.cache_A = np.zeros((B, Hq, Nb, D))
+        self.cache_L = np.full((B, Hq, Nb), NEG_INF)
+        self.begin_block()
+
+    def begin_block(self):
+        """A new block: the cache no longer describes this block's queries."""
+        self.valid = False
+        self.sim = np.full((self.B, self.Hq), np.nan)
+
+    def step(self, q, kin, vin, kp, vp, prefix_len: int, M: int,
+             tau: Optional[int], sel=None) -> StepResult:
+        B, Hq = self.B, self.Hq
+        tau_reuse = self.valid and (tau is None or M < tau)   # strict "M < tau"
+        if self.gamma is None:
+            head_reuse = np.full((B, Hq), tau_reuse)
+        else:
+            sim_ok = ~np.isnan(self.sim) & (self.sim > self.gamma[None, :])
+            head_reuse = tau_reuse & sim_ok
+
+        fresh_S = None
+        if sel is not None:
+            fresh_S = outblock_selected(q, kp, vp, prefix_len, self.scale, sel, residual=False)
+
+        for b in range(B):
+            for h in range(Hq):
+                if head_reuse[b, h]:
+                    continue            # keep the cached part and its similarity
+                g = kv_head(h, Hq, self.Hkv)
+                K = kp[b, g, :prefix_len]; V = vp[b, g, :prefix_len]
+                if sel is not None:     # sparse: block-external set = unselected keys
+                    keep = np.ones(prefix_len, dtype=bool)
+                    keep[np.asarray(sel[b, h], dtype=np.int64)] = False
+                    K, V = K[keep], V[keep]
+                a_new, l_new = attention_part(q[b, h], K, V, self.scale)
+                if self.gamma is not None and self.valid:
+                    self.sim[b, h] = cosine_similarity(a_new, self.cache_A[b, h])
+                self.cache_A[b, h] = a_new
+                self.cache_L[b, h] = l_new
+        self.valid = True
+
+        a_in, l_in = inblock(q, kin, vin, self.scale)
+        parts = [(self.cache_A, self.cache_L), (a_in, l_in)]
+        if fresh_S is not None:
+            parts.insert(0, fresh_S)
+        o, lse = merge(parts)
+        return StepResult(o, lse, not tau_reuse, head_reuse.copy(), self.sim.copy())
+
+
+def to64(t) -> np.ndarray:
+    """Exact widening of a torch (bf16/fp32) or numpy tensor to float64."""
+    if hasattr(t, "detach"):
+        return t.detach().to("cpu").double().numpy()
+    return np.asarray(t, dtype=np.float64)
