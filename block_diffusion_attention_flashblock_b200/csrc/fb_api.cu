@@ -1,0 +1,643 @@
+// Host side of libfb: argument checks, launch planning and the FlashBlock step
+// policy (FlashBlock summary, "Mécanisme Central" and "Stratégies de
+// Réutilisation Adaptatives").  Every entry point validates on the host before
+// touching CUDA, so a rejected call launches nothing.
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "fb_internal.cuh"
+
+namespace fb {
+
+// Per-device status word written by kernels whose bounded waits expire.
+__device__ int g_fb_status = 0;
+
+static uint64_t g_wait_limit_ns = 2000000000ull;
+uint64_t wait_limit_ns() { return g_wait_limit_ns; }
+
+int* device_status_ptr() {
+  int* p = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_fb_status) != cudaSuccess) return nullptr;
+  return p;
+}
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+RowMap make_rowmap(int B, int Hq, int Hkv, int Nb, int per_head, int tile_rows) {
+  RowMap rm;
+  rm.B = B; rm.Hq = Hq; rm.Hkv = Hkv; rm.G = Hq / Hkv; rm.Nb = Nb;
+  rm.per_head = per_head;
+  rm.rows_per_unit = per_head ? Nb : rm.G * Nb;
+  rm.row_tiles = (rm.rows_per_unit + tile_rows - 1) / tile_rows;
+  rm.units = per_head ? B * Hq : B * Hkv;
+  return rm;
+}
+
+// Split [0, nkeys) into nsplit ranges of keys_per_split (a multiple of
+// key_tile) so that tiles * nsplit fills the SMs ctas_per_sm deep.
+void plan_split(int64_t tiles, int64_t nkeys, int ctas_per_sm, int key_tile, int32_t* nsplit,
+                int64_t* keys_per_split) {
+  const int64_t target = (int64_t)num_sms() * ctas_per_sm;
+  const int64_t max_split = std::max<int64_t>(1, (nkeys + key_tile - 1) / key_tile);
+  int64_t ns = std::max<int64_t>(1, (target + tiles - 1) / tiles);
+  ns = std::min(ns, max_split);
+  int64_t kps = (nkeys + ns - 1) / ns;
+  kps = std::max<int64_t>(key_tile, (kps + key_tile - 1) / key_tile * key_tile);
+  ns = std::max<int64_t>(1, (nkeys + kps - 1) / kps);
+  *nsplit = (int32_t)ns;
+  *keys_per_split = kps;
+}
+
+// ------------------------------------------------------------- profiling --
+// Event pairs around launches, kept until fb_profile_read folds them in.
+struct ProfRecord {
+  int kind;
+  cudaEvent_t start, stop;
+  double bytes;
+};
+static struct {
+  bool on = false;
+  std::vector<ProfRecord> pending;
+  std::vector<cudaEvent_t> pool;
+  int64_t launches[FB_PROFILE_KINDS] = {0, 0, 0};
+  double ms[FB_PROFILE_KINDS] = {0, 0, 0};
+  double bytes[FB_PROFILE_KINDS] = {0, 0, 0};
+} g_prof;
+
+static cudaEvent_t prof_event() {
+  if (!g_prof.pool.empty()) {
+    cudaEvent_t e = g_prof.pool.back();
+    g_prof.pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Begin/end a profiled launch on stream s (no-ops while profiling is off).
+ProfScope::ProfScope(int kind, double bytes, cudaStream_t s) : kind_(kind), bytes_(bytes), s_(s) {
+  if (!g_prof.on) return;
+  start_ = prof_event();
+  cudaEventRecord(start_, s_);
+}
+ProfScope::~ProfScope() {
+  if (!g_prof.on || !start_) return;
+  cudaEvent_t stop = prof_event();
+  cudaEventRecord(stop, s_);
+  g_prof.pending.push_back({kind_, start_, stop, bytes_});
+}
+
+}  // namespace fb
+
+using namespace fb;
+
+// ------------------------------------------------------------------ checks --
+static inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static inline int esize(int dt) { return dt == FB_BF16 ? 2 : 4; }
+
+static fb_status check_strides(const int64_t* st, int es) {
+  for (int i = 0; i < 3; ++i) {
+    if (st[i] < 0) return FB_EINVAL;
+    if ((st[i] * es) % 16 != 0) return FB_EALIGN;
+  }
+  return FB_OK;
+}
+
+static fb_status check_desc(const fb_attn_desc* d) {
+  if (!d) return FB_EINVAL;
+  if (d->B < 1 || d->Hq < 1 || d->Hkv < 1 || d->Nb < 1 || d->D < 1) return FB_EINVAL;
+  if (d->Hq % d->Hkv != 0) return FB_EINVAL;
+  if ((d->in_dtype != FB_F32 && d->in_dtype != FB_BF16) || (d->out_dtype != FB_F32 && d->out_dtype != FB_BF16))
+    return FB_EDTYPE;
+  if (d->D != 64 && d->D != 128) return FB_EUNSUPPORTED;
+  if (!(d->scale >= 0.f) || isinf(d->scale)) return FB_EINVAL;
+  if (d->kp_capacity < 0) return FB_EINVAL;
+  fb_status s;
+  const int es = esize(d->in_dtype);
+  if ((s = check_strides(d->q_strides, es)) != FB_OK) return s;
+  if ((s = check_strides(d->kin_strides, es)) != FB_OK) return s;
+  if ((s = check_strides(d->kp_strides, es)) != FB_OK) return s;
+  if ((s = check_strides(d->o_strides, esize(d->out_dtype))) != FB_OK) return s;
+  return FB_OK;
+}
+
+static float scale_log2(const fb_attn_desc& d) {
+  const float sc = d.scale > 0.f ? d.scale : 1.0f / sqrtf((float)d.D);
+  return sc * kLog2e;
+}
+
+static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+static inline int64_t rows_of(const fb_attn_desc& d) { return (int64_t)d.B * d.Hq * d.Nb; }
+static inline size_t part_bytes(const fb_attn_desc& d, int32_t n) {
+  return align256((size_t)n * rows_of(d) * d.D * 4) + align256((size_t)n * rows_of(d) * 4);
+}
+
+// Upper bound of the split count of one pass over up to max_keys keys.
+static int32_t split_bound(const fb_attn_desc& d, int per_head, int64_t max_keys) {
+  const RowMap rm = make_rowmap(d.B, d.Hq, d.Hkv, d.Nb, per_head, generic_tile_rows(d.in_dtype == FB_BF16));
+  int32_t ns;
+  int64_t kps;
+  plan_split((int64_t)rm.units * rm.row_tiles, std::max<int64_t>(max_keys, 1),
+             generic_ctas_per_sm(d.D, d.in_dtype == FB_BF16), generic_key_tile(), &ns, &kps);
+  return ns;
+}
+
+// One attention pass of the block's queries over a key source.
+struct PassPlan {
+  AttnArgs a;
+  int32_t nsplit;
+};
+
+static PassPlan plan_pass(const fb_attn_desc& d, const void* q, const void* k, const void* v,
+                          const int64_t* kstr, int64_t nkeys, const int32_t* sel, int32_t sel_k,
+                          int32_t max_split) {
+  PassPlan p;
+  memset(&p.a, 0, sizeof(p.a));
+  AttnArgs& a = p.a;
+  const int bf16 = d.in_dtype == FB_BF16;
+  a.rm = make_rowmap(d.B, d.Hq, d.Hkv, d.Nb, sel != nullptr, generic_tile_rows(bf16));
+  a.q = q; a.q_sb = d.q_strides[0]; a.q_sh = d.q_strides[1]; a.q_st = d.q_strides[2];
+  a.k = k; a.v = v; a.k_sb = kstr[0]; a.k_sh = kstr[1]; a.k_st = kstr[2];
+  a.nkeys = sel ? sel_k : nkeys;
+  a.sel = sel; a.sel_k = sel_k;
+  a.key_rows = nkeys;
+  a.scale_log2 = scale_log2(d);
+  plan_split((int64_t)a.rm.units * a.rm.row_tiles, a.nkeys, generic_ctas_per_sm(d.D, bf16), generic_key_tile(),
+             &a.nsplit, &a.keys_per_split);
+  if (max_split > 0 && a.nsplit > max_split) {  // workspace sized smaller: fewer, longer splits
+    const int kt = generic_key_tile();
+    int64_t kps = (a.nkeys + max_split - 1) / max_split;
+    a.keys_per_split = std::max<int64_t>(kt, (kps + kt - 1) / kt * kt);
+    a.nsplit = (int32_t)std::max<int64_t>(1, (a.nkeys + a.keys_per_split - 1) / a.keys_per_split);
+  }
+  p.nsplit = a.nsplit;
+  return p;
+}
+
+// Algorithmic bytes of one attention pass: each key/value row of the source
+// read once per unit that needs it, Q read once, the final (A, L) written once.
+static double pass_bytes(const fb_attn_desc& d, const AttnArgs& a) {
+  const int es = esize(d.in_dtype);
+  const double kv = 2.0 * a.rm.units * (double)a.nkeys * d.D * es;
+  return kv + (double)rows_of(d) * d.D * es + (double)rows_of(d) * (d.D + 1) * 4;
+}
+
+static fb_status launch_pass(const fb_attn_desc& d, AttnArgs& a, float* pa, float* pl, cudaStream_t s) {
+  a.part_a = pa; a.part_l = pl;
+  a.part_stride_a = rows_of(d) * d.D;
+  a.part_stride_l = rows_of(d);
+  ProfScope prof(kProfPrefix, pass_bytes(d, a), s);
+  return launch_attn_generic(a, d.D, d.in_dtype == FB_BF16, s) == cudaSuccess ? FB_OK : FB_ECUDA;
+}
+
+static PartGroup group_of(const float* a, const float* l, int32_t n, const fb_attn_desc& d) {
+  PartGroup g;
+  g.a = a; g.l = l; g.count = n;
+  g.stride_a = rows_of(d) * d.D;
+  g.stride_l = rows_of(d);
+  return g;
+}
+
+// Merge `pl` into packed fp32 (A, L) at dst_a / dst_l.
+static fb_status merge_to_part(const fb_attn_desc& d, const PartList& pl, float* dst_a, float* dst_l,
+                               const int8_t* mask, int mask_active, cudaStream_t s) {
+  MergeArgs m;
+  memset(&m, 0, sizeof(m));
+  m.B = d.B; m.Hq = d.Hq; m.Nb = d.Nb; m.D = d.D;
+  m.parts = pl;
+  m.o = dst_a; m.o_sb = (int64_t)d.Hq * d.Nb * d.D; m.o_sh = (int64_t)d.Nb * d.D; m.o_st = d.D;
+  m.o_bf16 = 0;
+  m.lse = dst_l;
+  m.mask = mask; m.mask_active = mask_active;
+  double nparts = 0;
+  for (int i = 0; i < pl.ngroups; ++i) nparts += pl.g[i].count;
+  ProfScope prof(kProfAux, (nparts + 1) * rows_of(d) * (d.D + 1) * 4.0, s);
+  return launch_merge(m, s) == cudaSuccess ? FB_OK : FB_ECUDA;
+}
+
+static fb_status run_inblock(const fb_attn_desc& d, const void* q, const void* kin, const void* vin,
+                             const PartList& ext, void* o, float* lse, cudaStream_t s) {
+  PassPlan p = plan_pass(d, q, kin, vin, d.kin_strides, d.Nb, nullptr, 0, 1);
+  AttnArgs& a = p.a;
+  a.nsplit = 1;
+  a.keys_per_split = d.Nb;
+  a.merge_out = 1;
+  a.ext = ext;
+  a.o = o; a.o_sb = d.o_strides[0]; a.o_sh = d.o_strides[1]; a.o_st = d.o_strides[2];
+  a.o_bf16 = d.out_dtype == FB_BF16;
+  a.lse = lse;
+  double ext_parts = 0;
+  for (int i = 0; i < ext.ngroups; ++i) ext_parts += ext.g[i].count;
+  const int es = esize(d.in_dtype);
+  const double bytes = (double)rows_of(d) * d.D * es + 2.0 * d.B * d.Hkv * d.Nb * d.D * es +
+                       ext_parts * rows_of(d) * (d.D + 1) * 4.0 +
+                       (double)rows_of(d) * (d.D * esize(d.out_dtype) + (lse ? 4 : 0));
+  ProfScope prof(kProfInblock, bytes, s);
+  return launch_attn_generic(a, d.D, d.in_dtype == FB_BF16, s) == cudaSuccess ? FB_OK : FB_ECUDA;
+}
+
+// ------------------------------------------------------------- public API --
+extern "C" {
+
+const char* fb_status_string(fb_status s) {
+  switch (s) {
+    case FB_OK: return "FB_OK";
+    case FB_EINVAL: return "FB_EINVAL: invalid argument";
+    case FB_EALIGN: return "FB_EALIGN: pointer or stride not 16-byte aligned";
+    case FB_EDTYPE: return "FB_EDTYPE: unsupported dtype";
+    case FB_EUNSUPPORTED: return "FB_EUNSUPPORTED: unsupported configuration";
+    case FB_ESTATE: return "FB_ESTATE: handle state forbids the call";
+    case FB_ECUDA: return "FB_ECUDA: CUDA runtime error";
+    case FB_ETIMEOUT: return "FB_ETIMEOUT: a kernel wait expired";
+    case FB_ENOSPACE: return "FB_ENOSPACE: workspace too small";
+  }
+  return "unknown fb_status";
+}
+
+int32_t fb_version(void) { return (1 << 16) | 0; }
+
+fb_status fb_outblock_workspace_bytes(const fb_attn_desc* d, int64_t prefix_len, int32_t sel_k, size_t* bytes) {
+  fb_status st = check_desc(d);
+  if (st != FB_OK) return st;
+  if (!bytes || prefix_len < 0 || sel_k < 0) return FB_EINVAL;
+  size_t n = part_bytes(*d, std::max(split_bound(*d, 0, prefix_len), sel_k ? split_bound(*d, 1, sel_k) : 1));
+  if (sel_k) n += align256((size_t)d->B * d->Hq * ((prefix_len + 31) / 32) * 4);
+  *bytes = n;
+  return FB_OK;
+}
+
+fb_status fb_attn_outblock(const fb_attn_desc* d, const void* q, const void* kp, const void* vp,
+                           int64_t prefix_len, const int32_t* sel, int32_t sel_k, float* a_out, float* l_out,
+                           float* a_res, float* l_res, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  fb_status st = check_desc(d);
+  if (st != FB_OK) return st;
+  if (!q || !kp || !vp || !a_out || !l_out) return FB_EINVAL;
+  if (prefix_len < 0 || prefix_len > d->kp_capacity) return FB_EINVAL;
+  if (sel && (sel_k < 0 || sel_k > prefix_len)) return FB_EINVAL;
+  if (!sel && (a_res || l_res)) return FB_EINVAL;
+  if ((a_res == nullptr) != (l_res == nullptr)) return FB_EINVAL;
+  if (!al16(q) || !al16(kp) || !al16(vp) || !al16(a_out) || !al16(l_out) || !al16(sel) || !al16(a_res) ||
+      !al16(l_res) || !al16(ws))
+    return FB_EALIGN;
+  size_t need = 0;
+  if ((st = fb_outblock_workspace_bytes(d, prefix_len, sel ? sel_k : 0, &need)) != FB_OK) return st;
+  if (!ws || ws_bytes < need) return FB_ENOSPACE;
+
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint32_t* bitmap = nullptr;
+  const int64_t words = (prefix_len + 31) / 32;
+  if (sel) {
+    bitmap = reinterpret_cast<uint32_t*>(w);
+    w += align256((size_t)d->B * d->Hq * words * 4);
+  }
+  const int32_t cap = std::max(split_bound(*d, 0, prefix_len), sel ? split_bound(*d, 1, sel_k) : 1);
+  float* pa = reinterpret_cast<float*>(w);
+  float* pl = reinterpret_cast<float*>(w + align256((size_t)cap * rows_of(*d) * d->D * 4));
+
+  // pass 1: dense prefix, or the selected keys
+  PassPlan p = plan_pass(*d, q, kp, vp, d->kp_strides, prefix_len, sel, sel_k, cap);
+  if (p.nsplit == 1) {
+    if ((st = launch_pass(*d, p.a, a_out, l_out, stream)) != FB_OK) return st;
+  } else {
+    if ((st = launch_pass(*d, p.a, pa, pl, stream)) != FB_OK) return st;
+    PartList lst;
+    lst.ngroups = 1;
+    lst.g[0] = group_of(pa, pl, p.nsplit, *d);
+    if ((st = merge_to_part(*d, lst, a_out, l_out, nullptr, 0, stream)) != FB_OK) return st;
+  }
+  if (!sel || !a_res) return FB_OK;
+  // pass 2: the residual (prefix minus the selection)
+  if (launch_build_bitmap(sel, sel_k, d->B * d->Hq, bitmap, words, stream) != cudaSuccess) return FB_ECUDA;
+  PassPlan r = plan_pass(*d, q, kp, vp, d->kp_strides, prefix_len, nullptr, 0, cap);
+  r.a.excl = bitmap;
+  r.a.excl_words = words;
+  if (r.nsplit == 1) return launch_pass(*d, r.a, a_res, l_res, stream);
+  if ((st = launch_pass(*d, r.a, pa, pl, stream)) != FB_OK) return st;
+  PartList lst;
+  lst.ngroups = 1;
+  lst.g[0] = group_of(pa, pl, r.nsplit, *d);
+  return merge_to_part(*d, lst, a_res, l_res, nullptr, 0, stream);
+}
+
+static fb_status check_parts(int32_t nparts, const float* const* a, const float* const* l, int32_t maxn) {
+  if (nparts < 0 || nparts > maxn) return FB_EINVAL;
+  if (nparts > 0 && (!a || !l)) return FB_EINVAL;
+  for (int i = 0; i < nparts; ++i) {
+    if (!a[i] || !l[i]) return FB_EINVAL;
+    if (!al16(a[i]) || !al16(l[i])) return FB_EALIGN;
+  }
+  return FB_OK;
+}
+
+fb_status fb_attn_inblock(const fb_attn_desc* d, const void* q, const void* kin, const void* vin, int32_t nparts,
+                          const float* const* a_parts, const float* const* l_parts, void* o, float* lse,
+                          cudaStream_t stream) {
+  fb_status st = check_desc(d);
+  if (st != FB_OK) return st;
+  if (!q || !kin || !vin || !o) return FB_EINVAL;
+  if ((st = check_parts(nparts, a_parts, l_parts, FB_MAX_PARTS - 1)) != FB_OK) return st;
+  if (!al16(q) || !al16(kin) || !al16(vin) || !al16(o) || !al16(lse)) return FB_EALIGN;
+  PartList ext;
+  memset(&ext, 0, sizeof(ext));
+  ext.ngroups = nparts;
+  for (int i = 0; i < nparts; ++i) ext.g[i] = group_of(a_parts[i], l_parts[i], 1, *d);
+  return run_inblock(*d, q, kin, vin, ext, o, lse, stream);
+}
+
+fb_status fb_merge(const fb_attn_desc* d, int32_t nparts, const float* const* a_parts,
+                   const float* const* l_parts, void* o, float* lse, cudaStream_t stream) {
+  fb_status st = check_desc(d);
+  if (st != FB_OK) return st;
+  if (!o || nparts < 1) return FB_EINVAL;
+  if ((st = check_parts(nparts, a_parts, l_parts, FB_MAX_PARTS)) != FB_OK) return st;
+  if (!al16(o) || !al16(lse)) return FB_EALIGN;
+  MergeArgs m;
+  memset(&m, 0, sizeof(m));
+  m.B = d->B; m.Hq = d->Hq; m.Nb = d->Nb; m.D = d->D;
+  m.parts.ngroups = nparts;
+  for (int i = 0; i < nparts; ++i) m.parts.g[i] = group_of(a_parts[i], l_parts[i], 1, *d);
+  m.o = o; m.o_sb = d->o_strides[0]; m.o_sh = d->o_strides[1]; m.o_st = d->o_strides[2];
+  m.o_bf16 = d->out_dtype == FB_BF16;
+  m.lse = lse;
+  ProfScope prof(kProfAux, (double)nparts * rows_of(*d) * (d->D + 1) * 4.0 + rows_of(*d) * d->D * esize(d->out_dtype),
+                 stream);
+  return launch_merge(m, stream) == cudaSuccess ? FB_OK : FB_ECUDA;
+}
+
+fb_status fb_kv_append(const fb_attn_desc* d, void* kp, void* vp, int64_t prefix_len, const void* kin,
+                       const void* vin, cudaStream_t stream) {
+  fb_status st = check_desc(d);
+  if (st != FB_OK) return st;
+  if (!kp || !vp || !kin || !vin) return FB_EINVAL;
+  if (prefix_len < 0 || prefix_len + d->Nb > d->kp_capacity) return FB_EINVAL;
+  if (!al16(kp) || !al16(vp) || !al16(kin) || !al16(vin)) return FB_EALIGN;
+  ProfScope prof(kProfAux, 4.0 * d->B * d->Hkv * d->Nb * d->D * esize(d->in_dtype), stream);
+  return launch_kv_append(*d, kp, vp, prefix_len, kin, vin, stream) == cudaSuccess ? FB_OK : FB_ECUDA;
+}
+
+fb_status fb_get_device_status(cudaStream_t stream, fb_status* device_status) {
+  if (!device_status) return FB_EINVAL;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return FB_ECUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_fb_status, sizeof(int)) != cudaSuccess) return FB_ECUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_fb_status, &zero, sizeof(int)) != cudaSuccess) return FB_ECUDA;
+  }
+  *device_status = v == 0 ? FB_OK : static_cast<fb_status>(v);
+  return FB_OK;
+}
+
+fb_status fb_profile_enable(int32_t on) {
+  g_prof.on = on != 0;
+  return FB_OK;
+}
+
+fb_status fb_profile_read(int32_t reset, int64_t* launches, double* total_ms, double* alg_bytes) {
+  for (const ProfRecord& r : g_prof.pending) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess)
+      return FB_ECUDA;
+    g_prof.launches[r.kind] += 1;
+    g_prof.ms[r.kind] += ms;
+    g_prof.bytes[r.kind] += r.bytes;
+    g_prof.pool.push_back(r.start);
+    g_prof.pool.push_back(r.stop);
+  }
+  g_prof.pending.clear();
+  for (int k = 0; k < FB_PROFILE_KINDS; ++k) {
+    if (launches) launches[k] = g_prof.launches[k];
+    if (total_ms) total_ms[k] = g_prof.ms[k];
+    if (alg_bytes) alg_bytes[k] = g_prof.bytes[k];
+    if (reset) { g_prof.launches[k] = 0; g_prof.ms[k] = 0; g_prof.bytes[k] = 0; }
+  }
+  return FB_OK;
+}
+
+fb_status fb_debug_set_wait_limit_ns(uint64_t ns) {
+  g_wait_limit_ns = ns;
+  return FB_OK;
+}
+
+}  // extern "C"
+
+// -------------------------------------------------------------- the cache --
+struct fb_cache {
+  fb_attn_desc d;
+  int32_t flags;
+  int64_t max_prefix;
+  int32_t max_sel_k;
+  bool valid;
+  int32_t last_recomputed;
+  float* cache_a;     // block-external (or residual) part, packed fp32
+  float* cache_l;
+  float* part_a;      // split partials of the prefix / residual pass
+  float* part_l;
+  int32_t part_cap;
+  float* sel_a;       // split partials of the selected-keys pass (sparse)
+  float* sel_l;
+  int32_t sel_cap;
+  uint32_t* bitmap;   // sparse membership
+  int64_t bitmap_words;
+  int8_t* mask;       // gamma: reuse flags for the next step
+  float* sim;         // gamma: last similarity per (b, h)
+  float* gpart;       // gamma: per-chunk partial sums
+  int32_t* counters;  // gamma: per-head arrival counters (kept at zero)
+  int32_t chunks;
+};
+
+namespace {
+struct Carve {
+  size_t off = 0;
+  template <class T>
+  T* take(uint8_t* base, size_t bytes) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += align256(bytes);
+    return p;
+  }
+};
+
+fb_status layout_cache(const fb_attn_desc& d, int32_t flags, int64_t max_prefix, int32_t max_sel_k,
+                       uint8_t* base, fb_cache* c, size_t* total) {
+  Carve cv;
+  const int64_t rows = rows_of(d);
+  const int32_t part_cap = split_bound(d, 0, max_prefix);
+  const int32_t sel_cap = (flags & FB_CACHE_SPARSE) ? split_bound(d, 1, std::max(max_sel_k, 1)) : 0;
+  const int64_t words = (max_prefix + 31) / 32;
+  const int32_t chunks = (d.Nb + gamma_chunk_rows() - 1) / gamma_chunk_rows();
+  float* ca = cv.take<float>(base, rows * d.D * 4);
+  float* cl = cv.take<float>(base, rows * 4);
+  float* pa = cv.take<float>(base, (size_t)part_cap * rows * d.D * 4);
+  float* pl = cv.take<float>(base, (size_t)part_cap * rows * 4);
+  float* sa = nullptr; float* sl = nullptr; uint32_t* bm = nullptr;
+  if (flags & FB_CACHE_SPARSE) {
+    sa = cv.take<float>(base, (size_t)sel_cap * rows * d.D * 4);
+    sl = cv.take<float>(base, (size_t)sel_cap * rows * 4);
+    bm = cv.take<uint32_t>(base, (size_t)d.B * d.Hq * words * 4);
+  }
+  int8_t* mk = nullptr; float* sm = nullptr; float* gp = nullptr; int32_t* ct = nullptr;
+  if (flags & FB_CACHE_GAMMA) {
+    mk = cv.take<int8_t>(base, (size_t)d.B * d.Hq);
+    sm = cv.take<float>(base, (size_t)d.B * d.Hq * 4);
+    gp = cv.take<float>(base, (size_t)d.B * d.Hq * chunks * 3 * 4);
+    ct = cv.take<int32_t>(base, (size_t)d.B * d.Hq * 4);
+  }
+  *total = cv.off;
+  if (c) {
+    c->cache_a = ca; c->cache_l = cl; c->part_a = pa; c->part_l = pl; c->part_cap = part_cap;
+    c->sel_a = sa; c->sel_l = sl; c->sel_cap = sel_cap; c->bitmap = bm; c->bitmap_words = words;
+    c->mask = mk; c->sim = sm; c->gpart = gp; c->counters = ct; c->chunks = chunks;
+  }
+  return FB_OK;
+}
+}  // namespace
+
+extern "C" {
+
+fb_status fb_cache_workspace_bytes(const fb_attn_desc* d, int32_t flags, int64_t max_prefix, int32_t max_sel_k,
+                                   size_t* bytes) {
+  fb_status st = check_desc(d);
+  if (st != FB_OK) return st;
+  if (!bytes || max_prefix < 0 || max_sel_k < 0 || (flags & ~(FB_CACHE_SPARSE | FB_CACHE_GAMMA))) return FB_EINVAL;
+  return layout_cache(*d, flags, max_prefix, max_sel_k, nullptr, nullptr, bytes);
+}
+
+fb_status fb_cache_create(const fb_attn_desc* d, int32_t flags, int64_t max_prefix, int32_t max_sel_k,
+                          void* dev_mem, size_t bytes, cudaStream_t stream, fb_cache_t* out) {
+  size_t need = 0;
+  fb_status st = fb_cache_workspace_bytes(d, flags, max_prefix, max_sel_k, &need);
+  if (st != FB_OK) return st;
+  if (!out || !dev_mem) return FB_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(dev_mem) & 255u) != 0) return FB_EALIGN;
+  if (bytes < need) return FB_ENOSPACE;
+  fb_cache* c = new (std::nothrow) fb_cache;
+  if (!c) return FB_EINVAL;
+  memset(c, 0, sizeof(*c));
+  c->d = *d; c->flags = flags; c->max_prefix = max_prefix; c->max_sel_k = max_sel_k;
+  c->valid = false;
+  layout_cache(*d, flags, max_prefix, max_sel_k, static_cast<uint8_t*>(dev_mem), c, &need);
+  if (flags & FB_CACHE_GAMMA) {
+    if (cudaMemsetAsync(c->mask, 0, (size_t)d->B * d->Hq, stream) != cudaSuccess ||
+        cudaMemsetAsync(c->sim, 0xFF, (size_t)d->B * d->Hq * 4, stream) != cudaSuccess ||
+        cudaMemsetAsync(c->counters, 0, (size_t)d->B * d->Hq * 4, stream) != cudaSuccess) {
+      delete c;
+      return FB_ECUDA;
+    }
+  }
+  *out = c;
+  return FB_OK;
+}
+
+fb_status fb_cache_destroy(fb_cache_t c) {
+  if (!c) return FB_EINVAL;
+  delete c;
+  return FB_OK;
+}
+
+fb_status fb_cache_begin_block(fb_cache_t c, cudaStream_t stream) {
+  (void)stream;
+  if (!c) return FB_EINVAL;
+  c->valid = false;
+  return FB_OK;
+}
+
+fb_status fb_cache_last_step(fb_cache_t c, int32_t* recomputed) {
+  if (!c || !recomputed) return FB_EINVAL;
+  *recomputed = c->last_recomputed;
+  return FB_OK;
+}
+
+fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
+  if (!c || !a) return FB_EINVAL;
+  const fb_attn_desc& d = c->d;
+  if (!a->q || !a->kin || !a->vin || !a->kp || !a->vp || !a->o) return FB_EINVAL;
+  if (a->prefix_len < 0 || a->prefix_len > c->max_prefix || a->prefix_len > d.kp_capacity) return FB_EINVAL;
+  if (a->M < 0) return FB_EINVAL;
+  const bool sparse = a->sel != nullptr;
+  const bool gamma = a->gamma != nullptr;
+  if (sparse && !(c->flags & FB_CACHE_SPARSE)) return FB_ESTATE;
+  if (gamma && !(c->flags & FB_CACHE_GAMMA)) return FB_ESTATE;
+  if (sparse && gamma) return FB_EUNSUPPORTED;
+  if (sparse && (a->sel_k < 0 || a->sel_k > a->prefix_len || a->sel_k > c->max_sel_k)) return FB_EINVAL;
+  if (!al16(a->q) || !al16(a->kin) || !al16(a->vin) || !al16(a->kp) || !al16(a->vp) || !al16(a->o) ||
+      !al16(a->lse) || !al16(a->sel) || !al16(a->gamma))
+    return FB_EALIGN;
+
+  const bool tau_reuse = c->valid && (a->M < a->tau);
+  const int BH = d.B * d.Hq;
+  fb_status st;
+  PartList ext;
+  memset(&ext, 0, sizeof(ext));
+
+  if (gamma) {
+    PassPlan p = plan_pass(d, a->q, a->kp, a->vp, d.kp_strides, a->prefix_len, nullptr, 0, c->part_cap);
+    p.a.mask = c->mask;
+    p.a.mask_active = tau_reuse;
+    if ((st = launch_pass(d, p.a, c->part_a, c->part_l, s)) != FB_OK) return st;
+    GammaArgs g;
+    memset(&g, 0, sizeof(g));
+    g.B = d.B; g.Hq = d.Hq; g.Nb = d.Nb; g.D = d.D;
+    g.fresh.ngroups = 1;
+    g.fresh.g[0] = group_of(c->part_a, c->part_l, p.nsplit, d);
+    g.cache_a = c->cache_a; g.cache_l = c->cache_l;
+    g.mask = c->mask; g.gate_active = tau_reuse; g.cache_valid = c->valid;
+    g.gamma = a->gamma; g.sim = c->sim; g.partials = c->gpart; g.counters = c->counters;
+    g.chunks = c->chunks; g.reuse_out = a->reuse_out; g.sim_out = a->sim_out;
+    {
+      ProfScope prof(kProfAux, (p.nsplit + 2.0) * rows_of(d) * (d.D + 1) * 4.0, s);
+      if (launch_gamma_update(g, s) != cudaSuccess) return FB_ECUDA;
+    }
+  } else {
+    if (sparse) {
+      PassPlan p = plan_pass(d, a->q, a->kp, a->vp, d.kp_strides, a->prefix_len, a->sel, a->sel_k, c->sel_cap);
+      if ((st = launch_pass(d, p.a, c->sel_a, c->sel_l, s)) != FB_OK) return st;
+      ext.g[ext.ngroups++] = group_of(c->sel_a, c->sel_l, p.nsplit, d);
+    }
+    if (!tau_reuse) {
+      PassPlan p = plan_pass(d, a->q, a->kp, a->vp, d.kp_strides, a->prefix_len, nullptr, 0, c->part_cap);
+      if (sparse) {
+        if (launch_build_bitmap(a->sel, a->sel_k, BH, c->bitmap, (a->prefix_len + 31) / 32, s) != cudaSuccess)
+          return FB_ECUDA;
+        p.a.excl = c->bitmap;
+        p.a.excl_words = (a->prefix_len + 31) / 32;
+      }
+      if (p.nsplit == 1) {
+        if ((st = launch_pass(d, p.a, c->cache_a, c->cache_l, s)) != FB_OK) return st;
+      } else {
+        if ((st = launch_pass(d, p.a, c->part_a, c->part_l, s)) != FB_OK) return st;
+        PartList lst;
+        memset(&lst, 0, sizeof(lst));
+        lst.ngroups = 1;
+        lst.g[0] = group_of(c->part_a, c->part_l, p.nsplit, d);
+        if ((st = merge_to_part(d, lst, c->cache_a, c->cache_l, nullptr, 0, s)) != FB_OK) return st;
+      }
+    }
+    if (a->reuse_out && launch_fill_decision(a->reuse_out, BH, tau_reuse ? 1 : 0, s) != cudaSuccess)
+      return FB_ECUDA;
+    if (a->sim_out && cudaMemsetAsync(a->sim_out, 0xFF, (size_t)BH * 4, s) != cudaSuccess) return FB_ECUDA;
+  }
+  ext.g[ext.ngroups++] = group_of(c->cache_a, c->cache_l, 1, d);
+  if ((st = run_inblock(d, a->q, a->kin, a->vin, ext, a->o, a->lse, s)) != FB_OK) return st;
+  c->valid = true;
+  c->last_recomputed = !tau_reuse;
+  return FB_OK;
+}
+
+}  // extern "C"

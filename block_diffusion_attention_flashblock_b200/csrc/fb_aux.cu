@@ -1,0 +1,262 @@
+// Row-wise kernels of libfb: the N-way log-space merge, the gamma-gate
+// similarity/cache update, the KV-cache append and the sparse membership
+// bitmap (FlashBlock summary, "Mécanisme Central" and "Stratégies de
+// Réutilisation Adaptatives").
+#include "fb_internal.cuh"
+#include <math_constants.h>
+
+namespace fb {
+
+namespace {
+
+template <int D>
+struct Vec;  // D/32 fp32 values per lane
+template <>
+struct Vec<64> {
+  float v[2];
+  __device__ void load(const float* p) {
+    const float2 x = __ldg(reinterpret_cast<const float2*>(p));
+    v[0] = x.x; v[1] = x.y;
+  }
+  __device__ void store(float* p) const { *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]); }
+};
+template <>
+struct Vec<128> {
+  float v[4];
+  __device__ void load(const float* p) {
+    const float4 x = __ldg(reinterpret_cast<const float4*>(p));
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  }
+  __device__ void store(float* p) const { *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]); }
+};
+
+template <int D>
+__device__ __forceinline__ void store_out(void* o, int64_t off, bool bf16, const float* v) {
+  constexpr int E = D / 32;
+  if (bf16) {
+    __nv_bfloat16* p = static_cast<__nv_bfloat16*>(o) + off;
+#pragma unroll
+    for (int e = 0; e < E; e += 2)
+      *reinterpret_cast<__nv_bfloat162*>(p + e) = __floats2bfloat162_rn(v[e], v[e + 1]);
+  } else {
+    float* p = static_cast<float*>(o) + off;
+#pragma unroll
+    for (int e = 0; e < E; e += 2) *reinterpret_cast<float2*>(p + e) = make_float2(v[e], v[e + 1]);
+  }
+}
+
+// Merge all parts of one row (lane holds columns lane*E .. lane*E+E-1):
+// m = max L_p, w_p = e^{L_p - m}; returns sum w_p A_p / sum w_p and the LSE.
+template <int D>
+__device__ __forceinline__ float merge_row(const PartList& pl, int64_t row, int lane, float* out) {
+  constexpr int E = D / 32;
+  float m = -CUDART_INF_F;
+  for (int gi = 0; gi < pl.ngroups; ++gi) {
+    const PartGroup& g = pl.g[gi];
+    for (int p = 0; p < g.count; ++p) m = fmaxf(m, __ldg(g.l + p * g.stride_l + row));
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) out[e] = 0.f;
+  if (m == -CUDART_INF_F) return -CUDART_INF_F;
+  float wsum = 0.f;
+  for (int gi = 0; gi < pl.ngroups; ++gi) {
+    const PartGroup& g = pl.g[gi];
+    for (int p = 0; p < g.count; ++p) {
+      const float L = __ldg(g.l + p * g.stride_l + row);
+      if (L == -CUDART_INF_F) continue;
+      const float w = expf(L - m);
+      wsum += w;
+      Vec<D> a;
+      a.load(g.a + p * g.stride_a + row * D + lane * E);
+#pragma unroll
+      for (int e = 0; e < E; ++e) out[e] = fmaf(w, a.v[e], out[e]);
+    }
+  }
+  const float inv = 1.f / wsum;
+#pragma unroll
+  for (int e = 0; e < E; ++e) out[e] *= inv;
+  return m + logf(wsum);
+}
+
+}  // namespace
+
+// One warp per (b, h, i) row.
+template <int D>
+__global__ void __launch_bounds__(256) merge_kernel(const MergeArgs m) {
+  constexpr int E = D / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * 8 + warp;
+  const int64_t nrows = (int64_t)m.B * m.Hq * m.Nb;
+  if (row >= nrows) return;
+  const int64_t bh = row / m.Nb;
+  if (m.mask_active && m.mask[bh]) return;
+  const int b = (int)(bh / m.Hq), h = (int)(bh % m.Hq), i = (int)(row % m.Nb);
+  float out[E];
+  const float lse = merge_row<D>(m.parts, row, lane, out);
+  store_out<D>(m.o, b * m.o_sb + h * m.o_sh + i * m.o_st + lane * E, m.o_bf16, out);
+  if (m.lse && lane == 0) m.lse[row] = lse;
+}
+
+cudaError_t launch_merge(const MergeArgs& m, cudaStream_t s) {
+  const int64_t nrows = (int64_t)m.B * m.Hq * m.Nb;
+  const unsigned grid = (unsigned)((nrows + 7) / 8);
+  if (grid == 0) return cudaSuccess;
+  if (m.D == 64) merge_kernel<64><<<grid, 256, 0, s>>>(m);
+  else merge_kernel<128><<<grid, 256, 0, s>>>(m);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Gamma gate (summary, "Stratégies de Réutilisation Adaptatives", video
+// bullet): for every head that recomputed this step, merge its fresh split
+// partials into A_new, form <A_new, A_cached>, |A_new|^2, |A_cached|^2 over the
+// head's Nb x D values, write A_new into the cache, and let the last CTA of the
+// head turn the sums into sim = cos(A_new, A_cached) and the next step's
+// reuse flag sim > gamma[h].  Sums use a fixed order (lane tree, warp order,
+// chunk order), so the result does not depend on scheduling.
+// ---------------------------------------------------------------------------
+constexpr int kGammaRows = 64;
+int gamma_chunk_rows() { return kGammaRows; }
+
+template <int D>
+__global__ void __launch_bounds__(256) gamma_update_kernel(const GammaArgs g) {
+  constexpr int E = D / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y, chunk = blockIdx.x;
+  const int h = bh % g.Hq;
+  const bool reuse = g.gate_active && g.mask[bh];
+  if (reuse) {
+    if (chunk == 0 && threadIdx.x == 0) {
+      if (g.reuse_out) g.reuse_out[bh] = 1;
+      if (g.sim_out) g.sim_out[bh] = g.sim[bh];
+    }
+    return;
+  }
+  float dot = 0.f, na = 0.f, nc = 0.f;
+  const int r0 = chunk * kGammaRows;
+  const int r1 = min(r0 + kGammaRows, g.Nb);
+  for (int i = r0 + warp; i < r1; i += 8) {
+    const int64_t row = (int64_t)bh * g.Nb + i;
+    float a_new[E];
+    const float L = merge_row<D>(g.fresh, row, lane, a_new);
+    float* cp = g.cache_a + row * D + lane * E;
+    if (g.cache_valid) {
+      Vec<D> c;
+      c.load(cp);
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        dot = fmaf(a_new[e], c.v[e], dot);
+        na = fmaf(a_new[e], a_new[e], na);
+        nc = fmaf(c.v[e], c.v[e], nc);
+      }
+    }
+    Vec<D> w;
+#pragma unroll
+    for (int e = 0; e < E; ++e) w.v[e] = a_new[e];
+    w.store(cp);
+    if (lane == 0) g.cache_l[row] = L;
+  }
+  __shared__ float red[8][3];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    dot += __shfl_xor_sync(0xffffffffu, dot, off);
+    na += __shfl_xor_sync(0xffffffffu, na, off);
+    nc += __shfl_xor_sync(0xffffffffu, nc, off);
+  }
+  if (lane == 0) { red[warp][0] = dot; red[warp][1] = na; red[warp][2] = nc; }
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f;
+  for (int w = 0; w < 8; ++w) { s0 += red[w][0]; s1 += red[w][1]; s2 += red[w][2]; }
+  float* part = g.partials + ((int64_t)bh * g.chunks + chunk) * 3;
+  part[0] = s0; part[1] = s1; part[2] = s2;
+  if (chunk == 0 && g.reuse_out) g.reuse_out[bh] = 0;
+  __threadfence();
+  const int prev = atomicAdd(g.counters + bh, 1);
+  if (prev != g.chunks - 1) return;
+  __threadfence();
+  float t0 = 0.f, t1 = 0.f, t2 = 0.f;
+  const volatile float* all = g.partials + (int64_t)bh * g.chunks * 3;
+  for (int c = 0; c < g.chunks; ++c) { t0 += all[3 * c]; t1 += all[3 * c + 1]; t2 += all[3 * c + 2]; }
+  float sim = CUDART_NAN_F;
+  int8_t next = 0;
+  if (g.cache_valid) {
+    sim = (t1 > 0.f && t2 > 0.f) ? t0 / (sqrtf(t1) * sqrtf(t2)) : 0.f;
+    next = sim > g.gamma[h] ? 1 : 0;
+  }
+  g.sim[bh] = sim;
+  g.mask[bh] = next;
+  if (g.sim_out) g.sim_out[bh] = sim;
+  g.counters[bh] = 0;
+}
+
+cudaError_t launch_gamma_update(const GammaArgs& g, cudaStream_t s) {
+  dim3 grid(g.chunks, g.B * g.Hq);
+  if (g.D == 64) gamma_update_kernel<64><<<grid, 256, 0, s>>>(g);
+  else gamma_update_kernel<128><<<grid, 256, 0, s>>>(g);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// KV append: K_p/V_p rows [prefix_len, prefix_len + Nb) <- K_in/V_in, 16-byte
+// vectors, one thread per vector of K and of V.
+// ---------------------------------------------------------------------------
+__global__ void kv_append_kernel(uint8_t* kp, uint8_t* vp, const uint8_t* kin, const uint8_t* vin,
+                                 int32_t Hkv, int32_t Nb, int32_t vec_per_row, int64_t rows,
+                                 int64_t kp_sb, int64_t kp_sh, int64_t kp_st, int64_t kin_sb,
+                                 int64_t kin_sh, int64_t kin_st, int64_t prefix_len) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= rows * vec_per_row) return;
+  const int64_t r = idx / vec_per_row;
+  const int c = (int)(idx % vec_per_row);
+  const int i = (int)(r % Nb);
+  const int64_t bh = r / Nb;
+  const int h = (int)(bh % Hkv);
+  const int64_t b = bh / Hkv;
+  const int64_t src = b * kin_sb + h * kin_sh + i * kin_st + c * 16;
+  const int64_t dst = b * kp_sb + h * kp_sh + (prefix_len + i) * kp_st + c * 16;
+  *reinterpret_cast<uint4*>(kp + dst) = __ldg(reinterpret_cast<const uint4*>(kin + src));
+  *reinterpret_cast<uint4*>(vp + dst) = __ldg(reinterpret_cast<const uint4*>(vin + src));
+}
+
+cudaError_t launch_kv_append(const fb_attn_desc& d, void* kp, void* vp, int64_t prefix_len,
+                             const void* kin, const void* vin, cudaStream_t s) {
+  const int es = d.in_dtype == FB_BF16 ? 2 : 4;
+  const int vec = d.D * es / 16;
+  const int64_t rows = (int64_t)d.B * d.Hkv * d.Nb;
+  const int64_t n = rows * vec;
+  const int threads = 256;
+  const unsigned grid = (unsigned)((n + threads - 1) / threads);
+  kv_append_kernel<<<grid, threads, 0, s>>>(
+      static_cast<uint8_t*>(kp), static_cast<uint8_t*>(vp), static_cast<const uint8_t*>(kin),
+      static_cast<const uint8_t*>(vin), d.Hkv, d.Nb, vec, rows, d.kp_strides[0] * es, d.kp_strides[1] * es,
+      d.kp_strides[2] * es, d.kin_strides[0] * es, d.kin_strides[1] * es, d.kin_strides[2] * es, prefix_len);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Sparse membership bitmap: bit j of (b, h) set iff j is in sel[b, h, :].
+// ---------------------------------------------------------------------------
+__global__ void build_bitmap_kernel(const int32_t* sel, int32_t sel_k, uint32_t* bitmap, int64_t words) {
+  const int64_t bh = blockIdx.x;
+  uint32_t* w = bitmap + bh * words;
+  for (int64_t j = threadIdx.x; j < words; j += blockDim.x) w[j] = 0u;
+  __syncthreads();
+  const int32_t* s = sel + bh * sel_k;
+  for (int j = threadIdx.x; j < sel_k; j += blockDim.x) {
+    const int32_t key = s[j];
+    if (key >= 0 && (int64_t)(key >> 5) < words) atomicOr(w + (key >> 5), 1u << (key & 31));
+  }
+}
+
+cudaError_t launch_build_bitmap(const int32_t* sel, int32_t sel_k, int32_t BH, uint32_t* bitmap,
+                                int64_t words, cudaStream_t s) {
+  build_bitmap_kernel<<<BH, 256, 0, s>>>(sel, sel_k, bitmap, words);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fill_decision(int8_t* reuse_out, int32_t n, int8_t value, cudaStream_t s) {
+  return cudaMemsetAsync(reuse_out, value, (size_t)n, s);
+}
+
+}  // namespace fb

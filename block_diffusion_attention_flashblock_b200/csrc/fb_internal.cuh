@@ -1,0 +1,136 @@
+// Internal declarations shared by the libfb translation units.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include "fb.h"
+
+namespace fb {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// A group of `count` packed fp32 parts, part p at (a + p*stride_a, l + p*stride_l).
+struct PartGroup {
+  const float* a;
+  const float* l;
+  int32_t count;
+  int64_t stride_a, stride_l;
+};
+
+struct PartList {
+  int32_t ngroups;
+  PartGroup g[FB_MAX_PARTS];
+};
+
+// Where an attention kernel's (b, h, i) rows come from and how they are tiled.
+//   packed   (per_head = 0): unit = (b, kv head); its G*Nb rows are the block
+//            queries of the G query heads sharing that KV head, row r = g*Nb+i.
+//   per_head (per_head = 1): unit = (b, query head); rows are its Nb queries.
+struct RowMap {
+  int32_t B, Hq, Hkv, G, Nb;
+  int32_t per_head;
+  int32_t rows_per_unit;
+  int32_t row_tiles;       // tiles of the kernel's row count per unit
+  int32_t units;
+};
+
+// Arguments of the attention kernels (one launch = one key source).
+struct AttnArgs {
+  RowMap rm;
+  const void* q;
+  int64_t q_sb, q_sh, q_st;
+  const void* k;
+  const void* v;
+  int64_t k_sb, k_sh, k_st;
+  int64_t nkeys;               // keys in the source: [0, nkeys) or list entries
+  const int32_t* sel;          // per (b, query head) key list (per_head units only)
+  int32_t sel_k;
+  int64_t key_rows;            // rows addressable in the key source (list entries outside are skipped)
+  const uint32_t* excl;        // per (b, query head) bitmap: 1 = key excluded
+  int64_t excl_words;
+  int32_t nsplit;
+  int64_t keys_per_split;
+  const int8_t* mask;          // gamma: [B, Hq]; heads with mask=1 may be skipped
+  int32_t mask_active;         // 0: ignore mask
+  // epilogue 0: write part (A, L) of split s at part_a + s*part_stride_a ...
+  float* part_a;
+  float* part_l;
+  int64_t part_stride_a, part_stride_l;
+  // epilogue 1: merge with `ext` and write O / LSE
+  int32_t merge_out;
+  PartList ext;
+  void* o;
+  int64_t o_sb, o_sh, o_st;
+  int32_t o_bf16;
+  float* lse;
+  float scale_log2;            // softmax scale * log2(e)
+};
+
+// Profiling scope: brackets one launch with events on its stream when the
+// profiling hook is on (fb_profile_enable); kinds as in fb.h.
+enum { kProfPrefix = 0, kProfInblock = 1, kProfAux = 2 };
+class ProfScope {
+ public:
+  ProfScope(int kind, double alg_bytes, cudaStream_t s);
+  ~ProfScope();
+  ProfScope(const ProfScope&) = delete;
+  ProfScope& operator=(const ProfScope&) = delete;
+
+ private:
+  int kind_;
+  double bytes_;
+  cudaStream_t s_;
+  cudaEvent_t start_ = nullptr;
+};
+
+// Host-side planning helpers (fb_api.cu).
+int num_sms();
+RowMap make_rowmap(int B, int Hq, int Hkv, int Nb, int per_head, int tile_rows);
+void plan_split(int64_t tiles, int64_t nkeys, int ctas_per_sm, int key_tile,
+                int32_t* nsplit, int64_t* keys_per_split);
+
+// Launchers (return cudaGetLastError()).
+cudaError_t launch_attn_generic(const AttnArgs& a, int D, int in_bf16, cudaStream_t s);
+int generic_tile_rows(int in_bf16);
+int generic_key_tile();
+int generic_ctas_per_sm(int D, int in_bf16);
+
+struct MergeArgs {
+  int32_t B, Hq, Nb, D;
+  PartList parts;
+  void* o;
+  int64_t o_sb, o_sh, o_st;
+  int32_t o_bf16;
+  float* lse;
+  const int8_t* mask;       // rows of heads with mask=1 are skipped (or NULL)
+  int32_t mask_active;
+};
+cudaError_t launch_merge(const MergeArgs& m, cudaStream_t s);
+
+struct GammaArgs {
+  int32_t B, Hq, Nb, D;
+  PartList fresh;           // the fresh block-external part (split partials)
+  float* cache_a;           // packed [B, Hq, Nb, D]
+  float* cache_l;           // packed [B, Hq, Nb]
+  int8_t* mask;             // [B, Hq] reuse-next-step flags (read, then updated)
+  int32_t gate_active;      // host: cache valid && M < tau
+  int32_t cache_valid;      // host: a similarity can be formed
+  const float* gamma;       // device [Hq]
+  float* sim;               // device [B, Hq] state
+  float* partials;          // [B*Hq*chunks*3] scratch
+  int32_t* counters;        // [B*Hq], zero between launches
+  int32_t chunks;
+  int8_t* reuse_out;        // [B, Hq] or NULL
+  float* sim_out;           // [B, Hq] or NULL
+};
+cudaError_t launch_gamma_update(const GammaArgs& g, cudaStream_t s);
+int gamma_chunk_rows();
+
+cudaError_t launch_kv_append(const fb_attn_desc& d, void* kp, void* vp, int64_t prefix_len,
+                             const void* kin, const void* vin, cudaStream_t s);
+cudaError_t launch_build_bitmap(const int32_t* sel, int32_t sel_k, int32_t BH,
+                                uint32_t* bitmap, int64_t words, cudaStream_t s);
+cudaError_t launch_fill_decision(int8_t* reuse_out, int32_t n, int8_t value, cudaStream_t s);
+
+}  // namespace fb

@@ -251,3 +251,25 @@ class Workload:
 def get_spec(name: str, **overrides) -> WorkloadSpec:
     spec = SPECS[name]
     return spec.scaled(**overrides) if overrides else spec
+
+
+def tensor(shape, seed: int, std: float = 1.0, dtype: str = "bf16") -> torch.Tensor:
+    """A seeded N(0, std^2) tensor (fp32 draw, bf16 by round-to-nearest-even)."""
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed)))
+    x = g.standard_normal(size=tuple(shape), dtype=np.float32) * np.float32(std)
+    t = torch.from_numpy(x)
+    return t if dtype == "f32" else t.to(torch.bfloat16)
+
+
+def uniform(shape, seed: int, lo: float, hi: float) -> torch.Tensor:
+    """A seeded Uniform(lo, hi) fp32 tensor."""
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed)))
+    return torch.from_numpy(g.uniform(lo, hi, size=tuple(shape)).astype(np.float32))
+
+
+def random_selection(B: int, Hq: int, prefix_len: int, k: int, seed: int) -> torch.Tensor:
+    """k distinct ascending prefix positions per (b, h), int32 [B, Hq, k]."""
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed)))
+    out = np.stack([np.stack([np.sort(g.choice(prefix_len, size=k, replace=False)) for _ in range(Hq)])
+                    for _ in range(B)]).astype(np.int32)
+    return torch.from_numpy(out.reshape(B, Hq, k))

@@ -1,0 +1,210 @@
+"""GPU-vs-oracle parity through the C-ABI (needs a B200).
+
+Each test feeds the same seeded inputs to libfb (through its ctypes binding)
+and to the fp64 oracle, then compares element by element under the tolerances
+of tests/_gpu_common.py; reuse decisions and masks must agree bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+from block_diffusion_attention_flashblock_b200 import fb
+from block_diffusion_attention_flashblock_b200 import workloads as wl
+from oracle import flashblock_oracle as orc
+
+from _gpu_common import TOL, assert_lse_close, assert_o_close, compare_schedule
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    fb.lib()
+
+
+def _mk(B, Hq, Hkv, D, Nb, Lp, dtype, seed, cap_extra=64, std=1.0):
+    q = wl.tensor((B, Hq, Nb, D), seed, std, dtype)
+    kin = wl.tensor((B, Hkv, Nb, D), seed + 1, std, dtype)
+    vin = wl.tensor((B, Hkv, Nb, D), seed + 2, std, dtype)
+    kp = wl.tensor((B, Hkv, Lp + cap_extra, D), seed + 3, std, dtype)
+    vp = wl.tensor((B, Hkv, Lp + cap_extra, D), seed + 4, std, dtype)
+    return q, kin, vin, kp, vp
+
+
+SHAPES = [
+    # (B, Hq, Hkv, D, Nb, Lp, dtype)
+    (1, 4, 4, 64, 32, 256, "f32"),        # the tiny fp32 workload
+    (2, 4, 2, 128, 7, 300, "f32"),        # fp32, GQA, ragged
+    (1, 32, 8, 128, 32, 1000, "bf16"),    # dLLM shape, ragged prefix tail (1000 = 15*64 + 40)
+    (2, 8, 2, 64, 24, 700, "bf16"),       # D=64, G*Nb = 96 rows -> two row tiles
+    (1, 2, 2, 128, 200, 333, "bf16"),     # long block: several row tiles per head
+    (1, 32, 8, 128, 32, 8192, "bf16"),    # dLLM prefix at full size
+    (1, 8, 8, 128, 1, 129, "bf16"),       # one query, one key past a tile
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_outblock_dense(shape):
+    B, Hq, Hkv, D, Nb, Lp, dt = shape
+    q, kin, vin, kp, vp = _mk(B, Hq, Hkv, D, Nb, Lp, dt, seed=11)
+    qd, kpd, vpd = q.cuda(), kp.cuda(), vp.cuda()
+    a = torch.empty(B, Hq, Nb, D, device="cuda")
+    l = torch.empty(B, Hq, Nb, device="cuda")
+    desc = fb.make_desc(qd, kin.cuda(), kpd, a)
+    ws = torch.empty(fb.fb_outblock_workspace_bytes(desc, Lp), dtype=torch.uint8, device="cuda")
+    fb.fb_attn_outblock(desc, qd, kpd, vpd, Lp, a, l, ws)
+    A, L = orc.outblock(orc.to64(q), orc.to64(kp), orc.to64(vp), Lp, 1 / np.sqrt(D))
+    assert_o_close(a, A, TOL[dt], "A_out")
+    assert_lse_close(l, L, TOL[dt], "L_out")
+
+
+def test_outblock_empty_prefix():
+    q, kin, vin, kp, vp = _mk(1, 4, 2, 128, 16, 0, "bf16", seed=5)
+    qd, kpd = q.cuda(), kp.cuda()
+    a = torch.full((1, 4, 16, 128), 7.0, device="cuda")
+    l = torch.zeros(1, 4, 16, device="cuda")
+    desc = fb.make_desc(qd, kin.cuda(), kpd, a)
+    ws = torch.empty(fb.fb_outblock_workspace_bytes(desc, 0), dtype=torch.uint8, device="cuda")
+    fb.fb_attn_outblock(desc, qd, kpd, vp.cuda(), 0, a, l, ws)
+    assert torch.all(a == 0) and torch.all(torch.isneginf(l))
+
+
+@pytest.mark.parametrize("shape", [(1, 8, 2, 128, 32, 1500, 100, "bf16"), (1, 4, 4, 64, 32, 256, 40, "f32"),
+                                   (2, 8, 2, 128, 16, 3000, 0, "bf16"), (1, 4, 1, 128, 8, 200, 200, "bf16")],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_outblock_sparse_and_residual(shape):
+    B, Hq, Hkv, D, Nb, Lp, k, dt = shape
+    q, kin, vin, kp, vp = _mk(B, Hq, Hkv, D, Nb, Lp, dt, seed=21)
+    sel = wl.random_selection(B, Hq, Lp, k, seed=99)
+    qd, kpd, vpd = q.cuda(), kp.cuda(), vp.cuda()
+    aS = torch.empty(B, Hq, Nb, D, device="cuda"); lS = torch.empty(B, Hq, Nb, device="cuda")
+    aU = torch.empty_like(aS); lU = torch.empty_like(lS)
+    desc = fb.make_desc(qd, kin.cuda(), kpd, aS)
+    ws = torch.empty(fb.fb_outblock_workspace_bytes(desc, Lp, k), dtype=torch.uint8, device="cuda")
+    fb.fb_attn_outblock(desc, qd, kpd, vpd, Lp, aS, lS, ws, sel=sel.cuda(), sel_k=k, a_res=aU, l_res=lU)
+    sc = 1 / np.sqrt(D)
+    AS, LS = orc.outblock_selected(orc.to64(q), orc.to64(kp), orc.to64(vp), Lp, sc, sel.numpy(), residual=False)
+    AU, LU = orc.outblock_selected(orc.to64(q), orc.to64(kp), orc.to64(vp), Lp, sc, sel.numpy(), residual=True)
+    assert_o_close(aS, AS, TOL[dt], "A_S"); assert_lse_close(lS, LS, TOL[dt], "L_S")
+    assert_o_close(aU, AU, TOL[dt], "A_U"); assert_lse_close(lU, LU, TOL[dt], "L_U")
+
+
+def _random_parts(B, Hq, Nb, D, n, seed, empty_rows=True):
+    parts = []
+    for p in range(n):
+        A = wl.tensor((B, Hq, Nb, D), seed + 10 * p, 1.0, "f32")
+        L = wl.tensor((B, Hq, Nb), seed + 10 * p + 1, 3.0, "f32")
+        if empty_rows and p == 0:
+            L[..., ::5] = -float("inf")
+            A[..., ::5, :] = 0.0
+        parts.append((A, L))
+    return parts
+
+
+@pytest.mark.parametrize("nparts", [0, 1, 2])
+@pytest.mark.parametrize("shape", [(1, 32, 8, 128, 32, "bf16"), (1, 4, 4, 64, 32, "f32"),
+                                   (1, 3, 3, 128, 150, "bf16"), (2, 8, 4, 64, 5, "bf16")],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_inblock_merge(shape, nparts):
+    B, Hq, Hkv, D, Nb, dt = shape
+    q, kin, vin, kp, vp = _mk(B, Hq, Hkv, D, Nb, 8, dt, seed=31)
+    parts = _random_parts(B, Hq, Nb, D, nparts, seed=300)
+    o = torch.empty(B, Hq, Nb, D, device="cuda")
+    lse = torch.empty(B, Hq, Nb, device="cuda")
+    desc = fb.make_desc(q.cuda(), kin.cuda(), kp.cuda(), o)
+    fb.fb_attn_inblock(desc, q.cuda(), kin.cuda(), vin.cuda(), o, lse,
+                       [a.cuda() for a, _ in parts], [l.cuda() for _, l in parts])
+    Ai, Li = orc.inblock(orc.to64(q), orc.to64(kin), orc.to64(vin), 1 / np.sqrt(D))
+    A, L = orc.merge([(orc.to64(a), orc.to64(l)) for a, l in parts] + [(Ai, Li)])
+    assert_o_close(o, A, TOL[dt], "O"); assert_lse_close(lse, L, TOL[dt], "LSE")
+
+
+@pytest.mark.parametrize("nparts", [1, 2, 5, 8])
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+def test_merge_nway(nparts, out):
+    B, Hq, Nb, D = 2, 6, 37, 128
+    parts = _random_parts(B, Hq, Nb, D, nparts, seed=500)
+    if nparts >= 2:   # rows where every part is empty
+        for a, l in parts:
+            l[0, 0, 3] = -float("inf"); a[0, 0, 3] = 0.0
+    dt = torch.float32 if out == "f32" else torch.bfloat16
+    o = torch.empty(B, Hq, Nb, D, dtype=dt, device="cuda")
+    lse = torch.empty(B, Hq, Nb, device="cuda")
+    q = torch.empty(B, Hq, Nb, D, dtype=torch.bfloat16, device="cuda")
+    desc = fb.make_desc(q, q, q, o)
+    fb.fb_merge(desc, [a.cuda() for a, _ in parts], [l.cuda() for _, l in parts], o, lse)
+    A, L = orc.merge([(orc.to64(a), orc.to64(l)) for a, l in parts])
+    assert_o_close(o, A, 1e-6 if out == "f32" else 0.0, "merge O")
+    assert_lse_close(lse, L, 1e-6, "merge LSE")
+
+
+def test_kv_append_bit_exact():
+    B, Hkv, Nb, D, cap = 2, 3, 40, 128, 300
+    kp = wl.tensor((B, Hkv, cap, D), 1); vp = wl.tensor((B, Hkv, cap, D), 2)
+    kin = wl.tensor((B, Hkv, Nb, D), 3); vin = wl.tensor((B, Hkv, Nb, D), 4)
+    kpd, vpd = kp.cuda(), vp.cuda()
+    q = torch.empty(B, Hkv, Nb, D, dtype=torch.bfloat16, device="cuda")
+    desc = fb.make_desc(q, kin.cuda(), kpd, q)
+    fb.fb_kv_append(desc, kpd, vpd, 100, kin.cuda(), vin.cuda())
+    K, V, n = orc.kv_append(kp.float().numpy(), vp.float().numpy(), 100, kin.float().numpy(), vin.float().numpy())
+    assert n == 140
+    assert np.array_equal(kpd.float().cpu().numpy(), K) and np.array_equal(vpd.float().cpu().numpy(), V)
+    with pytest.raises(fb.FbError):
+        fb.fb_kv_append(desc, kpd, vpd, 270, kin.cuda(), vin.cuda())
+
+
+# ------------------------------------------------------------ schedules ---
+SCHEDULES = {
+    "tiny_f32": dict(),
+    "dllm_8k_small": dict(base="dllm_8k", prefix0=1000, blocks=2, steps=8),
+    "dllm_64k_small": dict(base="dllm_64k_b4", B=2, prefix0=2000, steps=16),
+    "video_small_mixed": dict(base="video_1560", Hq=6, Hkv=6, prefix0=3120, steps=5, sigma_range=(0.01, 1.0)),
+    "video_small": dict(base="video_1560", Hq=4, Hkv=4, prefix0=3120, steps=4),
+    "sparse_small": dict(base="sparse_32k_k2048", prefix0=4000, sel_k=256, Hq=8, Hkv=2),
+    "tau_zero": dict(base="dllm_8k", prefix0=500, blocks=1, steps=4, tau=0),
+    "tau_off": dict(base="dllm_8k", prefix0=500, blocks=1, steps=4, tau=None),
+    "nb1_gqa": dict(base="dllm_8k", Nb=1, prefix0=300, steps=3, m_model=("uniform", 0, 1), tau=1),
+}
+
+
+def _spec(name):
+    kw = dict(SCHEDULES[name])
+    base = kw.pop("base", name)
+    return wl.get_spec(base, **kw)
+
+
+@pytest.mark.parametrize("name", list(SCHEDULES))
+def test_step_schedule(name):
+    spec = _spec(name)
+    st = compare_schedule(spec)
+    if name == "tau_zero":
+        assert all(st["recomputed"])
+    if name == "tau_off":
+        assert st["recomputed"] == [True, False, False, False]
+    if name == "video_small_mixed":
+        r = np.array(st["reuse"])
+        assert 0 < r[2:].mean() < 1, "the mixed video case should both reuse and recompute"
+
+
+def test_step_bf16_output():
+    spec = wl.get_spec("dllm_8k", prefix0=700, blocks=1, steps=4)
+    compare_schedule(spec, out_dtype=torch.bfloat16)
+
+
+# ------------------------------------------------ full-size workloads ---
+def test_full_dllm_8k_all_heads():
+    """The benchmarked workload at its full size: 4 blocks x 8 steps, every head."""
+    compare_schedule(wl.get_spec("dllm_8k"), check_every=1)
+
+
+@pytest.mark.parametrize("name, groups", [
+    ("dllm_64k_b4", [(0, 0), (3, 7)]),
+    ("video_1560", [(0, 0), (0, 13), (0, 23)]),
+    ("sparse_32k_k2048", [(0, 0), (0, 5)]),
+])
+def test_full_size_sampled_heads(name, groups):
+    """Full-size workloads; the oracle recomputes only the sampled (b, kv-head) groups."""
+    spec = wl.get_spec(name)
+    compare_schedule(spec, groups=groups, check_every=1 if name != "dllm_64k_b4" else 5)
