@@ -239,7 +239,14 @@ static fb_status run_inblock(const fb_attn_desc& d, const void* q, const void* k
   a.nsplit = 1;
   a.keys_per_split = d.Nb;
   a.merge_out = 1;
-  a.ext = ext;
+  a.next = 0;
+  for (int gi = 0; gi < ext.ngroups; ++gi)
+    for (int p = 0; p < ext.g[gi].count; ++p) {
+      if (a.next >= FB_MAX_PARTS) return FB_EINVAL;
+      a.ext_a[a.next] = ext.g[gi].a + p * ext.g[gi].stride_a;
+      a.ext_l[a.next] = ext.g[gi].l + p * ext.g[gi].stride_l;
+      ++a.next;
+    }
   a.o = o; a.o_sb = d.o_strides[0]; a.o_sh = d.o_strides[1]; a.o_st = d.o_strides[2];
   a.o_bf16 = d.out_dtype == FB_BF16;
   a.lse = lse;
@@ -608,7 +615,17 @@ fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
     if (sparse) {
       PassPlan p = plan_pass(d, a->q, a->kp, a->vp, d.kp_strides, a->prefix_len, a->sel, a->sel_k, c->sel_cap);
       if ((st = launch_pass(d, p.a, c->sel_a, c->sel_l, s)) != FB_OK) return st;
-      ext.g[ext.ngroups++] = group_of(c->sel_a, c->sel_l, p.nsplit, d);
+      if (p.nsplit > FB_MAX_PARTS - 1) {
+        // fold the splits into split 0's slot (each row is read fully before it is written)
+        PartList lst;
+        memset(&lst, 0, sizeof(lst));
+        lst.ngroups = 1;
+        lst.g[0] = group_of(c->sel_a, c->sel_l, p.nsplit, d);
+        if ((st = merge_to_part(d, lst, c->sel_a, c->sel_l, nullptr, 0, s)) != FB_OK) return st;
+        ext.g[ext.ngroups++] = group_of(c->sel_a, c->sel_l, 1, d);
+      } else {
+        ext.g[ext.ngroups++] = group_of(c->sel_a, c->sel_l, p.nsplit, d);
+      }
     }
     if (!tau_reuse) {
       PassPlan p = plan_pass(d, a->q, a->kp, a->vp, d.kp_strides, a->prefix_len, nullptr, 0, c->part_cap);

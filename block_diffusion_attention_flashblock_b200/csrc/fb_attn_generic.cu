@@ -102,56 +102,43 @@ __device__ __forceinline__ uint32_t pack_bf16(float x, float y) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Merge epilogue: the weights of a row's in-kernel part (normaliser L_in) and
-// of its external parts, m = max L, w_p = e^{L_p - m}, 1 / sum w, LSE.
-struct ExtWeights {
-  float w_in, inv_sum, lse, m;
+// Split a pair of fp32 values into bf16 hi + lo parts (x = hi + lo to about
+// 2^-16 relative), so that P V with bf16 operands keeps fp32-level accuracy.
+__device__ __forceinline__ void split_bf16(float x, float y, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x - hf.x, y - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// Merge epilogue weights of one row: the in-kernel part has normaliser L_in,
+// the external parts L_p (prefetched in Lx); m = max, w = e^{L - m}.
+struct RowMerge {
+  float m, w_in, inv_sum, lse;
+  float w[FB_MAX_PARTS];
   bool empty;
 };
 
-__device__ __forceinline__ ExtWeights ext_weights(const PartList& ext, int64_t row, float L_in) {
+__device__ __forceinline__ RowMerge row_merge(int next, const float* Lx, float L_in) {
+  RowMerge r;
   float m = L_in;
-  for (int gi = 0; gi < ext.ngroups; ++gi) {
-    const PartGroup& g = ext.g[gi];
-    for (int p = 0; p < g.count; ++p) m = fmaxf(m, __ldg(g.l + p * g.stride_l + row));
-  }
-  ExtWeights w;
-  w.m = m;
-  w.empty = (m == -CUDART_INF_F);
-  if (w.empty) {
-    w.w_in = 0.f; w.inv_sum = 0.f; w.lse = -CUDART_INF_F;
-    return w;
-  }
+#pragma unroll
+  for (int p = 0; p < FB_MAX_PARTS; ++p)
+    if (p < next) m = fmaxf(m, Lx[p]);
+  r.m = m;
+  r.empty = (m == -CUDART_INF_F);
   float sum = 0.f;
-  w.w_in = (L_in == -CUDART_INF_F) ? 0.f : expf(L_in - m);
-  sum += w.w_in;
-  for (int gi = 0; gi < ext.ngroups; ++gi) {
-    const PartGroup& g = ext.g[gi];
-    for (int p = 0; p < g.count; ++p) {
-      const float L = __ldg(g.l + p * g.stride_l + row);
-      sum += (L == -CUDART_INF_F) ? 0.f : expf(L - m);
-    }
+  r.w_in = (r.empty || L_in == -CUDART_INF_F) ? 0.f : expf(L_in - m);
+  sum += r.w_in;
+#pragma unroll
+  for (int p = 0; p < FB_MAX_PARTS; ++p) {
+    r.w[p] = (p < next && !r.empty && Lx[p] != -CUDART_INF_F) ? expf(Lx[p] - m) : 0.f;
+    sum += r.w[p];
   }
-  w.inv_sum = 1.f / sum;
-  w.lse = m + logf(sum);
-  return w;
-}
-
-// Sum over external parts of w_p * A_p[row, col..col+1].
-__device__ __forceinline__ float2 ext_accum2(const PartList& ext, int64_t row, int D, int col, float m) {
-  float2 acc = make_float2(0.f, 0.f);
-  for (int gi = 0; gi < ext.ngroups; ++gi) {
-    const PartGroup& g = ext.g[gi];
-    for (int p = 0; p < g.count; ++p) {
-      const float L = __ldg(g.l + p * g.stride_l + row);
-      if (L == -CUDART_INF_F) continue;
-      const float w = expf(L - m);
-      const float2 v = __ldg(reinterpret_cast<const float2*>(g.a + p * g.stride_a + row * D + col));
-      acc.x += w * v.x;
-      acc.y += w * v.y;
-    }
-  }
-  return acc;
+  r.inv_sum = r.empty ? 0.f : 1.f / sum;
+  r.lse = r.empty ? -CUDART_INF_F : m + logf(sum);
+  return r;
 }
 
 }  // namespace
@@ -217,12 +204,24 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
   const int rA = warp * 16 + (lane >> 2);
   RowInfo rowi[2] = {map_row(rm, unit, row0 + rA), map_row(rm, unit, row0 + rA + 8)};
 
+  // Normalisers of the external parts of this thread's two rows, fetched
+  // early so the merge epilogue waits on memory only once per part.
+  float Lx[2][FB_MAX_PARTS];
+  if (a.merge_out) {
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const int64_t row = ((int64_t)rowi[rr].b * rm.Hq + rowi[rr].h) * rm.Nb + rowi[rr].i;
+#pragma unroll
+      for (int p = 0; p < FB_MAX_PARTS; ++p)
+        Lx[rr][p] = (p < a.next && rowi[rr].valid) ? __ldg(a.ext_l[p] + row) : -CUDART_INF_F;
+    }
+  }
+
   float o[DT][4];
 #pragma unroll
   for (int i = 0; i < DT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   float m_run[2] = {-CUDART_INF_F, -CUDART_INF_F};
   float l_run[2] = {0.f, 0.f};
-  uint32_t qf[KS][4];
 
   for (int t = 0; t < ntiles; ++t) {
     if (t + 1 < ntiles) {
@@ -233,13 +232,6 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
       cp_async_wait<0>();
     }
     __syncthreads();
-    if (t == 0) {
-#pragma unroll
-      for (int kk = 0; kk < KS; ++kk) {
-        const int r = warp * 16 + (lane & 15), ch = 2 * kk + (lane >> 4);
-        ldsm_x4(smem_u32(sQ + r * D + ((ch ^ (r & 7)) * 8)), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
-      }
-    }
     const __nv_bfloat16* cK = sK + (t & 1) * BN * D;
     const __nv_bfloat16* cV = sV + (t & 1) * BN * D;
 
@@ -249,13 +241,18 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
     for (int i = 0; i < NT; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < KS; ++kk) {
+      uint32_t qf[4];   // Q fragment, re-read from shared memory (keeps registers for P hi/lo)
+      {
+        const int r = warp * 16 + (lane & 15), ch = 2 * kk + (lane >> 4);
+        ldsm_x4(smem_u32(sQ + r * D + ((ch ^ (r & 7)) * 8)), qf[0], qf[1], qf[2], qf[3]);
+      }
 #pragma unroll
       for (int nt = 0; nt < NT; nt += 2) {
         const int r = (nt + (lane >> 4)) * 8 + (lane & 7), ch = 2 * kk + ((lane >> 3) & 1);
         uint32_t b0, b1, b2, b3;
         ldsm_x4(smem_u32(cK + r * D + ((ch ^ (r & 7)) * 8)), b0, b1, b2, b3);
-        mma_bf16(s[nt], qf[kk], b0, b1);
-        mma_bf16(s[nt + 1], qf[kk], b2, b3);
+        mma_bf16(s[nt], qf, b0, b1);
+        mma_bf16(s[nt + 1], qf, b2, b3);
       }
     }
 
@@ -306,20 +303,22 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
       o[i][0] *= alpha[0]; o[i][1] *= alpha[0];
       o[i][2] *= alpha[1]; o[i][3] *= alpha[1];
     }
-    uint32_t pf[NT][2];
+    // P = 2^(s - m) as bf16 hi + lo (P V below adds both products).
+    uint32_t pf[NT][2], pr[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const float p0 = exp2f(s[nt][0] - mref[0]), p1 = exp2f(s[nt][1] - mref[0]);
       const float p2 = exp2f(s[nt][2] - mref[1]), p3 = exp2f(s[nt][3] - mref[1]);
       l_run[0] += p0 + p1;
       l_run[1] += p2 + p3;
-      pf[nt][0] = pack_bf16(p0, p1);
-      pf[nt][1] = pack_bf16(p2, p3);
+      split_bf16(p0, p1, pf[nt][0], pr[nt][0]);
+      split_bf16(p2, p3, pf[nt][1], pr[nt][1]);
     }
-    // O += P V.
+    // O += P_hi V + P_lo V.
 #pragma unroll
     for (int kk = 0; kk < BN / 16; ++kk) {
       const uint32_t af[4] = {pf[2 * kk][0], pf[2 * kk][1], pf[2 * kk + 1][0], pf[2 * kk + 1][1]};
+      const uint32_t ar[4] = {pr[2 * kk][0], pr[2 * kk][1], pr[2 * kk + 1][0], pr[2 * kk + 1][1]};
 #pragma unroll
       for (int dt = 0; dt < DT; dt += 2) {
         const int r = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8, ch = dt + (lane >> 4);
@@ -327,6 +326,8 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
         ldsm_x4_t(smem_u32(cV + r * D + ((ch ^ (r & 7)) * 8)), b0, b1, b2, b3);
         mma_bf16(o[dt], af, b0, b1);
         mma_bf16(o[dt + 1], af, b2, b3);
+        mma_bf16(o[dt], ar, b0, b1);
+        mma_bf16(o[dt + 1], ar, b2, b3);
       }
     }
     __syncthreads();
@@ -372,18 +373,30 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
       const RowInfo& ri = rowi[rr];
       if (!ri.valid) continue;
       const int64_t row = ((int64_t)ri.b * Hq + ri.h) * Nb + ri.i;
-      const ExtWeights w = ext_weights(a.ext, row, Lrow[rr]);
+      const RowMerge w = row_merge(a.next, Lx[rr], Lrow[rr]);
+      const float win = w.w_in * inv[rr];
+      float2 acc[DT];
+#pragma unroll
+      for (int dt = 0; dt < DT; ++dt)
+        acc[dt] = make_float2(win * o[dt][2 * rr], win * o[dt][2 * rr + 1]);
+#pragma unroll
+      for (int p = 0; p < FB_MAX_PARTS; ++p) {
+        if (p >= a.next || w.w[p] == 0.f) continue;
+        const float* pa = a.ext_a[p] + row * D + 2 * (lane & 3);
+        float2 v[DT];
+#pragma unroll
+        for (int dt = 0; dt < DT; ++dt) v[dt] = __ldg(reinterpret_cast<const float2*>(pa + dt * 8));
+#pragma unroll
+        for (int dt = 0; dt < DT; ++dt) {
+          acc[dt].x = fmaf(w.w[p], v[dt].x, acc[dt].x);
+          acc[dt].y = fmaf(w.w[p], v[dt].y, acc[dt].y);
+        }
+      }
       const int64_t obase = ri.b * a.o_sb + ri.h * a.o_sh + ri.i * a.o_st;
 #pragma unroll
       for (int dt = 0; dt < DT; ++dt) {
         const int col = dt * 8 + 2 * (lane & 3);
-        float2 r2 = make_float2(0.f, 0.f);
-        if (!w.empty) {
-          const float2 e = ext_accum2(a.ext, row, D, col, w.m);
-          const float win = w.w_in * inv[rr];
-          r2.x = (e.x + win * o[dt][2 * rr]) * w.inv_sum;
-          r2.y = (e.y + win * o[dt][2 * rr + 1]) * w.inv_sum;
-        }
+        const float2 r2 = make_float2(acc[dt].x * w.inv_sum, acc[dt].y * w.inv_sum);
         if (a.o_bf16) {
           *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(a.o) + obase + col) =
               __floats2bfloat162_rn(r2.x, r2.y);
@@ -482,17 +495,28 @@ __global__ void __launch_bounds__(64 * (D / 64)) attn_f32_kernel(const AttnArgs 
       *reinterpret_cast<float4*>(pa + d) = make_float4(o[d] * inv, o[d + 1] * inv, o[d + 2] * inv, o[d + 3] * inv);
     if (half == 0) (a.part_l + split * a.part_stride_l)[row] = Lrow;
   } else {
-    const ExtWeights w = ext_weights(a.ext, row, Lrow);
+    float Lx[FB_MAX_PARTS];
+#pragma unroll
+    for (int p = 0; p < FB_MAX_PARTS; ++p) Lx[p] = p < a.next ? __ldg(a.ext_l[p] + row) : -CUDART_INF_F;
+    const RowMerge w = row_merge(a.next, Lx, Lrow);
     const int64_t obase = ri.b * a.o_sb + ri.h * a.o_sh + ri.i * a.o_st + half * DH;
     const float win = w.w_in * inv;
 #pragma unroll
-    for (int d = 0; d < DH; d += 2) {
-      float2 r2 = make_float2(0.f, 0.f);
-      if (!w.empty) {
-        const float2 e = ext_accum2(a.ext, row, D, half * DH + d, w.m);
-        r2.x = (e.x + win * o[d]) * w.inv_sum;
-        r2.y = (e.y + win * o[d + 1]) * w.inv_sum;
+    for (int d = 0; d < DH; ++d) o[d] *= win;
+#pragma unroll
+    for (int p = 0; p < FB_MAX_PARTS; ++p) {
+      if (p >= a.next || w.w[p] == 0.f) continue;
+      const float* pa = a.ext_a[p] + row * D + half * DH;
+#pragma unroll
+      for (int d = 0; d < DH; d += 4) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(pa + d));
+        o[d] = fmaf(w.w[p], v.x, o[d]); o[d + 1] = fmaf(w.w[p], v.y, o[d + 1]);
+        o[d + 2] = fmaf(w.w[p], v.z, o[d + 2]); o[d + 3] = fmaf(w.w[p], v.w, o[d + 3]);
       }
+    }
+#pragma unroll
+    for (int d = 0; d < DH; d += 2) {
+      const float2 r2 = make_float2(o[d] * w.inv_sum, o[d + 1] * w.inv_sum);
       if (a.o_bf16)
         *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(a.o) + obase + d) =
             __floats2bfloat162_rn(r2.x, r2.y);

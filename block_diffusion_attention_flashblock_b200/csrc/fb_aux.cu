@@ -47,13 +47,21 @@ __device__ __forceinline__ void store_out(void* o, int64_t off, bool bf16, const
 
 // Merge all parts of one row (lane holds columns lane*E .. lane*E+E-1):
 // m = max L_p, w_p = e^{L_p - m}; returns sum w_p A_p / sum w_p and the LSE.
+// Loads are issued in batches of independent requests (no load waits on a
+// branch over another load's value), so a row costs a few memory round trips.
 template <int D>
 __device__ __forceinline__ float merge_row(const PartList& pl, int64_t row, int lane, float* out) {
-  constexpr int E = D / 32;
+  constexpr int E = D / 32, U = 4;
   float m = -CUDART_INF_F;
   for (int gi = 0; gi < pl.ngroups; ++gi) {
     const PartGroup& g = pl.g[gi];
-    for (int p = 0; p < g.count; ++p) m = fmaxf(m, __ldg(g.l + p * g.stride_l + row));
+    for (int p0 = 0; p0 < g.count; p0 += 2 * U) {
+      float Ls[2 * U];
+#pragma unroll
+      for (int u = 0; u < 2 * U; ++u) Ls[u] = p0 + u < g.count ? __ldg(g.l + (p0 + u) * g.stride_l + row) : -CUDART_INF_F;
+#pragma unroll
+      for (int u = 0; u < 2 * U; ++u) m = fmaxf(m, Ls[u]);
+    }
   }
 #pragma unroll
   for (int e = 0; e < E; ++e) out[e] = 0.f;
@@ -61,15 +69,26 @@ __device__ __forceinline__ float merge_row(const PartList& pl, int64_t row, int 
   float wsum = 0.f;
   for (int gi = 0; gi < pl.ngroups; ++gi) {
     const PartGroup& g = pl.g[gi];
-    for (int p = 0; p < g.count; ++p) {
-      const float L = __ldg(g.l + p * g.stride_l + row);
-      if (L == -CUDART_INF_F) continue;
-      const float w = expf(L - m);
-      wsum += w;
-      Vec<D> a;
-      a.load(g.a + p * g.stride_a + row * D + lane * E);
+    for (int p0 = 0; p0 < g.count; p0 += U) {
+      float Ls[U];
+      Vec<D> A[U];
 #pragma unroll
-      for (int e = 0; e < E; ++e) out[e] = fmaf(w, a.v[e], out[e]);
+      for (int u = 0; u < U; ++u) {
+        const bool ok = p0 + u < g.count;
+        Ls[u] = ok ? __ldg(g.l + (p0 + u) * g.stride_l + row) : -CUDART_INF_F;
+        if (ok) A[u].load(g.a + (p0 + u) * g.stride_a + row * D + lane * E);
+        else {
+#pragma unroll
+          for (int e = 0; e < E; ++e) A[u].v[e] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const float w = Ls[u] == -CUDART_INF_F ? 0.f : expf(Ls[u] - m);
+        wsum += w;
+#pragma unroll
+        for (int e = 0; e < E; ++e) out[e] = fmaf(w, A[u].v[e], out[e]);
+      }
     }
   }
   const float inv = 1.f / wsum;

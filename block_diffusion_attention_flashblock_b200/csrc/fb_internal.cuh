@@ -57,9 +57,11 @@ struct AttnArgs {
   float* part_a;
   float* part_l;
   int64_t part_stride_a, part_stride_l;
-  // epilogue 1: merge with `ext` and write O / LSE
+  // epilogue 1: merge with up to FB_MAX_PARTS packed parts and write O / LSE
   int32_t merge_out;
-  PartList ext;
+  int32_t next;
+  const float* ext_a[FB_MAX_PARTS];
+  const float* ext_l[FB_MAX_PARTS];
   void* o;
   int64_t o_sb, o_sh, o_st;
   int32_t o_bf16;

@@ -159,9 +159,25 @@ def fb_outblock_workspace_bytes(desc: fb_attn_desc, prefix_len: int, sel_k: int 
     return n.value
 
 
+def _sel_ptr(sel: Optional[torch.Tensor]) -> Optional[int]:
+    """A selection list marks a sparse call even when it is empty (k = 0): an
+    empty tensor has no storage, so pass the address of a one-element stand-in."""
+    if sel is None:
+        return None
+    if sel.numel() == 0:
+        global _EMPTY_SEL
+        if _EMPTY_SEL is None or _EMPTY_SEL.device != sel.device:
+            _EMPTY_SEL = torch.zeros(4, dtype=torch.int32, device=sel.device)
+        return _EMPTY_SEL.data_ptr()
+    return sel.data_ptr()
+
+
+_EMPTY_SEL = None
+
+
 def fb_attn_outblock(desc, q, kp, vp, prefix_len, a_out, l_out, ws, sel=None, sel_k=0,
                      a_res=None, l_res=None, stream=None):
-    _check(lib().fb_attn_outblock(C.byref(desc), _ptr(q), _ptr(kp), _ptr(vp), prefix_len, _ptr(sel),
+    _check(lib().fb_attn_outblock(C.byref(desc), _ptr(q), _ptr(kp), _ptr(vp), prefix_len, _sel_ptr(sel),
                                   sel_k, _ptr(a_out), _ptr(l_out), _ptr(a_res), _ptr(l_res), _ptr(ws),
                                   ws.numel() * ws.element_size(), _stream(stream)), "fb_attn_outblock")
 
@@ -210,7 +226,7 @@ def fb_step(h, q, kin, vin, kp, vp, prefix_len, M, tau, o, lse=None, gamma=None,
     a = fb_step_args()
     a.q, a.kin, a.vin, a.kp, a.vp = _ptr(q), _ptr(kin), _ptr(vin), _ptr(kp), _ptr(vp)
     a.prefix_len, a.M, a.tau = prefix_len, M, tau
-    a.gamma, a.sel = _ptr(gamma), _ptr(sel)
+    a.gamma, a.sel = _ptr(gamma), _sel_ptr(sel)
     a.sel_k = 0 if sel is None else sel.shape[-1]
     a.o, a.lse, a.reuse_out, a.sim_out = _ptr(o), _ptr(lse), _ptr(reuse_out), _ptr(sim_out)
     _check(lib().fb_step(h, C.byref(a), _stream(stream)), "fb_step")

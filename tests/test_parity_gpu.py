@@ -136,7 +136,7 @@ def test_merge_nway(nparts, out):
     desc = fb.make_desc(q, q, q, o)
     fb.fb_merge(desc, [a.cuda() for a, _ in parts], [l.cuda() for _, l in parts], o, lse)
     A, L = orc.merge([(orc.to64(a), orc.to64(l)) for a, l in parts])
-    assert_o_close(o, A, 1e-6 if out == "f32" else 0.0, "merge O")
+    assert_o_close(o, A, 1e-6, "merge O")
     assert_lse_close(lse, L, 1e-6, "merge LSE")
 
 
