@@ -1,0 +1,574 @@
+// Block-external attention on the fifth-generation tensor cores (sm_100a):
+// the FlashBlock prefix pass, A_out with L_out = log Z_out over the prefix KV
+// cache (FlashBlock summary, "Mécanisme Central"), for bf16 inputs, D = 128.
+//
+// One CTA = one tile of 128 query rows (the block queries of the query heads
+// that share a KV head, packed) x one split of the prefix keys.  Warp roles:
+//   warp 0      TMA producer: Q once, then K and V tiles of 128 keys into a
+//               two-stage ring (cp.async.bulk.tensor, 128-byte swizzle, no
+//               multicast).
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma:
+//               S = Q K^T into one of two TMEM S buffers, and
+//               O += P_hi V + P_lo V into the TMEM O accumulator.
+//   warps 2..5  softmax, one query row per thread (TMEM lane = row): read S
+//               with tcgen05.ld, online max/sum in the log2 domain, write
+//               P = 2^(s - m) as bf16 hi + lo into swizzled shared memory for
+//               the PV product; the final O / l and L go to the split's part.
+// The running max is only moved (and O rescaled in TMEM) when a row's max
+// grows by more than 2^8, so P stays <= 256 and most tiles skip the rescale.
+// Every mbarrier wait is bounded; on expiry the CTA records FB_ETIMEOUT in
+// the device status word, drains its own TMA and MMA work, frees TMEM and
+// exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math_constants.h>
+
+#include "fb_internal.cuh"
+
+namespace fb {
+
+namespace {
+
+constexpr int kBM = 128, kBN = 128, kD = 128;
+constexpr int kThreads = 192;
+constexpr uint32_t kHalf = 16384;                 // [128 rows][64 bf16] 128B-swizzled block
+constexpr uint32_t kOffQ = 0;                     // Q: 2 halves
+constexpr uint32_t kOffK = kOffQ + 2 * kHalf;     // K: 2 stages x 2 halves
+constexpr uint32_t kOffV = kOffK + 4 * kHalf;     // V: 2 stages x 2 halves
+constexpr uint32_t kOffP = kOffV + 4 * kHalf;     // P: hi 2 halves, lo 2 halves
+constexpr uint32_t kOffBar = kOffP + 4 * kHalf;   // barriers and flags
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + slack for 1024-byte alignment
+constexpr uint32_t kTmemCols = 512;               // S0 [0,128) S1 [128,256) O [256,384)
+constexpr uint32_t kTmemO = 256;
+constexpr float kRescaleLog2 = 8.0f;
+
+// barrier slots
+enum {
+  B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 3, B_VFULL = 5, B_VEMPTY = 7, B_SFULL = 9, B_SFREE = 11,
+  B_PFULL = 13, B_PVDONE = 14, B_DRAIN = 15, B_COUNT = 16
+};
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Shared control block: first-failure flag, TMEM base.
+struct Ctl {
+  volatile int* abort;
+  int* status;
+  uint64_t limit_ns;
+};
+
+// Bounded wait for the phase of `parity` to complete.  Gives up when the limit
+// passes or another role has given up; the first to give up records the error.
+__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const Ctl& c) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try(bar, parity)) return true;
+    if (*c.abort) return false;
+    if (globaltimer() - t0 > c.limit_ns) {
+      if (atomicExch(const_cast<int*>(c.abort), 1) == 0) atomicCAS(c.status, 0, (int)FB_ETIMEOUT);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm, uint32_t bar, int c0, int c1,
+                                            int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+      "%5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+      : "memory");
+}
+
+// tcgen05 wrappers
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accum) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%"
+      "19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%"
+      "18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+      "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+      "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])),
+      "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+      "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])),
+      "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
+      "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
+      "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, 128-byte swizzle (layout code 2), sm_100
+// version bit 46; lbo/sbo in bytes.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16: D fp32, A/B bf16, M = 128, N = 128.
+constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t kIdescQK = kIdescBase;              // A, B K-major
+constexpr uint32_t kIdescPV = kIdescBase | (1u << 16);  // B (V) MN-major
+
+__device__ __forceinline__ uint32_t pack2_bf16(float x, float y) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+}  // namespace
+
+struct TcArgs {
+  int32_t B, Hq, Hkv, G, Nb;
+  int32_t mode;            // 0: unit (b, kv head), tile = hg heads x Nb queries; 1: unit (b, q head), 128 queries
+  int32_t hg;
+  int32_t tiles_per_unit;
+  int64_t nkeys;
+  int64_t keys_per_split;
+  float scale_log2;
+  float* part_a;
+  float* part_l;
+  int64_t part_stride_a, part_stride_l;
+  const int8_t* mask;
+  int32_t mask_active;
+  int* status;
+  uint64_t wait_limit_ns;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffBar + B_COUNT * 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBar + B_COUNT * 8 + 4);
+  auto bar = [&](int i) { return smem_addr(bars + i); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile_id = blockIdx.x, split = blockIdx.y;
+  const int unit = tile_id / a.tiles_per_unit, t = tile_id % a.tiles_per_unit;
+  int b, kvh, h0, i0;
+  if (a.mode == 0) {
+    b = unit / a.Hkv; kvh = unit % a.Hkv; h0 = kvh * a.G + t * a.hg; i0 = 0;
+  } else {
+    b = unit / a.Hq; h0 = unit % a.Hq; kvh = h0 / a.G; i0 = t * kBM;
+  }
+  // gamma gate: skip the tile when every query head in it reuses its cache
+  if (a.mask_active) {
+    const int hn = a.mode == 0 ? min(a.hg, a.G - t * a.hg) : 1;
+    bool all = true;
+    for (int h = h0; h < h0 + hn; ++h) all = all && a.mask[b * a.Hq + h];
+    if (all) return;
+  }
+  const int64_t kbeg = (int64_t)split * a.keys_per_split;
+  const int64_t kend = min(kbeg + a.keys_per_split, a.nkeys);
+  const int T = kend > kbeg ? (int)((kend - kbeg + kBN - 1) / kBN) : 0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < B_COUNT; ++i) {
+      uint32_t cnt = 1;
+      if (i == B_SFREE || i == B_SFREE + 1 || i == B_PFULL) cnt = 128;
+      mbar_init(bar(i), cnt);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Ctl ctl{abort_flag, a.status, a.wait_limit_ns};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && T > 0) {
+      int armed_k[2] = {-1, -1}, armed_v[2] = {-1, -1};
+      bool ok = true;
+      mbar_expect_tx(bar(B_QFULL), 2 * kHalf);
+      tma_load_4d(sbase + kOffQ, &tmQ, bar(B_QFULL), 0, i0, h0, b);
+      tma_load_4d(sbase + kOffQ + kHalf, &tmQ, bar(B_QFULL), 64, i0, h0, b);
+      for (int j = 0; j < T && ok; ++j) {
+        const int st = j & 1;
+        const int key0 = (int)(kbeg + (int64_t)j * kBN);
+        if (j >= 2) ok = wait_bounded(bar(B_KEMPTY + st), ((j >> 1) - 1) & 1, ctl);
+        if (!ok) break;
+        mbar_expect_tx(bar(B_KFULL + st), 2 * kHalf);
+        tma_load_4d(sbase + kOffK + st * 2 * kHalf, &tmK, bar(B_KFULL + st), 0, key0, kvh, b);
+        tma_load_4d(sbase + kOffK + st * 2 * kHalf + kHalf, &tmK, bar(B_KFULL + st), 64, key0, kvh, b);
+        armed_k[st] = j >> 1;
+        if (j >= 2) ok = wait_bounded(bar(B_VEMPTY + st), ((j >> 1) - 1) & 1, ctl);
+        if (!ok) break;
+        mbar_expect_tx(bar(B_VFULL + st), 2 * kHalf);
+        tma_load_4d(sbase + kOffV + st * 2 * kHalf, &tmV, bar(B_VFULL + st), 0, key0, kvh, b);
+        tma_load_4d(sbase + kOffV + st * 2 * kHalf + kHalf, &tmV, bar(B_VFULL + st), 64, key0, kvh, b);
+        armed_v[st] = j >> 1;
+      }
+      // Let every copy this thread started land before the CTA can exit.
+      const Ctl drain{abort_flag, a.status, a.wait_limit_ns};
+      wait_bounded(bar(B_QFULL), 0, drain);
+      for (int st = 0; st < 2; ++st) {
+        if (armed_k[st] >= 0) wait_bounded(bar(B_KFULL + st), armed_k[st] & 1, drain);
+        if (armed_v[st] >= 0) wait_bounded(bar(B_VFULL + st), armed_v[st] & 1, drain);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && T > 0) {
+      bool ok = wait_bounded(bar(B_QFULL), 0, ctl);
+      auto issue_pv = [&](int j) -> bool {
+        const int st = j & 1;
+        if (!wait_bounded(bar(B_PFULL), j & 1, ctl)) return false;
+        if (!wait_bounded(bar(B_VFULL + st), (j >> 1) & 1, ctl)) return false;
+        tc_fence_after();
+        const uint32_t vb = sbase + kOffV + st * 2 * kHalf;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {   // P_hi, then P_lo
+          const uint32_t pb = sbase + kOffP + part * 2 * kHalf;
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            const uint64_t ad = sw128_desc(pb + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(vb + kk * 2048, kHalf, 1024);
+            tc_mma(tmem + kTmemO, ad, bd, kIdescPV, (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        tc_commit(bar(B_VEMPTY + st));
+        tc_commit(bar(B_PVDONE));
+        return true;
+      };
+      for (int j = 0; j < T && ok; ++j) {
+        const int st = j & 1;
+        ok = wait_bounded(bar(B_KFULL + st), (j >> 1) & 1, ctl);
+        if (ok && j >= 2) ok = wait_bounded(bar(B_SFREE + st), ((j >> 1) - 1) & 1, ctl);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kb = sbase + kOffK + st * 2 * kHalf;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint64_t ad = sw128_desc(sbase + kOffQ + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sw128_desc(kb + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
+          tc_mma(tmem + st * kBN, ad, bd, kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(B_SFULL + st));
+        tc_commit(bar(B_KEMPTY + st));
+        if (j >= 1) ok = issue_pv(j - 1);
+      }
+      if (ok) issue_pv(T - 1);
+      // quiesce the tensor core before TMEM is freed
+      tc_commit(bar(B_DRAIN));
+      const Ctl drain{abort_flag, a.status, a.wait_limit_ns};
+      wait_bounded(bar(B_DRAIN), 0, drain);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
+    uint8_t* prow_hi = smem + kOffP + row * 128;
+    uint8_t* prow_lo = smem + kOffP + 2 * kHalf + row * 128;
+    float m = -CUDART_INF_F, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < T && ok; ++j) {
+      const int st = j & 1;
+      ok = wait_bounded(bar(B_SFULL + st), (j >> 1) & 1, ctl);
+      if (!ok) break;
+      tc_fence_after();
+      float s[kBN];
+#pragma unroll
+      for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tl + st * kBN + c * 32, s + c * 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(B_SFREE + st));
+      const int64_t key0 = kbeg + (int64_t)j * kBN;
+      const int nvalid = (int)min((int64_t)kBN, kend - key0);
+      float tmax = -CUDART_INF_F;
+#pragma unroll
+      for (int c = 0; c < kBN; ++c) {
+        s[c] = c < nvalid ? s[c] * a.scale_log2 : -CUDART_INF_F;
+        tmax = fmaxf(tmax, s[c]);
+      }
+      if (tmax > m + kRescaleLog2) {
+        // move the reference max; rescale what O already holds
+        if (j > 0 && m != -CUDART_INF_F) {
+          ok = wait_bounded(bar(B_PVDONE), (j - 1) & 1, ctl);
+          if (!ok) break;
+          tc_fence_after();
+          const float alpha = exp2f(m - tmax);
+          l *= alpha;
+#pragma unroll
+          for (int c = 0; c < kD / 32; ++c) {
+            float o[32];
+            tmem_ld32(tl + kTmemO + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+            tmem_st32(tl + kTmemO + c * 32, o);
+          }
+          tmem_wait_st();
+        }
+        m = tmax;
+      }
+      const float ref = (m == -CUDART_INF_F) ? 0.f : m;
+      float lsum = 0.f;
+#pragma unroll
+      for (int c = 0; c < kBN; ++c) {
+        s[c] = exp2f(s[c] - ref);
+        lsum += s[c];
+      }
+      l += lsum;
+      // P of the previous tile must be consumed before this one overwrites it
+      if (j > 0) {
+        ok = wait_bounded(bar(B_PVDONE), (j - 1) & 1, ctl);
+        if (!ok) break;
+      }
+#pragma unroll
+      for (int c = 0; c < kBN / 8; ++c) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float x = s[c * 8 + 2 * e], y = s[c * 8 + 2 * e + 1];
+          hi[e] = pack2_bf16(x, y);
+          const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162*>(&hi[e]);
+          const float2 hf = __bfloat1622float2(hb);
+          lo[e] = pack2_bf16(x - hf.x, y - hf.y);
+        }
+        const uint32_t off = (c >> 3) * kHalf + ((((uint32_t)c & 7u) ^ ((uint32_t)row & 7u)) << 4);
+        *reinterpret_cast<uint4*>(prow_hi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(prow_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      mbar_arrive(bar(B_PFULL));
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok && T > 0) ok = wait_bounded(bar(B_PVDONE), (T - 1) & 1, ctl);
+    if (ok) {
+      tc_fence_after();
+      int hh, ii;
+      bool valid;
+      if (a.mode == 0) {
+        const int g = t * a.hg + row / a.Nb;
+        ii = row % a.Nb;
+        hh = kvh * a.G + g;
+        valid = row < a.hg * a.Nb && g < a.G;
+      } else {
+        hh = h0;
+        ii = i0 + row;
+        valid = ii < a.Nb;
+      }
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float Lrow = l > 0.f ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
+      const int64_t r = ((int64_t)b * a.Hq + hh) * a.Nb + ii;
+      float* pa = a.part_a + split * a.part_stride_a + r * kD;
+#pragma unroll
+      for (int c = 0; c < kD / 32; ++c) {
+        float o[32];
+        if (T > 0) {
+          tmem_ld32(tl + kTmemO + c * 32, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0.f;
+        }
+        if (valid) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(pa + c * 32 + e) =
+                make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv);
+        }
+      }
+      if (valid) a.part_l[split * a.part_stride_l + r] = Lrow;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+  }
+}
+
+// ------------------------------------------------------------------ host --
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+bool map_4d(CUtensorMap* m, const void* base, uint64_t d1, uint64_t d2, uint64_t d3, int64_t s1, int64_t s2,
+            int64_t s3, uint32_t b1, uint32_t b2) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)kD, d1, d2, d3};
+  cuuint64_t strides[3] = {(cuuint64_t)s1 * 2, (cuuint64_t)s2 * 2, (cuuint64_t)s3 * 2};
+  cuuint32_t box[4] = {64, b1, b2, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+}  // namespace
+
+int* device_status_ptr();
+uint64_t wait_limit_ns();
+
+// Row tiling of the tcgen05 prefix pass, or false when the shape does not fit it.
+bool tc_tiling(const fb_attn_desc& d, int* mode, int* hg, int* tiles_per_unit, int* units) {
+  if (d.in_dtype != FB_BF16 || d.D != kD) return false;
+  const int G = d.Hq / d.Hkv;
+  if (d.Nb <= kBM && kBM % d.Nb == 0 && G * d.Nb >= 64) {
+    *mode = 0;
+    *hg = std::min(G, kBM / d.Nb);
+    *tiles_per_unit = (G + *hg - 1) / *hg;
+    *units = d.B * d.Hkv;
+    return true;
+  }
+  if (d.Nb >= 64) {
+    *mode = 1;
+    *hg = 1;
+    *tiles_per_unit = (d.Nb + kBM - 1) / kBM;
+    *units = d.B * d.Hq;
+    return true;
+  }
+  return false;
+}
+
+// Split count for `tiles` row tiles over nkeys keys: balance whole waves of
+// one CTA per SM against a fixed per-CTA cost (about two key tiles).
+void tc_plan_split(int64_t tiles, int64_t nkeys, int32_t max_split, int32_t* nsplit, int64_t* kps) {
+  const int64_t sms = num_sms();
+  const int64_t ktiles = std::max<int64_t>(1, (nkeys + kBN - 1) / kBN);
+  int64_t best_ns = 1;
+  double best = 1e300;
+  for (int64_t ns = 1; ns <= std::min<int64_t>(ktiles, std::max(1, max_split)); ++ns) {
+    const int64_t per = (ktiles + ns - 1) / ns;
+    const int64_t real_ns = (ktiles + per - 1) / per;
+    const int64_t waves = (tiles * real_ns + sms - 1) / sms;
+    const double cost = (double)waves * (per + 2) + 0.02 * real_ns;
+    if (cost < best) { best = cost; best_ns = real_ns; }
+  }
+  const int64_t per = (ktiles + best_ns - 1) / best_ns;
+  *kps = per * kBN;
+  *nsplit = (int32_t)((nkeys + *kps - 1) / *kps);
+  if (*nsplit < 1) *nsplit = 1;
+}
+
+cudaError_t launch_attn_tc(const fb_attn_desc& d, const void* q, const void* kp, const void* vp, int64_t nkeys,
+                           int32_t nsplit, int64_t kps, const int8_t* mask, int mask_active, float scale_log2,
+                           float* pa, float* pl, cudaStream_t s, bool* launched) {
+  *launched = false;
+  int mode, hg, tpu, units;
+  if (!tc_tiling(d, &mode, &hg, &tpu, &units) || nkeys <= 0) return cudaSuccess;
+  CUtensorMap tq, tk, tv;
+  const bool ok_q = mode == 0 ? map_4d(&tq, q, d.Nb, d.Hq, d.B, d.q_strides[2], d.q_strides[1], d.q_strides[0],
+                                       d.Nb, hg)
+                              : map_4d(&tq, q, d.Nb, d.Hq, d.B, d.q_strides[2], d.q_strides[1], d.q_strides[0],
+                                       kBM, 1);
+  if (!ok_q) return cudaSuccess;
+  if (!map_4d(&tk, kp, nkeys, d.Hkv, d.B, d.kp_strides[2], d.kp_strides[1], d.kp_strides[0], kBN, 1))
+    return cudaSuccess;
+  if (!map_4d(&tv, vp, nkeys, d.Hkv, d.B, d.kp_strides[2], d.kp_strides[1], d.kp_strides[0], kBN, 1))
+    return cudaSuccess;
+  TcArgs a;
+  a.B = d.B; a.Hq = d.Hq; a.Hkv = d.Hkv; a.G = d.Hq / d.Hkv; a.Nb = d.Nb;
+  a.mode = mode; a.hg = hg; a.tiles_per_unit = tpu;
+  a.nkeys = nkeys; a.keys_per_split = kps; a.scale_log2 = scale_log2;
+  a.part_a = pa; a.part_l = pl;
+  a.part_stride_a = (int64_t)d.B * d.Hq * d.Nb * d.D;
+  a.part_stride_l = (int64_t)d.B * d.Hq * d.Nb;
+  a.mask = mask; a.mask_active = mask_active;
+  a.status = device_status_ptr();
+  a.wait_limit_ns = wait_limit_ns();
+  if (!a.status) return cudaErrorInvalidValue;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  dim3 grid(units * tpu, nsplit);
+  attn_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, a);
+  *launched = true;
+  return cudaGetLastError();
+}
+
+int tc_units_tiles(const fb_attn_desc& d) {
+  int mode, hg, tpu, units;
+  if (!tc_tiling(d, &mode, &hg, &tpu, &units)) return 0;
+  return units * tpu;
+}
+
+}  // namespace fb
