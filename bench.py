@@ -10,9 +10,11 @@ tokens, 8 diffusion steps per block, 4 blocks, tau = 8).  Every diffusion step
 runs fb_step under the reuse policy, and every block ends with fb_kv_append.
 The metric is query tokens per second (B * Nb per diffusion step) with reuse
 on; the same schedule with tau = 0 (every step recomputes over the whole KV
-cache) is reported beside it.  L2 is flushed (a 256 MiB write) before every
+cache) is reported beside it.  L2 is flushed (a 1 GiB write) before every
 diffusion step, outside the event-timed interval, so each step reads the KV
-cache from HBM as it would between the layers of a model.
+cache from HBM as it would between the layers of a model; the flush also keeps
+the GPU busy long enough for the host to enqueue the next step, so the timed
+interval holds no host launch gaps.
 
 `--impl reference` times the fp64 CPU oracle on this host's cores on a
 bounded sample of the same schedule (the reference arm; there is no other
@@ -40,7 +42,7 @@ from block_diffusion_attention_flashblock_b200 import workloads as wl  # noqa: E
 
 METRIC = "block-diffusion attention step latency & query tok/s vs full-KV recompute"
 UNIT = "query tok/s"
-L2_FLUSH_BYTES = 256 << 20
+L2_FLUSH_BYTES = 1 << 30
 
 
 def _peaks():
@@ -127,6 +129,7 @@ class Schedule:
 def run_ours(args, spec, rank, world, device):
     from block_diffusion_attention_flashblock_b200 import fb
     torch.cuda.set_device(device)
+    fb.fb_debug_set_prefix_kernel({"auto": 0, "generic": 1, "tcgen05": 2}[args.prefix_kernel])
     sched = Schedule(spec, device)
     s = spec
     dt = s.torch_dtype
@@ -240,7 +243,8 @@ def run_ours(args, spec, rank, world, device):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": spec.dtype,
         "data": "synthetic (seeded; shapes of the pages' diffusion-LM workload)",
         "config": {"workload": _describe(spec), "query_tokens_per_step": sched.query_tokens,
-                   "diffusion_steps_per_step": len(sched.steps), "l2": "flushed (256 MiB write) before every "
+                   "prefix_kernel": args.prefix_kernel,
+                   "diffusion_steps_per_step": len(sched.steps), "l2": "flushed (1 GiB write) before every "
                    "diffusion step, outside the timed interval", "parallelism": f"replicas x{world}",
                    "full_steps_per_step": n_full},
         "step_latency": {"mean_us": 1e3 * ms_on / len(sched.steps), **per_kind},
@@ -326,6 +330,7 @@ def main():
     ap.add_argument("--workload", default="dllm_8k", choices=list(wl.SPECS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--prefix-kernel", default="auto", choices=["auto", "generic", "tcgen05"])
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
     spec = wl.get_spec(args.workload)

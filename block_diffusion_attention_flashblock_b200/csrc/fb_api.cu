@@ -149,13 +149,17 @@ static inline size_t part_bytes(const fb_attn_desc& d, int32_t n) {
   return align256((size_t)n * rows_of(d) * d.D * 4) + align256((size_t)n * rows_of(d) * 4);
 }
 
-// Upper bound of the split count of one pass over up to max_keys keys.
+// Upper bound of the split count of one pass over up to max_keys keys (both
+// the generic kernel's plan and, for dense prefix passes, the tcgen05 plan).
 static int32_t split_bound(const fb_attn_desc& d, int per_head, int64_t max_keys) {
   const RowMap rm = make_rowmap(d.B, d.Hq, d.Hkv, d.Nb, per_head, generic_tile_rows(d.in_dtype == FB_BF16));
   int32_t ns;
   int64_t kps;
   plan_split((int64_t)rm.units * rm.row_tiles, std::max<int64_t>(max_keys, 1),
              generic_ctas_per_sm(d.D, d.in_dtype == FB_BF16), generic_key_tile(), &ns, &kps);
+  int mode, hg, tpu, units;
+  if (!per_head && tc_tiling(d, &mode, &hg, &tpu, &units))
+    ns = std::max(ns, tc_split_cap((int64_t)units * tpu, max_keys));
   return ns;
 }
 
@@ -205,6 +209,50 @@ static fb_status launch_pass(const fb_attn_desc& d, AttnArgs& a, float* pa, floa
   a.part_stride_l = rows_of(d);
   ProfScope prof(kProfPrefix, pass_bytes(d, a), s);
   return launch_attn_generic(a, d.D, d.in_dtype == FB_BF16, s) == cudaSuccess ? FB_OK : FB_ECUDA;
+}
+
+// Dense block-external pass over prefix rows [0, nkeys): the tcgen05 kernel
+// when the shape and strides allow it, else the generic kernel.
+static int g_prefix_kernel = 0;  // 0 auto, 1 generic only, 2 tcgen05 whenever it applies
+
+struct PrefixPlan {
+  bool tc;
+  int32_t nsplit;
+  int64_t kps;
+  PassPlan gen;
+  TcMaps maps;
+};
+
+static PrefixPlan plan_prefix(const fb_attn_desc& d, const void* q, const void* kp, const void* vp, int64_t nkeys,
+                              int32_t cap) {
+  PrefixPlan p;
+  p.gen = plan_pass(d, q, kp, vp, d.kp_strides, nkeys, nullptr, 0, cap);
+  p.tc = false;
+  p.nsplit = p.gen.nsplit;
+  p.kps = p.gen.a.keys_per_split;
+  const int64_t min_keys = g_prefix_kernel == 2 ? 1 : 256;
+  if (g_prefix_kernel != 1 && nkeys >= min_keys && tc_make_maps(d, q, kp, vp, nkeys, &p.maps)) {
+    tc_plan_split((int64_t)p.maps.units * p.maps.tiles_per_unit, nkeys, cap, &p.nsplit, &p.kps);
+    p.tc = true;
+  }
+  return p;
+}
+
+static fb_status launch_prefix(const fb_attn_desc& d, PrefixPlan& p, int64_t nkeys, const int8_t* mask,
+                               int mask_active, float* pa, float* pl, cudaStream_t s) {
+  if (!p.tc) {
+    p.gen.a.mask = mask;
+    p.gen.a.mask_active = mask_active;
+    return launch_pass(d, p.gen.a, pa, pl, s);
+  }
+  const int es = esize(d.in_dtype);
+  const double bytes = 2.0 * d.B * d.Hkv * (double)nkeys * d.D * es + (double)rows_of(d) * d.D * es +
+                       (double)rows_of(d) * (d.D + 1) * 4;
+  ProfScope prof(kProfPrefix, bytes, s);
+  return launch_attn_tc(d, p.maps, nkeys, p.nsplit, p.kps, mask, mask_active, scale_log2(d), pa, pl, s) ==
+                 cudaSuccess
+             ? FB_OK
+             : FB_ECUDA;
 }
 
 static PartGroup group_of(const float* a, const float* l, int32_t n, const fb_attn_desc& d) {
@@ -319,12 +367,23 @@ fb_status fb_attn_outblock(const fb_attn_desc* d, const void* q, const void* kp,
   float* pl = reinterpret_cast<float*>(w + align256((size_t)cap * rows_of(*d) * d->D * 4));
 
   // pass 1: dense prefix, or the selected keys
+  if (!sel) {
+    PrefixPlan p = plan_prefix(*d, q, kp, vp, prefix_len, cap);
+    if (p.nsplit == 1) return launch_prefix(*d, p, prefix_len, nullptr, 0, a_out, l_out, stream);
+    if ((st = launch_prefix(*d, p, prefix_len, nullptr, 0, pa, pl, stream)) != FB_OK) return st;
+    PartList lst;
+    memset(&lst, 0, sizeof(lst));
+    lst.ngroups = 1;
+    lst.g[0] = group_of(pa, pl, p.nsplit, *d);
+    return merge_to_part(*d, lst, a_out, l_out, nullptr, 0, stream);
+  }
   PassPlan p = plan_pass(*d, q, kp, vp, d->kp_strides, prefix_len, sel, sel_k, cap);
   if (p.nsplit == 1) {
     if ((st = launch_pass(*d, p.a, a_out, l_out, stream)) != FB_OK) return st;
   } else {
     if ((st = launch_pass(*d, p.a, pa, pl, stream)) != FB_OK) return st;
     PartList lst;
+    memset(&lst, 0, sizeof(lst));
     lst.ngroups = 1;
     lst.g[0] = group_of(pa, pl, p.nsplit, *d);
     if ((st = merge_to_part(*d, lst, a_out, l_out, nullptr, 0, stream)) != FB_OK) return st;
@@ -338,6 +397,7 @@ fb_status fb_attn_outblock(const fb_attn_desc* d, const void* q, const void* kp,
   if (r.nsplit == 1) return launch_pass(*d, r.a, a_res, l_res, stream);
   if ((st = launch_pass(*d, r.a, pa, pl, stream)) != FB_OK) return st;
   PartList lst;
+  memset(&lst, 0, sizeof(lst));
   lst.ngroups = 1;
   lst.g[0] = group_of(pa, pl, r.nsplit, *d);
   return merge_to_part(*d, lst, a_res, l_res, nullptr, 0, stream);
@@ -435,6 +495,12 @@ fb_status fb_profile_read(int32_t reset, int64_t* launches, double* total_ms, do
     if (alg_bytes) alg_bytes[k] = g_prof.bytes[k];
     if (reset) { g_prof.launches[k] = 0; g_prof.ms[k] = 0; g_prof.bytes[k] = 0; }
   }
+  return FB_OK;
+}
+
+fb_status fb_debug_set_prefix_kernel(int32_t which) {
+  if (which < 0 || which > 2) return FB_EINVAL;
+  g_prefix_kernel = which;
   return FB_OK;
 }
 
@@ -594,10 +660,8 @@ fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
   memset(&ext, 0, sizeof(ext));
 
   if (gamma) {
-    PassPlan p = plan_pass(d, a->q, a->kp, a->vp, d.kp_strides, a->prefix_len, nullptr, 0, c->part_cap);
-    p.a.mask = c->mask;
-    p.a.mask_active = tau_reuse;
-    if ((st = launch_pass(d, p.a, c->part_a, c->part_l, s)) != FB_OK) return st;
+    PrefixPlan p = plan_prefix(d, a->q, a->kp, a->vp, a->prefix_len, c->part_cap);
+    if ((st = launch_prefix(d, p, a->prefix_len, c->mask, tau_reuse, c->part_a, c->part_l, s)) != FB_OK) return st;
     GammaArgs g;
     memset(&g, 0, sizeof(g));
     g.B = d.B; g.Hq = d.Hq; g.Nb = d.Nb; g.D = d.D;
@@ -628,17 +692,23 @@ fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
       }
     }
     if (!tau_reuse) {
-      PassPlan p = plan_pass(d, a->q, a->kp, a->vp, d.kp_strides, a->prefix_len, nullptr, 0, c->part_cap);
+      // dense: the whole prefix; sparse: the prefix minus each head's selection
+      PrefixPlan p;
       if (sparse) {
+        p.tc = false;
+        p.gen = plan_pass(d, a->q, a->kp, a->vp, d.kp_strides, a->prefix_len, nullptr, 0, c->part_cap);
+        p.nsplit = p.gen.nsplit;
         if (launch_build_bitmap(a->sel, a->sel_k, BH, c->bitmap, (a->prefix_len + 31) / 32, s) != cudaSuccess)
           return FB_ECUDA;
-        p.a.excl = c->bitmap;
-        p.a.excl_words = (a->prefix_len + 31) / 32;
+        p.gen.a.excl = c->bitmap;
+        p.gen.a.excl_words = (a->prefix_len + 31) / 32;
+      } else {
+        p = plan_prefix(d, a->q, a->kp, a->vp, a->prefix_len, c->part_cap);
       }
       if (p.nsplit == 1) {
-        if ((st = launch_pass(d, p.a, c->cache_a, c->cache_l, s)) != FB_OK) return st;
+        if ((st = launch_prefix(d, p, a->prefix_len, nullptr, 0, c->cache_a, c->cache_l, s)) != FB_OK) return st;
       } else {
-        if ((st = launch_pass(d, p.a, c->part_a, c->part_l, s)) != FB_OK) return st;
+        if ((st = launch_prefix(d, p, a->prefix_len, nullptr, 0, c->part_a, c->part_l, s)) != FB_OK) return st;
         PartList lst;
         memset(&lst, 0, sizeof(lst));
         lst.ngroups = 1;

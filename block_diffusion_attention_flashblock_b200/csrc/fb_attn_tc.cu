@@ -23,6 +23,8 @@
 #include <cudaTypedefs.h>
 #include <math_constants.h>
 
+#include <algorithm>
+
 #include "fb_internal.cuh"
 
 namespace fb {
@@ -83,15 +85,16 @@ struct Ctl {
 };
 
 // Bounded wait for the phase of `parity` to complete.  Gives up when the limit
-// passes or another role has given up; the first to give up records the error.
-__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const Ctl& c) {
+// passes or (unless `draining`) another role has given up; the first to give
+// up records the error.
+__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const Ctl& c, bool draining = false) {
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try(bar, parity)) return true;
-    if (*c.abort) return false;
+    if (!draining && *c.abort) return false;
     if (globaltimer() - t0 > c.limit_ns) {
       if (atomicExch(const_cast<int*>(c.abort), 1) == 0) atomicCAS(c.status, 0, (int)FB_ETIMEOUT);
       return false;
@@ -192,6 +195,7 @@ struct TcArgs {
   int32_t mask_active;
   int* status;
   uint64_t wait_limit_ns;
+  uint32_t q_bytes;        // bytes of one Q half-box (64 columns)
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -250,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && T > 0) {
       int armed_k[2] = {-1, -1}, armed_v[2] = {-1, -1};
       bool ok = true;
-      mbar_expect_tx(bar(B_QFULL), 2 * kHalf);
+      mbar_expect_tx(bar(B_QFULL), 2 * a.q_bytes);
       tma_load_4d(sbase + kOffQ, &tmQ, bar(B_QFULL), 0, i0, h0, b);
       tma_load_4d(sbase + kOffQ + kHalf, &tmQ, bar(B_QFULL), 64, i0, h0, b);
       for (int j = 0; j < T && ok; ++j) {
@@ -270,11 +274,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         armed_v[st] = j >> 1;
       }
       // Let every copy this thread started land before the CTA can exit.
-      const Ctl drain{abort_flag, a.status, a.wait_limit_ns};
-      wait_bounded(bar(B_QFULL), 0, drain);
+      wait_bounded(bar(B_QFULL), 0, ctl, true);
       for (int st = 0; st < 2; ++st) {
-        if (armed_k[st] >= 0) wait_bounded(bar(B_KFULL + st), armed_k[st] & 1, drain);
-        if (armed_v[st] >= 0) wait_bounded(bar(B_VFULL + st), armed_v[st] & 1, drain);
+        if (armed_k[st] >= 0) wait_bounded(bar(B_KFULL + st), armed_k[st] & 1, ctl, true);
+        if (armed_v[st] >= 0) wait_bounded(bar(B_VFULL + st), armed_v[st] & 1, ctl, true);
       }
     }
   } else if (warp == 1) {
@@ -321,8 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) issue_pv(T - 1);
       // quiesce the tensor core before TMEM is freed
       tc_commit(bar(B_DRAIN));
-      const Ctl drain{abort_flag, a.status, a.wait_limit_ns};
-      wait_bounded(bar(B_DRAIN), 0, drain);
+      wait_bounded(bar(B_DRAIN), 0, ctl, true);
     }
   } else {
     // ------------------------------------------------------------ softmax
@@ -333,9 +335,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* prow_lo = smem + kOffP + 2 * kHalf + row * 128;
     float m = -CUDART_INF_F, l = 0.f;
     bool ok = true;
+    // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform.
+    auto uniform = [](bool v) { return __all_sync(0xffffffffu, v); };
     for (int j = 0; j < T && ok; ++j) {
       const int st = j & 1;
-      ok = wait_bounded(bar(B_SFULL + st), (j >> 1) & 1, ctl);
+      ok = uniform(wait_bounded(bar(B_SFULL + st), (j >> 1) & 1, ctl));
       if (!ok) break;
       tc_fence_after();
       float s[kBN];
@@ -352,25 +356,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         s[c] = c < nvalid ? s[c] * a.scale_log2 : -CUDART_INF_F;
         tmax = fmaxf(tmax, s[c]);
       }
-      if (tmax > m + kRescaleLog2) {
-        // move the reference max; rescale what O already holds
-        if (j > 0 && m != -CUDART_INF_F) {
-          ok = wait_bounded(bar(B_PVDONE), (j - 1) & 1, ctl);
-          if (!ok) break;
-          tc_fence_after();
-          const float alpha = exp2f(m - tmax);
-          l *= alpha;
+      // Move this row's reference max when it grew by more than 2^8; rows whose
+      // O already holds values rescale it (alpha = 1 for the others).
+      const bool move = tmax > m + kRescaleLog2;
+      const bool scale_o = move && j > 0 && m != -CUDART_INF_F;
+      const float alpha = scale_o ? exp2f(m - tmax) : 1.f;
+      if (__any_sync(0xffffffffu, scale_o)) {
+        ok = uniform(wait_bounded(bar(B_PVDONE), (j - 1) & 1, ctl));
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < kD / 32; ++c) {
-            float o[32];
-            tmem_ld32(tl + kTmemO + c * 32, o);
-            tmem_wait_ld();
+        for (int c = 0; c < kD / 32; ++c) {
+          float o[32];
+          tmem_ld32(tl + kTmemO + c * 32, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= alpha;
-            tmem_st32(tl + kTmemO + c * 32, o);
-          }
-          tmem_wait_st();
+          for (int e = 0; e < 32; ++e) o[e] *= alpha;
+          tmem_st32(tl + kTmemO + c * 32, o);
         }
+        tmem_wait_st();
+      }
+      if (move) {
+        l *= alpha;
         m = tmax;
       }
       const float ref = (m == -CUDART_INF_F) ? 0.f : m;
@@ -383,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       l += lsum;
       // P of the previous tile must be consumed before this one overwrites it
       if (j > 0) {
-        ok = wait_bounded(bar(B_PVDONE), (j - 1) & 1, ctl);
+        ok = uniform(wait_bounded(bar(B_PVDONE), (j - 1) & 1, ctl));
         if (!ok) break;
       }
 #pragma unroll
@@ -406,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(B_PFULL));
     }
     // ------------------------------------------------------------ epilogue
-    if (ok && T > 0) ok = wait_bounded(bar(B_PVDONE), (T - 1) & 1, ctl);
+    if (ok && T > 0) ok = uniform(wait_bounded(bar(B_PVDONE), (T - 1) & 1, ctl));
     if (ok) {
       tc_fence_after();
       int hh, ii;
@@ -506,6 +513,22 @@ bool tc_tiling(const fb_attn_desc& d, int* mode, int* hg, int* tiles_per_unit, i
   return false;
 }
 
+bool tc_make_maps(const fb_attn_desc& d, const void* q, const void* kp, const void* vp, int64_t nkeys, TcMaps* m) {
+  if (nkeys <= 0 || !tc_tiling(d, &m->mode, &m->hg, &m->tiles_per_unit, &m->units)) return false;
+  const uint32_t qrows = m->mode == 0 ? (uint32_t)d.Nb : (uint32_t)kBM;
+  const uint32_t qheads = m->mode == 0 ? (uint32_t)m->hg : 1u;
+  return map_4d(&m->q, q, d.Nb, d.Hq, d.B, d.q_strides[2], d.q_strides[1], d.q_strides[0], qrows, qheads) &&
+         map_4d(&m->k, kp, nkeys, d.Hkv, d.B, d.kp_strides[2], d.kp_strides[1], d.kp_strides[0], kBN, 1) &&
+         map_4d(&m->v, vp, nkeys, d.Hkv, d.B, d.kp_strides[2], d.kp_strides[1], d.kp_strides[0], kBN, 1);
+}
+
+// Upper bound of the split count the planner may choose (sizes workspaces).
+int32_t tc_split_cap(int64_t tiles, int64_t max_keys) {
+  const int64_t ktiles = std::max<int64_t>(1, (max_keys + kBN - 1) / kBN);
+  const int64_t want = std::max<int64_t>(2, (4 * (int64_t)num_sms() + tiles - 1) / std::max<int64_t>(tiles, 1));
+  return (int32_t)std::min(ktiles, want);
+}
+
 // Split count for `tiles` row tiles over nkeys keys: balance whole waves of
 // one CTA per SM against a fixed per-CTA cost (about two key tiles).
 void tc_plan_split(int64_t tiles, int64_t nkeys, int32_t max_split, int32_t* nsplit, int64_t* kps) {
@@ -522,34 +545,21 @@ void tc_plan_split(int64_t tiles, int64_t nkeys, int32_t max_split, int32_t* nsp
   }
   const int64_t per = (ktiles + best_ns - 1) / best_ns;
   *kps = per * kBN;
-  *nsplit = (int32_t)((nkeys + *kps - 1) / *kps);
-  if (*nsplit < 1) *nsplit = 1;
+  *nsplit = (int32_t)std::max<int64_t>(1, (nkeys + *kps - 1) / *kps);
 }
 
-cudaError_t launch_attn_tc(const fb_attn_desc& d, const void* q, const void* kp, const void* vp, int64_t nkeys,
-                           int32_t nsplit, int64_t kps, const int8_t* mask, int mask_active, float scale_log2,
-                           float* pa, float* pl, cudaStream_t s, bool* launched) {
-  *launched = false;
-  int mode, hg, tpu, units;
-  if (!tc_tiling(d, &mode, &hg, &tpu, &units) || nkeys <= 0) return cudaSuccess;
-  CUtensorMap tq, tk, tv;
-  const bool ok_q = mode == 0 ? map_4d(&tq, q, d.Nb, d.Hq, d.B, d.q_strides[2], d.q_strides[1], d.q_strides[0],
-                                       d.Nb, hg)
-                              : map_4d(&tq, q, d.Nb, d.Hq, d.B, d.q_strides[2], d.q_strides[1], d.q_strides[0],
-                                       kBM, 1);
-  if (!ok_q) return cudaSuccess;
-  if (!map_4d(&tk, kp, nkeys, d.Hkv, d.B, d.kp_strides[2], d.kp_strides[1], d.kp_strides[0], kBN, 1))
-    return cudaSuccess;
-  if (!map_4d(&tv, vp, nkeys, d.Hkv, d.B, d.kp_strides[2], d.kp_strides[1], d.kp_strides[0], kBN, 1))
-    return cudaSuccess;
+cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys, int32_t nsplit, int64_t kps,
+                           const int8_t* mask, int mask_active, float scale_log2, float* pa, float* pl,
+                           cudaStream_t s) {
   TcArgs a;
   a.B = d.B; a.Hq = d.Hq; a.Hkv = d.Hkv; a.G = d.Hq / d.Hkv; a.Nb = d.Nb;
-  a.mode = mode; a.hg = hg; a.tiles_per_unit = tpu;
+  a.mode = m.mode; a.hg = m.hg; a.tiles_per_unit = m.tiles_per_unit;
   a.nkeys = nkeys; a.keys_per_split = kps; a.scale_log2 = scale_log2;
   a.part_a = pa; a.part_l = pl;
   a.part_stride_a = (int64_t)d.B * d.Hq * d.Nb * d.D;
   a.part_stride_l = (int64_t)d.B * d.Hq * d.Nb;
   a.mask = mask; a.mask_active = mask_active;
+  a.q_bytes = 64u * 2u * (uint32_t)(m.mode == 0 ? d.Nb * m.hg : kBM);
   a.status = device_status_ptr();
   a.wait_limit_ns = wait_limit_ns();
   if (!a.status) return cudaErrorInvalidValue;
@@ -559,16 +569,9 @@ cudaError_t launch_attn_tc(const fb_attn_desc& d, const void* q, const void* kp,
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  dim3 grid(units * tpu, nsplit);
-  attn_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, a);
-  *launched = true;
+  dim3 grid(m.units * m.tiles_per_unit, nsplit);
+  attn_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(m.q, m.k, m.v, a);
   return cudaGetLastError();
-}
-
-int tc_units_tiles(const fb_attn_desc& d) {
-  int mode, hg, tpu, units;
-  if (!tc_tiling(d, &mode, &hg, &tpu, &units)) return 0;
-  return units * tpu;
 }
 
 }  // namespace fb

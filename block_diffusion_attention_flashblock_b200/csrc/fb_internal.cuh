@@ -1,5 +1,6 @@
 // Internal declarations shared by the libfb translation units.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -97,6 +98,19 @@ cudaError_t launch_attn_generic(const AttnArgs& a, int D, int in_bf16, cudaStrea
 int generic_tile_rows(int in_bf16);
 int generic_key_tile();
 int generic_ctas_per_sm(int D, int in_bf16);
+
+// tcgen05 prefix pass (fb_attn_tc.cu).
+struct TcMaps {
+  CUtensorMap q, k, v;
+  int mode, hg, tiles_per_unit, units;
+};
+bool tc_tiling(const fb_attn_desc& d, int* mode, int* hg, int* tiles_per_unit, int* units);
+bool tc_make_maps(const fb_attn_desc& d, const void* q, const void* kp, const void* vp, int64_t nkeys, TcMaps* m);
+void tc_plan_split(int64_t tiles, int64_t nkeys, int32_t max_split, int32_t* nsplit, int64_t* kps);
+int32_t tc_split_cap(int64_t tiles, int64_t max_keys);
+cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys, int32_t nsplit, int64_t kps,
+                           const int8_t* mask, int mask_active, float scale_log2, float* pa, float* pl,
+                           cudaStream_t s);
 
 struct MergeArgs {
   int32_t B, Hq, Nb, D;

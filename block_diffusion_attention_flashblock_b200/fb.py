@@ -71,6 +71,7 @@ _SIGS = {
     "fb_get_device_status": (C.c_int, [_P, C.POINTER(C.c_int)]),
     "fb_debug_set_wait_limit_ns": (C.c_int, [C.c_uint64]),
     "fb_profile_enable": (C.c_int, [C.c_int32]),
+    "fb_debug_set_prefix_kernel": (C.c_int, [C.c_int32]),
     "fb_profile_read": (C.c_int, [C.c_int32, _P, _P, _P]),
 }
 
@@ -242,6 +243,13 @@ def fb_get_device_status(stream=None) -> int:
     s = C.c_int(0)
     _check(lib().fb_get_device_status(_stream(stream), C.byref(s)), "fb_get_device_status")
     return s.value
+
+
+PREFIX_AUTO, PREFIX_GENERIC, PREFIX_TC = 0, 1, 2
+
+
+def fb_debug_set_prefix_kernel(which: int):
+    _check(lib().fb_debug_set_prefix_kernel(which), "fb_debug_set_prefix_kernel")
 
 
 def fb_debug_set_wait_limit_ns(ns: int):

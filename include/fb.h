@@ -229,6 +229,11 @@ fb_status fb_get_device_status(cudaStream_t stream, fb_status* device_status);
 fb_status fb_profile_enable(int32_t on);
 fb_status fb_profile_read(int32_t reset, int64_t* launches, double* total_ms, double* alg_bytes);
 
+/* Test hook: which kernel runs dense block-external passes: 0 automatic (the
+ * tcgen05 kernel where the shape and strides allow it), 1 the generic
+ * mma.sync / FFMA kernel only, 2 the tcgen05 kernel whenever it applies. */
+fb_status fb_debug_set_prefix_kernel(int32_t which);
+
 /* Test hook: the bound of every barrier wait in later launches, in
  * nanoseconds (default 2e9).  0 makes any wait that is not already satisfied
  * expire at once.  Affects only the calling process. */

@@ -45,19 +45,53 @@ SHAPES = [
 ]
 
 
-@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
-def test_outblock_dense(shape):
+@pytest.fixture
+def prefix_kernel():
+    """Force one block-external kernel for a test, restore automatic choice after."""
+    def use(which):
+        fb.fb_debug_set_prefix_kernel(which)
+    yield use
+    fb.fb_debug_set_prefix_kernel(fb.PREFIX_AUTO)
+
+
+def _outblock_check(shape, seed=11):
     B, Hq, Hkv, D, Nb, Lp, dt = shape
-    q, kin, vin, kp, vp = _mk(B, Hq, Hkv, D, Nb, Lp, dt, seed=11)
+    q, kin, vin, kp, vp = _mk(B, Hq, Hkv, D, Nb, Lp, dt, seed=seed)
     qd, kpd, vpd = q.cuda(), kp.cuda(), vp.cuda()
-    a = torch.empty(B, Hq, Nb, D, device="cuda")
-    l = torch.empty(B, Hq, Nb, device="cuda")
+    a = torch.full((B, Hq, Nb, D), float("nan"), device="cuda")
+    l = torch.full((B, Hq, Nb), float("nan"), device="cuda")
     desc = fb.make_desc(qd, kin.cuda(), kpd, a)
     ws = torch.empty(fb.fb_outblock_workspace_bytes(desc, Lp), dtype=torch.uint8, device="cuda")
     fb.fb_attn_outblock(desc, qd, kpd, vpd, Lp, a, l, ws)
+    assert fb.fb_get_device_status() == fb.FB_OK
     A, L = orc.outblock(orc.to64(q), orc.to64(kp), orc.to64(vp), Lp, 1 / np.sqrt(D))
     assert_o_close(a, A, TOL[dt], "A_out")
     assert_lse_close(l, L, TOL[dt], "L_out")
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_outblock_dense(shape, prefix_kernel):
+    prefix_kernel(fb.PREFIX_GENERIC)
+    _outblock_check(shape)
+
+
+TC_SHAPES = [
+    # (B, Hq, Hkv, D, Nb, Lp, dtype): tcgen05 tilings
+    (1, 32, 8, 128, 32, 1000, "bf16"),    # 4 heads x 32 queries per tile, ragged last key tile (104 keys)
+    (1, 32, 8, 128, 32, 8192, "bf16"),    # dLLM prefix at full size
+    (2, 32, 8, 128, 64, 3000, "bf16"),    # 2 heads x 64 queries per tile, two tiles per KV head
+    (1, 8, 4, 128, 32, 500, "bf16"),      # G*Nb = 64: half-filled tiles
+    (1, 4, 4, 128, 200, 2000, "bf16"),    # one head per tile, 128 queries, ragged query tail
+    (1, 8, 2, 128, 1560, 1700, "bf16"),   # video-like block with GQA, 13 query tiles per head
+    (1, 2, 2, 128, 64, 129, "bf16"),      # second key tile holds one key
+    (1, 2, 1, 128, 64, 1, "bf16"),        # a single prefix key
+]
+
+
+@pytest.mark.parametrize("shape", TC_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_outblock_dense_tcgen05(shape, prefix_kernel):
+    prefix_kernel(fb.PREFIX_TC)
+    _outblock_check(shape, seed=13)
 
 
 def test_outblock_empty_prefix():
