@@ -204,9 +204,12 @@ def run_ours(args, spec, rank, world, device):
     clocks.start()
     ms_on, per_on, kinds_on, prof = timed(tau_on, args.steps, args.warmup, profile=True)
     clk = clocks.stop()
-    ms_full, per_full, _, _ = timed(0, args.steps, args.warmup)
+    if args.profile_run:
+        ms_full, per_full = float("nan"), []
+    else:
+        ms_full, per_full, _, _ = timed(0, args.steps, args.warmup)
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not args.profile_run:
         ms_e2e, _, _, _ = timed(tau_on, args.steps, args.warmup, e2e=True)
         item = sched.steps[0]
         h2d = sum(it["hq"].numel() * it["hq"].element_size() + 2 * it["hk"].numel() * it["hk"].element_size()
@@ -248,9 +251,9 @@ def run_ours(args, spec, rank, world, device):
                    "diffusion step, outside the timed interval", "parallelism": f"replicas x{world}",
                    "full_steps_per_step": n_full},
         "step_latency": {"mean_us": 1e3 * ms_on / len(sched.steps), **per_kind},
-        "full_recompute": {"value": world * sched.query_tokens / (ms_full * 1e-3), "ms_per_step": ms_full,
+        "full_recompute": None if args.profile_run else {"value": world * sched.query_tokens / (ms_full * 1e-3), "ms_per_step": ms_full,
                            "mean_step_us": 1e3 * ms_full / len(sched.steps)},
-        "speedup_vs_full_recompute": ms_full / ms_on,
+        "speedup_vs_full_recompute": None if args.profile_run else ms_full / ms_on,
         "e2e": e2e, "roofline": roof, "kernels": kernels, "gpu_launches": gpu_launches // 1,
         "gpu_launches_per_step": gpu_launches / args.steps, "clocks": clk,
     }
@@ -331,6 +334,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--prefix-kernel", default="auto", choices=["auto", "generic", "tcgen05"])
+    ap.add_argument("--profile-run", action="store_true",
+                    help="only the reuse-on schedule (no full-recompute, e2e or CPU legs): for ncu captures")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
     spec = wl.get_spec(args.workload)
@@ -351,7 +356,7 @@ def main():
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank == 0:
-        if world == 1:
+        if world == 1 and not args.profile_run:
             out["cpu_baseline"] = cpu_baseline(spec, args.cpu_budget)
         print(json.dumps(out))
 
