@@ -58,6 +58,7 @@ _SIGS = {
     "fb_outblock_workspace_bytes": (C.c_int, [_P, C.c_int64, C.c_int32, C.POINTER(C.c_size_t)]),
     "fb_attn_outblock": (C.c_int, [_P, _P, _P, _P, C.c_int64, _P, C.c_int32, _P, _P, _P, _P, _P,
                                    C.c_size_t, _P]),
+    "fb_attn_outblock_noalloc": (C.c_int, [_P, _P, _P, _P, C.c_int64, _P, _P, _P]),
     "fb_attn_inblock": (C.c_int, [_P, _P, _P, _P, C.c_int32, _P, _P, _P, _P, _P]),
     "fb_merge": (C.c_int, [_P, C.c_int32, _P, _P, _P, _P, _P]),
     "fb_kv_append": (C.c_int, [_P, _P, _P, C.c_int64, _P, _P, _P]),
@@ -181,6 +182,16 @@ def fb_attn_outblock(desc, q, kp, vp, prefix_len, a_out, l_out, ws, sel=None, se
     _check(lib().fb_attn_outblock(C.byref(desc), _ptr(q), _ptr(kp), _ptr(vp), prefix_len, _sel_ptr(sel),
                                   sel_k, _ptr(a_out), _ptr(l_out), _ptr(a_res), _ptr(l_res), _ptr(ws),
                                   ws.numel() * ws.element_size(), _stream(stream)), "fb_attn_outblock")
+
+
+FB_NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def fb_attn_outblock_noalloc(desc, q, kp, vp, prefix_len, a_out, l_out, stream=None):
+    """fb_attn_outblock (dense) with its scratch in the library's fixed array."""
+    _check(lib().fb_attn_outblock_noalloc(C.byref(desc), _ptr(q), _ptr(kp), _ptr(vp), prefix_len,
+                                          _ptr(a_out), _ptr(l_out), _stream(stream)),
+           "fb_attn_outblock_noalloc")
 
 
 def fb_attn_inblock(desc, q, kin, vin, o, lse=None, a_parts=(), l_parts=(), stream=None):

@@ -105,6 +105,34 @@ fb_status fb_attn_outblock(const fb_attn_desc* d, const void* q, const void* kp,
                            void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Dense block-external attention for callers that cannot allocate.  The pages
+ * have no counterpart: this is a library service, not part of the method.
+ *
+ * Same arguments and result as fb_attn_outblock with sel == NULL, but without
+ * a workspace argument: the split-KV partial results go to a fixed array of
+ * FB_NOALLOC_SCRATCH_BYTES inside the library.  It is for callers that cannot
+ * call cudaMalloc or pass scratch at call time. Examples: code whose host
+ * framework owns the whole device pool, plug-ins limited to memory their host
+ * hands them, and services that must not allocate while serving.
+ * - Every GPU on which the library is loaded keeps the array until the
+ *   process exits.
+ * - The first call on a device looks up the array's device address (with
+ *   that device current) and caches it.  Make that first call before any
+ *   stream capture.
+ * - All calls share the array, and it keeps the last call's contents; this
+ *   call overwrites everything it reads, so it needs no clearing.  Calls whose
+ *   work overlaps on the GPU (unordered streams) race on it.
+ * - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ * Errors: as fb_attn_outblock; FB_ENOSPACE when the call would need more than
+ *   FB_NOALLOC_SCRATCH_BYTES of scratch (fb_outblock_workspace_bytes with
+ *   sel_k = 0 gives the need).
+ * ------------------------------------------------------------------------- */
+#define FB_NOALLOC_SCRATCH_BYTES (64u << 20)
+fb_status fb_attn_outblock_noalloc(const fb_attn_desc* d, const void* q, const void* kp,
+                                   const void* vp, int64_t prefix_len,
+                                   float* a_out, float* l_out, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Block-internal attention fused with the log-space merge (summary,
  * "Mécanisme Central": A_in over J_in, merged with the block-external parts).
  *
