@@ -305,6 +305,10 @@ static fb_status run_inblock(const fb_attn_desc& d, const void* q, const void* k
                        ext_parts * rows_of(d) * (d.D + 1) * 4.0 +
                        (double)rows_of(d) * (d.D * esize(d.out_dtype) + (lse ? 4 : 0));
   ProfScope prof(kProfInblock, bytes, s);
+  if (inblock_small_applies(d, a.next))
+    return launch_inblock_small(d, q, kin, vin, a.next, a.ext_a, a.ext_l, o, lse, a.scale_log2, s) == cudaSuccess
+               ? FB_OK
+               : FB_ECUDA;
   return launch_attn_generic(a, d.D, d.in_dtype == FB_BF16, s) == cudaSuccess ? FB_OK : FB_ECUDA;
 }
 

@@ -178,6 +178,20 @@ __device__ __forceinline__ uint32_t pack2_bf16(float x, float y) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// 2^x on the MUFU unit (PTX ex2.approx; relative error about 2^-22, -inf -> 0).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// bf16 hi/lo split of a pair: hi = bf16(x), lo = bf16(x - hi).
+__device__ __forceinline__ void split_pair(float x, float y, uint32_t& hi, uint32_t& lo) {
+  hi = pack2_bf16(x, y);
+  const float hx = __uint_as_float(hi << 16), hy = __uint_as_float(hi & 0xFFFF0000u);
+  lo = pack2_bf16(x - hx, y - hy);
+}
+
 }  // namespace
 
 struct TcArgs {
@@ -350,17 +364,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(B_SFREE + st));
       const int64_t key0 = kbeg + (int64_t)j * kBN;
       const int nvalid = (int)min((int64_t)kBN, kend - key0);
-      float tmax = -CUDART_INF_F;
+      if (nvalid < kBN) {   // only the last tile of the last split is ragged
 #pragma unroll
-      for (int c = 0; c < kBN; ++c) {
-        s[c] = c < nvalid ? s[c] * a.scale_log2 : -CUDART_INF_F;
-        tmax = fmaxf(tmax, s[c]);
+        for (int c = 0; c < kBN; ++c)
+          if (c >= nvalid) s[c] = -CUDART_INF_F;
       }
+      // Row max of the raw scores (scale > 0 keeps the order), 8 chains.
+      float mx8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx8[e] = s[e];
+#pragma unroll
+      for (int c = 8; c < kBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+      const float tmax =
+          fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])), fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
+          a.scale_log2;
       // Move this row's reference max when it grew by more than 2^8; rows whose
       // O already holds values rescale it (alpha = 1 for the others).
       const bool move = tmax > m + kRescaleLog2;
       const bool scale_o = move && j > 0 && m != -CUDART_INF_F;
-      const float alpha = scale_o ? exp2f(m - tmax) : 1.f;
+      const float alpha = scale_o ? fast_exp2(m - tmax) : 1.f;
       if (__any_sync(0xffffffffu, scale_o)) {
         ok = uniform(wait_bounded(bar(B_PVDONE), (j - 1) & 1, ctl));
         if (!ok) break;
@@ -380,14 +402,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         l *= alpha;
         m = tmax;
       }
-      const float ref = (m == -CUDART_INF_F) ? 0.f : m;
-      float lsum = 0.f;
+      // p = 2^(s * scale - ref): one FFMA and one MUFU op per score; 8 sum chains.
+      const float nref = (m == -CUDART_INF_F) ? 0.f : -m;
+      float sm8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < kBN; ++c) {
-        s[c] = exp2f(s[c] - ref);
-        lsum += s[c];
+        s[c] = fast_exp2(fmaf(s[c], a.scale_log2, nref));
+        sm8[c & 7] += s[c];
       }
-      l += lsum;
+      l += ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
       // P of the previous tile must be consumed before this one overwrites it
       if (j > 0) {
         ok = uniform(wait_bounded(bar(B_PVDONE), (j - 1) & 1, ctl));
@@ -397,13 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < kBN / 8; ++c) {
         uint32_t hi[4], lo[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float x = s[c * 8 + 2 * e], y = s[c * 8 + 2 * e + 1];
-          hi[e] = pack2_bf16(x, y);
-          const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162*>(&hi[e]);
-          const float2 hf = __bfloat1622float2(hb);
-          lo[e] = pack2_bf16(x - hf.x, y - hf.y);
-        }
+        for (int e = 0; e < 4; ++e) split_pair(s[c * 8 + 2 * e], s[c * 8 + 2 * e + 1], hi[e], lo[e]);
         const uint32_t off = (c >> 3) * kHalf + ((((uint32_t)c & 7u) ^ ((uint32_t)row & 7u)) << 4);
         *reinterpret_cast<uint4*>(prow_hi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
         *reinterpret_cast<uint4*>(prow_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);

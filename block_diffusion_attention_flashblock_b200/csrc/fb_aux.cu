@@ -47,26 +47,15 @@ __device__ __forceinline__ void store_out(void* o, int64_t off, bool bf16, const
 
 // Merge all parts of one row (lane holds columns lane*E .. lane*E+E-1):
 // m = max L_p, w_p = e^{L_p - m}; returns sum w_p A_p / sum w_p and the LSE.
-// Loads are issued in batches of independent requests (no load waits on a
-// branch over another load's value), so a row costs a few memory round trips.
+// Parts are taken in batches of U whose loads are all issued before any is
+// used, with a running max across batches, so a row costs one memory round
+// trip per U parts; the summation order is fixed.
 template <int D>
 __device__ __forceinline__ float merge_row(const PartList& pl, int64_t row, int lane, float* out) {
-  constexpr int E = D / 32, U = 4;
-  float m = -CUDART_INF_F;
-  for (int gi = 0; gi < pl.ngroups; ++gi) {
-    const PartGroup& g = pl.g[gi];
-    for (int p0 = 0; p0 < g.count; p0 += 2 * U) {
-      float Ls[2 * U];
-#pragma unroll
-      for (int u = 0; u < 2 * U; ++u) Ls[u] = p0 + u < g.count ? __ldg(g.l + (p0 + u) * g.stride_l + row) : -CUDART_INF_F;
-#pragma unroll
-      for (int u = 0; u < 2 * U; ++u) m = fmaxf(m, Ls[u]);
-    }
-  }
+  constexpr int E = D / 32, U = 16;
+  float m = -CUDART_INF_F, wsum = 0.f;
 #pragma unroll
   for (int e = 0; e < E; ++e) out[e] = 0.f;
-  if (m == -CUDART_INF_F) return -CUDART_INF_F;
-  float wsum = 0.f;
   for (int gi = 0; gi < pl.ngroups; ++gi) {
     const PartGroup& g = pl.g[gi];
     for (int p0 = 0; p0 < g.count; p0 += U) {
@@ -75,12 +64,20 @@ __device__ __forceinline__ float merge_row(const PartList& pl, int64_t row, int 
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const bool ok = p0 + u < g.count;
-        Ls[u] = ok ? __ldg(g.l + (p0 + u) * g.stride_l + row) : -CUDART_INF_F;
-        if (ok) A[u].load(g.a + (p0 + u) * g.stride_a + row * D + lane * E);
-        else {
+        const int p = ok ? p0 + u : p0;
+        Ls[u] = __ldg(g.l + p * g.stride_l + row);
+        A[u].load(g.a + p * g.stride_a + row * D + lane * E);
+        if (!ok) Ls[u] = -CUDART_INF_F;
+      }
+      float bm = Ls[0];
 #pragma unroll
-          for (int e = 0; e < E; ++e) A[u].v[e] = 0.f;
-        }
+      for (int u = 1; u < U; ++u) bm = fmaxf(bm, Ls[u]);
+      if (bm > m) {
+        const float sc = (m == -CUDART_INF_F) ? 0.f : expf(m - bm);
+        wsum *= sc;
+#pragma unroll
+        for (int e = 0; e < E; ++e) out[e] *= sc;
+        m = bm;
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -90,6 +87,11 @@ __device__ __forceinline__ float merge_row(const PartList& pl, int64_t row, int 
         for (int e = 0; e < E; ++e) out[e] = fmaf(w, A[u].v[e], out[e]);
       }
     }
+  }
+  if (m == -CUDART_INF_F) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) out[e] = 0.f;
+    return -CUDART_INF_F;
   }
   const float inv = 1.f / wsum;
 #pragma unroll

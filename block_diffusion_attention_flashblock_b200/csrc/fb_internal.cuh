@@ -112,6 +112,12 @@ cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys
                            const int8_t* mask, int mask_active, float scale_log2, float* pa, float* pl,
                            cudaStream_t s);
 
+// Small-block in-block attention + merge (fb_inblock.cu).
+bool inblock_small_applies(const fb_attn_desc& d, int next);
+cudaError_t launch_inblock_small(const fb_attn_desc& d, const void* q, const void* kin, const void* vin, int next,
+                                 const float* const* ext_a, const float* const* ext_l, void* o, float* lse,
+                                 float scale_log2, cudaStream_t s);
+
 struct MergeArgs {
   int32_t B, Hq, Nb, D;
   PartList parts;

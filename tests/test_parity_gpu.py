@@ -139,7 +139,9 @@ def _random_parts(B, Hq, Nb, D, n, seed, empty_rows=True):
 
 @pytest.mark.parametrize("nparts", [0, 1, 2])
 @pytest.mark.parametrize("shape", [(1, 32, 8, 128, 32, "bf16"), (1, 4, 4, 64, 32, "f32"),
-                                   (1, 3, 3, 128, 150, "bf16"), (2, 8, 4, 64, 5, "bf16")],
+                                   (1, 3, 3, 128, 150, "bf16"), (2, 8, 4, 64, 5, "bf16"),
+                                   (2, 8, 2, 128, 5, "bf16"), (1, 8, 2, 128, 64, "bf16"),
+                                   (3, 4, 4, 128, 16, "bf16"), (1, 2, 1, 128, 1, "bf16")],
                          ids=lambda s: "x".join(map(str, s)))
 def test_inblock_merge(shape, nparts):
     B, Hq, Hkv, D, Nb, dt = shape
