@@ -213,11 +213,13 @@ static fb_status launch_pass(const fb_attn_desc& d, AttnArgs& a, float* pa, floa
 
 // Dense block-external pass over prefix rows [0, nkeys): the tcgen05 kernel
 // when the shape and strides allow it, else the generic kernel.
-static int g_prefix_kernel = 0;  // 0 auto, 1 generic only, 2 tcgen05 whenever it applies
+static int g_prefix_kernel = 0;  // 0 auto, 1 generic only, 2 tcgen05 whenever it applies, 3 as 2 without clusters
 
 struct PrefixPlan {
   bool tc;
-  int32_t nsplit;
+  int32_t nsplit;    // CTAs along the keys
+  int32_t cluster;   // > 1: the splits reduce inside one cluster
+  int32_t nparts;    // parts written: 1 when reduced in-kernel, else nsplit
   int64_t kps;
   PassPlan gen;
   TcMaps maps;
@@ -228,11 +230,14 @@ static PrefixPlan plan_prefix(const fb_attn_desc& d, const void* q, const void* 
   PrefixPlan p;
   p.gen = plan_pass(d, q, kp, vp, d.kp_strides, nkeys, nullptr, 0, cap);
   p.tc = false;
-  p.nsplit = p.gen.nsplit;
+  p.nsplit = p.nparts = p.gen.nsplit;
+  p.cluster = 1;
   p.kps = p.gen.a.keys_per_split;
-  const int64_t min_keys = g_prefix_kernel == 2 ? 1 : 256;
+  const int64_t min_keys = g_prefix_kernel >= 2 ? 1 : 256;
   if (g_prefix_kernel != 1 && nkeys >= min_keys && tc_make_maps(d, q, kp, vp, nkeys, &p.maps)) {
-    tc_plan_split((int64_t)p.maps.units * p.maps.tiles_per_unit, nkeys, cap, &p.nsplit, &p.kps);
+    tc_plan_split((int64_t)p.maps.units * p.maps.tiles_per_unit, nkeys, cap, g_prefix_kernel != 3, &p.nsplit,
+                  &p.kps, &p.cluster);
+    p.nparts = p.cluster > 1 ? 1 : p.nsplit;
     p.tc = true;
   }
   return p;
@@ -249,7 +254,7 @@ static fb_status launch_prefix(const fb_attn_desc& d, PrefixPlan& p, int64_t nke
   const double bytes = 2.0 * d.B * d.Hkv * (double)nkeys * d.D * es + (double)rows_of(d) * d.D * es +
                        (double)rows_of(d) * (d.D + 1) * 4;
   ProfScope prof(kProfPrefix, bytes, s);
-  return launch_attn_tc(d, p.maps, nkeys, p.nsplit, p.kps, mask, mask_active, scale_log2(d), pa, pl, s) ==
+  return launch_attn_tc(d, p.maps, nkeys, p.nsplit, p.kps, p.cluster, mask, mask_active, scale_log2(d), pa, pl, s) ==
                  cudaSuccess
              ? FB_OK
              : FB_ECUDA;
@@ -373,12 +378,12 @@ fb_status fb_attn_outblock(const fb_attn_desc* d, const void* q, const void* kp,
   // pass 1: dense prefix, or the selected keys
   if (!sel) {
     PrefixPlan p = plan_prefix(*d, q, kp, vp, prefix_len, cap);
-    if (p.nsplit == 1) return launch_prefix(*d, p, prefix_len, nullptr, 0, a_out, l_out, stream);
+    if (p.nparts == 1) return launch_prefix(*d, p, prefix_len, nullptr, 0, a_out, l_out, stream);
     if ((st = launch_prefix(*d, p, prefix_len, nullptr, 0, pa, pl, stream)) != FB_OK) return st;
     PartList lst;
     memset(&lst, 0, sizeof(lst));
     lst.ngroups = 1;
-    lst.g[0] = group_of(pa, pl, p.nsplit, *d);
+    lst.g[0] = group_of(pa, pl, p.nparts, *d);
     return merge_to_part(*d, lst, a_out, l_out, nullptr, 0, stream);
   }
   PassPlan p = plan_pass(*d, q, kp, vp, d->kp_strides, prefix_len, sel, sel_k, cap);
@@ -503,7 +508,7 @@ fb_status fb_profile_read(int32_t reset, int64_t* launches, double* total_ms, do
 }
 
 fb_status fb_debug_set_prefix_kernel(int32_t which) {
-  if (which < 0 || which > 2) return FB_EINVAL;
+  if (which < 0 || which > 3) return FB_EINVAL;
   g_prefix_kernel = which;
   return FB_OK;
 }
@@ -670,13 +675,13 @@ fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
     memset(&g, 0, sizeof(g));
     g.B = d.B; g.Hq = d.Hq; g.Nb = d.Nb; g.D = d.D;
     g.fresh.ngroups = 1;
-    g.fresh.g[0] = group_of(c->part_a, c->part_l, p.nsplit, d);
+    g.fresh.g[0] = group_of(c->part_a, c->part_l, p.nparts, d);
     g.cache_a = c->cache_a; g.cache_l = c->cache_l;
     g.mask = c->mask; g.gate_active = tau_reuse; g.cache_valid = c->valid;
     g.gamma = a->gamma; g.sim = c->sim; g.partials = c->gpart; g.counters = c->counters;
     g.chunks = c->chunks; g.reuse_out = a->reuse_out; g.sim_out = a->sim_out;
     {
-      ProfScope prof(kProfAux, (p.nsplit + 2.0) * rows_of(d) * (d.D + 1) * 4.0, s);
+      ProfScope prof(kProfAux, (p.nparts + 2.0) * rows_of(d) * (d.D + 1) * 4.0, s);
       if (launch_gamma_update(g, s) != cudaSuccess) return FB_ECUDA;
     }
   } else {
@@ -701,7 +706,8 @@ fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
       if (sparse) {
         p.tc = false;
         p.gen = plan_pass(d, a->q, a->kp, a->vp, d.kp_strides, a->prefix_len, nullptr, 0, c->part_cap);
-        p.nsplit = p.gen.nsplit;
+        p.nsplit = p.nparts = p.gen.nsplit;
+        p.cluster = 1;
         if (launch_build_bitmap(a->sel, a->sel_k, BH, c->bitmap, (a->prefix_len + 31) / 32, s) != cudaSuccess)
           return FB_ECUDA;
         p.gen.a.excl = c->bitmap;
@@ -709,14 +715,14 @@ fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
       } else {
         p = plan_prefix(d, a->q, a->kp, a->vp, a->prefix_len, c->part_cap);
       }
-      if (p.nsplit == 1) {
+      if (p.nparts == 1) {
         if ((st = launch_prefix(d, p, a->prefix_len, nullptr, 0, c->cache_a, c->cache_l, s)) != FB_OK) return st;
       } else {
         if ((st = launch_prefix(d, p, a->prefix_len, nullptr, 0, c->part_a, c->part_l, s)) != FB_OK) return st;
         PartList lst;
         memset(&lst, 0, sizeof(lst));
         lst.ngroups = 1;
-        lst.g[0] = group_of(c->part_a, c->part_l, p.nsplit, d);
+        lst.g[0] = group_of(c->part_a, c->part_l, p.nparts, d);
         if ((st = merge_to_part(d, lst, c->cache_a, c->cache_l, nullptr, 0, s)) != FB_OK) return st;
       }
     }

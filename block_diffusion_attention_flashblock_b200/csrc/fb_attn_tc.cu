@@ -157,6 +157,35 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Thread-block cluster helpers (split-KV reduction through distributed shared memory).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\nbarrier.cluster.wait.acquire;\n" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t map_rank(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 ld_dsmem_v4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+constexpr int kRedStride = 132;   // fp32 row stride of a CTA's staged part (bank spread)
+
 // Shared-memory matrix descriptor, 128-byte swizzle (layout code 2), sm_100
 // version bit 46; lbo/sbo in bytes.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -210,6 +239,7 @@ struct TcArgs {
   int* status;
   uint64_t wait_limit_ns;
   uint32_t q_bytes;        // bytes of one Q half-box (64 columns)
+  int32_t cluster;         // > 1: the gridDim.y splits form one cluster and reduce in-kernel
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -448,7 +478,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const float Lrow = l > 0.f ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
       const int64_t r = ((int64_t)b * a.Hq + hh) * a.Nb + ii;
-      float* pa = a.part_a + split * a.part_stride_a + r * kD;
+      // clustered: stage the normalised row in this CTA's shared memory (the
+      // K/V ring is idle now) for the cluster reduction below
+      float* pa = a.cluster > 1 ? reinterpret_cast<float*>(smem + kOffK) + row * kRedStride
+                                : a.part_a + split * a.part_stride_a + r * kD;
+      const bool store = a.cluster > 1 || valid;
 #pragma unroll
       for (int c = 0; c < kD / 32; ++c) {
         float o[32];
@@ -459,19 +493,70 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = 0.f;
         }
-        if (valid) {
+        if (store) {
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
             *reinterpret_cast<float4*>(pa + c * 32 + e) =
                 make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv);
         }
       }
-      if (valid) a.part_l[split * a.part_stride_l + r] = Lrow;
+      if (a.cluster > 1) reinterpret_cast<float*>(smem + kOffK + kBM * kRedStride * 4)[row] = Lrow;
+      else if (valid) a.part_l[split * a.part_stride_l + r] = Lrow;
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  if (a.cluster > 1) {
+    // Split-KV reduction over the cluster: rank c merges rows [c*R, c*R + R) of
+    // every rank's staged part (log-space merge, ranks in fixed order) and
+    // writes the final row.  32 threads per row, 4 columns per thread.
+    cluster_sync_all();
+    const int CS = a.cluster;
+    const uint32_t rank = cluster_rank();
+    const int R = (kBM + CS - 1) / CS;
+    const uint32_t sA = sbase + kOffK, sL = sbase + kOffK + kBM * kRedStride * 4;
+    const int lane4 = threadIdx.x & 31;
+    for (int rr = (int)rank * R + (int)(threadIdx.x >> 5); rr < min(kBM, ((int)rank + 1) * R); rr += kThreads / 32) {
+      int hh, ii;
+      bool valid;
+      if (a.mode == 0) {
+        const int g = t * a.hg + rr / a.Nb;
+        ii = rr % a.Nb;
+        hh = kvh * a.G + g;
+        valid = rr < a.hg * a.Nb && g < a.G;
+      } else {
+        hh = h0;
+        ii = i0 + rr;
+        valid = ii < a.Nb;
+      }
+      if (!valid) continue;
+      float m = -CUDART_INF_F;
+      float Ls[16];
+#pragma unroll
+      for (int p = 0; p < 16; ++p) {
+        Ls[p] = p < CS ? ld_dsmem_f32(map_rank(sL + rr * 4, p)) : -CUDART_INF_F;
+        m = fmaxf(m, Ls[p]);
+      }
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      float wsum = 0.f;
+#pragma unroll
+      for (int p = 0; p < 16; ++p) {
+        if (p >= CS || Ls[p] == -CUDART_INF_F) continue;
+        const float w = __expf(Ls[p] - m);
+        const float4 v = ld_dsmem_v4(map_rank(sA + (rr * kRedStride + lane4 * 4) * 4, p));
+        wsum += w;
+        acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
+        acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+      }
+      const int64_t r = ((int64_t)b * a.Hq + hh) * a.Nb + ii;
+      const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+      *reinterpret_cast<float4*>(a.part_a + r * kD + lane4 * 4) =
+          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+      if (lane4 == 0) a.part_l[r] = m == -CUDART_INF_F ? -CUDART_INF_F : m + __logf(wsum);
+    }
+    cluster_sync_all();   // keep every rank's shared memory alive until all reads are done
+  }
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
@@ -546,28 +631,74 @@ int32_t tc_split_cap(int64_t tiles, int64_t max_keys) {
   return (int32_t)std::min(ktiles, want);
 }
 
-// Split count for `tiles` row tiles over nkeys keys: balance whole waves of
-// one CTA per SM against a fixed per-CTA cost (about two key tiles).
-void tc_plan_split(int64_t tiles, int64_t nkeys, int32_t max_split, int32_t* nsplit, int64_t* kps) {
+// Largest number of clusters of `cs` CTAs that can run at once (0: not launchable).
+static int max_active_clusters(int cs) {
+  static int cache[64][17];
+  static bool init[64][17];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || cs < 2 || cs > 16) return 0;
+  if (init[dev][cs]) return cache[dev][cs];
+  int n = 0;
+  if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) == cudaSuccess &&
+      (cs <= 8 || cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                      cudaSuccess)) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, cs, 1);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 1;
+    at[0].val.clusterDim.y = cs;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, (void*)attn_tc_kernel, &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();
+  cache[dev][cs] = n;
+  init[dev][cs] = true;
+  return n;
+}
+
+// Split plan for `tiles` row tiles over nkeys keys.  Candidates: one split; up
+// to 16 splits reduced inside one cluster per tile; or more splits whose
+// partials a merge pass combines (at most max_split of them).  Cost = waves x
+// (key tiles per CTA + fixed CTA cost) + the merge pass when there is one.
+void tc_plan_split(int64_t tiles, int64_t nkeys, int32_t max_split, bool allow_cluster, int32_t* nsplit,
+                   int64_t* kps, int32_t* cluster) {
   const int64_t sms = num_sms();
   const int64_t ktiles = std::max<int64_t>(1, (nkeys + kBN - 1) / kBN);
-  int64_t best_ns = 1;
+  int64_t best_per = ktiles, best_cl = 1;
   double best = 1e300;
-  for (int64_t ns = 1; ns <= std::min<int64_t>(ktiles, std::max(1, max_split)); ++ns) {
+  for (int64_t ns = 1; ns <= ktiles; ++ns) {
     const int64_t per = (ktiles + ns - 1) / ns;
     const int64_t real_ns = (ktiles + per - 1) / per;
-    const int64_t waves = (tiles * real_ns + sms - 1) / sms;
-    const double cost = (double)waves * (per + 2) + 0.02 * real_ns;
-    if (cost < best) { best = cost; best_ns = real_ns; }
+    if (real_ns != ns) continue;
+    double cost;
+    int64_t cl = 1;
+    if (ns == 1) {
+      cost = (double)((tiles + sms - 1) / sms) * (per + 2);
+    } else if (allow_cluster && ns <= 16 && max_active_clusters((int)ns) > 0) {
+      const int64_t conc = max_active_clusters((int)ns);
+      cost = (double)((tiles + conc - 1) / conc) * (per + 2) + 0.5;
+      cl = ns;
+    } else if (ns <= max_split) {
+      cost = (double)((tiles * ns + sms - 1) / sms) * (per + 2) + 6.0;
+    } else {
+      continue;
+    }
+    if (cost < best) { best = cost; best_per = per; best_cl = cl; }
   }
-  const int64_t per = (ktiles + best_ns - 1) / best_ns;
-  *kps = per * kBN;
+  *kps = best_per * kBN;
   *nsplit = (int32_t)std::max<int64_t>(1, (nkeys + *kps - 1) / *kps);
+  *cluster = (int32_t)best_cl;
 }
 
 cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys, int32_t nsplit, int64_t kps,
-                           const int8_t* mask, int mask_active, float scale_log2, float* pa, float* pl,
-                           cudaStream_t s) {
+                           int32_t cluster, const int8_t* mask, int mask_active, float scale_log2, float* pa,
+                           float* pl, cudaStream_t s) {
   TcArgs a;
   a.B = d.B; a.Hq = d.Hq; a.Hkv = d.Hkv; a.G = d.Hq / d.Hkv; a.Nb = d.Nb;
   a.mode = m.mode; a.hg = m.hg; a.tiles_per_unit = m.tiles_per_unit;
@@ -579,6 +710,7 @@ cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys
   a.q_bytes = 64u * 2u * (uint32_t)(m.mode == 0 ? d.Nb * m.hg : kBM);
   a.status = device_status_ptr();
   a.wait_limit_ns = wait_limit_ns();
+  a.cluster = cluster > 1 ? nsplit : 1;
   if (!a.status) return cudaErrorInvalidValue;
   static bool attr = false;
   if (!attr) {
@@ -587,8 +719,23 @@ cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys
     attr = true;
   }
   dim3 grid(m.units * m.tiles_per_unit, nsplit);
-  attn_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(m.q, m.k, m.v, a);
-  return cudaGetLastError();
+  if (a.cluster <= 1) {
+    attn_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(m.q, m.k, m.v, a);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 1;
+  at[0].val.clusterDim.y = (unsigned)nsplit;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attn_tc_kernel, m.q, m.k, m.v, a);
 }
 
 }  // namespace fb

@@ -106,11 +106,12 @@ struct TcMaps {
 };
 bool tc_tiling(const fb_attn_desc& d, int* mode, int* hg, int* tiles_per_unit, int* units);
 bool tc_make_maps(const fb_attn_desc& d, const void* q, const void* kp, const void* vp, int64_t nkeys, TcMaps* m);
-void tc_plan_split(int64_t tiles, int64_t nkeys, int32_t max_split, int32_t* nsplit, int64_t* kps);
+void tc_plan_split(int64_t tiles, int64_t nkeys, int32_t max_split, bool allow_cluster, int32_t* nsplit,
+                   int64_t* kps, int32_t* cluster);
 int32_t tc_split_cap(int64_t tiles, int64_t max_keys);
 cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys, int32_t nsplit, int64_t kps,
-                           const int8_t* mask, int mask_active, float scale_log2, float* pa, float* pl,
-                           cudaStream_t s);
+                           int32_t cluster, const int8_t* mask, int mask_active, float scale_log2, float* pa,
+                           float* pl, cudaStream_t s);
 
 // Small-block in-block attention + merge (fb_inblock.cu).
 bool inblock_small_applies(const fb_attn_desc& d, int next);

@@ -259,7 +259,9 @@ fb_status fb_profile_read(int32_t reset, int64_t* launches, double* total_ms, do
 
 /* Test hook: which kernel runs dense block-external passes: 0 automatic (the
  * tcgen05 kernel where the shape and strides allow it), 1 the generic
- * mma.sync / FFMA kernel only, 2 the tcgen05 kernel whenever it applies. */
+ * mma.sync / FFMA kernel only, 2 the tcgen05 kernel whenever it applies,
+ * 3 as 2 but its key splits always go through a separate merge instead of
+ * the in-kernel cluster reduction. */
 fb_status fb_debug_set_prefix_kernel(int32_t which);
 
 /* Test hook: the bound of every barrier wait in later launches, in
