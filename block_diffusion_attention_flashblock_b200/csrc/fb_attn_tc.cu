@@ -10,10 +10,13 @@
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma:
 //               S = Q K^T into one of two TMEM S buffers, and
 //               O += P_hi V + P_lo V into the TMEM O accumulator.
-//   warps 2..5  softmax, one query row per thread (TMEM lane = row): read S
-//               with tcgen05.ld, online max/sum in the log2 domain, write
-//               P = 2^(s - m) as bf16 hi + lo into swizzled shared memory for
-//               the PV product; the final O / l and L go to the split's part.
+//   warps 2..9  softmax, two threads per query row (TMEM lane = row): warps
+//               w and w+4 share a TMEM lane quarter and take columns 0..63 and
+//               64..127 of S; they trade their row maxima (and at the end
+//               their row sums) through spare TMEM columns and a bounded
+//               mbarrier.  Each writes its half of P = 2^(s - m) as bf16 hi +
+//               lo into swizzled shared memory for the PV product; the final
+//               O / l and L go to the split's part.
 // The running max is only moved (and O rescaled in TMEM) when a row's max
 // grows by more than 2^8, so P stays <= 256 and most tiles skip the rescale.
 // Every mbarrier wait is bounded; on expiry the CTA records FB_ETIMEOUT in
@@ -32,7 +35,7 @@ namespace fb {
 namespace {
 
 constexpr int kBM = 128, kBN = 128, kD = 128;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr uint32_t kHalf = 16384;                 // [128 rows][64 bf16] 128B-swizzled block
 constexpr uint32_t kOffQ = 0;                     // Q: 2 halves
 constexpr uint32_t kOffK = kOffQ + 2 * kHalf;     // K: 2 stages x 2 halves
@@ -42,12 +45,13 @@ constexpr uint32_t kOffBar = kOffP + 4 * kHalf;   // barriers and flags
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + slack for 1024-byte alignment
 constexpr uint32_t kTmemCols = 512;               // S0 [0,128) S1 [128,256) O [256,384)
 constexpr uint32_t kTmemO = 256;
+constexpr uint32_t kTmemX = 384;                  // row-statistics exchange columns
 constexpr float kRescaleLog2 = 8.0f;
 
 // barrier slots
 enum {
   B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 3, B_VFULL = 5, B_VEMPTY = 7, B_SFULL = 9, B_SFREE = 11,
-  B_PFULL = 13, B_PVDONE = 14, B_DRAIN = 15, B_COUNT = 16
+  B_PFULL = 13, B_PVDONE = 14, B_DRAIN = 15, B_PAIR = 16, B_COUNT = 20
 };
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -153,6 +157,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
       "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
       "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
+}
+__device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
+  uint32_t r;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+  return __uint_as_float(r);
+}
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, float v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(__float_as_uint(v)) : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
@@ -276,7 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < B_COUNT; ++i) {
       uint32_t cnt = 1;
-      if (i == B_SFREE || i == B_SFREE + 1 || i == B_PFULL) cnt = 128;
+      if (i == B_SFREE || i == B_SFREE + 1 || i == B_PFULL) cnt = 256;
+      if (i >= B_PAIR) cnt = 64;
       mbar_init(bar(i), cnt);
     }
     *abort_flag = 0;
@@ -373,43 +386,63 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax
     const int q4 = warp & 3;
+    const int half = (warp - 2) >> 2;          // 0: columns 0..63, 1: columns 64..127
     const int row = q4 * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
-    uint8_t* prow_hi = smem + kOffP + row * 128;
-    uint8_t* prow_lo = smem + kOffP + 2 * kHalf + row * 128;
+    const uint32_t pair = bar(B_PAIR + q4);
+    uint8_t* prow_hi = smem + kOffP + half * kHalf + row * 128;
+    uint8_t* prow_lo = smem + kOffP + 2 * kHalf + half * kHalf + row * 128;
     float m = -CUDART_INF_F, l = 0.f;
     bool ok = true;
     // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform.
     auto uniform = [](bool v) { return __all_sync(0xffffffffu, v); };
+    // Trade one value per row with the partner warp through TMEM column
+    // kTmemX + 2*slot + half (phase `ph` of this lane quarter's pair barrier).
+    auto trade = [&](float mine, int slot, int ph, float& theirs) -> bool {
+      tmem_st1(tl + kTmemX + 2 * slot + half, mine);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(pair);
+      if (!uniform(wait_bounded(pair, ph & 1, ctl))) return false;
+      tc_fence_after();
+      theirs = tmem_ld1(tl + kTmemX + 2 * slot + (half ^ 1));
+      tmem_wait_ld();
+      return true;
+    };
     for (int j = 0; j < T && ok; ++j) {
       const int st = j & 1;
       ok = uniform(wait_bounded(bar(B_SFULL + st), (j >> 1) & 1, ctl));
       if (!ok) break;
       tc_fence_after();
-      float s[kBN];
-#pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tl + st * kBN + c * 32, s + c * 32);
+      float s[kBN / 2];
+      tmem_ld32(tl + st * kBN + half * 64, s);
+      tmem_ld32(tl + st * kBN + half * 64 + 32, s + 32);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(B_SFREE + st));
       const int64_t key0 = kbeg + (int64_t)j * kBN;
-      const int nvalid = (int)min((int64_t)kBN, kend - key0);
-      if (nvalid < kBN) {   // only the last tile of the last split is ragged
+      const int nvalid = (int)min((int64_t)kBN, kend - key0) - half * 64;
+      if (nvalid < 64) {   // only the last tile of the last split is ragged
 #pragma unroll
-        for (int c = 0; c < kBN; ++c)
+        for (int c = 0; c < 64; ++c)
           if (c >= nvalid) s[c] = -CUDART_INF_F;
       }
-      // Row max of the raw scores (scale > 0 keeps the order), 8 chains.
+      // Half-row max of the raw scores (scale > 0 keeps the order), 8 chains,
+      // then the partner's half: both threads of a row see the same max.
       float mx8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) mx8[e] = s[e];
 #pragma unroll
-      for (int c = 8; c < kBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-      const float tmax =
+      for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+      float tmax =
           fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])), fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
           a.scale_log2;
+      float other;
+      ok = trade(tmax, j & 1, j, other);
+      if (!ok) break;
+      tmax = fmaxf(tmax, other);
       // Move this row's reference max when it grew by more than 2^8; rows whose
-      // O already holds values rescale it (alpha = 1 for the others).
+      // O already holds values rescale their half of it (alpha = 1 otherwise).
       const bool move = tmax > m + kRescaleLog2;
       const bool scale_o = move && j > 0 && m != -CUDART_INF_F;
       const float alpha = scale_o ? fast_exp2(m - tmax) : 1.f;
@@ -418,13 +451,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < kD / 32; ++c) {
+        for (int c = 0; c < 2; ++c) {
           float o[32];
-          tmem_ld32(tl + kTmemO + c * 32, o);
+          tmem_ld32(tl + kTmemO + half * 64 + c * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] *= alpha;
-          tmem_st32(tl + kTmemO + c * 32, o);
+          tmem_st32(tl + kTmemO + half * 64 + c * 32, o);
         }
         tmem_wait_st();
       }
@@ -436,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float nref = (m == -CUDART_INF_F) ? 0.f : -m;
       float sm8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < kBN; ++c) {
+      for (int c = 0; c < 64; ++c) {
         s[c] = fast_exp2(fmaf(s[c], a.scale_log2, nref));
         sm8[c & 7] += s[c];
       }
@@ -447,11 +480,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
       }
 #pragma unroll
-      for (int c = 0; c < kBN / 8; ++c) {
+      for (int c = 0; c < 8; ++c) {
         uint32_t hi[4], lo[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) split_pair(s[c * 8 + 2 * e], s[c * 8 + 2 * e + 1], hi[e], lo[e]);
-        const uint32_t off = (c >> 3) * kHalf + ((((uint32_t)c & 7u) ^ ((uint32_t)row & 7u)) << 4);
+        const uint32_t off = (((uint32_t)c ^ ((uint32_t)row & 7u)) << 4);
         *reinterpret_cast<uint4*>(prow_hi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
         *reinterpret_cast<uint4*>(prow_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
@@ -461,7 +494,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ------------------------------------------------------------ epilogue
     if (ok && T > 0) ok = uniform(wait_bounded(bar(B_PVDONE), (T - 1) & 1, ctl));
+    float lo_other = 0.f;
+    if (ok) ok = trade(l, T & 1, T, lo_other);   // the row sum is the two halves' sum
     if (ok) {
+      l += lo_other;
       tc_fence_after();
       int hh, ii;
       bool valid;
@@ -480,14 +516,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t r = ((int64_t)b * a.Hq + hh) * a.Nb + ii;
       // clustered: stage the normalised row in this CTA's shared memory (the
       // K/V ring is idle now) for the cluster reduction below
-      float* pa = a.cluster > 1 ? reinterpret_cast<float*>(smem + kOffK) + row * kRedStride
-                                : a.part_a + split * a.part_stride_a + r * kD;
+      float* pa = (a.cluster > 1 ? reinterpret_cast<float*>(smem + kOffK) + row * kRedStride
+                                 : a.part_a + split * a.part_stride_a + r * kD) +
+                  half * 64;
       const bool store = a.cluster > 1 || valid;
 #pragma unroll
-      for (int c = 0; c < kD / 32; ++c) {
+      for (int c = 0; c < 2; ++c) {
         float o[32];
         if (T > 0) {
-          tmem_ld32(tl + kTmemO + c * 32, o);
+          tmem_ld32(tl + kTmemO + half * 64 + c * 32, o);
           tmem_wait_ld();
         } else {
 #pragma unroll
@@ -500,8 +537,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv);
         }
       }
-      if (a.cluster > 1) reinterpret_cast<float*>(smem + kOffK + kBM * kRedStride * 4)[row] = Lrow;
-      else if (valid) a.part_l[split * a.part_stride_l + r] = Lrow;
+      if (half == 0) {
+        if (a.cluster > 1) reinterpret_cast<float*>(smem + kOffK + kBM * kRedStride * 4)[row] = Lrow;
+        else if (valid) a.part_l[split * a.part_stride_l + r] = Lrow;
+      }
     }
   }
 

@@ -2,8 +2,10 @@
 // (FlashBlock summary, "Mécanisme Central": A_in over the block's own keys
 // J_in, then A = (e^{L_out-m} A_out + e^{L_in-m} A_in) / (...)).  This is the
 // whole reuse step of a diffusion LM, so it is built for latency:
-//   - one CTA = 64 packed query rows of one KV head (G query heads x Nb
-//     queries), 4 warps x 16 rows;
+//   - one CTA = 32 packed query rows of one KV head (G query heads x Nb
+//     queries); 4 warps: two 16-row slabs, and for each slab two warps that
+//     both form S and P but split the P V product and the epilogue by halves
+//     of the head dimension (shorter per-warp instruction chains);
 //   - every global load (Q, K_in, V_in and the cached external parts A, L) is
 //     issued at once with cp.async, so the kernel waits on memory once;
 //   - S = Q K_in^T and O = P V on mma.sync m16n8k16 (bf16 in, fp32 out) with
@@ -19,7 +21,7 @@ namespace fb {
 
 namespace {
 
-constexpr int kRows = 64;          // query rows per CTA
+constexpr int kRows = 32;          // query rows per CTA
 constexpr int kD = 128;
 constexpr int kExtStride = 132;    // fp32 row stride of staged external parts (bank spread)
 constexpr int kMaxExt = 2;
@@ -132,7 +134,8 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
   __syncthreads();
 
-  // ---- S = Q K^T for this warp's 16 rows ----
+  // ---- S = Q K^T for this warp's 16-row slab ----
+  const int slab = warp & 1, dh = warp >> 1;   // dh: which 64 columns of D this warp outputs
   float s[NT][4];
 #pragma unroll
   for (int n = 0; n < NT; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
@@ -140,7 +143,7 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   for (int kk = 0; kk < kD / 16; ++kk) {
     uint32_t qa[4];
     {
-      const int r = warp * 16 + (lane & 15), ch = 2 * kk + (lane >> 4);
+      const int r = slab * 16 + (lane & 15), ch = 2 * kk + (lane >> 4);
       ldsm4(saddr(sQ + swz(r, ch)), qa[0], qa[1], qa[2], qa[3]);
     }
 #pragma unroll
@@ -183,17 +186,18 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
     lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 1);
     lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 2);
   }
-  // ---- O = P V ----
-  float o[kD / 8][4];
+  // ---- O[:, dh*64 : dh*64+64] = P V ----
+  constexpr int DT = kD / 16;    // 8-column tiles in this warp's half
+  float o[DT][4];
 #pragma unroll
-  for (int d = 0; d < kD / 8; ++d) o[d][0] = o[d][1] = o[d][2] = o[d][3] = 0.f;
+  for (int d = 0; d < DT; ++d) o[d][0] = o[d][1] = o[d][2] = o[d][3] = 0.f;
 #pragma unroll
   for (int kk = 0; kk < KK; ++kk) {
     const uint32_t ah[4] = {ph[2 * kk][0], ph[2 * kk][1], ph[2 * kk + 1][0], ph[2 * kk + 1][1]};
     const uint32_t al[4] = {pl[2 * kk][0], pl[2 * kk][1], pl[2 * kk + 1][0], pl[2 * kk + 1][1]};
 #pragma unroll
-    for (int d = 0; d < kD / 8; d += 2) {
-      const int r = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8, ch = d + (lane >> 4);
+    for (int d = 0; d < DT; d += 2) {
+      const int r = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8, ch = dh * DT + d + (lane >> 4);
       uint32_t b0, b1, b2, b3;
       ldsm4t(saddr(sV + swz(r, ch)), b0, b1, b2, b3);
       mma16816(o[d], ah, b0, b1);
@@ -205,7 +209,7 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   // ---- merge with the external parts and store ----
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const int r = warp * 16 + (lane >> 2) + 8 * h;
+    const int r = slab * 16 + (lane >> 2) + 8 * h;
     const int rr = row0 + r;
     if (rr >= rows_unit) continue;
     const float Lin = lrow[h] > 0.f ? (mrow[h] + __log2f(lrow[h])) * kLn2 : -CUDART_INF_F;
@@ -229,8 +233,8 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
     const int g = rr / a.Nb, i = rr % a.Nb;
     const int64_t obase = b * a.o_sb + (int64_t)(kvh * a.G + g) * a.o_sh + (int64_t)i * a.o_st;
 #pragma unroll
-    for (int d = 0; d < kD / 8; ++d) {
-      const int col = d * 8 + 2 * (lane & 3);
+    for (int d = 0; d < DT; ++d) {
+      const int col = dh * 64 + d * 8 + 2 * (lane & 3);
       float x = win * o[d][2 * h], y = win * o[d][2 * h + 1];
 #pragma unroll
       for (int p = 0; p < kMaxExt; ++p) {
@@ -246,7 +250,7 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
       else
         *reinterpret_cast<float2*>(static_cast<float*>(a.o) + obase + col) = make_float2(x, y);
     }
-    if (a.lse && (lane & 3) == 0) a.lse[prow0 + r] = empty ? -CUDART_INF_F : m + logf(wsum);
+    if (a.lse && dh == 0 && (lane & 3) == 0) a.lse[prow0 + r] = empty ? -CUDART_INF_F : m + logf(wsum);
   }
 }
 
