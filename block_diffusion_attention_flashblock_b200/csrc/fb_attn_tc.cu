@@ -4,21 +4,26 @@
 //
 // One CTA = one tile of 128 query rows (the block queries of the query heads
 // that share a KV head, packed) x one split of the prefix keys.  Warp roles:
-//   warp 0      TMA producer: Q once, then K and V tiles of 128 keys into a
-//               two-stage ring (cp.async.bulk.tensor, 128-byte swizzle, no
-//               multicast).
+//   warp 0      TMA producers, no multicast: lane 0 loads Q once and then K
+//               tiles of 128 keys into a three-stage ring, lane 1 loads the V
+//               tiles into their own three-stage ring (128-byte swizzle).
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma:
-//               S = Q K^T into one of two TMEM S buffers, and
-//               O += P_hi V + P_lo V into the TMEM O accumulator.
+//               S = Q K^T (A, B in shared memory) into one of two TMEM S
+//               buffers, and O += P_hi V + P_lo V with P read from TMEM.
 //   warps 2..9  softmax, two threads per query row (TMEM lane = row): warps
 //               w and w+4 share a TMEM lane quarter and take columns 0..63 and
 //               64..127 of S; they trade their row maxima (and at the end
 //               their row sums) through spare TMEM columns and a bounded
-//               mbarrier.  Each writes its half of P = 2^(s - m) as bf16 hi +
-//               lo into swizzled shared memory for the PV product; the final
-//               O / l and L go to the split's part.
+//               mbarrier.  Each writes its half of P = 2^(s - m), as bf16 hi
+//               and lo parts, back into the TMEM columns its S tile came from;
+//               the final O / l and L go to the split's part.
+// P lives in the S buffer it replaces, so S_{j+2} may only overwrite it after
+// PV_j: the MMA thread issues in the order S_j, PV_{j-1}, S_{j+1}, PV_j, ...
+// and the tensor core runs its operations in issue order.
 // The running max is only moved (and O rescaled in TMEM) when a row's max
 // grows by more than 2^8, so P stays <= 256 and most tiles skip the rescale.
+// With a cluster launch, the key splits of one row tile reduce their parts
+// through distributed shared memory before anything reaches global memory.
 // Every mbarrier wait is bounded; on expiry the CTA records FB_ETIMEOUT in
 // the device status word, drains its own TMA and MMA work, frees TMEM and
 // exits.
@@ -36,22 +41,23 @@ namespace {
 
 constexpr int kBM = 128, kBN = 128, kD = 128;
 constexpr int kThreads = 320;
+constexpr int kStages = 3;                        // K and V ring depth
 constexpr uint32_t kHalf = 16384;                 // [128 rows][64 bf16] 128B-swizzled block
-constexpr uint32_t kOffQ = 0;                     // Q: 2 halves
-constexpr uint32_t kOffK = kOffQ + 2 * kHalf;     // K: 2 stages x 2 halves
-constexpr uint32_t kOffV = kOffK + 4 * kHalf;     // V: 2 stages x 2 halves
-constexpr uint32_t kOffP = kOffV + 4 * kHalf;     // P: hi 2 halves, lo 2 halves
-constexpr uint32_t kOffBar = kOffP + 4 * kHalf;   // barriers and flags
+constexpr uint32_t kTile = 2 * kHalf;             // one 128 x 128 bf16 tile
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffK = kOffQ + kTile;
+constexpr uint32_t kOffV = kOffK + kStages * kTile;
+constexpr uint32_t kOffBar = kOffV + kStages * kTile;   // barriers and flags
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + slack for 1024-byte alignment
-constexpr uint32_t kTmemCols = 512;               // S0 [0,128) S1 [128,256) O [256,384)
+constexpr uint32_t kTmemCols = 512;               // S/P buffers [0,128) [128,256), O [256,384)
 constexpr uint32_t kTmemO = 256;
 constexpr uint32_t kTmemX = 384;                  // row-statistics exchange columns
 constexpr float kRescaleLog2 = 8.0f;
 
 // barrier slots
 enum {
-  B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 3, B_VFULL = 5, B_VEMPTY = 7, B_SFULL = 9, B_SFREE = 11,
-  B_PFULL = 13, B_PVDONE = 14, B_DRAIN = 15, B_PAIR = 16, B_COUNT = 20
+  B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 10, B_SFULL = 13, B_PFULL = 15,
+  B_PVDONE = 17, B_DRAIN = 18, B_PAIR = 19, B_COUNT = 23
 };
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -127,6 +133,25 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
           d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+// D (TMEM) += A (TMEM, row per lane, bf16 pairs per column) x B (shared memory descriptor)
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accum) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(
+          d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%"
+      "18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+      "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
 }
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
@@ -288,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < B_COUNT; ++i) {
       uint32_t cnt = 1;
-      if (i == B_SFREE || i == B_SFREE + 1 || i == B_PFULL) cnt = 256;
+      if (i == B_PFULL || i == B_PFULL + 1) cnt = 256;
       if (i >= B_PAIR) cnt = 64;
       mbar_init(bar(i), cnt);
     }
@@ -307,54 +332,52 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Ctl ctl{abort_flag, a.status, a.wait_limit_ns};
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0 && T > 0) {
-      int armed_k[2] = {-1, -1}, armed_v[2] = {-1, -1};
+    // ------------------------------------------------------------ producers
+    if (lane < 2 && T > 0) {
+      // lane 0: Q, then the K ring; lane 1: the V ring
+      const bool is_k = lane == 0;
+      const CUtensorMap* tm = is_k ? &tmK : &tmV;
+      const int full = is_k ? B_KFULL : B_VFULL, empty = is_k ? B_KEMPTY : B_VEMPTY;
+      const uint32_t ring = sbase + (is_k ? kOffK : kOffV);
+      int armed[kStages] = {-1, -1, -1};
       bool ok = true;
-      mbar_expect_tx(bar(B_QFULL), 2 * a.q_bytes);
-      tma_load_4d(sbase + kOffQ, &tmQ, bar(B_QFULL), 0, i0, h0, b);
-      tma_load_4d(sbase + kOffQ + kHalf, &tmQ, bar(B_QFULL), 64, i0, h0, b);
+      if (is_k) {
+        mbar_expect_tx(bar(B_QFULL), 2 * a.q_bytes);
+        tma_load_4d(sbase + kOffQ, &tmQ, bar(B_QFULL), 0, i0, h0, b);
+        tma_load_4d(sbase + kOffQ + kHalf, &tmQ, bar(B_QFULL), 64, i0, h0, b);
+      }
       for (int j = 0; j < T && ok; ++j) {
-        const int st = j & 1;
+        const int st = j % kStages, round = j / kStages;
+        if (j >= kStages) ok = wait_bounded(bar(empty + st), (round - 1) & 1, ctl);
+        if (!ok) break;
         const int key0 = (int)(kbeg + (int64_t)j * kBN);
-        if (j >= 2) ok = wait_bounded(bar(B_KEMPTY + st), ((j >> 1) - 1) & 1, ctl);
-        if (!ok) break;
-        mbar_expect_tx(bar(B_KFULL + st), 2 * kHalf);
-        tma_load_4d(sbase + kOffK + st * 2 * kHalf, &tmK, bar(B_KFULL + st), 0, key0, kvh, b);
-        tma_load_4d(sbase + kOffK + st * 2 * kHalf + kHalf, &tmK, bar(B_KFULL + st), 64, key0, kvh, b);
-        armed_k[st] = j >> 1;
-        if (j >= 2) ok = wait_bounded(bar(B_VEMPTY + st), ((j >> 1) - 1) & 1, ctl);
-        if (!ok) break;
-        mbar_expect_tx(bar(B_VFULL + st), 2 * kHalf);
-        tma_load_4d(sbase + kOffV + st * 2 * kHalf, &tmV, bar(B_VFULL + st), 0, key0, kvh, b);
-        tma_load_4d(sbase + kOffV + st * 2 * kHalf + kHalf, &tmV, bar(B_VFULL + st), 64, key0, kvh, b);
-        armed_v[st] = j >> 1;
+        mbar_expect_tx(bar(full + st), kTile);
+        tma_load_4d(ring + st * kTile, tm, bar(full + st), 0, key0, kvh, b);
+        tma_load_4d(ring + st * kTile + kHalf, tm, bar(full + st), 64, key0, kvh, b);
+        armed[st] = round;
       }
       // Let every copy this thread started land before the CTA can exit.
-      wait_bounded(bar(B_QFULL), 0, ctl, true);
-      for (int st = 0; st < 2; ++st) {
-        if (armed_k[st] >= 0) wait_bounded(bar(B_KFULL + st), armed_k[st] & 1, ctl, true);
-        if (armed_v[st] >= 0) wait_bounded(bar(B_VFULL + st), armed_v[st] & 1, ctl, true);
-      }
+      if (is_k) wait_bounded(bar(B_QFULL), 0, ctl, true);
+      for (int st = 0; st < kStages; ++st)
+        if (armed[st] >= 0) wait_bounded(bar(full + st), armed[st] & 1, ctl, true);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && T > 0) {
       bool ok = wait_bounded(bar(B_QFULL), 0, ctl);
       auto issue_pv = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!wait_bounded(bar(B_PFULL), j & 1, ctl)) return false;
-        if (!wait_bounded(bar(B_VFULL + st), (j >> 1) & 1, ctl)) return false;
+        const int sb = j & 1, st = j % kStages;
+        if (!wait_bounded(bar(B_PFULL + sb), (j >> 1) & 1, ctl)) return false;
+        if (!wait_bounded(bar(B_VFULL + st), (j / kStages) & 1, ctl)) return false;
         tc_fence_after();
-        const uint32_t vb = sbase + kOffV + st * 2 * kHalf;
+        const uint32_t vb = sbase + kOffV + st * kTile;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {   // P_hi, then P_lo
-          const uint32_t pb = sbase + kOffP + part * 2 * kHalf;
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk) {
-            const uint64_t ad = sw128_desc(pb + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
             const uint64_t bd = sw128_desc(vb + kk * 2048, kHalf, 1024);
-            tc_mma(tmem + kTmemO, ad, bd, kIdescPV, (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
+            tc_mma_ts(tmem + kTmemO, tmem + sb * kBN + part * 64 + kk * 8, bd, kIdescPV,
+                      (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
           }
         }
         tc_commit(bar(B_VEMPTY + st));
@@ -362,19 +385,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       for (int j = 0; j < T && ok; ++j) {
-        const int st = j & 1;
-        ok = wait_bounded(bar(B_KFULL + st), (j >> 1) & 1, ctl);
-        if (ok && j >= 2) ok = wait_bounded(bar(B_SFREE + st), ((j >> 1) - 1) & 1, ctl);
+        const int sb = j & 1, st = j % kStages;
+        ok = wait_bounded(bar(B_KFULL + st), (j / kStages) & 1, ctl);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t kb = sbase + kOffK + st * 2 * kHalf;
+        const uint32_t kb = sbase + kOffK + st * kTile;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint64_t ad = sw128_desc(sbase + kOffQ + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = sw128_desc(kb + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
-          tc_mma(tmem + st * kBN, ad, bd, kIdescQK, kk > 0 ? 1u : 0u);
+          tc_mma(tmem + sb * kBN, ad, bd, kIdescQK, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar(B_SFULL + st));
+        tc_commit(bar(B_SFULL + sb));
         tc_commit(bar(B_KEMPTY + st));
         if (j >= 1) ok = issue_pv(j - 1);
       }
@@ -390,8 +412,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = q4 * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
     const uint32_t pair = bar(B_PAIR + q4);
-    uint8_t* prow_hi = smem + kOffP + half * kHalf + row * 128;
-    uint8_t* prow_lo = smem + kOffP + 2 * kHalf + half * kHalf + row * 128;
     float m = -CUDART_INF_F, l = 0.f;
     bool ok = true;
     // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform.
@@ -410,16 +430,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
     for (int j = 0; j < T && ok; ++j) {
-      const int st = j & 1;
-      ok = uniform(wait_bounded(bar(B_SFULL + st), (j >> 1) & 1, ctl));
+      const int sb = j & 1;
+      ok = uniform(wait_bounded(bar(B_SFULL + sb), (j >> 1) & 1, ctl));
       if (!ok) break;
       tc_fence_after();
-      float s[kBN / 2];
-      tmem_ld32(tl + st * kBN + half * 64, s);
-      tmem_ld32(tl + st * kBN + half * 64 + 32, s + 32);
+      float s[64];
+      tmem_ld32(tl + sb * kBN + half * 64, s);
+      tmem_ld32(tl + sb * kBN + half * 64 + 32, s + 32);
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(B_SFREE + st));
       const int64_t key0 = kbeg + (int64_t)j * kBN;
       const int nvalid = (int)min((int64_t)kBN, kend - key0) - half * 64;
       if (nvalid < 64) {   // only the last tile of the last split is ragged
@@ -428,7 +446,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (c >= nvalid) s[c] = -CUDART_INF_F;
       }
       // Half-row max of the raw scores (scale > 0 keeps the order), 8 chains,
-      // then the partner's half: both threads of a row see the same max.
+      // then the partner's half: both threads of a row see the same max.  The
+      // trade also orders both halves' reads of S before either writes P over it.
       float mx8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) mx8[e] = s[e];
@@ -474,23 +493,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         sm8[c & 7] += s[c];
       }
       l += ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
-      // P of the previous tile must be consumed before this one overwrites it
-      if (j > 0) {
-        ok = uniform(wait_bounded(bar(B_PVDONE), (j - 1) & 1, ctl));
-        if (!ok) break;
-      }
+      // P (bf16 pairs, lower key in the low half) over this tile's S columns:
+      // hi parts at [sb*128, sb*128+64), lo parts at [sb*128+64, sb*128+128).
+      uint32_t hi[32], lo[32];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) split_pair(s[c * 8 + 2 * e], s[c * 8 + 2 * e + 1], hi[e], lo[e]);
-        const uint32_t off = (((uint32_t)c ^ ((uint32_t)row & 7u)) << 4);
-        *reinterpret_cast<uint4*>(prow_hi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(prow_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      for (int e = 0; e < 32; ++e) split_pair(s[2 * e], s[2 * e + 1], hi[e], lo[e]);
+      tmem_st32u(tl + sb * kBN + half * 32, hi);
+      tmem_st32u(tl + sb * kBN + 64 + half * 32, lo);
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(B_PFULL));
+      mbar_arrive(bar(B_PFULL + sb));
     }
     // ------------------------------------------------------------ epilogue
     if (ok && T > 0) ok = uniform(wait_bounded(bar(B_PVDONE), (T - 1) & 1, ctl));
@@ -515,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float Lrow = l > 0.f ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
       const int64_t r = ((int64_t)b * a.Hq + hh) * a.Nb + ii;
       // clustered: stage the normalised row in this CTA's shared memory (the
-      // K/V ring is idle now) for the cluster reduction below
+      // K/V rings are idle now) for the cluster reduction below
       float* pa = (a.cluster > 1 ? reinterpret_cast<float*>(smem + kOffK) + row * kRedStride
                                  : a.part_a + split * a.part_stride_a + r * kD) +
                   half * 64;
