@@ -365,20 +365,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && T > 0) {
       bool ok = wait_bounded(bar(B_QFULL), 0, ctl);
+      // Descriptors are built once; a shared-memory offset moves the start
+      // address field (bits 0..13, in 16-byte units), so each MMA only adds a
+      // constant (the whole CTA's shared memory stays below 2^18 bytes).
+      const uint64_t dQ = sw128_desc(sbase + kOffQ, 16, 1024);
+      const uint64_t dK = sw128_desc(sbase + kOffK, 16, 1024);
+      const uint64_t dV = sw128_desc(sbase + kOffV, kHalf, 1024);
       auto issue_pv = [&](int j) -> bool {
         const int sb = j & 1, st = j % kStages;
         if (!wait_bounded(bar(B_PFULL + sb), (j >> 1) & 1, ctl)) return false;
         if (!wait_bounded(bar(B_VFULL + st), (j / kStages) & 1, ctl)) return false;
         tc_fence_after();
-        const uint32_t vb = sbase + kOffV + st * kTile;
+        const uint64_t dVs = dV + (uint64_t)((st * kTile) >> 4);
+        const uint32_t pt = tmem + sb * kBN;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {   // P_hi, then P_lo
 #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk) {
-            const uint64_t bd = sw128_desc(vb + kk * 2048, kHalf, 1024);
-            tc_mma_ts(tmem + kTmemO, tmem + sb * kBN + part * 64 + kk * 8, bd, kIdescPV,
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            tc_mma_ts(tmem + kTmemO, pt + part * 64 + kk * 8, dVs + (uint64_t)((kk * 2048) >> 4), kIdescPV,
                       (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
-          }
         }
         tc_commit(bar(B_VEMPTY + st));
         tc_commit(bar(B_PVDONE));
@@ -389,12 +394,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = wait_bounded(bar(B_KFULL + st), (j / kStages) & 1, ctl);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t kb = sbase + kOffK + st * kTile;
+        const uint64_t dKs = dK + (uint64_t)((st * kTile) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint64_t ad = sw128_desc(sbase + kOffQ + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sw128_desc(kb + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
-          tc_mma(tmem + sb * kBN, ad, bd, kIdescQK, kk > 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4);
+          tc_mma(tmem + sb * kBN, dQ + off, dKs + off, kIdescQK, kk > 0 ? 1u : 0u);
         }
         tc_commit(bar(B_SFULL + sb));
         tc_commit(bar(B_KEMPTY + st));
