@@ -112,6 +112,19 @@ __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const C
   }
 }
 
+// Wait for a phase: an inline non-blocking test first (the common case is a
+// phase that already completed), the bounded polling loop only otherwise.
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, const Ctl& c, bool draining = false) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  if (ok) return true;
+  return wait_bounded(bar, parity, c, draining);
+}
+
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm, uint32_t bar, int c0, int c1,
                                             int c2, int c3) {
   asm volatile(
@@ -348,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int j = 0; j < T && ok; ++j) {
         const int st = j % kStages, round = j / kStages;
-        if (j >= kStages) ok = wait_bounded(bar(empty + st), (round - 1) & 1, ctl);
+        if (j >= kStages) ok = wait_phase(bar(empty + st), (round - 1) & 1, ctl);
         if (!ok) break;
         const int key0 = (int)(kbeg + (int64_t)j * kBN);
         mbar_expect_tx(bar(full + st), kTile);
@@ -357,14 +370,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         armed[st] = round;
       }
       // Let every copy this thread started land before the CTA can exit.
-      if (is_k) wait_bounded(bar(B_QFULL), 0, ctl, true);
+      if (is_k) wait_phase(bar(B_QFULL), 0, ctl, true);
       for (int st = 0; st < kStages; ++st)
-        if (armed[st] >= 0) wait_bounded(bar(full + st), armed[st] & 1, ctl, true);
+        if (armed[st] >= 0) wait_phase(bar(full + st), armed[st] & 1, ctl, true);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && T > 0) {
-      bool ok = wait_bounded(bar(B_QFULL), 0, ctl);
+      bool ok = wait_phase(bar(B_QFULL), 0, ctl);
       // Descriptors are built once; a shared-memory offset moves the start
       // address field (bits 0..13, in 16-byte units), so each MMA only adds a
       // constant (the whole CTA's shared memory stays below 2^18 bytes).
@@ -373,8 +386,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dV = sw128_desc(sbase + kOffV, kHalf, 1024);
       auto issue_pv = [&](int j) -> bool {
         const int sb = j & 1, st = j % kStages;
-        if (!wait_bounded(bar(B_PFULL + sb), (j >> 1) & 1, ctl)) return false;
-        if (!wait_bounded(bar(B_VFULL + st), (j / kStages) & 1, ctl)) return false;
+        if (!wait_phase(bar(B_PFULL + sb), (j >> 1) & 1, ctl)) return false;
+        if (!wait_phase(bar(B_VFULL + st), (j / kStages) & 1, ctl)) return false;
         tc_fence_after();
         const uint64_t dVs = dV + (uint64_t)((st * kTile) >> 4);
         const uint32_t pt = tmem + sb * kBN;
@@ -391,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       for (int j = 0; j < T && ok; ++j) {
         const int sb = j & 1, st = j % kStages;
-        ok = wait_bounded(bar(B_KFULL + st), (j / kStages) & 1, ctl);
+        ok = wait_phase(bar(B_KFULL + st), (j / kStages) & 1, ctl);
         if (!ok) break;
         tc_fence_after();
         const uint64_t dKs = dK + (uint64_t)((st * kTile) >> 4);
@@ -407,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) issue_pv(T - 1);
       // quiesce the tensor core before TMEM is freed
       tc_commit(bar(B_DRAIN));
-      wait_bounded(bar(B_DRAIN), 0, ctl, true);
+      wait_phase(bar(B_DRAIN), 0, ctl, true);
     }
   } else {
     // ------------------------------------------------------------ softmax
@@ -427,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(pair);
-      if (!uniform(wait_bounded(pair, ph & 1, ctl))) return false;
+      if (!uniform(wait_phase(pair, ph & 1, ctl))) return false;
       tc_fence_after();
       theirs = tmem_ld1(tl + kTmemX + 2 * slot + (half ^ 1));
       tmem_wait_ld();
@@ -435,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     for (int j = 0; j < T && ok; ++j) {
       const int sb = j & 1;
-      ok = uniform(wait_bounded(bar(B_SFULL + sb), (j >> 1) & 1, ctl));
+      ok = uniform(wait_phase(bar(B_SFULL + sb), (j >> 1) & 1, ctl));
       if (!ok) break;
       tc_fence_after();
       float s[64];
@@ -470,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool scale_o = move && j > 0 && m != -CUDART_INF_F;
       const float alpha = scale_o ? fast_exp2(m - tmax) : 1.f;
       if (__any_sync(0xffffffffu, scale_o)) {
-        ok = uniform(wait_bounded(bar(B_PVDONE), (j - 1) & 1, ctl));
+        ok = uniform(wait_phase(bar(B_PVDONE), (j - 1) & 1, ctl));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -509,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(B_PFULL + sb));
     }
     // ------------------------------------------------------------ epilogue
-    if (ok && T > 0) ok = uniform(wait_bounded(bar(B_PVDONE), (T - 1) & 1, ctl));
+    if (ok && T > 0) ok = uniform(wait_phase(bar(B_PVDONE), (T - 1) & 1, ctl));
     float lo_other = 0.f;
     if (ok) ok = trade(l, T & 1, T, lo_other);   // the row sum is the two halves' sum
     if (ok) {
