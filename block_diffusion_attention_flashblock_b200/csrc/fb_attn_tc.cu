@@ -7,9 +7,11 @@
 //   warp 0      TMA producers, no multicast: lane 0 loads Q once and then K
 //               tiles of 128 keys into a three-stage ring, lane 1 loads the V
 //               tiles into their own three-stage ring (128-byte swizzle).
-//   warp 1      allocates TMEM; one thread issues tcgen05.mma:
-//               S = Q K^T (A, B in shared memory) into one of two TMEM S
-//               buffers, and O += P_hi V + P_lo V with P read from TMEM.
+//   warp 1      allocates TMEM; one thread issues S = Q K^T (tcgen05.mma, A
+//               and B in shared memory) into one of two TMEM S buffers.
+//   warp 10     one thread issues O += P_hi V + P_lo V with P read from TMEM.
+//               Two issuing threads on different SM sub-partitions keep the
+//               tensor core fed while each waits on its own barriers.
 //   warps 2..9  softmax, two threads per query row (TMEM lane = row): warps
 //               w and w+4 share a TMEM lane quarter and take columns 0..63 and
 //               64..127 of S; they trade their row maxima (and at the end
@@ -17,9 +19,8 @@
 //               mbarrier.  Each writes its half of P = 2^(s - m), as bf16 hi
 //               and lo parts, back into the TMEM columns its S tile came from;
 //               the final O / l and L go to the split's part.
-// P lives in the S buffer it replaces, so S_{j+2} may only overwrite it after
-// PV_j: the MMA thread issues in the order S_j, PV_{j-1}, S_{j+1}, PV_j, ...
-// and the tensor core runs its operations in issue order.
+// P lives in the S buffer it replaces, so S_{j+2} is only issued once PV_j
+// has completed (a completion barrier per buffer).
 // The running max is only moved (and O rescaled in TMEM) when a row's max
 // grows by more than 2^8, so P stays <= 256 and most tiles skip the rescale.
 // With a cluster launch, the key splits of one row tile reduce their parts
@@ -40,7 +41,7 @@ namespace fb {
 namespace {
 
 constexpr int kBM = 128, kBN = 128, kD = 128;
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kStages = 3;                        // K and V ring depth
 constexpr uint32_t kHalf = 16384;                 // [128 rows][64 bf16] 128B-swizzled block
 constexpr uint32_t kTile = 2 * kHalf;             // one 128 x 128 bf16 tile
@@ -57,7 +58,7 @@ constexpr float kRescaleLog2 = 8.0f;
 // barrier slots
 enum {
   B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 10, B_SFULL = 13, B_PFULL = 15,
-  B_PVDONE = 17, B_DRAIN = 18, B_PAIR = 19, B_COUNT = 23
+  B_PVDONE = 17, B_DRAIN = 19, B_PAIR = 21, B_COUNT = 25
 };
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -374,37 +375,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int st = 0; st < kStages; ++st)
         if (armed[st] >= 0) wait_phase(bar(full + st), armed[st] & 1, ctl, true);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && T > 0) {
-      bool ok = wait_phase(bar(B_QFULL), 0, ctl);
-      // Descriptors are built once; a shared-memory offset moves the start
-      // address field (bits 0..13, in 16-byte units), so each MMA only adds a
-      // constant (the whole CTA's shared memory stays below 2^18 bytes).
+  } else if (warp == 1 || warp == 10) {
+    // ------------------------------------------------------------ MMA issuers
+    // Descriptors are built once; a shared-memory offset moves the start
+    // address field (bits 0..13, in 16-byte units), so each MMA only adds a
+    // constant (the whole CTA's shared memory stays below 2^18 bytes).
+    if (lane == 0 && T > 0 && warp == 1) {
+      // S_j = Q K_j^T into buffer j & 1, once K_j has landed and PV_{j-2} has
+      // finished reading the P that buffer held
       const uint64_t dQ = sw128_desc(sbase + kOffQ, 16, 1024);
       const uint64_t dK = sw128_desc(sbase + kOffK, 16, 1024);
-      const uint64_t dV = sw128_desc(sbase + kOffV, kHalf, 1024);
-      auto issue_pv = [&](int j) -> bool {
-        const int sb = j & 1, st = j % kStages;
-        if (!wait_phase(bar(B_PFULL + sb), (j >> 1) & 1, ctl)) return false;
-        if (!wait_phase(bar(B_VFULL + st), (j / kStages) & 1, ctl)) return false;
-        tc_fence_after();
-        const uint64_t dVs = dV + (uint64_t)((st * kTile) >> 4);
-        const uint32_t pt = tmem + sb * kBN;
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {   // P_hi, then P_lo
-#pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
-            tc_mma_ts(tmem + kTmemO, pt + part * 64 + kk * 8, dVs + (uint64_t)((kk * 2048) >> 4), kIdescPV,
-                      (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(bar(B_VEMPTY + st));
-        tc_commit(bar(B_PVDONE));
-        return true;
-      };
+      bool ok = wait_phase(bar(B_QFULL), 0, ctl);
       for (int j = 0; j < T && ok; ++j) {
         const int sb = j & 1, st = j % kStages;
         ok = wait_phase(bar(B_KFULL + st), (j / kStages) & 1, ctl);
+        if (ok && j >= 2) ok = wait_phase(bar(B_PVDONE + sb), ((j >> 1) - 1) & 1, ctl);
         if (!ok) break;
         tc_fence_after();
         const uint64_t dKs = dK + (uint64_t)((st * kTile) >> 4);
@@ -415,14 +400,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_commit(bar(B_SFULL + sb));
         tc_commit(bar(B_KEMPTY + st));
-        if (j >= 1) ok = issue_pv(j - 1);
       }
-      if (ok) issue_pv(T - 1);
-      // quiesce the tensor core before TMEM is freed
+      // quiesce this thread's tensor-core work before TMEM is freed
       tc_commit(bar(B_DRAIN));
       wait_phase(bar(B_DRAIN), 0, ctl, true);
     }
-  } else {
+    if (lane == 0 && T > 0 && warp == 10) {
+      // O += P_j V_j (hi then lo) once softmax has written P_j and V_j landed
+      const uint64_t dV = sw128_desc(sbase + kOffV, kHalf, 1024);
+      bool ok = true;
+      for (int j = 0; j < T && ok; ++j) {
+        const int sb = j & 1, st = j % kStages;
+        ok = wait_phase(bar(B_PFULL + sb), (j >> 1) & 1, ctl);
+        if (ok) ok = wait_phase(bar(B_VFULL + st), (j / kStages) & 1, ctl);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t dVs = dV + (uint64_t)((st * kTile) >> 4);
+        const uint32_t pt = tmem + sb * kBN;
+#pragma unroll
+        for (int part = 0; part < 2; ++part)   // P_hi, then P_lo
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            tc_mma_ts(tmem + kTmemO, pt + part * 64 + kk * 8, dVs + (uint64_t)((kk * 2048) >> 4), kIdescPV,
+                      (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(B_VEMPTY + st));
+        tc_commit(bar(B_PVDONE + sb));
+      }
+      tc_commit(bar(B_DRAIN + 1));
+      wait_phase(bar(B_DRAIN + 1), 0, ctl, true);
+    }
+  } else if (warp >= 2 && warp <= 9) {
     // ------------------------------------------------------------ softmax
     const int q4 = warp & 3;
     const int half = (warp - 2) >> 2;          // 0: columns 0..63, 1: columns 64..127
@@ -483,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool scale_o = move && j > 0 && m != -CUDART_INF_F;
       const float alpha = scale_o ? fast_exp2(m - tmax) : 1.f;
       if (__any_sync(0xffffffffu, scale_o)) {
-        ok = uniform(wait_phase(bar(B_PVDONE), (j - 1) & 1, ctl));
+        ok = uniform(wait_phase(bar(B_PVDONE + ((j - 1) & 1)), ((j - 1) >> 1) & 1, ctl));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -522,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(B_PFULL + sb));
     }
     // ------------------------------------------------------------ epilogue
-    if (ok && T > 0) ok = uniform(wait_phase(bar(B_PVDONE), (T - 1) & 1, ctl));
+    if (ok && T > 0) ok = uniform(wait_phase(bar(B_PVDONE + ((T - 1) & 1)), ((T - 1) >> 1) & 1, ctl));
     float lo_other = 0.f;
     if (ok) ok = trade(l, T & 1, T, lo_other);   // the row sum is the two halves' sum
     if (ok) {
