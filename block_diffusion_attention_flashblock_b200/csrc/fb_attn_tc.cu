@@ -8,19 +8,20 @@
 //               tiles of 128 keys into a three-stage ring, lane 1 loads the V
 //               tiles into their own three-stage ring (128-byte swizzle).
 //   warp 1      allocates TMEM; one thread issues S = Q K^T (tcgen05.mma, A
-//               and B in shared memory) into one of two TMEM S buffers.
+//               and B in shared memory) into one of three TMEM S buffers.
 //   warp 10     one thread issues O += P_hi V + P_lo V with P read from TMEM.
 //               Two issuing threads on different SM sub-partitions keep the
 //               tensor core fed while each waits on its own barriers.
 //   warps 2..9  softmax, two threads per query row (TMEM lane = row): warps
 //               w and w+4 share a TMEM lane quarter and take columns 0..63 and
 //               64..127 of S; they trade their row maxima (and at the end
-//               their row sums) through spare TMEM columns and a bounded
+//               their row sums) through shared memory and a bounded
 //               mbarrier.  Each writes its half of P = 2^(s - m), as bf16 hi
 //               and lo parts, back into the TMEM columns its S tile came from;
 //               the final O / l and L go to the split's part.
-// P lives in the S buffer it replaces, so S_{j+2} is only issued once PV_j
-// has completed (a completion barrier per buffer).
+// P lives in the S buffer it replaces, so S_{j+3} is only issued once PV_j
+// has completed (a completion barrier per buffer); three buffers leave two
+// softmax tiles for the chain P_j -> PV_j -> S_{j+3}.
 // The running max is only moved (and O rescaled in TMEM) when a row's max
 // grows by more than 2^8, so P stays <= 256 and most tiles skip the rescale.
 // With a cluster launch, the key splits of one row tile reduce their parts
@@ -48,17 +49,19 @@ constexpr uint32_t kTile = 2 * kHalf;             // one 128 x 128 bf16 tile
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kTile;
 constexpr uint32_t kOffV = kOffK + kStages * kTile;
-constexpr uint32_t kOffBar = kOffV + kStages * kTile;   // barriers and flags
-constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + slack for 1024-byte alignment
-constexpr uint32_t kTmemCols = 512;               // S/P buffers [0,128) [128,256), O [256,384)
-constexpr uint32_t kTmemO = 256;
-constexpr uint32_t kTmemX = 384;                  // row-statistics exchange columns
+constexpr uint32_t kOffBar = kOffV + kStages * kTile;   // barriers and flags (256 bytes)
+constexpr uint32_t kOffX = kOffBar + 256;               // row-statistics exchange, 2 x 2 x 128 fp32
+constexpr uint32_t kSmemSlack = 768;                    // the aligned base may sit up to this far in
+constexpr uint32_t kSmemBytes = kOffX + 2048 + kSmemSlack;
+constexpr int kSBuf = 3;                          // S/P buffers in TMEM
+constexpr uint32_t kTmemCols = 512;               // S/P buffers [0,128) [128,256) [256,384), O [384,512)
+constexpr uint32_t kTmemO = 384;
 constexpr float kRescaleLog2 = 8.0f;
 
 // barrier slots
 enum {
-  B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 10, B_SFULL = 13, B_PFULL = 15,
-  B_PVDONE = 17, B_DRAIN = 19, B_PAIR = 21, B_COUNT = 25
+  B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 10, B_SFULL = 13, B_PFULL = 16,
+  B_PVDONE = 19, B_DRAIN = 22, B_PAIR = 24, B_COUNT = 28
 };
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -298,6 +301,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if (smem - smem_raw > (ptrdiff_t)kSmemSlack) {   // the layout would not fit: report, touch nothing
+    if (threadIdx.x == 0) atomicCAS(a.status, 0, (int)FB_EUNSUPPORTED);
+    return;
+  }
   const uint32_t sbase = smem_addr(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffBar + B_COUNT * 8);
@@ -327,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < B_COUNT; ++i) {
       uint32_t cnt = 1;
-      if (i == B_PFULL || i == B_PFULL + 1) cnt = 256;
+      if (i >= B_PFULL && i < B_PFULL + kSBuf) cnt = 256;
       if (i >= B_PAIR) cnt = 64;
       mbar_init(bar(i), cnt);
     }
@@ -381,15 +388,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // address field (bits 0..13, in 16-byte units), so each MMA only adds a
     // constant (the whole CTA's shared memory stays below 2^18 bytes).
     if (lane == 0 && T > 0 && warp == 1) {
-      // S_j = Q K_j^T into buffer j & 1, once K_j has landed and PV_{j-2} has
+      // S_j = Q K_j^T into buffer j % 3, once K_j has landed and PV_{j-3} has
       // finished reading the P that buffer held
       const uint64_t dQ = sw128_desc(sbase + kOffQ, 16, 1024);
       const uint64_t dK = sw128_desc(sbase + kOffK, 16, 1024);
       bool ok = wait_phase(bar(B_QFULL), 0, ctl);
       for (int j = 0; j < T && ok; ++j) {
-        const int sb = j & 1, st = j % kStages;
+        const int sb = j % kSBuf, st = j % kStages;
         ok = wait_phase(bar(B_KFULL + st), (j / kStages) & 1, ctl);
-        if (ok && j >= 2) ok = wait_phase(bar(B_PVDONE + sb), ((j >> 1) - 1) & 1, ctl);
+        if (ok && j >= kSBuf) ok = wait_phase(bar(B_PVDONE + sb), (j / kSBuf - 1) & 1, ctl);
         if (!ok) break;
         tc_fence_after();
         const uint64_t dKs = dK + (uint64_t)((st * kTile) >> 4);
@@ -410,8 +417,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dV = sw128_desc(sbase + kOffV, kHalf, 1024);
       bool ok = true;
       for (int j = 0; j < T && ok; ++j) {
-        const int sb = j & 1, st = j % kStages;
-        ok = wait_phase(bar(B_PFULL + sb), (j >> 1) & 1, ctl);
+        const int sb = j % kSBuf, st = j % kStages;
+        ok = wait_phase(bar(B_PFULL + sb), (j / kSBuf) & 1, ctl);
         if (ok) ok = wait_phase(bar(B_VFULL + st), (j / kStages) & 1, ctl);
         if (!ok) break;
         tc_fence_after();
@@ -436,26 +443,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = q4 * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
     const uint32_t pair = bar(B_PAIR + q4);
+    float* xch = reinterpret_cast<float*>(smem + kOffX);   // [slot][half][row]
     float m = -CUDART_INF_F, l = 0.f;
     bool ok = true;
     // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform.
     auto uniform = [](bool v) { return __all_sync(0xffffffffu, v); };
-    // Trade one value per row with the partner warp through TMEM column
-    // kTmemX + 2*slot + half (phase `ph` of this lane quarter's pair barrier).
+    // Trade one value per row with the partner warp through shared memory
+    // slot `slot` (phase `ph` of this lane quarter's pair barrier; the barrier
+    // arrive/wait orders the store before the partner's load).
     auto trade = [&](float mine, int slot, int ph, float& theirs) -> bool {
-      tmem_st1(tl + kTmemX + 2 * slot + half, mine);
-      tmem_wait_st();
-      tc_fence_before();
+      xch[(slot * 2 + half) * kBM + row] = mine;
       mbar_arrive(pair);
       if (!uniform(wait_phase(pair, ph & 1, ctl))) return false;
-      tc_fence_after();
-      theirs = tmem_ld1(tl + kTmemX + 2 * slot + (half ^ 1));
-      tmem_wait_ld();
+      theirs = xch[(slot * 2 + (half ^ 1)) * kBM + row];
       return true;
     };
     for (int j = 0; j < T && ok; ++j) {
-      const int sb = j & 1;
-      ok = uniform(wait_phase(bar(B_SFULL + sb), (j >> 1) & 1, ctl));
+      const int sb = j % kSBuf;
+      ok = uniform(wait_phase(bar(B_SFULL + sb), (j / kSBuf) & 1, ctl));
       if (!ok) break;
       tc_fence_after();
       float s[64];
@@ -490,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool scale_o = move && j > 0 && m != -CUDART_INF_F;
       const float alpha = scale_o ? fast_exp2(m - tmax) : 1.f;
       if (__any_sync(0xffffffffu, scale_o)) {
-        ok = uniform(wait_phase(bar(B_PVDONE + ((j - 1) & 1)), ((j - 1) >> 1) & 1, ctl));
+        ok = uniform(wait_phase(bar(B_PVDONE + (j - 1) % kSBuf), ((j - 1) / kSBuf) & 1, ctl));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -529,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(B_PFULL + sb));
     }
     // ------------------------------------------------------------ epilogue
-    if (ok && T > 0) ok = uniform(wait_phase(bar(B_PVDONE + ((T - 1) & 1)), ((T - 1) >> 1) & 1, ctl));
+    if (ok && T > 0) ok = uniform(wait_phase(bar(B_PVDONE + (T - 1) % kSBuf), ((T - 1) / kSBuf) & 1, ctl));
     float lo_other = 0.f;
     if (ok) ok = trade(l, T & 1, T, lo_other);   // the row sum is the two halves' sum
     if (ok) {
