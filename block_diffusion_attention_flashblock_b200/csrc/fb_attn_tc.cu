@@ -4,9 +4,10 @@
 //
 // One CTA = one tile of 128 query rows (the block queries of the query heads
 // that share a KV head, packed) x one split of the prefix keys.  Warp roles:
-//   warp 0      TMA producers, no multicast: lane 0 loads Q once and then K
-//               tiles of 128 keys into a three-stage ring, lane 1 loads the V
-//               tiles into their own three-stage ring (128-byte swizzle).
+//   warp 0      TMA producer, no multicast: Q once, then K tiles of 128 keys
+//               into a three-stage ring (128-byte swizzle).
+//   warp 11     TMA producer of the V tiles, its own three-stage ring (a warp
+//               of its own, so a wait on one ring never stalls the other).
 //   warp 1      allocates TMEM; one thread issues S = Q K^T (tcgen05.mma, A
 //               and B in shared memory) into one of three TMEM S buffers.
 //   warp 10     one thread issues O += P_hi V + P_lo V with P read from TMEM.
@@ -42,7 +43,7 @@ namespace fb {
 namespace {
 
 constexpr int kBM = 128, kBN = 128, kD = 128;
-constexpr int kThreads = 352;
+constexpr int kThreads = 384;
 constexpr int kStages = 3;                        // K and V ring depth
 constexpr uint32_t kHalf = 16384;                 // [128 rows][64 bf16] 128B-swizzled block
 constexpr uint32_t kTile = 2 * kHalf;             // one 128 x 128 bf16 tile
@@ -352,11 +353,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const Ctl ctl{abort_flag, a.status, a.wait_limit_ns};
 
-  if (warp == 0) {
+  if (warp == 0 || warp == 11) {
     // ------------------------------------------------------------ producers
-    if (lane < 2 && T > 0) {
-      // lane 0: Q, then the K ring; lane 1: the V ring
-      const bool is_k = lane == 0;
+    if (lane == 0 && T > 0) {
+      // warp 0: Q, then the K ring; warp 11: the V ring
+      const bool is_k = warp == 0;
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(is_k ? &tmK : &tmV)) : "memory");
+      if (is_k) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQ)) : "memory");
       const CUtensorMap* tm = is_k ? &tmK : &tmV;
       const int full = is_k ? B_KFULL : B_VFULL, empty = is_k ? B_KEMPTY : B_VEMPTY;
       const uint32_t ring = sbase + (is_k ? kOffK : kOffV);
