@@ -236,8 +236,7 @@ static PrefixPlan plan_prefix(const fb_attn_desc& d, const void* q, const void* 
   const int64_t min_keys = g_prefix_kernel >= 2 ? 1 : 256;
   if (g_prefix_kernel != 1 && nkeys >= min_keys && tc_make_maps(d, q, kp, vp, nkeys, &p.maps)) {
     tc_plan_split((int64_t)p.maps.units * p.maps.tiles_per_unit, nkeys, cap, g_prefix_kernel != 3, &p.nsplit,
-                  &p.kps, &p.cluster);
-    p.nparts = p.cluster > 1 ? 1 : p.nsplit;
+                  &p.kps, &p.cluster, &p.nparts);
     p.tc = true;
   }
   return p;
@@ -286,7 +285,8 @@ static fb_status merge_to_part(const fb_attn_desc& d, const PartList& pl, float*
 }
 
 static fb_status run_inblock(const fb_attn_desc& d, const void* q, const void* kin, const void* vin,
-                             const PartList& ext, void* o, float* lse, cudaStream_t s) {
+                             const PartList& ext, void* o, float* lse, cudaStream_t s, float* cache_a = nullptr,
+                             float* cache_l = nullptr) {
   PassPlan p = plan_pass(d, q, kin, vin, d.kin_strides, d.Nb, nullptr, 0, 1);
   AttnArgs& a = p.a;
   a.nsplit = 1;
@@ -311,9 +311,11 @@ static fb_status run_inblock(const fb_attn_desc& d, const void* q, const void* k
                        (double)rows_of(d) * (d.D * esize(d.out_dtype) + (lse ? 4 : 0));
   ProfScope prof(kProfInblock, bytes, s);
   if (inblock_small_applies(d, a.next))
-    return launch_inblock_small(d, q, kin, vin, a.next, a.ext_a, a.ext_l, o, lse, a.scale_log2, s) == cudaSuccess
+    return launch_inblock_small(d, q, kin, vin, a.next, a.ext_a, a.ext_l, o, lse, cache_a, cache_l, a.scale_log2,
+                                s) == cudaSuccess
                ? FB_OK
                : FB_ECUDA;
+  if (cache_a) return FB_EUNSUPPORTED;   // callers only ask for the cache write where the small kernel runs
   return launch_attn_generic(a, d.D, d.in_dtype == FB_BF16, s) == cudaSuccess ? FB_OK : FB_ECUDA;
 }
 
@@ -714,6 +716,19 @@ fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
         p.gen.a.excl_words = (a->prefix_len + 31) / 32;
       } else {
         p = plan_prefix(d, a->q, a->kp, a->vp, a->prefix_len, c->part_cap);
+      }
+      // the in-block kernel can take the split parts itself and write their
+      // merge into the cache, saving a merge pass
+      if (!sparse && p.nparts > 1 && inblock_small_applies(d, p.nparts)) {
+        if ((st = launch_prefix(d, p, a->prefix_len, nullptr, 0, c->part_a, c->part_l, s)) != FB_OK) return st;
+        ext.g[ext.ngroups++] = group_of(c->part_a, c->part_l, p.nparts, d);
+        if (a->reuse_out && launch_fill_decision(a->reuse_out, BH, 0, s) != cudaSuccess) return FB_ECUDA;
+        if (a->sim_out && cudaMemsetAsync(a->sim_out, 0xFF, (size_t)BH * 4, s) != cudaSuccess) return FB_ECUDA;
+        if ((st = run_inblock(d, a->q, a->kin, a->vin, ext, a->o, a->lse, s, c->cache_a, c->cache_l)) != FB_OK)
+          return st;
+        c->valid = true;
+        c->last_recomputed = 1;
+        return FB_OK;
       }
       if (p.nparts == 1) {
         if ((st = launch_prefix(d, p, a->prefix_len, nullptr, 0, c->cache_a, c->cache_l, s)) != FB_OK) return st;

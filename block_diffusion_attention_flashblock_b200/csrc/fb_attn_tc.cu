@@ -25,8 +25,10 @@
 // softmax tiles for the chain P_j -> PV_j -> S_{j+3}.
 // The running max is only moved (and O rescaled in TMEM) when a row's max
 // grows by more than 2^8, so P stays <= 256 and most tiles skip the rescale.
-// With a cluster launch, the key splits of one row tile reduce their parts
-// through distributed shared memory before anything reaches global memory.
+// With a cluster launch, each cluster of key splits of one row tile reduces
+// its parts through distributed shared memory before anything reaches global
+// memory (one part per cluster).  The last split also takes the ragged
+// remainder of the keys.
 // Every mbarrier wait is bounded; on expiry the CTA records FB_ETIMEOUT in
 // the device status word, drains its own TMA and MMA work, frees TMEM and
 // exits.
@@ -294,7 +296,7 @@ struct TcArgs {
   int* status;
   uint64_t wait_limit_ns;
   uint32_t q_bytes;        // bytes of one Q half-box (64 columns)
-  int32_t cluster;         // > 1: the gridDim.y splits form one cluster and reduce in-kernel
+  int32_t cluster;         // > 1: clusters of this many consecutive splits reduce in-kernel
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -329,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (all) return;
   }
   const int64_t kbeg = (int64_t)split * a.keys_per_split;
-  const int64_t kend = min(kbeg + a.keys_per_split, a.nkeys);
+  const int64_t kend = split == (int)gridDim.y - 1 ? a.nkeys : min(kbeg + a.keys_per_split, a.nkeys);
   const int T = kend > kbeg ? (int)((kend - kbeg + kBN - 1) / kBN) : 0;
 
   if (threadIdx.x == 0) {
@@ -634,9 +636,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int64_t r = ((int64_t)b * a.Hq + hh) * a.Nb + ii;
       const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-      *reinterpret_cast<float4*>(a.part_a + r * kD + lane4 * 4) =
+      const int part = split / CS;
+      *reinterpret_cast<float4*>(a.part_a + part * a.part_stride_a + r * kD + lane4 * 4) =
           make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-      if (lane4 == 0) a.part_l[r] = m == -CUDART_INF_F ? -CUDART_INF_F : m + __logf(wsum);
+      if (lane4 == 0) a.part_l[part * a.part_stride_l + r] = m == -CUDART_INF_F ? -CUDART_INF_F : m + __logf(wsum);
     }
     cluster_sync_all();   // keep every rank's shared memory alive until all reads are done
   }
@@ -745,38 +748,36 @@ static int max_active_clusters(int cs) {
   return n;
 }
 
-// Split plan for `tiles` row tiles over nkeys keys.  Candidates: one split; up
-// to 16 splits reduced inside one cluster per tile; or more splits whose
-// partials a merge pass combines (at most max_split of them).  Cost = waves x
-// (key tiles per CTA + fixed CTA cost) + the merge pass when there is one.
-void tc_plan_split(int64_t tiles, int64_t nkeys, int32_t max_split, bool allow_cluster, int32_t* nsplit,
-                   int64_t* kps, int32_t* cluster) {
+// Split plan for `tiles` row tiles over nkeys keys: nsplit splits of kps keys
+// (the last one takes the rest), grouped into clusters of `cluster` splits
+// that reduce in-kernel (1: no cluster), leaving nparts parts per row for a
+// later merge.  Candidates are scored as waves of concurrently resident CTAs
+// (or clusters) x (the longest split in key tiles + a fixed cost of about two
+// tiles), plus a small cost per extra part; nparts is at most max_parts.
+void tc_plan_split(int64_t tiles, int64_t nkeys, int32_t max_parts, bool allow_cluster, int32_t* nsplit,
+                   int64_t* kps, int32_t* cluster, int32_t* nparts) {
   const int64_t sms = num_sms();
   const int64_t ktiles = std::max<int64_t>(1, (nkeys + kBN - 1) / kBN);
-  int64_t best_per = ktiles, best_cl = 1;
   double best = 1e300;
-  for (int64_t ns = 1; ns <= ktiles; ++ns) {
-    const int64_t per = (ktiles + ns - 1) / ns;
-    const int64_t real_ns = (ktiles + per - 1) / per;
-    if (real_ns != ns) continue;
-    double cost;
-    int64_t cl = 1;
-    if (ns == 1) {
-      cost = (double)((tiles + sms - 1) / sms) * (per + 2);
-    } else if (allow_cluster && ns <= 16 && max_active_clusters((int)ns) > 0) {
-      const int64_t conc = max_active_clusters((int)ns);
-      cost = (double)((tiles + conc - 1) / conc) * (per + 2) + 0.5;
-      cl = ns;
-    } else if (ns <= max_split) {
-      cost = (double)((tiles * ns + sms - 1) / sms) * (per + 2) + 6.0;
-    } else {
-      continue;
+  int64_t b_ns = 1, b_cs = 1, b_per = ktiles;
+  for (int cs = 1; cs <= (allow_cluster ? 16 : 1); ++cs) {
+    const int64_t conc = cs == 1 ? sms : (int64_t)max_active_clusters(cs);
+    if (conc <= 0) continue;
+    for (int64_t nc = 1; nc * cs <= ktiles; ++nc) {
+      const int64_t ns = nc * cs;
+      const int64_t parts = cs == 1 ? ns : nc;
+      if (parts > std::max(1, max_parts)) break;
+      const int64_t per = ktiles / ns, last = ktiles - (ns - 1) * per;
+      const int64_t units = cs == 1 ? tiles * ns : tiles * nc;
+      const int64_t waves = (units + conc - 1) / conc;
+      const double cost = (double)waves * (last + 2) + (parts > 1 ? 1.5 + 0.1 * parts : 0.0) + 0.01 * ns;
+      if (cost < best) { best = cost; b_ns = ns; b_cs = cs; b_per = per; }
     }
-    if (cost < best) { best = cost; best_per = per; best_cl = cl; }
   }
-  *kps = best_per * kBN;
-  *nsplit = (int32_t)std::max<int64_t>(1, (nkeys + *kps - 1) / *kps);
-  *cluster = (int32_t)best_cl;
+  *nsplit = (int32_t)b_ns;
+  *kps = b_per * kBN;
+  *cluster = (int32_t)b_cs;
+  *nparts = (int32_t)(b_cs == 1 ? b_ns : b_ns / b_cs);
 }
 
 cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys, int32_t nsplit, int64_t kps,
@@ -793,7 +794,7 @@ cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys
   a.q_bytes = 64u * 2u * (uint32_t)(m.mode == 0 ? d.Nb * m.hg : kBM);
   a.status = device_status_ptr();
   a.wait_limit_ns = wait_limit_ns();
-  a.cluster = cluster > 1 ? nsplit : 1;
+  a.cluster = cluster > 1 ? cluster : 1;
   if (!a.status) return cudaErrorInvalidValue;
   static bool attr = false;
   if (!attr) {
@@ -814,7 +815,7 @@ cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = 1;
-  at[0].val.clusterDim.y = (unsigned)nsplit;
+  at[0].val.clusterDim.y = (unsigned)cluster;
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;

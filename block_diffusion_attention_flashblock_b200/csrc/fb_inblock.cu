@@ -6,13 +6,16 @@
 //     queries); 4 warps: two 16-row slabs, and for each slab two warps that
 //     both form S and P but split the P V product and the epilogue by halves
 //     of the head dimension (shorter per-warp instruction chains);
-//   - every global load (Q, K_in, V_in and the cached external parts A, L) is
-//     issued at once with cp.async, so the kernel waits on memory once;
+//   - every global load (Q, K_in, V_in and the external parts A, L) is issued
+//     up front with cp.async in three groups (Q and K_in; V_in; the parts), so
+//     S and the softmax start while V_in and the parts are still arriving;
 //   - S = Q K_in^T and O = P V on mma.sync m16n8k16 (bf16 in, fp32 out) with
 //     the block's keys padded to NB in {16, 32, 64}; P V uses a bf16 hi + lo
 //     split of P so the product keeps fp32-level accuracy;
-//   - the merge with up to two external parts reads them from shared memory
-//     and writes O (bf16 or fp32) and the merged natural-log LSE.
+//   - the merge with up to four external parts reads them from shared memory
+//     and writes O (bf16 or fp32) and the merged natural-log LSE; on a full
+//     step it can also write the merged external part (the block-external
+//     attention combined over its key splits) into the cache.
 #include <math_constants.h>
 
 #include "fb_internal.cuh"
@@ -24,7 +27,7 @@ namespace {
 constexpr int kRows = 32;          // query rows per CTA
 constexpr int kD = 128;
 constexpr int kExtStride = 132;    // fp32 row stride of staged external parts (bank spread)
-constexpr int kMaxExt = 2;
+constexpr int kMaxExt = 4;
 
 __device__ __forceinline__ uint32_t saddr(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 __device__ __forceinline__ void cp16(uint32_t dst, const void* src, int bytes) {
@@ -80,6 +83,8 @@ struct InblockArgs {
   int64_t o_sb, o_sh, o_st;
   int32_t o_bf16;
   float* lse;
+  float* cache_a;     // non-null: also store merge(external parts) here (packed fp32)
+  float* cache_l;
   float scale_log2;
 };
 
@@ -117,8 +122,15 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
     const bool ok = r < a.Nb;
     const int64_t off = b * a.k_sb + (int64_t)kvh * a.k_sh + (int64_t)(ok ? r : 0) * a.k_st + ch * 8;
     cp16(saddr(sK + swz(r, ch)), a.k + off, ok ? 16 : 0);
+  }
+  asm volatile("cp.async.commit_group;\n" ::: "memory");   // group: Q, K_in
+  for (int c = tid; c < NB * 16; c += 128) {
+    const int r = c >> 4, ch = c & 15;
+    const bool ok = r < a.Nb;
+    const int64_t off = b * a.k_sb + (int64_t)kvh * a.k_sh + (int64_t)(ok ? r : 0) * a.k_st + ch * 8;
     cp16(saddr(sV + swz(r, ch)), a.v + off, ok ? 16 : 0);
   }
+  asm volatile("cp.async.commit_group;\n" ::: "memory");   // group: V_in
   for (int p = 0; p < a.next; ++p) {
     for (int c = tid; c < kRows * 32; c += 128) {
       const int r = c >> 5, ch = c & 31;
@@ -131,7 +143,7 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
       cp4(saddr(sL + p * kRows + r), ok ? a.ext_l[p] + prow0 + r : a.ext_l[p], ok ? 4 : 0);
     }
   }
-  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 2;\n" ::: "memory");   // group: parts
   __syncthreads();
 
   // ---- S = Q K^T for this warp's 16-row slab ----
@@ -186,6 +198,8 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
     lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 1);
     lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 2);
   }
+  asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+  __syncthreads();
   // ---- O[:, dh*64 : dh*64+64] = P V ----
   constexpr int DT = kD / 16;    // 8-column tiles in this warp's half
   float o[DT][4];
@@ -206,6 +220,8 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
       mma16816(o[d + 1], al, b2, b3);
     }
   }
+  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+  __syncthreads();
   // ---- merge with the external parts and store ----
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
@@ -222,34 +238,39 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
     }
     const bool empty = m == -CUDART_INF_F;
     const float w_in = (empty || Lin == -CUDART_INF_F) ? 0.f : __expf(Lin - m);
-    float wx[kMaxExt], wsum = w_in;
+    float wx[kMaxExt], wext = 0.f;
 #pragma unroll
     for (int p = 0; p < kMaxExt; ++p) {
       wx[p] = (empty || Lx[p] == -CUDART_INF_F) ? 0.f : __expf(Lx[p] - m);
-      wsum += wx[p];
+      wext += wx[p];
     }
+    const float wsum = w_in + wext;
     const float inv = empty ? 0.f : 1.f / wsum;
+    const float inv_ext = wext > 0.f ? 1.f / wext : 0.f;
     const float win = lrow[h] > 0.f ? w_in / lrow[h] : 0.f;
     const int g = rr / a.Nb, i = rr % a.Nb;
     const int64_t obase = b * a.o_sb + (int64_t)(kvh * a.G + g) * a.o_sh + (int64_t)i * a.o_st;
 #pragma unroll
     for (int d = 0; d < DT; ++d) {
       const int col = dh * 64 + d * 8 + 2 * (lane & 3);
-      float x = win * o[d][2 * h], y = win * o[d][2 * h + 1];
+      float ex = 0.f, ey = 0.f;   // sum of w_p A_p over the external parts
 #pragma unroll
       for (int p = 0; p < kMaxExt; ++p) {
         if (wx[p] == 0.f) continue;
         const float2 e = *reinterpret_cast<const float2*>(sE + (p * kRows + r) * kExtStride + col);
-        x = fmaf(wx[p], e.x, x);
-        y = fmaf(wx[p], e.y, y);
+        ex = fmaf(wx[p], e.x, ex);
+        ey = fmaf(wx[p], e.y, ey);
       }
-      x *= inv;
-      y *= inv;
+      if (a.cache_a)
+        *reinterpret_cast<float2*>(a.cache_a + (prow0 + r) * kD + col) = make_float2(ex * inv_ext, ey * inv_ext);
+      const float x = (win * o[d][2 * h] + ex) * inv, y = (win * o[d][2 * h + 1] + ey) * inv;
       if (a.o_bf16)
         *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(a.o) + obase + col) = __floats2bfloat162_rn(x, y);
       else
         *reinterpret_cast<float2*>(static_cast<float*>(a.o) + obase + col) = make_float2(x, y);
     }
+    if (a.cache_l && dh == 0 && (lane & 3) == 0)
+      a.cache_l[prow0 + r] = wext > 0.f ? m + logf(wext) : -CUDART_INF_F;
     if (a.lse && dh == 0 && (lane & 3) == 0) a.lse[prow0 + r] = empty ? -CUDART_INF_F : m + logf(wsum);
   }
 }
@@ -261,7 +282,7 @@ bool inblock_small_applies(const fb_attn_desc& d, int next) {
 
 cudaError_t launch_inblock_small(const fb_attn_desc& d, const void* q, const void* kin, const void* vin, int next,
                                  const float* const* ext_a, const float* const* ext_l, void* o, float* lse,
-                                 float scale_log2, cudaStream_t s) {
+                                 float* cache_a, float* cache_l, float scale_log2, cudaStream_t s) {
   InblockArgs a;
   memset(&a, 0, sizeof(a));
   a.B = d.B; a.Hq = d.Hq; a.Hkv = d.Hkv; a.G = d.Hq / d.Hkv; a.Nb = d.Nb;
@@ -276,6 +297,8 @@ cudaError_t launch_inblock_small(const fb_attn_desc& d, const void* q, const voi
   a.o = o; a.o_sb = d.o_strides[0]; a.o_sh = d.o_strides[1]; a.o_st = d.o_strides[2];
   a.o_bf16 = d.out_dtype == FB_BF16;
   a.lse = lse;
+  a.cache_a = cache_a;
+  a.cache_l = cache_l;
   a.scale_log2 = scale_log2;
   const int NB = d.Nb <= 16 ? 16 : d.Nb <= 32 ? 32 : 64;
   const size_t smem = (size_t)(kRows + 2 * NB) * kD * 2 + (size_t)kMaxExt * kRows * (kExtStride + 1) * 4;

@@ -106,8 +106,8 @@ struct TcMaps {
 };
 bool tc_tiling(const fb_attn_desc& d, int* mode, int* hg, int* tiles_per_unit, int* units);
 bool tc_make_maps(const fb_attn_desc& d, const void* q, const void* kp, const void* vp, int64_t nkeys, TcMaps* m);
-void tc_plan_split(int64_t tiles, int64_t nkeys, int32_t max_split, bool allow_cluster, int32_t* nsplit,
-                   int64_t* kps, int32_t* cluster);
+void tc_plan_split(int64_t tiles, int64_t nkeys, int32_t max_parts, bool allow_cluster, int32_t* nsplit,
+                   int64_t* kps, int32_t* cluster, int32_t* nparts);
 int32_t tc_split_cap(int64_t tiles, int64_t max_keys);
 cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys, int32_t nsplit, int64_t kps,
                            int32_t cluster, const int8_t* mask, int mask_active, float scale_log2, float* pa,
@@ -117,7 +117,7 @@ cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys
 bool inblock_small_applies(const fb_attn_desc& d, int next);
 cudaError_t launch_inblock_small(const fb_attn_desc& d, const void* q, const void* kin, const void* vin, int next,
                                  const float* const* ext_a, const float* const* ext_l, void* o, float* lse,
-                                 float scale_log2, cudaStream_t s);
+                                 float* cache_a, float* cache_l, float scale_log2, cudaStream_t s);
 
 struct MergeArgs {
   int32_t B, Hq, Nb, D;

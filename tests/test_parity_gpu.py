@@ -145,7 +145,7 @@ def _random_parts(B, Hq, Nb, D, n, seed, empty_rows=True):
     return parts
 
 
-@pytest.mark.parametrize("nparts", [0, 1, 2])
+@pytest.mark.parametrize("nparts", [0, 1, 2, 4, 7])
 @pytest.mark.parametrize("shape", [(1, 32, 8, 128, 32, "bf16"), (1, 4, 4, 64, 32, "f32"),
                                    (1, 3, 3, 128, 150, "bf16"), (2, 8, 4, 64, 5, "bf16"),
                                    (2, 8, 2, 128, 5, "bf16"), (1, 8, 2, 128, 64, "bf16"),
