@@ -4,24 +4,28 @@
                     [--workload dllm_8k] [--no-e2e]
 
 A timed "step" is one pass of the whole hot path over one workload: the
-diffusion-LM schedule of one attention layer (dllm_8k: B 1, 32 query / 8 KV
-heads, head dim 128, prefix 8192 tokens growing by 32 per block, blocks of 32
-tokens, 8 diffusion steps per block, 4 blocks, tau = 8).  Every diffusion step
-runs fb_step under the reuse policy, and every block ends with fb_kv_append.
-The metric is query tokens per second (B * Nb per diffusion step) with reuse
-on; the same schedule with tau = 0 (every step recomputes over the whole KV
-cache) is reported beside it.  L2 is flushed (a 1 GiB write) before every
-diffusion step, outside the event-timed interval, so each step reads the KV
-cache from HBM as it would between the layers of a model; the flush also keeps
-the GPU busy long enough for the host to enqueue the next step, so the timed
-interval holds no host launch gaps.
+diffusion-LM schedule (dllm_8k: B 1, 32 query / 8 KV heads, head dim 128,
+prefix 8192 tokens growing by 32 per block, blocks of 32 tokens, 8 diffusion
+steps per block, 4 blocks, tau = 8) for each of NL attention layers, every
+layer with its own KV cache, cache state and inputs.  Every diffusion step
+runs fb_step for each layer in turn under the reuse policy, and every block
+ends with fb_kv_append.  NL is chosen so that the layers' KV caches together
+exceed twice the L2: as between the layers of a model, each layer's data has
+left L2 by the time its next step runs.  L2 is also flushed (a 1 GiB write)
+before every timed step, outside the timed interval.
 
-Each diffusion step is captured once as a CUDA graph (fb_step plus, at a
-block's end, fb_kv_append; the reuse decisions are taken on the host while
-capturing, in schedule order) and the timed region replays them; the same
-steps as eager library calls are reported under "eager", and the per-kernel
-breakdown behind "roofline" comes from a separate eager pass with CUDA events
-around every launch.
+The metric is query tokens per second: B * Nb per layer-step (one fb_step of
+one layer, all heads), over all layer-steps of the timed step.  The same
+schedule with tau = 0 (every step recomputes over the whole KV cache) is
+reported beside it, and the per-step latencies follow from the two.
+
+The whole step is captured once as a CUDA graph (the reuse decisions are taken
+on the host while capturing, in schedule order) and replayed between two CUDA
+events; the same calls made eagerly are reported under "eager", and "e2e"
+repeats the eager pass with every layer-step's inputs copied from pinned host
+memory and its outputs read back.  The roofline comes from graphs of one
+library call repeated over the layers (so no per-launch event overhead enters
+the duration), with launch counts and algorithmic bytes from a profiled pass.
 
 `--impl reference` times the fp64 CPU oracle on this host's cores on a
 bounded sample of the same schedule (the reference arm; there is no other
@@ -117,213 +121,246 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------- ours ---
-class Schedule:
-    """All inputs of one workload pass, resident on the device, plus host copies for e2e."""
+L2_BYTES = 126 << 20
 
-    def __init__(self, spec, device):
-        self.spec = spec
+
+def n_layers(spec) -> int:
+    """Independent layer states stepped in turn: enough that the layers' KV
+    caches together exceed twice the L2 (so each layer's data has left L2 by
+    the time its next step runs), at least 2, at most 8."""
+    kv = 2 * spec.B * spec.Hkv * spec.lcap * spec.D * (4 if spec.dtype == "f32" else 2)
+    return int(min(8, max(2, -(-2 * L2_BYTES // kv))))
+
+
+class Layers:
+    """NL attention layers of one workload, each with its own KV cache, cache
+    state, per-step inputs and outputs, all resident on the device (plus
+    pinned host copies of layer 0's inputs for the end-to-end leg)."""
+
+    def __init__(self, spec, device, nl):
+        from block_diffusion_attention_flashblock_b200 import fb
+        self.spec, self.nl = spec, nl
         w = wl.Workload(spec)
         kp, vp = w.prefix_kv()
-        self.kp, self.vp = kp.to(device), vp.to(device)
-        self.steps = []
-        for st in w.schedule():
-            self.steps.append(dict(st=st, q=st.q.to(device), kin=st.kin.to(device), vin=st.vin.to(device),
-                                   sel=None if st.sel is None else st.sel.to(device),
-                                   hq=st.q.pin_memory(), hk=st.kin.pin_memory(), hv=st.vin.pin_memory()))
-        self.query_tokens = spec.B * spec.Nb * len(self.steps)
+        self.steps = list(w.schedule())
+        dt = spec.torch_dtype
+        self.L = []
+        for _ in range(nl):
+            d = dict(kp=kp.to(device), vp=vp.to(device),
+                     o=torch.empty(spec.B, spec.Hq, spec.Nb, spec.D, dtype=dt, device=device),
+                     lse=torch.empty(spec.B, spec.Hq, spec.Nb, dtype=torch.float32, device=device),
+                     x=[dict(q=st.q.to(device), kin=st.kin.to(device), vin=st.vin.to(device),
+                             sel=None if st.sel is None else st.sel.to(device)) for st in self.steps])
+            d["layer"] = fb.FlashBlockLayer(d["x"][0]["q"], d["x"][0]["kin"], d["kp"], d["o"],
+                                            max_prefix=spec.lcap, gamma=spec.gamma is not None,
+                                            sparse=spec.sel_k is not None, max_sel_k=spec.sel_k or 0)
+            self.L.append(d)
+        self.host = [dict(q=st.q.pin_memory(), kin=st.kin.pin_memory(), vin=st.vin.pin_memory()) for st in self.steps]
+        self.query_tokens = spec.B * spec.Nb * len(self.steps) * nl   # layer-steps x B x Nb
+
+    def close(self):
+        for d in self.L:
+            d["layer"].close()
 
 
 def run_ours(args, spec, rank, world, device):
     from block_diffusion_attention_flashblock_b200 import fb
     torch.cuda.set_device(device)
-    fb.fb_debug_set_prefix_kernel({"auto": 0, "generic": 1, "tcgen05": 2}[args.prefix_kernel])
-    sched = Schedule(spec, device)
+    fb.fb_debug_set_prefix_kernel({"auto": 0, "generic": 1, "tcgen05": 2, "tcgen05-nocluster": 3}[args.prefix_kernel])
+    nl = n_layers(spec)
+    S = Layers(spec, device, nl)
     s = spec
-    dt = s.torch_dtype
-    o = torch.empty(s.B, s.Hq, s.Nb, s.D, dtype=dt, device=device)
-    lse = torch.empty(s.B, s.Hq, s.Nb, dtype=torch.float32, device=device)
-    q_like = torch.empty(s.B, s.Hq, s.Nb, s.D, dtype=dt, device=device)
-    k_like = torch.empty(s.B, s.Hkv, s.Nb, s.D, dtype=dt, device=device)
-    layer = fb.FlashBlockLayer(q_like, k_like, sched.kp, o, max_prefix=s.lcap, gamma=s.gamma is not None,
-                               sparse=s.sel_k is not None, max_sel_k=s.sel_k or 0)
     gamma = torch.full((s.Hq,), s.gamma, device=device) if s.gamma is not None else None
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
-    ho = torch.empty(o.shape, dtype=dt, pin_memory=True)
-    hl = torch.empty(lse.shape, dtype=torch.float32, pin_memory=True)
+    nsteps = len(S.steps)
 
-    def one_pass(tau, events, e2e=False, kinds=None):
-        for item in sched.steps:
-            st = item["st"]
-            if st.step == 0:
-                layer.begin_block()
-            flush.zero_()                                   # evict the KV cache from L2
+    def schedule(tau, e2e=False):
+        """The whole schedule: per diffusion step, every layer's fb_step (and at
+        a block's end its fb_kv_append).  Returns the recompute decisions."""
+        rec = []
+        for t, st in enumerate(S.steps):
+            for li, d in enumerate(S.L):
+                x = d["x"][t]
+                if st.step == 0:
+                    d["layer"].begin_block()
+                if e2e:
+                    h = S.host[t]
+                    x["q"].copy_(h["q"], non_blocking=True)
+                    x["kin"].copy_(h["kin"], non_blocking=True)
+                    x["vin"].copy_(h["vin"], non_blocking=True)
+                d["layer"].step(x["q"], x["kin"], x["vin"], d["kp"], d["vp"], st.prefix_len, st.M, tau, d["o"],
+                                d["lse"], gamma, x["sel"])
+                if st.last_in_block:
+                    fb.fb_kv_append(d["layer"].desc, d["kp"], d["vp"], st.prefix_len, x["kin"], x["vin"])
+                if e2e:
+                    ho[t].copy_(d["o"], non_blocking=True)
+                    hl[t].copy_(d["lse"], non_blocking=True)
+            rec.append(S.L[0]["layer"].last_recomputed())
+        return rec
+
+    def timed_region(fn, steps, warmup):
+        """Flush L2, then time fn() between two CUDA events; max over ranks."""
+        for _ in range(warmup):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        ev = []
+        for _ in range(steps):
+            flush.zero_()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            if e2e:
-                item["q"].copy_(item["hq"], non_blocking=True)
-                item["kin"].copy_(item["hk"], non_blocking=True)
-                item["vin"].copy_(item["hv"], non_blocking=True)
-            layer.step(item["q"], item["kin"], item["vin"], sched.kp, sched.vp, st.prefix_len, st.M, tau, o,
-                       lse, gamma, item["sel"])
-            if st.last_in_block:
-                fb.fb_kv_append(layer.desc, sched.kp, sched.vp, st.prefix_len, item["kin"], item["vin"])
-            if e2e:
-                ho.copy_(o, non_blocking=True)
-                hl.copy_(lse, non_blocking=True)
+            fn()
             e1.record(stream)
-            events.append((e0, e1, layer.last_recomputed()))
+            ev.append((e0, e1))
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        if world > 1:
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return t.item()
 
-    def timed(tau, steps, warmup, e2e=False, profile=False):
-        for _ in range(warmup):
-            one_pass(tau, [], e2e)
+    def graph_of(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            out = fn()
         torch.cuda.synchronize()
-        if world > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize()
-        if profile:
-            fb.fb_profile_read(reset=True)
-            fb.fb_profile_enable(True)
-        events = []
-        for _ in range(steps):
-            one_pass(tau, events, e2e)
-        torch.cuda.synchronize()
-        if profile:
-            fb.fb_profile_enable(False)
-        if world > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize()
-        ms = [a.elapsed_time(b) for a, b, _ in events]
-        kinds = [k for _, _, k in events]
-        total = torch.tensor([sum(ms)], dtype=torch.float64, device=device)
-        if world > 1:
-            torch.distributed.all_reduce(total, op=torch.distributed.ReduceOp.MAX)
-        prof = fb.fb_profile_read(reset=True) if profile else None
-        return total.item() / steps, ms, kinds, prof
-
-    def capture(tau):
-        """One CUDA graph per diffusion step: its fb_step and, at a block's end,
-        the append.  The reuse decisions are taken on the host while capturing,
-        in schedule order, exactly as an eager pass takes them."""
-        graphs = []
-        for item in sched.steps:
-            st = item["st"]
-            if st.step == 0:
-                layer.begin_block()
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, capture_error_mode="thread_local"):
-                layer.step(item["q"], item["kin"], item["vin"], sched.kp, sched.vp, st.prefix_len, st.M, tau, o,
-                           lse, gamma, item["sel"])
-                if st.last_in_block:
-                    fb.fb_kv_append(layer.desc, sched.kp, sched.vp, st.prefix_len, item["kin"], item["vin"])
-            graphs.append((g, layer.last_recomputed()))
-        torch.cuda.synchronize()
-        return graphs
-
-    def timed_graphs(graphs, steps, warmup):
-        def run(events):
-            for g, rec in graphs:
-                flush.zero_()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                g.replay()
-                e1.record(stream)
-                events.append((e0, e1, rec))
-        for _ in range(warmup):
-            run([])
-        torch.cuda.synchronize()
-        if world > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize()
-        events = []
-        for _ in range(steps):
-            run(events)
-        torch.cuda.synchronize()
-        if world > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize()
-        ms = [a.elapsed_time(b) for a, b, _ in events]
-        total = torch.tensor([sum(ms)], dtype=torch.float64, device=device)
-        if world > 1:
-            torch.distributed.all_reduce(total, op=torch.distributed.ReduceOp.MAX)
-        return total.item() / steps, ms, [k for _, _, k in events]
+        return g, out
 
     tau_on = s.tau if s.tau is not None else fb.FB_TAU_OFF
+    ho = [torch.empty(S.L[0]["o"].shape, dtype=S.L[0]["o"].dtype, pin_memory=True) for _ in S.steps]
+    hl = [torch.empty(S.L[0]["lse"].shape, dtype=torch.float32, pin_memory=True) for _ in S.steps]
     props = torch.cuda.get_device_properties(device)
     try:
         smi_id = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
     except AttributeError:
         smi_id = str(device.index)
     clocks = ClockSampler(smi_id)
-    # eager library calls (no per-kernel events inside the timed steps)
-    ms_eager, _, _, _ = timed(tau_on, args.steps, args.warmup)
-    # the same steps replayed from CUDA graphs (the headline number)
+
+    # eager library calls
+    ms_eager = timed_region(lambda: schedule(tau_on), args.steps, args.warmup)
+    # the whole schedule as one CUDA graph (the headline number)
+    g_on, rec_on = graph_of(lambda: schedule(tau_on))
     clocks.start()
-    if args.eager:
-        ms_on, per_on, kinds_on = ms_eager, *timed(tau_on, args.steps, 0)[1:3]
-    else:
-        graphs_on = capture(tau_on)
-        ms_on, per_on, kinds_on = timed_graphs(graphs_on, args.steps, args.warmup)
+    ms_on = timed_region(g_on.replay, args.steps, args.warmup)
     clk = clocks.stop()
-    # per-kernel CUDA events around every launch, in a separate eager pass
-    _, _, _, prof = timed(tau_on, args.steps, 1, profile=True)
-    if args.profile_run:
-        ms_full, per_full = float("nan"), []
-    elif args.eager:
-        ms_full, per_full, _, _ = timed(0, args.steps, args.warmup)
-    else:
-        graphs_full = capture(0)
-        ms_full, per_full, _ = timed_graphs(graphs_full, args.steps, args.warmup)
+    del g_on
+    # per-kernel launch counts and algorithmic bytes (one eager pass, events per launch)
+    fb.fb_profile_read(reset=True)
+    fb.fb_profile_enable(True)
+    schedule(tau_on)
+    torch.cuda.synchronize()
+    fb.fb_profile_enable(False)
+    prof = fb.fb_profile_read(reset=True)
+    ms_full = None
+    if not args.profile_run:
+        g_full, _ = graph_of(lambda: schedule(0))
+        ms_full = timed_region(g_full.replay, args.steps, args.warmup)
+        del g_full
     e2e = None
     if not args.no_e2e and not args.profile_run:
-        ms_e2e, _, _, _ = timed(tau_on, args.steps, args.warmup, e2e=True)
-        item = sched.steps[0]
-        h2d = sum(it["hq"].numel() * it["hq"].element_size() + 2 * it["hk"].numel() * it["hk"].element_size()
-                  for it in sched.steps)
-        d2h = len(sched.steps) * (ho.numel() * ho.element_size() + hl.numel() * hl.element_size())
-        e2e = {"value": world * sched.query_tokens / (ms_e2e * 1e-3), "unit": UNIT,
-               "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-    layer.close()
-    assert fb.fb_get_device_status() == fb.FB_OK
+        ms_e2e = timed_region(lambda: schedule(tau_on, e2e=True), args.steps, args.warmup)
+        h2d = nl * sum(h["q"].numel() * h["q"].element_size() + 2 * h["kin"].numel() * h["kin"].element_size()
+                       for h in S.host)
+        d2h = nl * (sum(x.numel() * x.element_size() for x in ho) + sum(x.numel() * x.element_size() for x in hl))
+        e2e = {"value": world * S.query_tokens / (ms_e2e * 1e-3), "unit": UNIT, "ms_per_step": ms_e2e,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "note": "eager calls; every layer-step copies its Q, K_in, V_in from pinned host memory and reads "
+                       "its O and LSE back, inside the timed region"}
 
-    # roofline of the dominant kernel kind (largest event-timed share)
-    hbm, tf, tf_sus, peak_src = _peaks()
-    dom = max(prof, key=lambda k: prof[k][1])
-    n, tot_ms, byts = prof[dom]
-    achieved = (byts / n) / ((tot_ms / n) * 1e-3) / 1e9
-    traffic = _ncu_traffic(dom, spec.name)
-    roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-            "frac": achieved / hbm, "peak_source": f"{peak_src} hbm_gbs",
-            "traffic": traffic, "alg_bytes_per_launch": byts / n, "avg_launch_us": 1e3 * tot_ms / n,
-            "launches": n}
-    kernels = {k: {"launches": v[0], "total_ms_per_step": v[1] / args.steps,
-                   "avg_us": (1e3 * v[1] / v[0]) if v[0] else None,
-                   "achieved_GBps": (v[2] / (v[1] * 1e-3) / 1e9) if v[1] else None} for k, v in prof.items()}
-    n_full = sum(kinds_on) // args.steps
+    # Per-kind launch durations without per-launch event overhead: a graph of
+    # R rounds over the layers of one library call, L2 flushed before it.
+    R = 4
+    st_mid = S.steps[0]
+    P = st_mid.prefix_len
+    parts = []
+    for d in S.L:
+        a = torch.empty(s.B, s.Hq, s.Nb, s.D, dtype=torch.float32, device=device)
+        l = torch.empty(s.B, s.Hq, s.Nb, dtype=torch.float32, device=device)
+        ws = torch.empty(max(16, fb.fb_outblock_workspace_bytes(d["layer"].desc, P)), dtype=torch.uint8,
+                         device=device)
+        parts.append((a, l, ws))
+
+    def call_prefix():
+        for d, (a, l, ws) in zip(S.L, parts):
+            x = d["x"][0]
+            fb.fb_attn_outblock(d["layer"].desc, x["q"], d["kp"], d["vp"], P, a, l, ws)
+
+    def call_inblock():
+        for d, (a, l, ws) in zip(S.L, parts):
+            x = d["x"][0]
+            fb.fb_attn_inblock(d["layer"].desc, x["q"], x["kin"], x["vin"], d["o"], d["lse"], [a], [l])
+
+    call_prefix()
     per_kind = {}
-    for kind in (True, False):
-        xs = [m for m, k in zip(per_on, kinds_on) if k == kind]
-        if xs:
-            per_kind["full_step_us" if kind else "reuse_step_us"] = 1e3 * statistics.mean(xs)
+    for kind, fn in (("prefix_attention", call_prefix), ("inblock_merge", call_inblock)):
+        fb.fb_profile_read(reset=True)
+        fb.fb_profile_enable(True)
+        fn()
+        torch.cuda.synchronize()
+        fb.fb_profile_enable(False)
+        pk = fb.fb_profile_read(reset=True)
+        g, _ = graph_of(lambda: [fn() for _ in range(R)])
+        ms = timed_region(g.replay, args.steps, args.warmup)
+        del g
+        calls = R * nl
+        byts = sum(v[2] for v in pk.values()) / nl
+        per_kind[kind] = {"call": "fb_attn_outblock" if kind == "prefix_attention" else
+                          "fb_attn_inblock (one cached external part)",
+                          "kernels_per_call": sum(v[0] for v in pk.values()) / nl,
+                          "avg_call_us": 1e3 * ms / calls, "alg_bytes_per_call": byts,
+                          "achieved_GBps": byts / (ms * 1e-3 / calls) / 1e9}
+    assert fb.fb_get_device_status() == fb.FB_OK
+    S.close()
+
+    hbm, tf, tf_sus, peak_src = _peaks()
+    # the dominant kind: launches in the schedule x its graph-timed duration
+    share = {k: prof[k][0] * per_kind[k]["avg_call_us"] / max(1e-9, per_kind[k]["kernels_per_call"])
+             for k in per_kind}
+    dom = max(share, key=share.get)
+    pkd = per_kind[dom]
+    traffic = _ncu_traffic(dom, spec.name)
+    roof = {"kernel": dom, "call": pkd["call"], "bound": "hbm", "achieved": pkd["achieved_GBps"], "peak": hbm,
+            "unit": "GB/s", "frac": pkd["achieved_GBps"] / hbm, "peak_source": f"{peak_src} hbm_gbs (burst)",
+            "traffic": traffic, "alg_bytes_per_launch": pkd["alg_bytes_per_call"],
+            "avg_launch_us": pkd["avg_call_us"],
+            "timing": f"CUDA events around one graph of {R * nl} calls ({nl} layers x {R}), L2 flushed before"}
+    kernels = {k: {"launches_per_step": v[0], "alg_bytes_per_step": v[2]} for k, v in prof.items()}
+    n_full = sum(rec_on)
+    layer_steps = nsteps * nl
+    step_lat = {"mean_us": 1e3 * ms_on / layer_steps}
+    if ms_full is not None:
+        t_full = ms_full / layer_steps
+        step_lat["full_step_us"] = 1e3 * t_full
+        if nsteps > n_full:
+            step_lat["reuse_step_us_derived"] = 1e3 * (ms_on / nl - n_full * t_full) / (nsteps - n_full)
     gpu_launches = sum(v[0] for v in prof.values())
     return {
-        "metric": METRIC, "value": world * sched.query_tokens / (ms_on * 1e-3), "unit": UNIT,
+        "metric": METRIC, "value": world * S.query_tokens / (ms_on * 1e-3), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_on,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": spec.dtype,
         "data": "synthetic (seeded; shapes of the pages' diffusion-LM workload)",
-        "config": {"workload": _describe(spec), "query_tokens_per_step": sched.query_tokens,
-                   "prefix_kernel": args.prefix_kernel,
-                   "diffusion_steps_per_step": len(sched.steps), "l2": "flushed (1 GiB write) before every "
-                   "diffusion step, outside the timed interval", "parallelism": f"replicas x{world}",
-                   "full_steps_per_step": n_full},
-        "step_latency": {"mean_us": 1e3 * ms_on / len(sched.steps), **per_kind},
-        "timing": "CUDA graph per diffusion step, replayed" if not args.eager else "eager library calls",
-        "eager": {"value": world * sched.query_tokens / (ms_eager * 1e-3), "ms_per_step": ms_eager},
-        "full_recompute": None if args.profile_run else {"value": world * sched.query_tokens / (ms_full * 1e-3), "ms_per_step": ms_full,
-                           "mean_step_us": 1e3 * ms_full / len(sched.steps)},
-        "speedup_vs_full_recompute": None if args.profile_run else ms_full / ms_on,
-        "e2e": e2e, "roofline": roof, "kernels": kernels, "gpu_launches": gpu_launches // 1,
-        "gpu_launches_per_step": gpu_launches / args.steps, "clocks": clk,
+        "config": {"workload": _describe(spec), "layers": nl,
+                   "query_tokens_per_step": S.query_tokens,
+                   "prefix_kernel": args.prefix_kernel, "diffusion_steps_per_layer": nsteps,
+                   "l2": f"flushed (1 GiB write) before every timed step; inside it {nl} layers with their own "
+                         f"KV caches are stepped in turn, so each layer's data has left L2 when it runs",
+                   "parallelism": f"replicas x{world}", "full_steps_per_layer": n_full},
+        "step_latency": step_lat,
+        "timing": "one CUDA graph of the whole schedule (all layers), replayed; CUDA events around each replay",
+        "eager": {"value": world * S.query_tokens / (ms_eager * 1e-3), "ms_per_step": ms_eager},
+        "full_recompute": None if ms_full is None else {
+            "value": world * S.query_tokens / (ms_full * 1e-3), "ms_per_step": ms_full,
+            "mean_step_us": 1e3 * ms_full / layer_steps},
+        "speedup_vs_full_recompute": None if ms_full is None else ms_full / ms_on,
+        "e2e": e2e, "roofline": roof, "per_call": per_kind, "kernels": kernels,
+        "gpu_launches": gpu_launches * args.steps, "gpu_launches_per_step": gpu_launches, "clocks": clk,
     }
 
 
@@ -401,8 +438,7 @@ def main():
     ap.add_argument("--workload", default="dllm_8k", choices=list(wl.SPECS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
-    ap.add_argument("--prefix-kernel", default="auto", choices=["auto", "generic", "tcgen05"])
-    ap.add_argument("--eager", action="store_true", help="time eager library calls instead of graph replays")
+    ap.add_argument("--prefix-kernel", default="auto", choices=["auto", "generic", "tcgen05", "tcgen05-nocluster"])
     ap.add_argument("--profile-run", action="store_true",
                     help="only the reuse-on schedule (no full-recompute, e2e or CPU legs): for ncu captures")
     args = ap.parse_args()

@@ -19,7 +19,8 @@
 //               their row sums) through shared memory and a bounded
 //               mbarrier.  Each writes its half of P = 2^(s - m), as bf16 hi
 //               and lo parts, back into the TMEM columns its S tile came from;
-//               the final O / l and L go to the split's part.
+//               the final O / l and L are staged in shared memory and leave
+//               as whole rows (512 contiguous bytes per warp store).
 // P lives in the S buffer it replaces, so S_{j+3} is only issued once PV_j
 // has completed (a completion barrier per buffer); three buffers leave two
 // softmax tiles for the chain P_j -> PV_j -> S_{j+3}.
@@ -27,8 +28,9 @@
 // grows by more than 2^8, so P stays <= 256 and most tiles skip the rescale.
 // With a cluster launch, each cluster of key splits of one row tile reduces
 // its parts through distributed shared memory before anything reaches global
-// memory (one part per cluster).  The last split also takes the ragged
-// remainder of the keys.
+// memory (one part per cluster): every rank sends each other rank the rows
+// that rank owns with one bulk shared-to-shared copy, and each owner merges
+// its rows.  The last split also takes the ragged remainder of the keys.
 // Every mbarrier wait is bounded; on expiry the CTA records FB_ETIMEOUT in
 // the device status word, drains its own TMA and MMA work, frees TMEM and
 // exits.
@@ -64,7 +66,7 @@ constexpr float kRescaleLog2 = 8.0f;
 // barrier slots
 enum {
   B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 10, B_SFULL = 13, B_PFULL = 16,
-  B_PVDONE = 19, B_DRAIN = 22, B_PAIR = 24, B_COUNT = 28
+  B_PVDONE = 19, B_DRAIN = 22, B_PAIR = 24, B_RECV = 28, B_COUNT = 29
 };
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -203,14 +205,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
       "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
 }
-__device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
-  uint32_t r;
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
-  return __uint_as_float(r);
-}
-__device__ __forceinline__ void tmem_st1(uint32_t taddr, float v) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(__float_as_uint(v)) : "memory");
-}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -228,20 +222,46 @@ __device__ __forceinline__ uint32_t map_rank(uint32_t local, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
   return r;
 }
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
-}
-__device__ __forceinline__ float4 ld_dsmem_v4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr)
+// Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory into
+// another cluster rank's, completing on that rank's mbarrier (no multicast).
+__device__ __forceinline__ void bulk_to_rank(uint32_t dst_cluster, uint32_t src, uint32_t bytes,
+                                             uint32_t bar_cluster) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   dst_cluster),
+               "r"(src), "r"(bytes), "r"(bar_cluster)
                : "memory");
-  return v;
 }
-constexpr int kRedStride = 132;   // fp32 row stride of a CTA's staged part (bank spread)
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Epilogue staging, inside the idle K/V rings: this CTA's normalised rows
+// [128][kRedStride] fp32 (columns 0..127 = O, column 128 = L), then, with a
+// cluster launch, the rows this rank owns as received from every rank
+// [ranks x rows per rank <= 143][kRedStride].
+constexpr int kRedStride = 132;
+constexpr uint32_t kRowBytes = kRedStride * 4u;   // 528, a multiple of 16
+constexpr uint32_t kRecvOff = 128u * kRowBytes;
+static_assert(kRecvOff + 144u * kRowBytes <= 2u * 3u * 32768u, "epilogue staging must fit in the K/V rings");
+
+// This thread's 64 output columns (a half row of O in TMEM, zero when the
+// split had no keys), scaled by inv, handed to put(float4 index, value).
+template <class F>
+__device__ __forceinline__ void load_o_scaled(uint32_t tl, int half, int T, float inv, F&& put) {
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    float o[32];
+    if (T > 0) {
+      tmem_ld32(tl + kTmemO + half * 64 + c * 32, o);
+      tmem_wait_ld();
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < 32; e += 4)
+      put((c * 32 + e) / 4, make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv));
+  }
+}
 
 // Shared-memory matrix descriptor, 128-byte swizzle (layout code 2), sm_100
 // version bit 46; lbo/sbo in bytes.
@@ -259,10 +279,6 @@ constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3
 constexpr uint32_t kIdescQK = kIdescBase;              // A, B K-major
 constexpr uint32_t kIdescPV = kIdescBase | (1u << 16);  // B (V) MN-major
 
-__device__ __forceinline__ uint32_t pack2_bf16(float x, float y) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
 
 // 2^x on the MUFU unit (PTX ex2.approx; relative error about 2^-22, -inf -> 0).
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -271,11 +287,15 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// bf16 hi/lo split of a pair: hi = bf16(x), lo = bf16(x - hi).
+// bf16 hi/lo split of a pair by truncation, on integer and FADD pipes only:
+// hi = the upper 16 bits of x (exact remainder x - hi in fp32), lo = the upper
+// 16 bits of that remainder, so x - hi - lo < 2^-14 |x|.  Lower key in the low
+// half of each packed word.
 __device__ __forceinline__ void split_pair(float x, float y, uint32_t& hi, uint32_t& lo) {
-  hi = pack2_bf16(x, y);
-  const float hx = __uint_as_float(hi << 16), hy = __uint_as_float(hi & 0xFFFF0000u);
-  lo = pack2_bf16(x - hx, y - hy);
+  const uint32_t xb = __float_as_uint(x), yb = __float_as_uint(y);
+  hi = __byte_perm(xb, yb, 0x7632);
+  const float rx = x - __uint_as_float(xb & 0xFFFF0000u), ry = y - __uint_as_float(yb & 0xFFFF0000u);
+  lo = __byte_perm(__float_as_uint(rx), __float_as_uint(ry), 0x7632);
 }
 
 }  // namespace
@@ -330,6 +350,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int h = h0; h < h0 + hn; ++h) all = all && a.mask[b * a.Hq + h];
     if (all) return;
   }
+  // Row rr of the tile: its row in the part layout, and whether it exists.
+  auto row_index = [&](int rr, int64_t& r) -> bool {
+    int hh, ii;
+    bool valid;
+    if (a.mode == 0) {
+      const int g = t * a.hg + rr / a.Nb;
+      ii = rr % a.Nb;
+      hh = kvh * a.G + g;
+      valid = rr < a.hg * a.Nb && g < a.G;
+    } else {
+      hh = h0;
+      ii = i0 + rr;
+      valid = ii < a.Nb;
+    }
+    r = ((int64_t)b * a.Hq + hh) * a.Nb + ii;
+    return valid;
+  };
+  if (warp == 1 && lane == 1) {
+    // warm the address translation of the part rows this CTA writes at the end
+    int64_t r0;
+    row_index(0, r0);
+    const int part = a.cluster > 1 ? split / a.cluster : split;
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.part_a + part * a.part_stride_a + r0 * kD));
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.part_l + part * a.part_stride_l + r0));
+  }
   const int64_t kbeg = (int64_t)split * a.keys_per_split;
   const int64_t kend = split == (int)gridDim.y - 1 ? a.nkeys : min(kbeg + a.keys_per_split, a.nkeys);
   const int T = kend > kbeg ? (int)((kend - kbeg + kBN - 1) / kBN) : 0;
@@ -338,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < B_COUNT; ++i) {
       uint32_t cnt = 1;
       if (i >= B_PFULL && i < B_PFULL + kSBuf) cnt = 256;
-      if (i >= B_PAIR) cnt = 64;
+      if (i >= B_PAIR && i < B_PAIR + 4) cnt = 64;
       mbar_init(bar(i), cnt);
     }
     *abort_flag = 0;
@@ -544,104 +589,85 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) ok = trade(l, T & 1, T, lo_other);   // the row sum is the two halves' sum
     if (ok) {
       l += lo_other;
-      tc_fence_after();
-      int hh, ii;
-      bool valid;
-      if (a.mode == 0) {
-        const int g = t * a.hg + row / a.Nb;
-        ii = row % a.Nb;
-        hh = kvh * a.G + g;
-        valid = row < a.hg * a.Nb && g < a.G;
-      } else {
-        hh = h0;
-        ii = i0 + row;
-        valid = ii < a.Nb;
-      }
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const float Lrow = l > 0.f ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
-      const int64_t r = ((int64_t)b * a.Hq + hh) * a.Nb + ii;
-      // clustered: stage the normalised row in this CTA's shared memory (the
-      // K/V rings are idle now) for the cluster reduction below
-      float* pa = (a.cluster > 1 ? reinterpret_cast<float*>(smem + kOffK) + row * kRedStride
-                                 : a.part_a + split * a.part_stride_a + r * kD) +
-                  half * 64;
-      const bool store = a.cluster > 1 || valid;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        float o[32];
-        if (T > 0) {
-          tmem_ld32(tl + kTmemO + half * 64 + c * 32, o);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0.f;
-        }
-        if (store) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(pa + c * 32 + e) =
-                make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv);
-        }
-      }
-      if (half == 0) {
-        if (a.cluster > 1) reinterpret_cast<float*>(smem + kOffK + kBM * kRedStride * 4)[row] = Lrow;
-        else if (valid) a.part_l[split * a.part_stride_l + r] = Lrow;
-      }
+      // stage the normalised row and its L in this CTA's shared memory (the
+      // K/V rings are idle now)
+      tc_fence_after();
+      float* st = reinterpret_cast<float*>(smem + kOffK) + row * kRedStride;
+      load_o_scaled(tl, half, T, inv,
+                    [&](int c, float4 v) { *reinterpret_cast<float4*>(st + half * 64 + c * 4) = v; });
+      if (half == 0) st[128] = Lrow;
+      fence_proxy_async_smem();   // the rows may leave by bulk copy
     }
   }
 
+  const int CS = a.cluster;
+  const int R = (kBM + CS - 1) / CS;   // rows owned by each cluster rank
+  const int rank = CS > 1 ? (int)cluster_rank() : 0;
+  const int own = CS > 1 ? max(0, min(R, kBM - rank * R)) : 0;
+  if (CS > 1 && threadIdx.x == 0) mbar_expect_tx(bar(B_RECV), (uint32_t)(CS * own) * kRowBytes);
   tc_fence_before();
   __syncthreads();
-  if (a.cluster > 1) {
-    // Split-KV reduction over the cluster: rank c merges rows [c*R, c*R + R) of
-    // every rank's staged part (log-space merge, ranks in fixed order) and
-    // writes the final row.  32 threads per row, 4 columns per thread.
-    cluster_sync_all();
-    const int CS = a.cluster;
-    const uint32_t rank = cluster_rank();
-    const int R = (kBM + CS - 1) / CS;
-    const uint32_t sA = sbase + kOffK, sL = sbase + kOffK + kBM * kRedStride * 4;
-    const int lane4 = threadIdx.x & 31;
-    for (int rr = (int)rank * R + (int)(threadIdx.x >> 5); rr < min(kBM, ((int)rank + 1) * R); rr += kThreads / 32) {
-      int hh, ii;
-      bool valid;
-      if (a.mode == 0) {
-        const int g = t * a.hg + rr / a.Nb;
-        ii = rr % a.Nb;
-        hh = kvh * a.G + g;
-        valid = rr < a.hg * a.Nb && g < a.G;
-      } else {
-        hh = h0;
-        ii = i0 + rr;
-        valid = ii < a.Nb;
-      }
-      if (!valid) continue;
-      float m = -CUDART_INF_F;
-      float Ls[16];
-#pragma unroll
-      for (int p = 0; p < 16; ++p) {
-        Ls[p] = p < CS ? ld_dsmem_f32(map_rank(sL + rr * 4, p)) : -CUDART_INF_F;
-        m = fmaxf(m, Ls[p]);
-      }
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      float wsum = 0.f;
-#pragma unroll
-      for (int p = 0; p < 16; ++p) {
-        if (p >= CS || Ls[p] == -CUDART_INF_F) continue;
-        const float w = __expf(Ls[p] - m);
-        const float4 v = ld_dsmem_v4(map_rank(sA + (rr * kRedStride + lane4 * 4) * 4, p));
-        wsum += w;
-        acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
-        acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
-      }
-      const int64_t r = ((int64_t)b * a.Hq + hh) * a.Nb + ii;
-      const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-      const int part = split / CS;
-      *reinterpret_cast<float4*>(a.part_a + part * a.part_stride_a + r * kD + lane4 * 4) =
-          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-      if (lane4 == 0) a.part_l[part * a.part_stride_l + r] = m == -CUDART_INF_F ? -CUDART_INF_F : m + __logf(wsum);
+  const int nwarps = kThreads / 32;
+  const float* stage = reinterpret_cast<const float*>(smem + kOffK);
+  if (CS <= 1) {
+    // one row per warp: 512 contiguous bytes per store instruction
+    for (int rr = warp; rr < kBM; rr += nwarps) {
+      int64_t r;
+      if (!row_index(rr, r)) continue;
+      *reinterpret_cast<float4*>(a.part_a + split * a.part_stride_a + r * kD + lane * 4) =
+          *reinterpret_cast<const float4*>(stage + rr * kRedStride + lane * 4);
+      if (lane == 0) a.part_l[split * a.part_stride_l + r] = stage[rr * kRedStride + 128];
     }
-    cluster_sync_all();   // keep every rank's shared memory alive until all reads are done
+  } else {
+    // Split-KV reduction over the cluster.  Rank c owns rows [c*R, c*R + R).
+    // Once every rank is past its main loop, each rank sends each owner that
+    // owner's block of its staged rows with one bulk copy into the owner's
+    // receive area (slot p*R + i for rank p's row c*R + i), completing on
+    // the owner's receive barrier; the owner merges its rows in log space,
+    // ranks in fixed order, and writes the cluster's part.
+    cluster_sync_all();
+    if (threadIdx.x == 0) {
+      for (int o = 0; o < CS; ++o) {
+        const int n = max(0, min(R, kBM - o * R));
+        if (n == 0) continue;
+        bulk_to_rank(map_rank(sbase + kOffK + kRecvOff + (uint32_t)(rank * R) * kRowBytes, (uint32_t)o),
+                     sbase + kOffK + (uint32_t)(o * R) * kRowBytes, (uint32_t)n * kRowBytes,
+                     map_rank(bar(B_RECV), (uint32_t)o));
+      }
+    }
+    // waited on even after a failure elsewhere in this CTA (draining), so no copy
+    // into this CTA is still in flight when it exits
+    if (wait_phase(bar(B_RECV), 0, ctl, true)) {
+      const float* recv = reinterpret_cast<const float*>(smem + kOffK + kRecvOff);
+      for (int rl = warp; rl < own; rl += nwarps) {
+        int64_t r;
+        if (!row_index(rank * R + rl, r)) continue;
+        float m = -CUDART_INF_F;
+#pragma unroll 1
+        for (int p = 0; p < CS; ++p) m = fmaxf(m, recv[(p * R + rl) * kRedStride + 128]);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float wsum = 0.f;
+#pragma unroll 1
+        for (int p = 0; p < CS; ++p) {
+          const float* rowp = recv + (p * R + rl) * kRedStride;
+          const float Lp = rowp[128];
+          if (Lp == -CUDART_INF_F) continue;
+          const float w = __expf(Lp - m);
+          const float4 v = *reinterpret_cast<const float4*>(rowp + lane * 4);
+          wsum += w;
+          acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
+          acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+        }
+        const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+        const int part = split / CS;
+        *reinterpret_cast<float4*>(a.part_a + part * a.part_stride_a + r * kD + lane * 4) =
+            make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        if (lane == 0) a.part_l[part * a.part_stride_l + r] = m == -CUDART_INF_F ? -CUDART_INF_F : m + __logf(wsum);
+      }
+    }
+    cluster_sync_all();   // every copy out of this CTA's staging has landed
   }
   if (warp == 1) {
     tc_fence_after();

@@ -108,6 +108,16 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   // KV head are consecutive in the packed (b, h, i) order of parts and LSE.
   const int64_t prow0 = ((int64_t)b * a.Hq + (int64_t)kvh * a.G) * a.Nb + row0;
 
+  if (tid == 0) {
+    // warm the address translation of the rows this CTA stores at the end
+    const int g = min(row0 / a.Nb, a.G - 1), i = row0 % a.Nb;
+    const size_t esz = a.o_bf16 ? 2 : 4;
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(static_cast<const char*>(a.o) +
+                                                  (b * a.o_sb + (int64_t)(kvh * a.G + g) * a.o_sh +
+                                                   (int64_t)i * a.o_st) * esz));
+    if (a.cache_a) asm volatile("prefetch.global.L2 [%0];" ::"l"(a.cache_a + prow0 * kD));
+    if (a.lse) asm volatile("prefetch.global.L2 [%0];" ::"l"(a.lse + prow0));
+  }
   // ---- one batch of asynchronous loads ----
   for (int c = tid; c < kRows * 16; c += 128) {
     const int r = c >> 4, ch = c & 15;
