@@ -234,7 +234,7 @@ static PrefixPlan plan_prefix(const fb_attn_desc& d, const void* q, const void* 
   p.cluster = 1;
   p.kps = p.gen.a.keys_per_split;
   const int64_t min_keys = g_prefix_kernel >= 2 ? 1 : 256;
-  if (g_prefix_kernel != 1 && nkeys >= min_keys && tc_make_maps(d, q, kp, vp, nkeys, &p.maps)) {
+  if (g_prefix_kernel != 1 && nkeys >= min_keys && tc_make_maps(d, q, kp, vp, nkeys, d.kp_strides, &p.maps)) {
     tc_plan_split((int64_t)p.maps.units * p.maps.tiles_per_unit, nkeys, cap, g_prefix_kernel != 3, &p.nsplit,
                   &p.kps, &p.cluster, &p.nparts);
     p.tc = true;
@@ -284,9 +284,32 @@ static fb_status merge_to_part(const fb_attn_desc& d, const PartList& pl, float*
   return launch_merge(m, s) == cudaSuccess ? FB_OK : FB_ECUDA;
 }
 
+// Merge `pl` into the output O (the descriptor's output dtype and strides) and LSE.
+static fb_status merge_to_out(const fb_attn_desc& d, const PartList& pl, void* o, float* lse, cudaStream_t s) {
+  MergeArgs m;
+  memset(&m, 0, sizeof(m));
+  m.B = d.B; m.Hq = d.Hq; m.Nb = d.Nb; m.D = d.D;
+  m.parts = pl;
+  m.o = o; m.o_sb = d.o_strides[0]; m.o_sh = d.o_strides[1]; m.o_st = d.o_strides[2];
+  m.o_bf16 = d.out_dtype == FB_BF16;
+  m.lse = lse;
+  double nparts = 0;
+  for (int i = 0; i < pl.ngroups; ++i) nparts += pl.g[i].count;
+  ProfScope prof(kProfAux, nparts * rows_of(d) * (d.D + 1) * 4.0 + rows_of(d) * (d.D * esize(d.out_dtype) + 4.0),
+                 s);
+  return launch_merge(m, s) == cudaSuccess ? FB_OK : FB_ECUDA;
+}
+
+// Block-internal attention merged with the external parts `ext` into O and
+// LSE.  Small blocks: one fused kernel (which can also write the merge of the
+// external parts into cache_a / cache_l).  Larger bf16 blocks with a parts
+// workspace (ws_a / ws_l, ws_cap parts): the tcgen05 attention kernel over
+// the block's own keys writes split parts there, and the merge kernel
+// combines them with ext.  Otherwise the generic kernel, fused with the merge.
 static fb_status run_inblock(const fb_attn_desc& d, const void* q, const void* kin, const void* vin,
                              const PartList& ext, void* o, float* lse, cudaStream_t s, float* cache_a = nullptr,
-                             float* cache_l = nullptr) {
+                             float* cache_l = nullptr, float* ws_a = nullptr, float* ws_l = nullptr,
+                             int32_t ws_cap = 0) {
   PassPlan p = plan_pass(d, q, kin, vin, d.kin_strides, d.Nb, nullptr, 0, 1);
   AttnArgs& a = p.a;
   a.nsplit = 1;
@@ -309,13 +332,32 @@ static fb_status run_inblock(const fb_attn_desc& d, const void* q, const void* k
   const double bytes = (double)rows_of(d) * d.D * es + 2.0 * d.B * d.Hkv * d.Nb * d.D * es +
                        ext_parts * rows_of(d) * (d.D + 1) * 4.0 +
                        (double)rows_of(d) * (d.D * esize(d.out_dtype) + (lse ? 4 : 0));
-  ProfScope prof(kProfInblock, bytes, s);
-  if (inblock_small_applies(d, a.next))
+  if (inblock_small_applies(d, a.next)) {
+    ProfScope prof(kProfInblock, bytes, s);
     return launch_inblock_small(d, q, kin, vin, a.next, a.ext_a, a.ext_l, o, lse, cache_a, cache_l, a.scale_log2,
                                 s) == cudaSuccess
                ? FB_OK
                : FB_ECUDA;
+  }
   if (cache_a) return FB_EUNSUPPORTED;   // callers only ask for the cache write where the small kernel runs
+  TcMaps maps;
+  if (ws_a && ws_cap >= 1 && g_prefix_kernel != 1 && d.Nb >= 128 && ext.ngroups < 8 &&
+      tc_make_maps(d, q, kin, vin, d.Nb, d.kin_strides, &maps)) {
+    int32_t ns, cl, np;
+    int64_t kps;
+    tc_plan_split((int64_t)maps.units * maps.tiles_per_unit, d.Nb, ws_cap, false, &ns, &kps, &cl, &np);
+    {
+      const double tc_bytes = (double)rows_of(d) * d.D * es + 2.0 * d.B * d.Hkv * d.Nb * d.D * es +
+                              (double)np * rows_of(d) * (d.D + 1) * 4.0;
+      ProfScope prof(kProfInblock, tc_bytes, s);
+      if (launch_attn_tc(d, maps, d.Nb, ns, kps, 1, nullptr, 0, a.scale_log2, ws_a, ws_l, s) != cudaSuccess)
+        return FB_ECUDA;
+    }
+    PartList all = ext;
+    all.g[all.ngroups++] = group_of(ws_a, ws_l, np, d);
+    return merge_to_out(d, all, o, lse, s);
+  }
+  ProfScope prof(kProfInblock, bytes, s);
   return launch_attn_generic(a, d.D, d.in_dtype == FB_BF16, s) == cudaSuccess ? FB_OK : FB_ECUDA;
 }
 
@@ -746,7 +788,11 @@ fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
     if (a->sim_out && cudaMemsetAsync(a->sim_out, 0xFF, (size_t)BH * 4, s) != cudaSuccess) return FB_ECUDA;
   }
   ext.g[ext.ngroups++] = group_of(c->cache_a, c->cache_l, 1, d);
-  if ((st = run_inblock(d, a->q, a->kin, a->vin, ext, a->o, a->lse, s)) != FB_OK) return st;
+  // the split parts of the prefix pass are consumed by now: their slots take
+  // the block-internal pass's parts
+  if ((st = run_inblock(d, a->q, a->kin, a->vin, ext, a->o, a->lse, s, nullptr, nullptr, c->part_a, c->part_l,
+                        c->part_cap)) != FB_OK)
+    return st;
   c->valid = true;
   c->last_recomputed = !tau_reuse;
   return FB_OK;

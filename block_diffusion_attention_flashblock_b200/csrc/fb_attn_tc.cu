@@ -41,6 +41,7 @@
 #include <algorithm>
 
 #include "fb_internal.cuh"
+#include "fb_ptx.cuh"
 
 namespace fb {
 
@@ -69,32 +70,12 @@ enum {
   B_PVDONE = 19, B_DRAIN = 22, B_PAIR = 24, B_RECV = 28, B_COUNT = 29
 };
 
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
+using ptx::globaltimer;
+using ptx::mbar_arrive;
+using ptx::mbar_expect_tx;
+using ptx::mbar_init;
+using ptx::mbar_try;
+using ptx::smem_addr;
 
 // Shared control block: first-failure flag, TMEM base.
 struct Ctl {
@@ -231,9 +212,7 @@ __device__ __forceinline__ void bulk_to_rank(uint32_t dst_cluster, uint32_t src,
                "r"(src), "r"(bytes), "r"(bar_cluster)
                : "memory");
 }
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
+using ptx::fence_proxy_async_smem;
 // Epilogue staging, inside the idle K/V rings: this CTA's normalised rows
 // [128][kRedStride] fp32 (columns 0..127 = O, column 128 = L), then, with a
 // cluster launch, the rows this rank owns as received from every rank
@@ -350,30 +329,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int h = h0; h < h0 + hn; ++h) all = all && a.mask[b * a.Hq + h];
     if (all) return;
   }
-  // Row rr of the tile: its row in the part layout, and whether it exists.
-  auto row_index = [&](int rr, int64_t& r) -> bool {
-    int hh, ii;
-    bool valid;
-    if (a.mode == 0) {
-      const int g = t * a.hg + rr / a.Nb;
-      ii = rr % a.Nb;
-      hh = kvh * a.G + g;
-      valid = rr < a.hg * a.Nb && g < a.G;
-    } else {
-      hh = h0;
-      ii = i0 + rr;
-      valid = ii < a.Nb;
-    }
-    r = ((int64_t)b * a.Hq + hh) * a.Nb + ii;
-    return valid;
-  };
+  // The tile's rows [0, nrows) exist and are the consecutive rows
+  // [rbase, rbase + nrows) of the packed (b, h, i) part layout.
+  int64_t rbase;
+  int nrows;
+  if (a.mode == 0) {
+    rbase = ((int64_t)b * a.Hq + (int64_t)kvh * a.G + (int64_t)t * a.hg) * a.Nb;
+    nrows = min(a.hg, a.G - t * a.hg) * a.Nb;
+  } else {
+    rbase = ((int64_t)b * a.Hq + h0) * a.Nb + i0;
+    nrows = min(kBM, a.Nb - i0);
+  }
   if (warp == 1 && lane == 1) {
     // warm the address translation of the part rows this CTA writes at the end
-    int64_t r0;
-    row_index(0, r0);
     const int part = a.cluster > 1 ? split / a.cluster : split;
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.part_a + part * a.part_stride_a + r0 * kD));
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.part_l + part * a.part_stride_l + r0));
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.part_a + part * a.part_stride_a + rbase * kD));
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.part_l + part * a.part_stride_l + rbase));
   }
   const int64_t kbeg = (int64_t)split * a.keys_per_split;
   const int64_t kend = split == (int)gridDim.y - 1 ? a.nkeys : min(kbeg + a.keys_per_split, a.nkeys);
@@ -612,14 +583,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nwarps = kThreads / 32;
   const float* stage = reinterpret_cast<const float*>(smem + kOffK);
   if (CS <= 1) {
-    // one row per warp: 512 contiguous bytes per store instruction
-    for (int rr = warp; rr < kBM; rr += nwarps) {
-      int64_t r;
-      if (!row_index(rr, r)) continue;
-      *reinterpret_cast<float4*>(a.part_a + split * a.part_stride_a + r * kD + lane * 4) =
-          *reinterpret_cast<const float4*>(stage + rr * kRedStride + lane * 4);
-      if (lane == 0) a.part_l[split * a.part_stride_l + r] = stage[rr * kRedStride + 128];
+    // The tile's rows are one contiguous range of the part: every thread
+    // copies up to 11 of its 16-byte pieces, all loads before all stores, a
+    // warp covering 512 contiguous bytes per store instruction.
+    constexpr int kPieces = (kBM * 32 + kThreads - 1) / kThreads;
+    float* dst = a.part_a + split * a.part_stride_a + rbase * kD;
+    float4 v[kPieces];
+#pragma unroll
+    for (int k = 0; k < kPieces; ++k) {
+      const int idx = threadIdx.x + k * kThreads, rr = idx >> 5;
+      if (rr < nrows) v[k] = *reinterpret_cast<const float4*>(stage + rr * kRedStride + (idx & 31) * 4);
     }
+#pragma unroll
+    for (int k = 0; k < kPieces; ++k) {
+      const int idx = threadIdx.x + k * kThreads, rr = idx >> 5;
+      if (rr < nrows) *reinterpret_cast<float4*>(dst + (size_t)idx * 4) = v[k];
+    }
+    if ((int)threadIdx.x < nrows) a.part_l[split * a.part_stride_l + rbase + threadIdx.x] = stage[threadIdx.x * kRedStride + 128];
   } else {
     // Split-KV reduction over the cluster.  Rank c owns rows [c*R, c*R + R).
     // Once every rank is past its main loop, each rank sends each owner that
@@ -641,9 +621,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // into this CTA is still in flight when it exits
     if (wait_phase(bar(B_RECV), 0, ctl, true)) {
       const float* recv = reinterpret_cast<const float*>(smem + kOffK + kRecvOff);
-      for (int rl = warp; rl < own; rl += nwarps) {
-        int64_t r;
-        if (!row_index(rank * R + rl, r)) continue;
+      const int own_valid = min(own, nrows - rank * R);
+#pragma unroll 2
+      for (int rl = warp; rl < own_valid; rl += nwarps) {
+        const int64_t r = rbase + rank * R + rl;
         float m = -CUDART_INF_F;
 #pragma unroll 1
         for (int p = 0; p < CS; ++p) m = fmaxf(m, recv[(p * R + rl) * kRedStride + 128]);
@@ -727,13 +708,14 @@ bool tc_tiling(const fb_attn_desc& d, int* mode, int* hg, int* tiles_per_unit, i
   return false;
 }
 
-bool tc_make_maps(const fb_attn_desc& d, const void* q, const void* kp, const void* vp, int64_t nkeys, TcMaps* m) {
+bool tc_make_maps(const fb_attn_desc& d, const void* q, const void* k, const void* v, int64_t nkeys,
+                  const int64_t* kstr, TcMaps* m) {
   if (nkeys <= 0 || !tc_tiling(d, &m->mode, &m->hg, &m->tiles_per_unit, &m->units)) return false;
   const uint32_t qrows = m->mode == 0 ? (uint32_t)d.Nb : (uint32_t)kBM;
   const uint32_t qheads = m->mode == 0 ? (uint32_t)m->hg : 1u;
   return map_4d(&m->q, q, d.Nb, d.Hq, d.B, d.q_strides[2], d.q_strides[1], d.q_strides[0], qrows, qheads) &&
-         map_4d(&m->k, kp, nkeys, d.Hkv, d.B, d.kp_strides[2], d.kp_strides[1], d.kp_strides[0], kBN, 1) &&
-         map_4d(&m->v, vp, nkeys, d.Hkv, d.B, d.kp_strides[2], d.kp_strides[1], d.kp_strides[0], kBN, 1);
+         map_4d(&m->k, k, nkeys, d.Hkv, d.B, kstr[2], kstr[1], kstr[0], kBN, 1) &&
+         map_4d(&m->v, v, nkeys, d.Hkv, d.B, kstr[2], kstr[1], kstr[0], kBN, 1);
 }
 
 // Upper bound of the split count the planner may choose (sizes workspaces).
@@ -796,7 +778,10 @@ void tc_plan_split(int64_t tiles, int64_t nkeys, int32_t max_parts, bool allow_c
       const int64_t per = ktiles / ns, last = ktiles - (ns - 1) * per;
       const int64_t units = cs == 1 ? tiles * ns : tiles * nc;
       const int64_t waves = (units + conc - 1) / conc;
-      const double cost = (double)waves * (last + 2) + (parts > 1 ? 1.5 + 0.1 * parts : 0.0) + 0.01 * ns;
+      // a cluster's in-kernel reduction (two cluster barriers and the
+      // shared-to-shared copies) costs about four key tiles per CTA
+      const double cost = (double)waves * (last + 2 + (cs > 1 ? 4 : 0)) + (parts > 1 ? 1.5 + 0.1 * parts : 0.0) +
+                          0.01 * ns;
       if (cost < best) { best = cost; b_ns = ns; b_cs = cs; b_per = per; }
     }
   }

@@ -2,40 +2,37 @@
 // (FlashBlock summary, "Mécanisme Central": A_in over the block's own keys
 // J_in, then A = (e^{L_out-m} A_out + e^{L_in-m} A_in) / (...)).  This is the
 // whole reuse step of a diffusion LM, so it is built for latency:
-//   - one CTA = 32 packed query rows of one KV head (G query heads x Nb
-//     queries); 4 warps: two 16-row slabs, and for each slab two warps that
-//     both form S and P but split the P V product and the epilogue by halves
-//     of the head dimension (shorter per-warp instruction chains);
-//   - every global load (Q, K_in, V_in and the external parts A, L) is issued
-//     up front with cp.async in three groups (Q and K_in; V_in; the parts), so
-//     S and the softmax start while V_in and the parts are still arriving;
+//   - one CTA = 16 packed query rows of one KV head (G query heads x Nb
+//     queries) and 4 warps; every warp forms S and P for the 16 rows (one
+//     m16 tile) and owns a quarter (32 columns) of the head dimension in the
+//     P V product, the merge and the stores, which keeps each warp's
+//     dependent instruction chain short;
+//   - every load (Q, K_in, V_in rows and the external parts' A rows) is one
+//     bulk copy per row, issued up front on three mbarriers (Q and K_in;
+//     V_in; the parts), so S and the softmax start while V_in and the parts
+//     are still arriving; the parts' L values are plain loads issued first;
 //   - S = Q K_in^T and O = P V on mma.sync m16n8k16 (bf16 in, fp32 out) with
 //     the block's keys padded to NB in {16, 32, 64}; P V uses a bf16 hi + lo
 //     split of P so the product keeps fp32-level accuracy;
-//   - the merge with up to four external parts reads them from shared memory
-//     and writes O (bf16 or fp32) and the merged natural-log LSE; on a full
-//     step it can also write the merged external part (the block-external
-//     attention combined over its key splits) into the cache.
+//   - the merge with NX (0..4, a template parameter) external parts reads
+//     them from shared memory; O rows (bf16 or fp32) and, on a full step, the
+//     merged external part for the cache are staged in shared memory and
+//     leave as whole-row bulk stores; LSE is written directly.
 #include <math_constants.h>
 
 #include "fb_internal.cuh"
+#include "fb_ptx.cuh"
 
 namespace fb {
 
 namespace {
 
-constexpr int kRows = 32;          // query rows per CTA
+constexpr int kRows = 16;          // query rows per CTA (one m16 tile)
 constexpr int kD = 128;
-constexpr int kExtStride = 132;    // fp32 row stride of staged external parts (bank spread)
+constexpr int kRowE = kD + 8;      // bf16 row stride of staged Q, K, V (272 bytes: conflict-free ldmatrix)
+constexpr int kExtStride = 132;    // fp32 row stride of staged parts and output rows (bank spread)
 constexpr int kMaxExt = 4;
 
-__device__ __forceinline__ uint32_t saddr(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
-__device__ __forceinline__ void cp16(uint32_t dst, const void* src, int bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(bytes));
-}
-__device__ __forceinline__ void cp4(uint32_t dst, const void* src, int bytes) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(dst), "l"(src), "r"(bytes));
-}
 __device__ __forceinline__ void ldsm4(uint32_t a, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(a));
@@ -63,8 +60,6 @@ __device__ __forceinline__ void split2(float x, float y, uint32_t& hi, uint32_t&
   const __nv_bfloat162 l = __floats2bfloat162_rn(x - hx, y - hy);
   lo = *reinterpret_cast<const uint32_t*>(&l);
 }
-// swizzled offset (elements) of 16-byte chunk `ch` of row `r` in a [rows][128] bf16 tile
-__device__ __forceinline__ int swz(int r, int ch) { return r * kD + ((ch ^ (r & 7)) << 3); }
 
 }  // namespace
 
@@ -86,93 +81,112 @@ struct InblockArgs {
   float* cache_a;     // non-null: also store merge(external parts) here (packed fp32)
   float* cache_l;
   float scale_log2;
+  int* status;
+  uint64_t wait_limit_ns;
 };
 
-template <int NB>
+// Bounded wait on phase 0 of a load barrier; the first expiry is recorded.
+__device__ __forceinline__ bool wait_loaded(uint32_t bar, const InblockArgs& a) {
+  if (ptx::mbar_test(bar, 0)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  while (!ptx::mbar_try(bar, 0)) {
+    if (ptx::globaltimer() - t0 > a.wait_limit_ns) {
+      atomicCAS(a.status, 0, (int)FB_ETIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+template <int NB, int NX>
 __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a) {
   constexpr int NT = NB / 8;     // key n-tiles of S
   constexpr int KK = NB / 16;    // key k-steps of P V
+  constexpr int NXS = NX > 0 ? NX : 1;
   extern __shared__ __align__(128) uint8_t sm[];
-  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(sm);             // [64][128]
-  __nv_bfloat16* sK = sQ + kRows * kD;                                   // [NB][128]
-  __nv_bfloat16* sV = sK + NB * kD;                                      // [NB][128]
-  float* sE = reinterpret_cast<float*>(sV + NB * kD);                    // [next][64][132]
-  float* sL = sE + kMaxExt * kRows * kExtStride;                         // [next][64]
+  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(sm);             // [16][kRowE]
+  __nv_bfloat16* sK = sQ + kRows * kRowE;                                // [NB][kRowE]
+  __nv_bfloat16* sV = sK + NB * kRowE;                                   // [NB][kRowE]
+  float* sE = reinterpret_cast<float*>(sV + NB * kRowE);                 // [NX][16][kExtStride]
+  float* sL = sE + NXS * kRows * kExtStride;                             // [NX][16]
+  float* sO = sL + NXS * kRows;                                          // [16][kExtStride] output rows
+  float* sC = sO + kRows * kExtStride;                                   // [16][kExtStride] cache rows
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + kRows * kExtStride);  // Q+K, V, parts
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int unit = blockIdx.x / a.tiles_per_unit, tile = blockIdx.x % a.tiles_per_unit;
   const int b = unit / a.Hkv, kvh = unit % a.Hkv;
   const int rows_unit = a.G * a.Nb;
   const int row0 = tile * kRows;
+  const int nq = min(kRows, rows_unit - row0);   // rows of this CTA that exist
   // packed row r -> (query head kvh*G + r / Nb, query r % Nb); the rows of one
   // KV head are consecutive in the packed (b, h, i) order of parts and LSE.
   const int64_t prow0 = ((int64_t)b * a.Hq + (int64_t)kvh * a.G) * a.Nb + row0;
+  const uint32_t bar_qk = ptx::smem_addr(bars), bar_v = bar_qk + 8, bar_e = bar_qk + 16;
 
+  // ---- every load is one bulk copy per row, issued up front ----
   if (tid == 0) {
-    // warm the address translation of the rows this CTA stores at the end
-    const int g = min(row0 / a.Nb, a.G - 1), i = row0 % a.Nb;
-    const size_t esz = a.o_bf16 ? 2 : 4;
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(static_cast<const char*>(a.o) +
-                                                  (b * a.o_sb + (int64_t)(kvh * a.G + g) * a.o_sh +
-                                                   (int64_t)i * a.o_st) * esz));
-    if (a.cache_a) asm volatile("prefetch.global.L2 [%0];" ::"l"(a.cache_a + prow0 * kD));
-    if (a.lse) asm volatile("prefetch.global.L2 [%0];" ::"l"(a.lse + prow0));
+    ptx::mbar_init(bar_qk, 1);
+    ptx::mbar_init(bar_v, 1);
+    ptx::mbar_init(bar_e, 1);
+    ptx::fence_mbar_init();
+    ptx::mbar_expect_tx(bar_qk, (uint32_t)(nq + a.Nb) * (kD * 2));
+    ptx::mbar_expect_tx(bar_v, (uint32_t)a.Nb * (kD * 2));
+    ptx::mbar_expect_tx(bar_e, (uint32_t)(NX * nq) * (kD * 4));
   }
-  // ---- one batch of asynchronous loads ----
-  for (int c = tid; c < kRows * 16; c += 128) {
-    const int r = c >> 4, ch = c & 15;
-    const int rr = row0 + r;
-    const bool ok = rr < rows_unit;
-    const int g = ok ? rr / a.Nb : 0, i = ok ? rr % a.Nb : 0;
-    const __nv_bfloat16* src = a.q + b * a.q_sb + (int64_t)(kvh * a.G + g) * a.q_sh + (int64_t)i * a.q_st + ch * 8;
-    cp16(saddr(sQ + swz(r, ch)), ok ? src : a.q, ok ? 16 : 0);
-  }
-  for (int c = tid; c < NB * 16; c += 128) {
-    const int r = c >> 4, ch = c & 15;
-    const bool ok = r < a.Nb;
-    const int64_t off = b * a.k_sb + (int64_t)kvh * a.k_sh + (int64_t)(ok ? r : 0) * a.k_st + ch * 8;
-    cp16(saddr(sK + swz(r, ch)), a.k + off, ok ? 16 : 0);
-  }
-  asm volatile("cp.async.commit_group;\n" ::: "memory");   // group: Q, K_in
-  for (int c = tid; c < NB * 16; c += 128) {
-    const int r = c >> 4, ch = c & 15;
-    const bool ok = r < a.Nb;
-    const int64_t off = b * a.k_sb + (int64_t)kvh * a.k_sh + (int64_t)(ok ? r : 0) * a.k_st + ch * 8;
-    cp16(saddr(sV + swz(r, ch)), a.v + off, ok ? 16 : 0);
-  }
-  asm volatile("cp.async.commit_group;\n" ::: "memory");   // group: V_in
-  for (int p = 0; p < a.next; ++p) {
-    for (int c = tid; c < kRows * 32; c += 128) {
-      const int r = c >> 5, ch = c & 31;
-      const bool ok = row0 + r < rows_unit;
-      cp16(saddr(sE + (p * kRows + r) * kExtStride + ch * 4), ok ? a.ext_a[p] + (prow0 + r) * kD + ch * 4 : a.ext_a[p],
-           ok ? 16 : 0);
-    }
-    for (int r = tid; r < kRows; r += 128) {
-      const bool ok = row0 + r < rows_unit;
-      cp4(saddr(sL + p * kRows + r), ok ? a.ext_l[p] + prow0 + r : a.ext_l[p], ok ? 4 : 0);
-    }
-  }
-  asm volatile("cp.async.commit_group;\ncp.async.wait_group 2;\n" ::: "memory");   // group: parts
+  float lx = -CUDART_INF_F;   // L of part tid / 16, row tid % 16 (read early, stored after P V)
+  if (tid < NX * kRows && (tid & 15) < nq) lx = a.ext_l[tid >> 4][prow0 + (tid & 15)];
   __syncthreads();
+  if (warp == 0) {
+    if (lane < kRows) {
+      const int r = lane;
+      if (r < nq) {
+        const int rr = row0 + r, g = rr / a.Nb, i = rr % a.Nb;
+        ptx::bulk_g2s(ptx::smem_addr(sQ + r * kRowE),
+                      a.q + b * a.q_sb + (int64_t)(kvh * a.G + g) * a.q_sh + (int64_t)i * a.q_st, kD * 2, bar_qk);
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < kD / 8; ++c) reinterpret_cast<uint4*>(sQ + r * kRowE)[c] = make_uint4(0, 0, 0, 0);
+      }
+    }
+  } else if (warp == 1 || warp == 2) {
+    const bool isk = warp == 1;
+    __nv_bfloat16* dst = isk ? sK : sV;
+    const __nv_bfloat16* src = (isk ? a.k : a.v) + b * a.k_sb + (int64_t)kvh * a.k_sh;
+#pragma unroll 1
+    for (int r = lane; r < NB; r += 32) {
+      if (r < a.Nb) {
+        ptx::bulk_g2s(ptx::smem_addr(dst + r * kRowE), src + (int64_t)r * a.k_st, kD * 2, isk ? bar_qk : bar_v);
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < kD / 8; ++c) reinterpret_cast<uint4*>(dst + r * kRowE)[c] = make_uint4(0, 0, 0, 0);
+      }
+    }
+  } else if (NX > 0) {
+    const int p = lane >> 4, r = lane & 15;
+#pragma unroll
+    for (int pp = 0; pp < NX; pp += 2)
+      if (pp + p < NX && r < nq)
+        ptx::bulk_g2s(ptx::smem_addr(sE + ((pp + p) * kRows + r) * kExtStride), a.ext_a[pp + p] + (prow0 + r) * kD,
+                      kD * 4, bar_e);
+  }
+  __syncthreads();   // zero-filled rows
+  bool ok = wait_loaded(bar_qk, a);
 
-  // ---- S = Q K^T for this warp's 16-row slab ----
-  const int slab = warp & 1, dh = warp >> 1;   // dh: which 64 columns of D this warp outputs
+  // ---- S = Q K^T for the CTA's 16 rows (every warp) ----
+  const int dq = warp;   // this warp's quarter of D: columns dq*32 .. dq*32+31
   float s[NT][4];
 #pragma unroll
   for (int n = 0; n < NT; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
 #pragma unroll
   for (int kk = 0; kk < kD / 16; ++kk) {
     uint32_t qa[4];
-    {
-      const int r = slab * 16 + (lane & 15), ch = 2 * kk + (lane >> 4);
-      ldsm4(saddr(sQ + swz(r, ch)), qa[0], qa[1], qa[2], qa[3]);
-    }
+    ldsm4(ptx::smem_addr(sQ + (lane & 15) * kRowE + (2 * kk + (lane >> 4)) * 8), qa[0], qa[1], qa[2], qa[3]);
 #pragma unroll
     for (int n = 0; n < NT; n += 2) {
       const int r = (n + (lane >> 4)) * 8 + (lane & 7), ch = 2 * kk + ((lane >> 3) & 1);
       uint32_t b0, b1, b2, b3;
-      ldsm4(saddr(sK + swz(r, ch)), b0, b1, b2, b3);
+      ldsm4(ptx::smem_addr(sK + r * kRowE + ch * 8), b0, b1, b2, b3);
       mma16816(s[n], qa, b0, b1);
       if (n + 1 < NT) mma16816(s[n + 1], qa, b2, b3);
     }
@@ -208,10 +222,9 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
     lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 1);
     lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 2);
   }
-  asm volatile("cp.async.wait_group 1;\n" ::: "memory");
-  __syncthreads();
-  // ---- O[:, dh*64 : dh*64+64] = P V ----
-  constexpr int DT = kD / 16;    // 8-column tiles in this warp's half
+  ok = wait_loaded(bar_v, a) && ok;
+  // ---- O[:, dq*32 : dq*32+32] = P V ----
+  constexpr int DT = 4;    // 8-column tiles in this warp's quarter
   float o[DT][4];
 #pragma unroll
   for (int d = 0; d < DT; ++d) o[d][0] = o[d][1] = o[d][2] = o[d][3] = 0.f;
@@ -221,36 +234,37 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
     const uint32_t al[4] = {pl[2 * kk][0], pl[2 * kk][1], pl[2 * kk + 1][0], pl[2 * kk + 1][1]};
 #pragma unroll
     for (int d = 0; d < DT; d += 2) {
-      const int r = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8, ch = dh * DT + d + (lane >> 4);
+      const int r = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8, ch = dq * DT + d + (lane >> 4);
       uint32_t b0, b1, b2, b3;
-      ldsm4t(saddr(sV + swz(r, ch)), b0, b1, b2, b3);
+      ldsm4t(ptx::smem_addr(sV + r * kRowE + ch * 8), b0, b1, b2, b3);
       mma16816(o[d], ah, b0, b1);
       mma16816(o[d + 1], ah, b2, b3);
       mma16816(o[d], al, b0, b1);
       mma16816(o[d + 1], al, b2, b3);
     }
   }
-  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
-  __syncthreads();
-  // ---- merge with the external parts and store ----
+  if (tid < NX * kRows) sL[tid] = lx;
+  ok = wait_loaded(bar_e, a) && ok;
+  __syncthreads();   // sL
+  // ---- merge with the external parts; rows staged for whole-row stores ----
+  const bool obf = a.o_bf16 != 0;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const int r = slab * 16 + (lane >> 2) + 8 * h;
-    const int rr = row0 + r;
-    if (rr >= rows_unit) continue;
+    const int r = (lane >> 2) + 8 * h;
+    if (r >= nq) continue;
     const float Lin = lrow[h] > 0.f ? (mrow[h] + __log2f(lrow[h])) * kLn2 : -CUDART_INF_F;
-    float Lx[kMaxExt];
     float m = Lin;
+    float Lx[NXS];
 #pragma unroll
-    for (int p = 0; p < kMaxExt; ++p) {
-      Lx[p] = p < a.next ? sL[p * kRows + r] : -CUDART_INF_F;
+    for (int p = 0; p < NX; ++p) {
+      Lx[p] = sL[p * kRows + r];
       m = fmaxf(m, Lx[p]);
     }
     const bool empty = m == -CUDART_INF_F;
     const float w_in = (empty || Lin == -CUDART_INF_F) ? 0.f : __expf(Lin - m);
-    float wx[kMaxExt], wext = 0.f;
+    float wx[NXS], wext = 0.f;
 #pragma unroll
-    for (int p = 0; p < kMaxExt; ++p) {
+    for (int p = 0; p < NX; ++p) {
       wx[p] = (empty || Lx[p] == -CUDART_INF_F) ? 0.f : __expf(Lx[p] - m);
       wext += wx[p];
     }
@@ -258,34 +272,58 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
     const float inv = empty ? 0.f : 1.f / wsum;
     const float inv_ext = wext > 0.f ? 1.f / wext : 0.f;
     const float win = lrow[h] > 0.f ? w_in / lrow[h] : 0.f;
-    const int g = rr / a.Nb, i = rr % a.Nb;
-    const int64_t obase = b * a.o_sb + (int64_t)(kvh * a.G + g) * a.o_sh + (int64_t)i * a.o_st;
 #pragma unroll
     for (int d = 0; d < DT; ++d) {
-      const int col = dh * 64 + d * 8 + 2 * (lane & 3);
-      float ex = 0.f, ey = 0.f;   // sum of w_p A_p over the external parts
+      const int col = dq * 32 + d * 8 + 2 * (lane & 3);
+      float ex = 0.f, ey = 0.f;   // sum of w_p A_p over the external parts (a part with w = 0 may hold -inf rows)
 #pragma unroll
-      for (int p = 0; p < kMaxExt; ++p) {
-        if (wx[p] == 0.f) continue;
+      for (int p = 0; p < NX; ++p) {
         const float2 e = *reinterpret_cast<const float2*>(sE + (p * kRows + r) * kExtStride + col);
-        ex = fmaf(wx[p], e.x, ex);
-        ey = fmaf(wx[p], e.y, ey);
+        ex = wx[p] == 0.f ? ex : fmaf(wx[p], e.x, ex);
+        ey = wx[p] == 0.f ? ey : fmaf(wx[p], e.y, ey);
       }
-      if (a.cache_a)
-        *reinterpret_cast<float2*>(a.cache_a + (prow0 + r) * kD + col) = make_float2(ex * inv_ext, ey * inv_ext);
+      if (a.cache_a) *reinterpret_cast<float2*>(sC + r * kExtStride + col) = make_float2(ex * inv_ext, ey * inv_ext);
       const float x = (win * o[d][2 * h] + ex) * inv, y = (win * o[d][2 * h + 1] + ey) * inv;
-      if (a.o_bf16)
-        *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(a.o) + obase + col) = __floats2bfloat162_rn(x, y);
+      if (obf)
+        reinterpret_cast<__nv_bfloat162*>(sO + r * kExtStride)[col >> 1] = __floats2bfloat162_rn(x, y);
       else
-        *reinterpret_cast<float2*>(static_cast<float*>(a.o) + obase + col) = make_float2(x, y);
+        *reinterpret_cast<float2*>(sO + r * kExtStride + col) = make_float2(x, y);
     }
-    if (a.cache_l && dh == 0 && (lane & 3) == 0)
-      a.cache_l[prow0 + r] = wext > 0.f ? m + logf(wext) : -CUDART_INF_F;
-    if (a.lse && dh == 0 && (lane & 3) == 0) a.lse[prow0 + r] = empty ? -CUDART_INF_F : m + logf(wsum);
+    if (dq == 0 && (lane & 3) == 0) {
+      if (a.cache_l) a.cache_l[prow0 + r] = wext > 0.f ? m + logf(wext) : -CUDART_INF_F;
+      if (a.lse) a.lse[prow0 + r] = empty ? -CUDART_INF_F : m + logf(wsum);
+    }
+  }
+  ptx::fence_proxy_async_smem();
+  __syncthreads();
+  // ---- whole-row stores: lanes 0..15 the output rows, 16..31 the cache rows (warp 0) ----
+  if (ok && warp == 0) {
+    const int r = lane & 15;
+    if (r < nq && lane < 16) {
+      const int rr = row0 + r, g = rr / a.Nb, i = rr % a.Nb;
+      const int64_t obase = b * a.o_sb + (int64_t)(kvh * a.G + g) * a.o_sh + (int64_t)i * a.o_st;
+      void* dst = obf ? static_cast<void*>(static_cast<__nv_bfloat16*>(a.o) + obase)
+                      : static_cast<void*>(static_cast<float*>(a.o) + obase);
+      ptx::bulk_s2g(dst, ptx::smem_addr(sO + r * kExtStride), obf ? kD * 2 : kD * 4);
+      ptx::bulk_commit();
+    } else if (r < nq && a.cache_a) {
+      ptx::bulk_s2g(a.cache_a + (prow0 + r) * kD, ptx::smem_addr(sC + r * kExtStride), kD * 4);
+      ptx::bulk_commit();
+    }
+    ptx::bulk_wait_read();
+  }
+  if (!ok && tid == 0) {
+    // a load wait expired: let every copy into shared memory land before exit
+    wait_loaded(bar_qk, a);
+    wait_loaded(bar_v, a);
+    wait_loaded(bar_e, a);
   }
 }
 
 // ------------------------------------------------------------------ host --
+int* device_status_ptr();
+uint64_t wait_limit_ns();
+
 bool inblock_small_applies(const fb_attn_desc& d, int next) {
   return d.in_dtype == FB_BF16 && d.D == kD && d.Nb <= 64 && next <= kMaxExt;
 }
@@ -310,22 +348,34 @@ cudaError_t launch_inblock_small(const fb_attn_desc& d, const void* q, const voi
   a.cache_a = cache_a;
   a.cache_l = cache_l;
   a.scale_log2 = scale_log2;
+  a.status = device_status_ptr();
+  a.wait_limit_ns = wait_limit_ns();
+  if (!a.status) return cudaErrorInvalidValue;
   const int NB = d.Nb <= 16 ? 16 : d.Nb <= 32 ? 32 : 64;
-  const size_t smem = (size_t)(kRows + 2 * NB) * kD * 2 + (size_t)kMaxExt * kRows * (kExtStride + 1) * 4;
+  const int nxs = next > 0 ? next : 1;
+  const size_t smem = (size_t)(kRows + 2 * NB) * kRowE * 2 + (size_t)nxs * kRows * (kExtStride + 1) * 4 +
+                      2 * (size_t)kRows * kExtStride * 4 + 3 * 8;
   const dim3 grid(d.B * d.Hkv * a.tiles_per_unit);
-  static bool attr[3] = {false, false, false};
-  auto run = [&](auto kern, int idx) -> cudaError_t {
-    if (!attr[idx]) {
+  // instances above the default 48 KB of dynamic shared memory opt in once
+  static bool opted[3][kMaxExt + 1] = {};
+  auto run = [&](void (*kern)(InblockArgs), int nbi) -> cudaError_t {
+    if (smem > 48 * 1024 && !opted[nbi][next]) {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
-      attr[idx] = true;
+      opted[nbi][next] = true;
     }
     kern<<<grid, 128, smem, s>>>(a);
     return cudaGetLastError();
   };
-  if (NB == 16) return run(inblock_small_kernel<16>, 0);
-  if (NB == 32) return run(inblock_small_kernel<32>, 1);
-  return run(inblock_small_kernel<64>, 2);
+#define FB_INB_CASE(nb, nx) \
+  if (NB == nb && next == nx) return run(inblock_small_kernel<nb, nx>, nb == 16 ? 0 : nb == 32 ? 1 : 2);
+#define FB_INB_NB(nb) FB_INB_CASE(nb, 0) FB_INB_CASE(nb, 1) FB_INB_CASE(nb, 2) FB_INB_CASE(nb, 3) FB_INB_CASE(nb, 4)
+  FB_INB_NB(16)
+  FB_INB_NB(32)
+  FB_INB_NB(64)
+#undef FB_INB_NB
+#undef FB_INB_CASE
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace fb

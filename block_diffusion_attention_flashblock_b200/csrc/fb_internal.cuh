@@ -105,7 +105,9 @@ struct TcMaps {
   int mode, hg, tiles_per_unit, units;
 };
 bool tc_tiling(const fb_attn_desc& d, int* mode, int* hg, int* tiles_per_unit, int* units);
-bool tc_make_maps(const fb_attn_desc& d, const void* q, const void* kp, const void* vp, int64_t nkeys, TcMaps* m);
+// Tensor maps for a pass over keys [0, nkeys) of K/V with (b, h, t) strides kstr.
+bool tc_make_maps(const fb_attn_desc& d, const void* q, const void* k, const void* v, int64_t nkeys,
+                  const int64_t* kstr, TcMaps* m);
 void tc_plan_split(int64_t tiles, int64_t nkeys, int32_t max_parts, bool allow_cluster, int32_t* nsplit,
                    int64_t* kps, int32_t* cluster, int32_t* nparts);
 int32_t tc_split_cap(int64_t tiles, int64_t max_keys);
