@@ -167,6 +167,7 @@ def run_ours(args, spec, rank, world, device):
     from block_diffusion_attention_flashblock_b200 import fb
     torch.cuda.set_device(device)
     fb.fb_debug_set_prefix_kernel({"auto": 0, "generic": 1, "tcgen05": 2, "tcgen05-nocluster": 3}[args.prefix_kernel])
+    fb.fb_debug_set_pdl(not args.no_pdl)
     nl = n_layers(spec)
     S = Layers(spec, device, nl)
     s = spec
@@ -349,6 +350,7 @@ def run_ours(args, spec, rank, world, device):
         "config": {"workload": _describe(spec), "layers": nl,
                    "query_tokens_per_step": S.query_tokens,
                    "prefix_kernel": args.prefix_kernel, "diffusion_steps_per_layer": nsteps,
+                   "programmatic_dependent_launch": not args.no_pdl,
                    "l2": f"flushed (1 GiB write) before every timed step; inside it {nl} layers with their own "
                          f"KV caches are stepped in turn, so each layer's data has left L2 when it runs",
                    "parallelism": f"replicas x{world}", "full_steps_per_layer": n_full},
@@ -437,6 +439,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="dllm_8k", choices=list(wl.SPECS))
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-pdl", action="store_true", help="launch kernels in plain stream order")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--prefix-kernel", default="auto", choices=["auto", "generic", "tcgen05", "tcgen05-nocluster"])
     ap.add_argument("--profile-run", action="store_true",

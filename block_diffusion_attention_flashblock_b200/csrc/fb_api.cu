@@ -20,6 +20,8 @@ __device__ int g_fb_status = 0;
 
 static uint64_t g_wait_limit_ns = 2000000000ull;
 uint64_t wait_limit_ns() { return g_wait_limit_ns; }
+static bool g_pdl = true;
+bool pdl_enabled() { return g_pdl; }
 
 int* device_status_ptr() {
   int* p = nullptr;
@@ -315,14 +317,20 @@ static fb_status run_inblock(const fb_attn_desc& d, const void* q, const void* k
   a.nsplit = 1;
   a.keys_per_split = d.Nb;
   a.merge_out = 1;
-  a.next = 0;
+  // the external parts, flattened (the small kernel takes up to 4)
+  const float* fa[FB_MAX_PARTS];
+  const float* fl[FB_MAX_PARTS];
+  int nflat = 0;
   for (int gi = 0; gi < ext.ngroups; ++gi)
     for (int p = 0; p < ext.g[gi].count; ++p) {
-      if (a.next >= FB_MAX_PARTS) return FB_EINVAL;
-      a.ext_a[a.next] = ext.g[gi].a + p * ext.g[gi].stride_a;
-      a.ext_l[a.next] = ext.g[gi].l + p * ext.g[gi].stride_l;
-      ++a.next;
+      if (nflat < FB_MAX_PARTS) {
+        fa[nflat] = ext.g[gi].a + p * ext.g[gi].stride_a;
+        fl[nflat] = ext.g[gi].l + p * ext.g[gi].stride_l;
+      }
+      ++nflat;
     }
+  a.next = std::min(nflat, (int)FB_MAX_PARTS);
+  for (int i = 0; i < a.next; ++i) { a.ext_a[i] = fa[i]; a.ext_l[i] = fl[i]; }
   a.o = o; a.o_sb = d.o_strides[0]; a.o_sh = d.o_strides[1]; a.o_st = d.o_strides[2];
   a.o_bf16 = d.out_dtype == FB_BF16;
   a.lse = lse;
@@ -332,13 +340,14 @@ static fb_status run_inblock(const fb_attn_desc& d, const void* q, const void* k
   const double bytes = (double)rows_of(d) * d.D * es + 2.0 * d.B * d.Hkv * d.Nb * d.D * es +
                        ext_parts * rows_of(d) * (d.D + 1) * 4.0 +
                        (double)rows_of(d) * (d.D * esize(d.out_dtype) + (lse ? 4 : 0));
-  if (inblock_small_applies(d, a.next)) {
+  if (inblock_small_applies(d, nflat)) {
     ProfScope prof(kProfInblock, bytes, s);
-    return launch_inblock_small(d, q, kin, vin, a.next, a.ext_a, a.ext_l, o, lse, cache_a, cache_l, a.scale_log2,
-                                s) == cudaSuccess
+    return launch_inblock_small(d, q, kin, vin, nflat, fa, fl, o, lse, cache_a, cache_l, a.scale_log2, s) ==
+                   cudaSuccess
                ? FB_OK
                : FB_ECUDA;
   }
+  if (nflat > FB_MAX_PARTS) return FB_EINVAL;
   if (cache_a) return FB_EUNSUPPORTED;   // callers only ask for the cache write where the small kernel runs
   TcMaps maps;
   if (ws_a && ws_cap >= 1 && g_prefix_kernel != 1 && d.Nb >= 128 && ext.ngroups < 8 &&
@@ -554,6 +563,11 @@ fb_status fb_profile_read(int32_t reset, int64_t* launches, double* total_ms, do
 fb_status fb_debug_set_prefix_kernel(int32_t which) {
   if (which < 0 || which > 3) return FB_EINVAL;
   g_prefix_kernel = which;
+  return FB_OK;
+}
+
+fb_status fb_debug_set_pdl(int32_t on) {
+  g_pdl = on != 0;
   return FB_OK;
 }
 

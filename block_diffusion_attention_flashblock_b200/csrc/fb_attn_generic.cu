@@ -16,6 +16,7 @@
 // Both take the same AttnArgs; numerics: scores in the log2 domain
 // (s * scale * log2 e), online max/sum per row, exp2f, fp32 accumulation.
 #include "fb_internal.cuh"
+#include "fb_ptx.cuh"
 #include <math_constants.h>
 
 namespace fb {
@@ -144,6 +145,7 @@ __device__ __forceinline__ RowMerge row_merge(int next, const float* Lx, float L
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
+  ptx::pdl_prologue();
   constexpr int BM = 64, BN = 64, CH = D / 8, NT = BN / 8, DT = D / 8, KS = D / 16;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem_raw);
@@ -410,6 +412,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(64 * (D / 64)) attn_f32_kernel(const AttnArgs a) {
+  ptx::pdl_prologue();
   constexpr int TPR = D / 64, BM = 64, BN = 32, DH = 64;
   constexpr int NTH = BM * TPR;
   __shared__ __align__(16) float sK[BN * D];
@@ -541,16 +544,14 @@ static cudaError_t launch_mma(const AttnArgs& a, cudaStream_t s) {
     attr_set = true;
   }
   dim3 grid(a.rm.units * a.rm.row_tiles, a.nsplit);
-  attn_mma_kernel<D><<<grid, 128, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_k(attn_mma_kernel<D>, grid, dim3(128), smem, s, a);
 }
 
 cudaError_t launch_attn_generic(const AttnArgs& a, int D, int in_bf16, cudaStream_t s) {
   if (in_bf16) return D == 64 ? launch_mma<64>(a, s) : launch_mma<128>(a, s);
   dim3 grid(a.rm.units * a.rm.row_tiles, a.nsplit);
-  if (D == 64) attn_f32_kernel<64><<<grid, 64, 0, s>>>(a);
-  else attn_f32_kernel<128><<<grid, 128, 0, s>>>(a);
-  return cudaGetLastError();
+  if (D == 64) return launch_k(attn_f32_kernel<64>, grid, dim3(64), 0, s, a);
+  return launch_k(attn_f32_kernel<128>, grid, dim3(128), 0, s, a);
 }
 
 }  // namespace fb

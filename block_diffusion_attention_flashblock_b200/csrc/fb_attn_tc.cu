@@ -301,6 +301,7 @@ struct TcArgs {
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
+  ptx::pdl_prologue();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   if (smem - smem_raw > (ptrdiff_t)kSmemSlack) {   // the layout would not fit: report, touch nothing
@@ -814,22 +815,21 @@ cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys
     attr = true;
   }
   dim3 grid(m.units * m.tiles_per_unit, nsplit);
-  if (a.cluster <= 1) {
-    attn_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(m.q, m.k, m.v, a);
-    return cudaGetLastError();
-  }
+  if (a.cluster <= 1) return launch_k(attn_tc_kernel, grid, dim3(kThreads), kSmemBytes, s, m.q, m.k, m.v, a);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = s;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = 1;
   at[0].val.clusterDim.y = (unsigned)cluster;
   at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, attn_tc_kernel, m.q, m.k, m.v, a);
 }
 

@@ -3,6 +3,7 @@
 // bitmap (FlashBlock summary, "Mécanisme Central" and "Stratégies de
 // Réutilisation Adaptatives").
 #include "fb_internal.cuh"
+#include "fb_ptx.cuh"
 #include <math_constants.h>
 
 namespace fb {
@@ -104,6 +105,7 @@ __device__ __forceinline__ float merge_row(const PartList& pl, int64_t row, int 
 // One warp per (b, h, i) row.
 template <int D>
 __global__ void __launch_bounds__(256) merge_kernel(const MergeArgs m) {
+  ptx::pdl_prologue();
   constexpr int E = D / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * 8 + warp;
@@ -122,9 +124,8 @@ cudaError_t launch_merge(const MergeArgs& m, cudaStream_t s) {
   const int64_t nrows = (int64_t)m.B * m.Hq * m.Nb;
   const unsigned grid = (unsigned)((nrows + 7) / 8);
   if (grid == 0) return cudaSuccess;
-  if (m.D == 64) merge_kernel<64><<<grid, 256, 0, s>>>(m);
-  else merge_kernel<128><<<grid, 256, 0, s>>>(m);
-  return cudaGetLastError();
+  if (m.D == 64) return launch_k(merge_kernel<64>, grid, dim3(256), 0, s, m);
+  return launch_k(merge_kernel<128>, grid, dim3(256), 0, s, m);
 }
 
 // ---------------------------------------------------------------------------
@@ -141,6 +142,7 @@ int gamma_chunk_rows() { return kGammaRows; }
 
 template <int D>
 __global__ void __launch_bounds__(256) gamma_update_kernel(const GammaArgs g) {
+  ptx::pdl_prologue();
   constexpr int E = D / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y, chunk = blockIdx.x;
@@ -213,9 +215,8 @@ __global__ void __launch_bounds__(256) gamma_update_kernel(const GammaArgs g) {
 
 cudaError_t launch_gamma_update(const GammaArgs& g, cudaStream_t s) {
   dim3 grid(g.chunks, g.B * g.Hq);
-  if (g.D == 64) gamma_update_kernel<64><<<grid, 256, 0, s>>>(g);
-  else gamma_update_kernel<128><<<grid, 256, 0, s>>>(g);
-  return cudaGetLastError();
+  if (g.D == 64) return launch_k(gamma_update_kernel<64>, grid, dim3(256), 0, s, g);
+  return launch_k(gamma_update_kernel<128>, grid, dim3(256), 0, s, g);
 }
 
 // ---------------------------------------------------------------------------
@@ -226,6 +227,7 @@ __global__ void kv_append_kernel(uint8_t* kp, uint8_t* vp, const uint8_t* kin, c
                                  int32_t Hkv, int32_t Nb, int32_t vec_per_row, int64_t rows,
                                  int64_t kp_sb, int64_t kp_sh, int64_t kp_st, int64_t kin_sb,
                                  int64_t kin_sh, int64_t kin_st, int64_t prefix_len) {
+  ptx::pdl_prologue();
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= rows * vec_per_row) return;
   const int64_t r = idx / vec_per_row;
@@ -248,17 +250,18 @@ cudaError_t launch_kv_append(const fb_attn_desc& d, void* kp, void* vp, int64_t 
   const int64_t n = rows * vec;
   const int threads = 256;
   const unsigned grid = (unsigned)((n + threads - 1) / threads);
-  kv_append_kernel<<<grid, threads, 0, s>>>(
-      static_cast<uint8_t*>(kp), static_cast<uint8_t*>(vp), static_cast<const uint8_t*>(kin),
-      static_cast<const uint8_t*>(vin), d.Hkv, d.Nb, vec, rows, d.kp_strides[0] * es, d.kp_strides[1] * es,
-      d.kp_strides[2] * es, d.kin_strides[0] * es, d.kin_strides[1] * es, d.kin_strides[2] * es, prefix_len);
-  return cudaGetLastError();
+  return launch_k(kv_append_kernel, dim3(grid), dim3(threads), 0, s, static_cast<uint8_t*>(kp),
+                  static_cast<uint8_t*>(vp), static_cast<const uint8_t*>(kin), static_cast<const uint8_t*>(vin),
+                  (int32_t)d.Hkv, (int32_t)d.Nb, (int32_t)vec, rows, d.kp_strides[0] * es, d.kp_strides[1] * es,
+                  d.kp_strides[2] * es, d.kin_strides[0] * es, d.kin_strides[1] * es, d.kin_strides[2] * es,
+                  prefix_len);
 }
 
 // ---------------------------------------------------------------------------
 // Sparse membership bitmap: bit j of (b, h) set iff j is in sel[b, h, :].
 // ---------------------------------------------------------------------------
 __global__ void build_bitmap_kernel(const int32_t* sel, int32_t sel_k, uint32_t* bitmap, int64_t words) {
+  ptx::pdl_prologue();
   const int64_t bh = blockIdx.x;
   uint32_t* w = bitmap + bh * words;
   for (int64_t j = threadIdx.x; j < words; j += blockDim.x) w[j] = 0u;
@@ -272,8 +275,7 @@ __global__ void build_bitmap_kernel(const int32_t* sel, int32_t sel_k, uint32_t*
 
 cudaError_t launch_build_bitmap(const int32_t* sel, int32_t sel_k, int32_t BH, uint32_t* bitmap,
                                 int64_t words, cudaStream_t s) {
-  build_bitmap_kernel<<<BH, 256, 0, s>>>(sel, sel_k, bitmap, words);
-  return cudaGetLastError();
+  return launch_k(build_bitmap_kernel, dim3(BH), dim3(256), 0, s, sel, sel_k, bitmap, words);
 }
 
 cudaError_t launch_fill_decision(int8_t* reuse_out, int32_t n, int8_t value, cudaStream_t s) {

@@ -100,6 +100,7 @@ __device__ __forceinline__ bool wait_loaded(uint32_t bar, const InblockArgs& a) 
 
 template <int NB, int NX>
 __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a) {
+  ptx::pdl_prologue();
   constexpr int NT = NB / 8;     // key n-tiles of S
   constexpr int KK = NB / 16;    // key k-steps of P V
   constexpr int NXS = NX > 0 ? NX : 1;
@@ -134,8 +135,14 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
     ptx::mbar_expect_tx(bar_v, (uint32_t)a.Nb * (kD * 2));
     ptx::mbar_expect_tx(bar_e, (uint32_t)(NX * nq) * (kD * 4));
   }
-  float lx = -CUDART_INF_F;   // L of part tid / 16, row tid % 16 (read early, stored after P V)
-  if (tid < NX * kRows && (tid & 15) < nq) lx = a.ext_l[tid >> 4][prow0 + (tid & 15)];
+  // L of (part, row) = (idx / 16, idx % 16) for idx = tid, tid + 128: read
+  // early, stored to shared memory after P V
+  float lx[2] = {-CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int idx = tid + k * 128;
+    if (idx < NX * kRows && (idx & 15) < nq) lx[k] = a.ext_l[idx >> 4][prow0 + (idx & 15)];
+  }
   __syncthreads();
   if (warp == 0) {
     if (lane < kRows) {
@@ -243,7 +250,9 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
       mma16816(o[d + 1], al, b2, b3);
     }
   }
-  if (tid < NX * kRows) sL[tid] = lx;
+#pragma unroll
+  for (int k = 0; k < 2; ++k)
+    if (tid + k * 128 < NX * kRows) sL[tid + k * 128] = lx[k];
   ok = wait_loaded(bar_e, a) && ok;
   __syncthreads();   // sL
   // ---- merge with the external parts; rows staged for whole-row stores ----
@@ -364,8 +373,7 @@ cudaError_t launch_inblock_small(const fb_attn_desc& d, const void* q, const voi
       if (e != cudaSuccess) return e;
       opted[nbi][next] = true;
     }
-    kern<<<grid, 128, smem, s>>>(a);
-    return cudaGetLastError();
+    return launch_k(kern, grid, dim3(128), smem, s, a);
   };
 #define FB_INB_CASE(nb, nx) \
   if (NB == nb && next == nx) return run(inblock_small_kernel<nb, nx>, nb == 16 ? 0 : nb == 32 ? 1 : 2);

@@ -87,6 +87,26 @@ class ProfScope {
   cudaEvent_t start_ = nullptr;
 };
 
+// Kernel launch with programmatic dependent launch allowed (when enabled):
+// the next kernel in the stream may start its launch while this one drains;
+// every kernel begins with ptx::pdl_prologue(), so it touches no global
+// memory before the kernels it depends on have completed.
+bool pdl_enabled();
+template <class... KArgs, class... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 // Host-side planning helpers (fb_api.cu).
 int num_sms();
 RowMap make_rowmap(int B, int Hq, int Hkv, int Nb, int per_head, int tile_rows);

@@ -269,6 +269,13 @@ fb_status fb_debug_set_prefix_kernel(int32_t which);
  * expire at once.  Affects only the calling process. */
 fb_status fb_debug_set_wait_limit_ns(uint64_t ns);
 
+/* Tuning hook: 1 (default) launches every kernel with programmatic dependent
+ * launch allowed, so a kernel's launch overlaps the tail of the one before it
+ * in the stream (each kernel waits for its predecessors before it touches
+ * global memory); 0 launches them in plain stream order.  Affects only the
+ * calling process. */
+fb_status fb_debug_set_pdl(int32_t on);
+
 #ifdef __cplusplus
 }
 #endif
