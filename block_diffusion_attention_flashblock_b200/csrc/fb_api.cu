@@ -225,6 +225,8 @@ struct PrefixPlan {
   int64_t kps;
   PassPlan gen;
   TcMaps maps;
+  const uint32_t* excl;   // non-null: per (b, query head) bitmap of keys the pass leaves out
+  int64_t excl_words;
 };
 
 static PrefixPlan plan_prefix(const fb_attn_desc& d, const void* q, const void* kp, const void* vp, int64_t nkeys,
@@ -235,6 +237,8 @@ static PrefixPlan plan_prefix(const fb_attn_desc& d, const void* q, const void* 
   p.nsplit = p.nparts = p.gen.nsplit;
   p.cluster = 1;
   p.kps = p.gen.a.keys_per_split;
+  p.excl = nullptr;
+  p.excl_words = 0;
   const int64_t min_keys = g_prefix_kernel >= 2 ? 1 : 256;
   if (g_prefix_kernel != 1 && nkeys >= min_keys && tc_make_maps(d, q, kp, vp, nkeys, d.kp_strides, &p.maps)) {
     tc_plan_split((int64_t)p.maps.units * p.maps.tiles_per_unit, nkeys, cap, g_prefix_kernel != 3, &p.nsplit,
@@ -249,13 +253,16 @@ static fb_status launch_prefix(const fb_attn_desc& d, PrefixPlan& p, int64_t nke
   if (!p.tc) {
     p.gen.a.mask = mask;
     p.gen.a.mask_active = mask_active;
+    p.gen.a.excl = p.excl;
+    p.gen.a.excl_words = p.excl_words;
     return launch_pass(d, p.gen.a, pa, pl, s);
   }
   const int es = esize(d.in_dtype);
   const double bytes = 2.0 * d.B * d.Hkv * (double)nkeys * d.D * es + (double)rows_of(d) * d.D * es +
                        (double)rows_of(d) * (d.D + 1) * 4;
   ProfScope prof(kProfPrefix, bytes, s);
-  return launch_attn_tc(d, p.maps, nkeys, p.nsplit, p.kps, p.cluster, mask, mask_active, scale_log2(d), pa, pl, s) ==
+  return launch_attn_tc(d, p.maps, nkeys, p.nsplit, p.kps, p.cluster, mask, mask_active, scale_log2(d), pa, pl, s,
+                        p.excl, p.excl_words) ==
                  cudaSuccess
              ? FB_OK
              : FB_ECUDA;
@@ -453,15 +460,15 @@ fb_status fb_attn_outblock(const fb_attn_desc* d, const void* q, const void* kp,
   if (!sel || !a_res) return FB_OK;
   // pass 2: the residual (prefix minus the selection)
   if (launch_build_bitmap(sel, sel_k, d->B * d->Hq, bitmap, words, stream) != cudaSuccess) return FB_ECUDA;
-  PassPlan r = plan_pass(*d, q, kp, vp, d->kp_strides, prefix_len, nullptr, 0, cap);
-  r.a.excl = bitmap;
-  r.a.excl_words = words;
-  if (r.nsplit == 1) return launch_pass(*d, r.a, a_res, l_res, stream);
-  if ((st = launch_pass(*d, r.a, pa, pl, stream)) != FB_OK) return st;
+  PrefixPlan r = plan_prefix(*d, q, kp, vp, prefix_len, cap);
+  r.excl = bitmap;
+  r.excl_words = words;
+  if (r.nparts == 1) return launch_prefix(*d, r, prefix_len, nullptr, 0, a_res, l_res, stream);
+  if ((st = launch_prefix(*d, r, prefix_len, nullptr, 0, pa, pl, stream)) != FB_OK) return st;
   PartList lst;
   memset(&lst, 0, sizeof(lst));
   lst.ngroups = 1;
-  lst.g[0] = group_of(pa, pl, r.nsplit, *d);
+  lst.g[0] = group_of(pa, pl, r.nparts, *d);
   return merge_to_part(*d, lst, a_res, l_res, nullptr, 0, stream);
 }
 
@@ -760,18 +767,12 @@ fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
     }
     if (!tau_reuse) {
       // dense: the whole prefix; sparse: the prefix minus each head's selection
-      PrefixPlan p;
+      PrefixPlan p = plan_prefix(d, a->q, a->kp, a->vp, a->prefix_len, c->part_cap);
       if (sparse) {
-        p.tc = false;
-        p.gen = plan_pass(d, a->q, a->kp, a->vp, d.kp_strides, a->prefix_len, nullptr, 0, c->part_cap);
-        p.nsplit = p.nparts = p.gen.nsplit;
-        p.cluster = 1;
         if (launch_build_bitmap(a->sel, a->sel_k, BH, c->bitmap, (a->prefix_len + 31) / 32, s) != cudaSuccess)
           return FB_ECUDA;
-        p.gen.a.excl = c->bitmap;
-        p.gen.a.excl_words = (a->prefix_len + 31) / 32;
-      } else {
-        p = plan_prefix(d, a->q, a->kp, a->vp, a->prefix_len, c->part_cap);
+        p.excl = c->bitmap;
+        p.excl_words = (a->prefix_len + 31) / 32;
       }
       // the in-block kernel can take the split parts itself and write their
       // merge into the cache, saving a merge pass

@@ -296,6 +296,8 @@ struct TcArgs {
   uint64_t wait_limit_ns;
   uint32_t q_bytes;        // bytes of one Q half-box (64 columns)
   int32_t cluster;         // > 1: clusters of this many consecutive splits reduce in-kernel
+  const uint32_t* excl;    // non-null: per (b, query head) bitmap of excluded keys (sparse residual pass)
+  int64_t excl_words;
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -480,8 +482,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       theirs = xch[(slot * 2 + (half ^ 1)) * kBM + row];
       return true;
     };
+    // sparse residual pass: this row's bitmap of excluded keys (a padding row
+    // reads the tile's last real row, whose result is discarded)
+    const uint32_t* exrow = nullptr;
+    if (a.excl) {
+      const int rr = min(row, nrows - 1);
+      const int hh = a.mode == 0 ? kvh * a.G + t * a.hg + rr / a.Nb : h0;
+      exrow = a.excl + ((int64_t)b * a.Hq + hh) * a.excl_words;
+    }
     for (int j = 0; j < T && ok; ++j) {
       const int sb = j % kSBuf;
+      const int64_t key0 = kbeg + (int64_t)j * kBN;
+      uint32_t ex0 = 0u, ex1 = 0u;   // exclusion bits of this thread's 64 keys, loaded before the wait
+      if (exrow) {
+        const int64_t w0 = (key0 + half * 64) >> 5;
+        if (w0 < a.excl_words) ex0 = __ldg(exrow + w0);
+        if (w0 + 1 < a.excl_words) ex1 = __ldg(exrow + w0 + 1);
+      }
       ok = uniform(wait_phase(bar(B_SFULL + sb), (j / kSBuf) & 1, ctl));
       if (!ok) break;
       tc_fence_after();
@@ -489,12 +506,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(tl + sb * kBN + half * 64, s);
       tmem_ld32(tl + sb * kBN + half * 64 + 32, s + 32);
       tmem_wait_ld();
-      const int64_t key0 = kbeg + (int64_t)j * kBN;
       const int nvalid = (int)min((int64_t)kBN, kend - key0) - half * 64;
       if (nvalid < 64) {   // only the last tile of the last split is ragged
 #pragma unroll
         for (int c = 0; c < 64; ++c)
           if (c >= nvalid) s[c] = -CUDART_INF_F;
+      }
+      if (exrow) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (((c < 32 ? ex0 : ex1) >> (c & 31)) & 1u) s[c] = -CUDART_INF_F;
       }
       // Half-row max of the raw scores (scale > 0 keeps the order), 8 chains,
       // then the partner's half: both threads of a row see the same max.  The
@@ -794,7 +815,7 @@ void tc_plan_split(int64_t tiles, int64_t nkeys, int32_t max_parts, bool allow_c
 
 cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys, int32_t nsplit, int64_t kps,
                            int32_t cluster, const int8_t* mask, int mask_active, float scale_log2, float* pa,
-                           float* pl, cudaStream_t s) {
+                           float* pl, cudaStream_t s, const uint32_t* excl, int64_t excl_words) {
   TcArgs a;
   a.B = d.B; a.Hq = d.Hq; a.Hkv = d.Hkv; a.G = d.Hq / d.Hkv; a.Nb = d.Nb;
   a.mode = m.mode; a.hg = m.hg; a.tiles_per_unit = m.tiles_per_unit;
@@ -807,6 +828,8 @@ cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys
   a.status = device_status_ptr();
   a.wait_limit_ns = wait_limit_ns();
   a.cluster = cluster > 1 ? cluster : 1;
+  a.excl = excl;
+  a.excl_words = excl_words;
   if (!a.status) return cudaErrorInvalidValue;
   static bool attr = false;
   if (!attr) {
