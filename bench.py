@@ -366,6 +366,29 @@ def run_ours(args, spec, rank, world, device):
     }
 
 
+def kernels_only(spec, device, n):
+    """N full steps then N reuse steps of one layer (the first block's steps
+    0 and 1 at its size), with an L2 flush before each: the launches an ncu
+    capture of the hot kernels needs, in the configuration bench.py times."""
+    from block_diffusion_attention_flashblock_b200 import fb
+    torch.cuda.set_device(device)
+    S = Layers(spec, device, 1)
+    d = S.L[0]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    gamma = torch.full((spec.Hq,), spec.gamma, device=device) if spec.gamma is not None else None
+    st0 = S.steps[0]
+    x = d["x"][0]
+    for tau in (0, fb.FB_TAU_OFF):   # every step recomputes; then every step reuses the cache
+        for _ in range(n):
+            flush.zero_()
+            d["layer"].step(x["q"], x["kin"], x["vin"], d["kp"], d["vp"], st0.prefix_len, 0, tau, d["o"], d["lse"],
+                            gamma, x["sel"])
+    torch.cuda.synchronize()
+    assert fb.fb_get_device_status() == fb.FB_OK
+    S.close()
+    print(json.dumps({"kernels_only": spec.name, "full_steps": n, "reuse_steps": n}))
+
+
 def _ncu_traffic(kind, workload):
     """Per-launch DRAM bytes of this kernel from the committed ncu summary, if it
     was taken on the current kernel source (else None)."""
@@ -442,6 +465,9 @@ def main():
     ap.add_argument("--no-pdl", action="store_true", help="launch kernels in plain stream order")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--prefix-kernel", default="auto", choices=["auto", "generic", "tcgen05", "tcgen05-nocluster"])
+    ap.add_argument("--kernels-only", type=int, default=0, metavar="N",
+                    help="run N full and N reuse steps of one layer of the workload, untimed, and exit "
+                         "(a small case for ncu captures)")
     ap.add_argument("--profile-run", action="store_true",
                     help="only the reuse-on schedule (no full-recompute, e2e or CPU legs): for ncu captures")
     args = ap.parse_args()
@@ -460,6 +486,9 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
     device = torch.device("cuda", local)
+    if args.kernels_only:
+        kernels_only(spec, device, args.kernels_only)
+        return
     out = run_ours(args, spec, rank, world, device)
     if world > 1:
         torch.distributed.destroy_process_group()

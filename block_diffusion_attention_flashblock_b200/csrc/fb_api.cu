@@ -22,6 +22,8 @@ static uint64_t g_wait_limit_ns = 2000000000ull;
 uint64_t wait_limit_ns() { return g_wait_limit_ns; }
 static bool g_pdl = true;
 bool pdl_enabled() { return g_pdl; }
+static bool g_stall = false;
+bool debug_stall() { return g_stall; }
 
 int* device_status_ptr() {
   int* p = nullptr;
@@ -570,6 +572,11 @@ fb_status fb_profile_read(int32_t reset, int64_t* launches, double* total_ms, do
 fb_status fb_debug_set_prefix_kernel(int32_t which) {
   if (which < 0 || which > 3) return FB_EINVAL;
   g_prefix_kernel = which;
+  return FB_OK;
+}
+
+fb_status fb_debug_set_stall(int32_t on) {
+  g_stall = on != 0;
   return FB_OK;
 }
 

@@ -67,7 +67,7 @@ constexpr float kRescaleLog2 = 8.0f;
 // barrier slots
 enum {
   B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 10, B_SFULL = 13, B_PFULL = 16,
-  B_PVDONE = 19, B_DRAIN = 22, B_PAIR = 24, B_RECV = 28, B_COUNT = 29
+  B_PVDONE = 19, B_DRAIN = 22, B_PAIR = 24, B_RECV = 28, B_STALL = 29, B_COUNT = 30
 };
 
 using ptx::globaltimer;
@@ -84,18 +84,24 @@ struct Ctl {
   uint64_t limit_ns;
 };
 
+// A drain (waiting for this CTA's own copies or MMAs before it exits) is
+// bounded by at least this, whatever the configured limit, so a short test
+// limit never lets a CTA exit with its own asynchronous work in flight.
+constexpr uint64_t kDrainLimitNs = 1000000000ull;
+
 // Bounded wait for the phase of `parity` to complete.  Gives up when the limit
 // passes or (unless `draining`) another role has given up; the first to give
 // up records the error.
 __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const Ctl& c, bool draining = false) {
   if (mbar_try(bar, parity)) return true;
+  const uint64_t limit = draining ? (c.limit_ns > kDrainLimitNs ? c.limit_ns : kDrainLimitNs) : c.limit_ns;
   const uint64_t t0 = globaltimer();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try(bar, parity)) return true;
     if (!draining && *c.abort) return false;
-    if (globaltimer() - t0 > c.limit_ns) {
+    if (globaltimer() - t0 > limit) {
       if (atomicExch(const_cast<int*>(c.abort), 1) == 0) atomicCAS(c.status, 0, (int)FB_ETIMEOUT);
       return false;
     }
@@ -298,6 +304,7 @@ struct TcArgs {
   int32_t cluster;         // > 1: clusters of this many consecutive splits reduce in-kernel
   const uint32_t* excl;    // non-null: per (b, query head) bitmap of excluded keys (sparse residual pass)
   int64_t excl_words;
+  int32_t stall;           // test hook: the S issuer first waits on a barrier nothing completes
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -416,7 +423,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // finished reading the P that buffer held
       const uint64_t dQ = sw128_desc(sbase + kOffQ, 16, 1024);
       const uint64_t dK = sw128_desc(sbase + kOffK, 16, 1024);
-      bool ok = wait_phase(bar(B_QFULL), 0, ctl);
+      bool ok = !a.stall || wait_phase(bar(B_STALL), 0, ctl);
+      ok = ok && wait_phase(bar(B_QFULL), 0, ctl);
       for (int j = 0; j < T && ok; ++j) {
         const int sb = j % kSBuf, st = j % kStages;
         ok = wait_phase(bar(B_KFULL + st), (j / kStages) & 1, ctl);
@@ -830,6 +838,7 @@ cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys
   a.cluster = cluster > 1 ? cluster : 1;
   a.excl = excl;
   a.excl_words = excl_words;
+  a.stall = debug_stall() ? 1 : 0;
   if (!a.status) return cudaErrorInvalidValue;
   static bool attr = false;
   if (!attr) {

@@ -83,14 +83,19 @@ struct InblockArgs {
   float scale_log2;
   int* status;
   uint64_t wait_limit_ns;
+  int32_t stall;      // test hook: thread 0 first waits on a barrier nothing completes
 };
 
-// Bounded wait on phase 0 of a load barrier; the first expiry is recorded.
-__device__ __forceinline__ bool wait_loaded(uint32_t bar, const InblockArgs& a) {
+// Bounded wait on phase 0 of a load barrier; the first expiry is recorded.  A
+// drain (the last wait before exit after an expiry) is bounded by at least
+// one second whatever the configured limit, so the CTA never exits with a
+// copy into its shared memory in flight.
+__device__ __forceinline__ bool wait_loaded(uint32_t bar, const InblockArgs& a, bool drain = false) {
   if (ptx::mbar_test(bar, 0)) return true;
+  const uint64_t limit = drain && a.wait_limit_ns < 1000000000ull ? 1000000000ull : a.wait_limit_ns;
   const uint64_t t0 = ptx::globaltimer();
   while (!ptx::mbar_try(bar, 0)) {
-    if (ptx::globaltimer() - t0 > a.wait_limit_ns) {
+    if (ptx::globaltimer() - t0 > limit) {
       atomicCAS(a.status, 0, (int)FB_ETIMEOUT);
       return false;
     }
@@ -112,7 +117,7 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   float* sL = sE + NXS * kRows * kExtStride;                             // [NX][16]
   float* sO = sL + NXS * kRows;                                          // [16][kExtStride] output rows
   float* sC = sO + kRows * kExtStride;                                   // [16][kExtStride] cache rows
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + kRows * kExtStride);  // Q+K, V, parts
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + kRows * kExtStride);  // Q+K, V, parts, (test) stall
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int unit = blockIdx.x / a.tiles_per_unit, tile = blockIdx.x % a.tiles_per_unit;
@@ -130,6 +135,7 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
     ptx::mbar_init(bar_qk, 1);
     ptx::mbar_init(bar_v, 1);
     ptx::mbar_init(bar_e, 1);
+    ptx::mbar_init(bar_e + 8, 1);
     ptx::fence_mbar_init();
     ptx::mbar_expect_tx(bar_qk, (uint32_t)(nq + a.Nb) * (kD * 2));
     ptx::mbar_expect_tx(bar_v, (uint32_t)a.Nb * (kD * 2));
@@ -178,7 +184,8 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
                       kD * 4, bar_e);
   }
   __syncthreads();   // zero-filled rows
-  bool ok = wait_loaded(bar_qk, a);
+  bool ok = !(a.stall && tid == 0) || wait_loaded(bar_e + 8, a);
+  ok = wait_loaded(bar_qk, a) && ok;
 
   // ---- S = Q K^T for the CTA's 16 rows (every warp) ----
   const int dq = warp;   // this warp's quarter of D: columns dq*32 .. dq*32+31
@@ -323,9 +330,9 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   }
   if (!ok && tid == 0) {
     // a load wait expired: let every copy into shared memory land before exit
-    wait_loaded(bar_qk, a);
-    wait_loaded(bar_v, a);
-    wait_loaded(bar_e, a);
+    wait_loaded(bar_qk, a, true);
+    wait_loaded(bar_v, a, true);
+    wait_loaded(bar_e, a, true);
   }
 }
 
@@ -359,11 +366,12 @@ cudaError_t launch_inblock_small(const fb_attn_desc& d, const void* q, const voi
   a.scale_log2 = scale_log2;
   a.status = device_status_ptr();
   a.wait_limit_ns = wait_limit_ns();
+  a.stall = debug_stall() ? 1 : 0;
   if (!a.status) return cudaErrorInvalidValue;
   const int NB = d.Nb <= 16 ? 16 : d.Nb <= 32 ? 32 : 64;
   const int nxs = next > 0 ? next : 1;
   const size_t smem = (size_t)(kRows + 2 * NB) * kRowE * 2 + (size_t)nxs * kRows * (kExtStride + 1) * 4 +
-                      2 * (size_t)kRows * kExtStride * 4 + 3 * 8;
+                      2 * (size_t)kRows * kExtStride * 4 + 4 * 8;
   const dim3 grid(d.B * d.Hkv * a.tiles_per_unit);
   // instances above the default 48 KB of dynamic shared memory opt in once
   static bool opted[3][kMaxExt + 1] = {};

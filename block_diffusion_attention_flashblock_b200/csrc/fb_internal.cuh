@@ -92,6 +92,7 @@ class ProfScope {
 // every kernel begins with ptx::pdl_prologue(), so it touches no global
 // memory before the kernels it depends on have completed.
 bool pdl_enabled();
+bool debug_stall();   // test hook: kernels first wait on a barrier nothing completes
 template <class... KArgs, class... Args>
 cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
   cudaLaunchConfig_t cfg = {};

@@ -269,6 +269,13 @@ fb_status fb_debug_set_prefix_kernel(int32_t which);
  * expire at once.  Affects only the calling process. */
 fb_status fb_debug_set_wait_limit_ns(uint64_t ns);
 
+/* Test hook: when on, each tcgen05 prefix/in-block kernel and each small
+ * in-block kernel launched afterwards first waits on a barrier that nothing
+ * completes, so that wait runs out after the configured limit and the launch
+ * records FB_ETIMEOUT (every CTA still drains its own copies and MMAs before
+ * it returns).  Off by default.  Affects only the calling process. */
+fb_status fb_debug_set_stall(int32_t on);
+
 /* Tuning hook: 1 (default) launches every kernel with programmatic dependent
  * launch allowed, so a kernel's launch overlaps the tail of the one before it
  * in the stream (each kernel waits for its predecessors before it touches
