@@ -189,6 +189,10 @@ static PassPlan plan_pass(const fb_attn_desc& d, const void* q, const void* k, c
   a.scale_log2 = scale_log2(d);
   plan_split((int64_t)a.rm.units * a.rm.row_tiles, a.nkeys, generic_ctas_per_sm(d.D, bf16), generic_key_tile(),
              &a.nsplit, &a.keys_per_split);
+  if (sel && a.keys_per_split > generic_max_gather_keys()) {   // a CTA stages at most this many list entries
+    a.keys_per_split = generic_max_gather_keys();
+    a.nsplit = (int32_t)std::max<int64_t>(1, (a.nkeys + a.keys_per_split - 1) / a.keys_per_split);
+  }
   if (max_split > 0 && a.nsplit > max_split) {  // workspace sized smaller: fewer, longer splits
     const int kt = generic_key_tile();
     int64_t kps = (a.nkeys + max_split - 1) / max_split;

@@ -21,6 +21,9 @@
 
 namespace fb {
 
+// Longest key-list slice one CTA of a gather pass stages in shared memory.
+constexpr int kMaxGatherKeys = 4096;
+
 namespace {
 
 struct RowInfo {
@@ -168,9 +171,18 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
   const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
   const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(a.k) + b * a.k_sb + kvh * a.k_sh;
   const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(a.v) + b * a.k_sb + kvh * a.k_sh;
-  const int32_t* sel = nullptr;
-  if (a.sel) {  // per_head units: one list per (b, query head)
-    sel = a.sel + (int64_t)unit * a.sel_k;
+  // per_head units with a key list: this split's slice of the (b, query head)
+  // list is staged in shared memory first, so a tile's gather does not wait
+  // on its own index loads
+  // (slices longer than kMaxGatherKeys, which the host gives no staging
+  // space, read their indices directly)
+  int32_t* sSel = reinterpret_cast<int32_t*>(sV + 2 * BN * D);
+  const bool gather = a.sel != nullptr;
+  const bool staged = gather && a.keys_per_split <= kMaxGatherKeys;
+  const int32_t* sel = gather ? a.sel + (int64_t)unit * a.sel_k : nullptr;
+  if (staged) {
+    for (int64_t k = kbeg + tid; k < kend; k += 128) sSel[k - kbeg] = __ldg(sel + k);
+    __syncthreads();
   }
 
   // Q tile -> smem (swizzled 16-byte chunks: chunk c of row r at c ^ (r & 7)).
@@ -187,7 +199,8 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
     for (int c = tid; c < BN * CH; c += 128) {
       const int r = c / CH, ch = c % CH;
       const int64_t key = key0 + r;
-      int64_t phys = key < kend ? (sel ? (int64_t)__ldg(sel + key) : key) : -1;
+      int64_t phys = key < kend ? (staged ? (int64_t)sSel[key - kbeg] : gather ? (int64_t)__ldg(sel + key) : key)
+                                : -1;
       const bool ok = phys >= 0 && phys < a.key_rows;
       if (!ok) phys = 0;
       const int off = r * D + ((ch ^ (r & 7)) * 8);
@@ -528,6 +541,7 @@ __global__ void __launch_bounds__(64 * (D / 64)) attn_f32_kernel(const AttnArgs 
 
 // ---------------------------------------------------------------------------
 int generic_tile_rows(int) { return 64; }
+int generic_max_gather_keys() { return kMaxGatherKeys; }
 int generic_key_tile() { return 64; }
 int generic_ctas_per_sm(int D, int in_bf16) {
   if (!in_bf16) return 4;
@@ -536,10 +550,14 @@ int generic_ctas_per_sm(int D, int in_bf16) {
 
 template <int D>
 static cudaError_t launch_mma(const AttnArgs& a, cudaStream_t s) {
-  constexpr int smem = (64 * D + 4 * 64 * D) * 2;
+  // Q, two K and two V stages, and (gather passes) the split's key list
+  constexpr int base = (64 * D + 4 * 64 * D) * 2;
+  const int smem =
+      base + (a.sel && a.keys_per_split <= kMaxGatherKeys ? (int)((a.keys_per_split * 4 + 15) / 16 * 16) : 0);
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(attn_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         base + kMaxGatherKeys * 4);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }

@@ -118,6 +118,7 @@ void plan_split(int64_t tiles, int64_t nkeys, int ctas_per_sm, int key_tile,
 cudaError_t launch_attn_generic(const AttnArgs& a, int D, int in_bf16, cudaStream_t s);
 int generic_tile_rows(int in_bf16);
 int generic_key_tile();
+int generic_max_gather_keys();   // longest key-list slice per CTA of a gather pass
 int generic_ctas_per_sm(int D, int in_bf16);
 
 // tcgen05 prefix pass (fb_attn_tc.cu).
