@@ -166,7 +166,7 @@ class Layers:
 def run_ours(args, spec, rank, world, device):
     from block_diffusion_attention_flashblock_b200 import fb
     torch.cuda.set_device(device)
-    fb.fb_debug_set_prefix_kernel({"auto": 0, "generic": 1, "tcgen05": 2, "tcgen05-nocluster": 3}[args.prefix_kernel])
+    fb.fb_debug_set_prefix_kernel({"auto": 0, "generic": 1, "tcgen05": 2, "tcgen05-nocluster": 3, "tcgen05-cluster": 4}[args.prefix_kernel])
     fb.fb_debug_set_pdl(not args.no_pdl)
     nl = n_layers(spec)
     S = Layers(spec, device, nl)
@@ -464,7 +464,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-pdl", action="store_true", help="launch kernels in plain stream order")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
-    ap.add_argument("--prefix-kernel", default="auto", choices=["auto", "generic", "tcgen05", "tcgen05-nocluster"])
+    ap.add_argument("--prefix-kernel", default="auto", choices=["auto", "generic", "tcgen05", "tcgen05-nocluster", "tcgen05-cluster"])
     ap.add_argument("--kernels-only", type=int, default=0, metavar="N",
                     help="run N full and N reuse steps of one layer of the workload, untimed, and exit "
                          "(a small case for ncu captures)")

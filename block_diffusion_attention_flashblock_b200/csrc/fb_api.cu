@@ -221,7 +221,8 @@ static fb_status launch_pass(const fb_attn_desc& d, AttnArgs& a, float* pa, floa
 
 // Dense block-external pass over prefix rows [0, nkeys): the tcgen05 kernel
 // when the shape and strides allow it, else the generic kernel.
-static int g_prefix_kernel = 0;  // 0 auto, 1 generic only, 2 tcgen05 whenever it applies, 3 as 2 without clusters
+static int g_prefix_kernel = 0;  // 0 auto, 1 generic only, 2 tcgen05 whenever it applies, 3 as 2 without
+                                 // clusters, 4 as 2 with the cluster reduction taken at no cost in the plan
 
 struct PrefixPlan {
   bool tc;
@@ -248,7 +249,7 @@ static PrefixPlan plan_prefix(const fb_attn_desc& d, const void* q, const void* 
   const int64_t min_keys = g_prefix_kernel >= 2 ? 1 : 256;
   if (g_prefix_kernel != 1 && nkeys >= min_keys && tc_make_maps(d, q, kp, vp, nkeys, d.kp_strides, &p.maps)) {
     tc_plan_split((int64_t)p.maps.units * p.maps.tiles_per_unit, nkeys, cap, g_prefix_kernel != 3, &p.nsplit,
-                  &p.kps, &p.cluster, &p.nparts);
+                  &p.kps, &p.cluster, &p.nparts, g_prefix_kernel == 4 ? 0.0 : 4.0);
     p.tc = true;
   }
   return p;
@@ -574,7 +575,7 @@ fb_status fb_profile_read(int32_t reset, int64_t* launches, double* total_ms, do
 }
 
 fb_status fb_debug_set_prefix_kernel(int32_t which) {
-  if (which < 0 || which > 3) return FB_EINVAL;
+  if (which < 0 || which > 4) return FB_EINVAL;
   g_prefix_kernel = which;
   return FB_OK;
 }

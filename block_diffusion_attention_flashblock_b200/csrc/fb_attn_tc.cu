@@ -793,7 +793,7 @@ static int max_active_clusters(int cs) {
 // (or clusters) x (the longest split in key tiles + a fixed cost of about two
 // tiles), plus a small cost per extra part; nparts is at most max_parts.
 void tc_plan_split(int64_t tiles, int64_t nkeys, int32_t max_parts, bool allow_cluster, int32_t* nsplit,
-                   int64_t* kps, int32_t* cluster, int32_t* nparts) {
+                   int64_t* kps, int32_t* cluster, int32_t* nparts, double cluster_cost) {
   const int64_t sms = num_sms();
   const int64_t ktiles = std::max<int64_t>(1, (nkeys + kBN - 1) / kBN);
   double best = 1e300;
@@ -809,9 +809,9 @@ void tc_plan_split(int64_t tiles, int64_t nkeys, int32_t max_parts, bool allow_c
       const int64_t units = cs == 1 ? tiles * ns : tiles * nc;
       const int64_t waves = (units + conc - 1) / conc;
       // a cluster's in-kernel reduction (two cluster barriers and the
-      // shared-to-shared copies) costs about four key tiles per CTA
-      const double cost = (double)waves * (last + 2 + (cs > 1 ? 4 : 0)) + (parts > 1 ? 1.5 + 0.1 * parts : 0.0) +
-                          0.01 * ns;
+      // shared-to-shared copies) costs cluster_cost key tiles per CTA
+      const double cost = (double)waves * (last + 2 + (cs > 1 ? cluster_cost : 0.0)) +
+                          (parts > 1 ? 1.5 + 0.1 * parts : 0.0) + 0.01 * ns;
       if (cost < best) { best = cost; b_ns = ns; b_cs = cs; b_per = per; }
     }
   }

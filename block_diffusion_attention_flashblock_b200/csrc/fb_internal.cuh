@@ -131,7 +131,7 @@ bool tc_tiling(const fb_attn_desc& d, int* mode, int* hg, int* tiles_per_unit, i
 bool tc_make_maps(const fb_attn_desc& d, const void* q, const void* k, const void* v, int64_t nkeys,
                   const int64_t* kstr, TcMaps* m);
 void tc_plan_split(int64_t tiles, int64_t nkeys, int32_t max_parts, bool allow_cluster, int32_t* nsplit,
-                   int64_t* kps, int32_t* cluster, int32_t* nparts);
+                   int64_t* kps, int32_t* cluster, int32_t* nparts, double cluster_cost = 4.0);
 int32_t tc_split_cap(int64_t tiles, int64_t max_keys);
 cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys, int32_t nsplit, int64_t kps,
                            int32_t cluster, const int8_t* mask, int mask_active, float scale_log2, float* pa,

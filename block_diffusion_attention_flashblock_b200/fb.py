@@ -258,7 +258,7 @@ def fb_get_device_status(stream=None) -> int:
     return s.value
 
 
-PREFIX_AUTO, PREFIX_GENERIC, PREFIX_TC, PREFIX_TC_NO_CLUSTER = 0, 1, 2, 3
+PREFIX_AUTO, PREFIX_GENERIC, PREFIX_TC, PREFIX_TC_NO_CLUSTER, PREFIX_TC_CLUSTER = 0, 1, 2, 3, 4
 
 
 def fb_debug_set_prefix_kernel(which: int):

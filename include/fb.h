@@ -261,7 +261,9 @@ fb_status fb_profile_read(int32_t reset, int64_t* launches, double* total_ms, do
  * tcgen05 kernel where the shape and strides allow it), 1 the generic
  * mma.sync / FFMA kernel only, 2 the tcgen05 kernel whenever it applies,
  * 3 as 2 but its key splits always go through a separate merge instead of
- * the in-kernel cluster reduction. */
+ * the in-kernel cluster reduction, 4 as 2 with the split planner charging
+ * nothing for the cluster reduction (so it is taken wherever it saves
+ * waves or parts). */
 fb_status fb_debug_set_prefix_kernel(int32_t which);
 
 /* Test hook: the bound of every barrier wait in later launches, in

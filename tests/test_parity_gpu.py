@@ -92,13 +92,20 @@ TC_SHAPES = [
 @pytest.mark.parametrize("mode", ["cluster", "merge"])
 def test_outblock_dense_tcgen05(shape, mode, prefix_kernel):
     """tcgen05 prefix pass; key splits reduced in-kernel across a cluster, or by the merge pass."""
-    prefix_kernel(fb.PREFIX_TC if mode == "cluster" else fb.PREFIX_TC_NO_CLUSTER)
+    prefix_kernel(fb.PREFIX_TC_CLUSTER if mode == "cluster" else fb.PREFIX_TC_NO_CLUSTER)
     _outblock_check(shape, seed=13)
 
 
 @pytest.mark.parametrize("name", ["dllm_8k_small", "dllm_64k_small", "video_small_mixed"])
 def test_step_schedule_tcgen05_no_cluster(name, prefix_kernel):
     prefix_kernel(fb.PREFIX_TC_NO_CLUSTER)
+    compare_schedule(_spec(name))
+
+
+@pytest.mark.parametrize("name", ["dllm_8k_small", "dllm_64k_small", "sparse_small"])
+def test_step_schedule_tcgen05_cluster(name, prefix_kernel):
+    """The split planner takes the in-kernel cluster reduction wherever it saves waves or parts."""
+    prefix_kernel(fb.PREFIX_TC_CLUSTER)
     compare_schedule(_spec(name))
 
 
