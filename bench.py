@@ -312,25 +312,38 @@ def run_ours(args, spec, rank, world, device):
         del g
         calls = R * nl
         byts = sum(v[2] for v in pk.values()) / nl
+        nk = P if kind == "prefix_attention" else s.Nb
+        flops = 4.0 * s.B * s.Hq * s.Nb * nk * s.D   # Q K^T and P V, algorithmic
         per_kind[kind] = {"call": "fb_attn_outblock" if kind == "prefix_attention" else
-                          "fb_attn_inblock (one cached external part)",
+                          "fb_attn_inblock (one cached external part; above 64-token blocks this public call runs "
+                          "the generic kernel, fb_step the tcgen05 pass)",
                           "kernels_per_call": sum(v[0] for v in pk.values()) / nl,
-                          "avg_call_us": 1e3 * ms / calls, "alg_bytes_per_call": byts,
-                          "achieved_GBps": byts / (ms * 1e-3 / calls) / 1e9}
+                          "own_kernels_per_call": pk[kind][0] / nl,
+                          "avg_call_us": 1e3 * ms / calls, "alg_bytes_per_call": byts, "alg_flops_per_call": flops,
+                          "achieved_GBps": byts / (ms * 1e-3 / calls) / 1e9,
+                          "achieved_TFLOPs": flops / (ms * 1e-3 / calls) / 1e12}
     assert fb.fb_get_device_status() == fb.FB_OK
     S.close()
 
     hbm, tf, tf_sus, peak_src = _peaks()
-    # the dominant kind: launches in the schedule x its graph-timed duration
-    share = {k: prof[k][0] * per_kind[k]["avg_call_us"] / max(1e-9, per_kind[k]["kernels_per_call"])
+    # the dominant kind: its calls in the schedule x the graph-timed call duration
+    share = {k: prof[k][0] / max(1e-9, per_kind[k]["own_kernels_per_call"]) * per_kind[k]["avg_call_us"]
              for k in per_kind}
     dom = max(share, key=share.get)
     pkd = per_kind[dom]
     traffic = _ncu_traffic(dom, spec.name)
-    roof = {"kernel": dom, "call": pkd["call"], "bound": "hbm", "achieved": pkd["achieved_GBps"], "peak": hbm,
-            "unit": "GB/s", "frac": pkd["achieved_GBps"] / hbm, "peak_source": f"{peak_src} hbm_gbs (burst)",
+    # bound: the tensor pipe when the call's algorithmic flop per byte exceeds
+    # the ridge of the measured peaks, else HBM
+    ridge = tf * 1e12 / (hbm * 1e9)
+    tensor = pkd["alg_flops_per_call"] / pkd["alg_bytes_per_call"] > ridge
+    roof = {"kernel": dom, "call": pkd["call"], "bound": "tensor" if tensor else "hbm",
+            "achieved": pkd["achieved_TFLOPs"] if tensor else pkd["achieved_GBps"],
+            "peak": tf if tensor else hbm, "unit": "TFLOP/s" if tensor else "GB/s",
+            "frac": pkd["achieved_TFLOPs"] / tf if tensor else pkd["achieved_GBps"] / hbm,
+            "peak_source": f"{peak_src} " + ("bf16_tflops (burst)" if tensor else "hbm_gbs (burst)"),
+            "frac_hbm": pkd["achieved_GBps"] / hbm, "frac_tensor": pkd["achieved_TFLOPs"] / tf,
             "traffic": traffic, "alg_bytes_per_launch": pkd["alg_bytes_per_call"],
-            "avg_launch_us": pkd["avg_call_us"],
+            "alg_flops_per_launch": pkd["alg_flops_per_call"], "avg_launch_us": pkd["avg_call_us"],
             "timing": f"CUDA events around one graph of {R * nl} calls ({nl} layers x {R}), L2 flushed before"}
     kernels = {k: {"launches_per_step": v[0], "alg_bytes_per_step": v[2]} for k, v in prof.items()}
     n_full = sum(rec_on)

@@ -460,8 +460,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int part = 0; part < 2; ++part)   // P_hi, then P_lo
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk)
-            tc_mma_ts(tmem + kTmemO, pt + part * 64 + kk * 8, dVs + (uint64_t)((kk * 2048) >> 4), kIdescPV,
-                      (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
+            tc_mma_ts(tmem + kTmemO, pt + (kk >> 2) * 64 + part * 32 + (kk & 3) * 8,
+                      dVs + (uint64_t)((kk * 2048) >> 4), kIdescPV, (j > 0 || part > 0 || kk > 0) ? 1u : 0u);
         tc_commit(bar(B_VEMPTY + st));
         tc_commit(bar(B_PVDONE + sb));
       }
@@ -510,29 +510,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = uniform(wait_phase(bar(B_SFULL + sb), (j / kSBuf) & 1, ctl));
       if (!ok) break;
       tc_fence_after();
+      // this thread's 64 scores, ragged tail and excluded keys masked to -inf
       float s[64];
-      tmem_ld32(tl + sb * kBN + half * 64, s);
-      tmem_ld32(tl + sb * kBN + half * 64 + 32, s + 32);
-      tmem_wait_ld();
       const int nvalid = (int)min((int64_t)kBN, kend - key0) - half * 64;
-      if (nvalid < 64) {   // only the last tile of the last split is ragged
+      auto load_s = [&]() {
+        tmem_ld32(tl + sb * kBN + half * 64, s);
+        tmem_ld32(tl + sb * kBN + half * 64 + 32, s + 32);
+        tmem_wait_ld();
+        if (nvalid < 64) {   // only the last tile of the last split is ragged
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c >= nvalid) s[c] = -CUDART_INF_F;
-      }
-      if (exrow) {
+          for (int c = 0; c < 64; ++c)
+            if (c >= nvalid) s[c] = -CUDART_INF_F;
+        }
+        if (exrow) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (((c < 32 ? ex0 : ex1) >> (c & 31)) & 1u) s[c] = -CUDART_INF_F;
-      }
-      // Half-row max of the raw scores (scale > 0 keeps the order), 8 chains,
-      // then the partner's half: both threads of a row see the same max.  The
-      // trade also orders both halves' reads of S before either writes P over it.
+          for (int c = 0; c < 64; ++c)
+            if (((c < 32 ? ex0 : ex1) >> (c & 31)) & 1u) s[c] = -CUDART_INF_F;
+        }
+      };
+      // p = 2^(s * scale - ref) in place: one FFMA and one MUFU op per score,
+      // 8 sum chains
+      auto exp_pass = [&](float ref) -> float {
+        const float nref = (ref == -CUDART_INF_F) ? 0.f : -ref;
+        float sm8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          s[c] = fast_exp2(fmaf(s[c], a.scale_log2, nref));
+          sm8[c & 7] += s[c];
+        }
+        return ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
+      };
+      load_s();
+      // Half-row max of the raw scores (scale > 0 keeps the order).  Once the
+      // row has a reference max m, P is formed against it in the same pass
+      // (the common case: the tile's max stays within m + 2^8); the row's
+      // first tile takes the max first.  The partner's half is traded either
+      // way, so both threads of a row see the same max.
+      const bool two_pass = __any_sync(0xffffffffu, m == -CUDART_INF_F);
       float mx8[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mx8[e] = s[e];
+      for (int e = 0; e < 8; ++e) mx8[e] = -CUDART_INF_F;
+      float psum = 0.f;
+      if (two_pass) {
 #pragma unroll
-      for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+        for (int c = 0; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+      } else {
+        const float nref = -m;
+        float sm8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+          s[c] = fast_exp2(fmaf(s[c], a.scale_log2, nref));
+          sm8[c & 7] += s[c];
+        }
+        psum = ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
+      }
       float tmax =
           fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])), fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
           a.scale_log2;
@@ -564,22 +596,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         l *= alpha;
         m = tmax;
       }
-      // p = 2^(s * scale - ref): one FFMA and one MUFU op per score; 8 sum chains.
-      const float nref = (m == -CUDART_INF_F) ? 0.f : -m;
-      float sm8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        s[c] = fast_exp2(fmaf(s[c], a.scale_log2, nref));
-        sm8[c & 7] += s[c];
+      // P again from the scores (still in TMEM: each half writes P only over
+      // its own columns) when a row of the warp moved its reference, or on
+      // the first tile
+      if (two_pass || __any_sync(0xffffffffu, move)) {
+        if (!two_pass) load_s();
+        psum = exp_pass(m);
       }
-      l += ((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7]));
-      // P (bf16 pairs, lower key in the low half) over this tile's S columns:
-      // hi parts at [sb*128, sb*128+64), lo parts at [sb*128+64, sb*128+128).
+      l += psum;
+      // P (bf16 pairs, lower key in the low half) over this half's own S
+      // columns: hi parts at half*64 + [0, 32), lo parts at half*64 + [32, 64).
       uint32_t hi[32], lo[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) split_pair(s[2 * e], s[2 * e + 1], hi[e], lo[e]);
-      tmem_st32u(tl + sb * kBN + half * 32, hi);
-      tmem_st32u(tl + sb * kBN + 64 + half * 32, lo);
+      tmem_st32u(tl + sb * kBN + half * 64, hi);
+      tmem_st32u(tl + sb * kBN + half * 64 + 32, lo);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(B_PFULL + sb));

@@ -96,6 +96,35 @@ def test_outblock_dense_tcgen05(shape, mode, prefix_kernel):
     _outblock_check(shape, seed=13)
 
 
+@pytest.mark.parametrize("which", ["generic", "tcgen05", "tcgen05-cluster"])
+def test_outblock_rising_and_falling_scores(which, prefix_kernel):
+    """Scores that grow along the prefix (KV head 0) force the running max to
+    move on every key tile, so O is rescaled in place many times; scores that
+    fall (KV head 1) never move it after the first tile."""
+    prefix_kernel({"generic": fb.PREFIX_GENERIC, "tcgen05": fb.PREFIX_TC_NO_CLUSTER,
+                   "tcgen05-cluster": fb.PREFIX_TC_CLUSTER}[which])
+    # 8 row tiles x 64 key tiles (ragged last): several key tiles per CTA
+    B, Hq, Hkv, D, Nb, Lp = 1, 32, 8, 128, 32, 8100
+    q = wl.tensor((B, Hq, Nb, D), 61, 0.5, "f32").abs().to(torch.bfloat16)
+    ramp = torch.arange(Lp + 64, dtype=torch.float32) * 0.02
+    sign = torch.tensor([1.0, -1.0] * (Hkv // 2)).view(1, Hkv, 1, 1)
+    kp = (wl.tensor((B, Hkv, Lp + 64, D), 62, 0.5, "f32") + sign * ramp.view(1, 1, -1, 1)).to(torch.bfloat16)
+    vp = wl.tensor((B, Hkv, Lp + 64, D), 63, 1.0, "bf16")
+    kin = wl.tensor((B, Hkv, Nb, D), 64, 1.0, "bf16")
+    qd, kpd, vpd = q.cuda(), kp.cuda(), vp.cuda()
+    a = torch.full((B, Hq, Nb, D), float("nan"), device="cuda")
+    l = torch.full((B, Hq, Nb), float("nan"), device="cuda")
+    desc = fb.make_desc(qd, kin.cuda(), kpd, a)
+    ws = torch.empty(fb.fb_outblock_workspace_bytes(desc, Lp), dtype=torch.uint8, device="cuda")
+    fb.fb_attn_outblock(desc, qd, kpd, vpd, Lp, a, l, ws)
+    assert fb.fb_get_device_status() == fb.FB_OK
+    A, L = orc.outblock(orc.to64(q), orc.to64(kp), orc.to64(vp), Lp, 1 / np.sqrt(D))
+    for h0 in range(0, Hq, Hq // Hkv):   # the heads of each KV head separately (their scales differ)
+        h1 = h0 + Hq // Hkv
+        assert_o_close(a[:, h0:h1], A[:, h0:h1], TOL["bf16"], f"A_out heads {h0}..{h1 - 1}")
+        assert_lse_close(l[:, h0:h1], L[:, h0:h1], TOL["bf16"], f"L_out heads {h0}..{h1 - 1}")
+
+
 @pytest.mark.parametrize("name", ["dllm_8k_small", "dllm_64k_small", "video_small_mixed"])
 def test_step_schedule_tcgen05_no_cluster(name, prefix_kernel):
     prefix_kernel(fb.PREFIX_TC_NO_CLUSTER)
