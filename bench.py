@@ -124,6 +124,14 @@ class ClockSampler:
 L2_BYTES = 126 << 20
 
 
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The slowest rank's time: every rank takes part, every rank gets the max."""
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.item()
+
+
 def n_layers(spec) -> int:
     """Independent layer states stepped in turn: enough that the layers' KV
     caches together exceed twice the L2 (so each layer's data has left L2 by
@@ -221,11 +229,7 @@ def run_ours(args, spec, rank, world, device):
         if world > 1:
             torch.distributed.barrier()
         torch.cuda.synchronize()
-        ms = sum(a.elapsed_time(b) for a, b in ev) / steps
-        t = torch.tensor([ms], dtype=torch.float64, device=device)
-        if world > 1:
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return t.item()
+        return max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / steps, world, device)
 
     def graph_of(fn):
         g = torch.cuda.CUDAGraph()
@@ -275,9 +279,31 @@ def run_ours(args, spec, rank, world, device):
                "note": "eager calls; every layer-step copies its Q, K_in, V_in from pinned host memory and reads "
                        "its O and LSE back, inside the timed region"}
 
+    # Reuse-step latency, measured directly: after one full step per layer, a
+    # graph of R rounds over the layers of a step that reuses the cache (the
+    # block's step 1 inputs, M = 0 with tau on; the gamma gate, where on,
+    # still decides per head), L2 flushed before it.
+    R = 4
+    st1 = S.steps[1] if len(S.steps) > 1 else S.steps[0]
+    for d in S.L:
+        x = d["x"][0]
+        d["layer"].begin_block()
+        d["layer"].step(x["q"], x["kin"], x["vin"], d["kp"], d["vp"], S.steps[0].prefix_len, 0, 0, d["o"], d["lse"],
+                        gamma, x["sel"])
+
+    def reuse_round():
+        for d in S.L:
+            x = d["x"][1 if len(S.steps) > 1 else 0]
+            d["layer"].step(x["q"], x["kin"], x["vin"], d["kp"], d["vp"], st1.prefix_len, 0, tau_on, d["o"],
+                            d["lse"], gamma, x["sel"])
+
+    g_reuse, _ = graph_of(lambda: [reuse_round() for _ in range(R)])
+    reuse_recomputed = S.L[0]["layer"].last_recomputed()
+    ms_reuse = timed_region(g_reuse.replay, args.steps, args.warmup)
+    del g_reuse
+
     # Per-kind launch durations without per-launch event overhead: a graph of
     # R rounds over the layers of one library call, L2 flushed before it.
-    R = 4
     st_mid = S.steps[0]
     P = st_mid.prefix_len
     parts = []
@@ -352,8 +378,9 @@ def run_ours(args, spec, rank, world, device):
     if ms_full is not None:
         t_full = ms_full / layer_steps
         step_lat["full_step_us"] = 1e3 * t_full
-        if nsteps > n_full:
-            step_lat["reuse_step_us_derived"] = 1e3 * (ms_on / nl - n_full * t_full) / (nsteps - n_full)
+    step_lat["reuse_step_us"] = 1e3 * ms_reuse / (R * nl)
+    if reuse_recomputed:
+        step_lat["reuse_step_note"] = "the gate recomputed at least one head in the measured reuse step"
     gpu_launches = sum(v[0] for v in prof.values())
     return {
         "metric": METRIC, "value": world * S.query_tokens / (ms_on * 1e-3), "unit": UNIT,

@@ -93,6 +93,13 @@ SPECS = {
         name="dllm_64k_b4", B=4, Hq=32, Hkv=8, D=128, prefix0=65536, Nb=64,
         steps=16, blocks=1, dtype="bf16", std=0.5,
         m_model=("binomial", 64, 0.1), pert_std=0.05, tau=16, seed=2026_0002),
+    # context-length sweep of the long-context shape at B = 1 (the pages'
+    # latency-growth claim, 100k to 800k tokens of context)
+    **{f"dllm_ctx_{n // 1000}k": WorkloadSpec(
+        name=f"dllm_ctx_{n // 1000}k", B=1, Hq=32, Hkv=8, D=128, prefix0=n, Nb=64,
+        steps=16, blocks=1, dtype="bf16", std=0.5,
+        m_model=("binomial", 64, 0.1), pert_std=0.05, tau=16, seed=2026_0010 + i)
+       for i, n in enumerate((100_000, 200_000, 400_000, 800_000))},
     "video_1560": WorkloadSpec(
         name="video_1560", B=1, Hq=24, Hkv=24, D=128, prefix0=31200, Nb=1560,
         steps=8, blocks=1, dtype="bf16", std=1.0, m_model=("all",),
