@@ -120,3 +120,15 @@ def test_cache_and_step_checks(L):
     assert L.fb_cache_begin_block(h, None) == fb.FB_OK
     assert L.fb_cache_destroy(h) == fb.FB_OK
     assert L.fb_cache_destroy(None) == fb.FB_EINVAL
+
+
+def test_debug_hooks_validate_and_reset(L):
+    assert L.fb_debug_set_prefix_kernel(5) == fb.FB_EINVAL
+    assert L.fb_debug_set_prefix_kernel(-1) == fb.FB_EINVAL
+    for which in (4, 3, 2, 1, 0):
+        assert L.fb_debug_set_prefix_kernel(which) == fb.FB_OK
+    for on in (0, 1):
+        assert L.fb_debug_set_pdl(on) == fb.FB_OK
+        assert L.fb_debug_set_stall(on) == fb.FB_OK
+    assert L.fb_debug_set_stall(0) == fb.FB_OK
+    assert L.fb_debug_set_wait_limit_ns(2_000_000_000) == fb.FB_OK
