@@ -100,6 +100,12 @@ SPECS = {
         steps=16, blocks=1, dtype="bf16", std=0.5,
         m_model=("binomial", 64, 0.1), pert_std=0.05, tau=16, seed=2026_0010 + i)
        for i, n in enumerate((100_000, 200_000, 400_000, 800_000))},
+    # small blocks (NEXT-2): the dllm_8k layer with blocks of 4 tokens; tau 2
+    # reuses while at most one token changed, about as often as dllm_8k's tau 8
+    "dllm_8k_nb4": WorkloadSpec(
+        name="dllm_8k_nb4", B=1, Hq=32, Hkv=8, D=128, prefix0=8192, Nb=4, steps=8,
+        blocks=4, dtype="bf16", std=0.5, m_model=("binomial", 4, 0.15),
+        pert_std=0.05, tau=2, seed=2026_0020),
     "video_1560": WorkloadSpec(
         name="video_1560", B=1, Hq=24, Hkv=24, D=128, prefix0=31200, Nb=1560,
         steps=8, blocks=1, dtype="bf16", std=1.0, m_model=("all",),
@@ -109,6 +115,14 @@ SPECS = {
         Nb=32, steps=8, blocks=1, dtype="bf16", std=0.5,
         m_model=("binomial", 32, 0.15), pert_std=0.05, tau=8, sel_k=2048,
         seed=2026_0004),
+    # sparse density sweep (NEXT-3, top-k by score only): 20, 30 and 40 % of
+    # the 32k prefix selected
+    **{f"sparse_32k_d{pct}": WorkloadSpec(
+        name=f"sparse_32k_d{pct}", B=1, Hq=32, Hkv=8, D=128, prefix0=32768,
+        Nb=32, steps=8, blocks=1, dtype="bf16", std=0.5,
+        m_model=("binomial", 32, 0.15), pert_std=0.05, tau=8, sel_k=32768 * pct // 100,
+        seed=2026_0030 + pct)
+       for pct in (20, 30, 40)},
 }
 
 

@@ -247,6 +247,8 @@ SCHEDULES = {
     "tau_zero": dict(base="dllm_8k", prefix0=500, blocks=1, steps=4, tau=0),
     "tau_off": dict(base="dllm_8k", prefix0=500, blocks=1, steps=4, tau=None),
     "nb1_gqa": dict(base="dllm_8k", Nb=1, prefix0=300, steps=3, m_model=("uniform", 0, 1), tau=1),
+    "nb4_small": dict(base="dllm_8k_nb4", prefix0=1000, blocks=2),
+    "sparse_d40_small": dict(base="sparse_32k_d40", prefix0=3000, sel_k=1200, Hq=8, Hkv=2),
 }
 
 
@@ -283,6 +285,8 @@ def test_full_dllm_8k_all_heads():
 @pytest.mark.parametrize("name, groups", [
     ("dllm_64k_b4", [(0, 0), (3, 7)]),
     ("dllm_ctx_200k", [(0, 0), (0, 7)]),
+    ("dllm_8k_nb4", [(0, 0), (0, 5)]),
+    ("sparse_32k_d40", [(0, 0), (0, 6)]),
     ("video_1560", [(0, 0), (0, 13), (0, 23)]),
     ("sparse_32k_k2048", [(0, 0), (0, 5)]),
 ])
