@@ -232,8 +232,9 @@ struct PrefixPlan {
   int64_t kps;
   PassPlan gen;
   TcMaps maps;
-  const uint32_t* excl;   // non-null: per (b, query head) bitmap of keys the pass leaves out
+  const uint32_t* excl;   // non-null: per (b, query head) key bitmap
   int64_t excl_words;
+  bool excl_invert;       // false: the pass leaves out the set keys; true: it covers only them
 };
 
 static PrefixPlan plan_prefix(const fb_attn_desc& d, const void* q, const void* kp, const void* vp, int64_t nkeys,
@@ -246,6 +247,7 @@ static PrefixPlan plan_prefix(const fb_attn_desc& d, const void* q, const void* 
   p.kps = p.gen.a.keys_per_split;
   p.excl = nullptr;
   p.excl_words = 0;
+  p.excl_invert = false;
   const int64_t min_keys = g_prefix_kernel >= 2 ? 1 : 256;
   if (g_prefix_kernel != 1 && nkeys >= min_keys && tc_make_maps(d, q, kp, vp, nkeys, d.kp_strides, &p.maps)) {
     tc_plan_split((int64_t)p.maps.units * p.maps.tiles_per_unit, nkeys, cap, g_prefix_kernel != 3, &p.nsplit,
@@ -269,7 +271,7 @@ static fb_status launch_prefix(const fb_attn_desc& d, PrefixPlan& p, int64_t nke
                        (double)rows_of(d) * (d.D + 1) * 4;
   ProfScope prof(kProfPrefix, bytes, s);
   return launch_attn_tc(d, p.maps, nkeys, p.nsplit, p.kps, p.cluster, mask, mask_active, scale_log2(d), pa, pl, s,
-                        p.excl, p.excl_words) ==
+                        p.excl, p.excl_words, p.excl_invert) ==
                  cudaSuccess
              ? FB_OK
              : FB_ECUDA;
@@ -762,26 +764,50 @@ fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
       if (launch_gamma_update(g, s) != cudaSuccess) return FB_ECUDA;
     }
   } else {
+    bool bitmap_built = false;
     if (sparse) {
-      PassPlan p = plan_pass(d, a->q, a->kp, a->vp, d.kp_strides, a->prefix_len, a->sel, a->sel_k, c->sel_cap);
-      if ((st = launch_pass(d, p.a, c->sel_a, c->sel_l, s)) != FB_OK) return st;
-      if (p.nsplit > FB_MAX_PARTS - 1) {
+      // Selected keys: gathered row by row per query head, or — when the
+      // selection covers more than 1/G of the prefix, so gathering per query
+      // head would read more than the whole prefix once per KV head — a dense
+      // pass over the prefix that leaves out every key not selected.
+      int32_t nsel = 0;
+      PrefixPlan sp;
+      sp.tc = false;
+      if ((int64_t)a->sel_k * (d.Hq / d.Hkv) > a->prefix_len) {
+        sp = plan_prefix(d, a->q, a->kp, a->vp, a->prefix_len, c->sel_cap);
+      }
+      if (sp.tc) {
+        if (launch_build_bitmap(a->sel, a->sel_k, BH, c->bitmap, (a->prefix_len + 31) / 32, s) != cudaSuccess)
+          return FB_ECUDA;
+        bitmap_built = true;
+        sp.excl = c->bitmap;
+        sp.excl_words = (a->prefix_len + 31) / 32;
+        sp.excl_invert = true;
+        if ((st = launch_prefix(d, sp, a->prefix_len, nullptr, 0, c->sel_a, c->sel_l, s)) != FB_OK) return st;
+        nsel = sp.nparts;
+      } else {
+        PassPlan p = plan_pass(d, a->q, a->kp, a->vp, d.kp_strides, a->prefix_len, a->sel, a->sel_k, c->sel_cap);
+        if ((st = launch_pass(d, p.a, c->sel_a, c->sel_l, s)) != FB_OK) return st;
+        nsel = p.nsplit;
+      }
+      if (nsel > FB_MAX_PARTS - 1) {
         // fold the splits into split 0's slot (each row is read fully before it is written)
         PartList lst;
         memset(&lst, 0, sizeof(lst));
         lst.ngroups = 1;
-        lst.g[0] = group_of(c->sel_a, c->sel_l, p.nsplit, d);
+        lst.g[0] = group_of(c->sel_a, c->sel_l, nsel, d);
         if ((st = merge_to_part(d, lst, c->sel_a, c->sel_l, nullptr, 0, s)) != FB_OK) return st;
         ext.g[ext.ngroups++] = group_of(c->sel_a, c->sel_l, 1, d);
       } else {
-        ext.g[ext.ngroups++] = group_of(c->sel_a, c->sel_l, p.nsplit, d);
+        ext.g[ext.ngroups++] = group_of(c->sel_a, c->sel_l, nsel, d);
       }
     }
     if (!tau_reuse) {
       // dense: the whole prefix; sparse: the prefix minus each head's selection
       PrefixPlan p = plan_prefix(d, a->q, a->kp, a->vp, a->prefix_len, c->part_cap);
       if (sparse) {
-        if (launch_build_bitmap(a->sel, a->sel_k, BH, c->bitmap, (a->prefix_len + 31) / 32, s) != cudaSuccess)
+        if (!bitmap_built &&
+            launch_build_bitmap(a->sel, a->sel_k, BH, c->bitmap, (a->prefix_len + 31) / 32, s) != cudaSuccess)
           return FB_ECUDA;
         p.excl = c->bitmap;
         p.excl_words = (a->prefix_len + 31) / 32;

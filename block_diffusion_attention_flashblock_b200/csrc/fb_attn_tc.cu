@@ -302,8 +302,9 @@ struct TcArgs {
   uint64_t wait_limit_ns;
   uint32_t q_bytes;        // bytes of one Q half-box (64 columns)
   int32_t cluster;         // > 1: clusters of this many consecutive splits reduce in-kernel
-  const uint32_t* excl;    // non-null: per (b, query head) bitmap of excluded keys (sparse residual pass)
+  const uint32_t* excl;    // non-null: per (b, query head) key bitmap (sparse passes)
   int64_t excl_words;
+  int32_t excl_invert;     // 0: a set bit excludes the key (residual pass); 1: a clear bit does (selected-keys pass)
   int32_t stall;           // test hook: the S issuer first waits on a barrier nothing completes
 };
 
@@ -506,6 +507,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t w0 = (key0 + half * 64) >> 5;
         if (w0 < a.excl_words) ex0 = __ldg(exrow + w0);
         if (w0 + 1 < a.excl_words) ex1 = __ldg(exrow + w0 + 1);
+        if (a.excl_invert) {
+          ex0 = ~ex0;
+          ex1 = ~ex1;
+        }
       }
       ok = uniform(wait_phase(bar(B_SFULL + sb), (j / kSBuf) & 1, ctl));
       if (!ok) break;
@@ -854,7 +859,8 @@ void tc_plan_split(int64_t tiles, int64_t nkeys, int32_t max_parts, bool allow_c
 
 cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys, int32_t nsplit, int64_t kps,
                            int32_t cluster, const int8_t* mask, int mask_active, float scale_log2, float* pa,
-                           float* pl, cudaStream_t s, const uint32_t* excl, int64_t excl_words) {
+                           float* pl, cudaStream_t s, const uint32_t* excl, int64_t excl_words,
+                           bool excl_invert) {
   TcArgs a;
   a.B = d.B; a.Hq = d.Hq; a.Hkv = d.Hkv; a.G = d.Hq / d.Hkv; a.Nb = d.Nb;
   a.mode = m.mode; a.hg = m.hg; a.tiles_per_unit = m.tiles_per_unit;
@@ -869,6 +875,7 @@ cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys
   a.cluster = cluster > 1 ? cluster : 1;
   a.excl = excl;
   a.excl_words = excl_words;
+  a.excl_invert = excl_invert ? 1 : 0;
   a.stall = debug_stall() ? 1 : 0;
   if (!a.status) return cudaErrorInvalidValue;
   static bool attr = false;

@@ -135,7 +135,8 @@ void tc_plan_split(int64_t tiles, int64_t nkeys, int32_t max_parts, bool allow_c
 int32_t tc_split_cap(int64_t tiles, int64_t max_keys);
 cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys, int32_t nsplit, int64_t kps,
                            int32_t cluster, const int8_t* mask, int mask_active, float scale_log2, float* pa,
-                           float* pl, cudaStream_t s, const uint32_t* excl = nullptr, int64_t excl_words = 0);
+                           float* pl, cudaStream_t s, const uint32_t* excl = nullptr, int64_t excl_words = 0,
+                           bool excl_invert = false);
 
 // Small-block in-block attention + merge (fb_inblock.cu).
 bool inblock_small_applies(const fb_attn_desc& d, int next);
