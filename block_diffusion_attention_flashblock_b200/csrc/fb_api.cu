@@ -640,7 +640,10 @@ fb_status layout_cache(const fb_attn_desc& d, int32_t flags, int64_t max_prefix,
   Carve cv;
   const int64_t rows = rows_of(d);
   const int32_t part_cap = split_bound(d, 0, max_prefix);
-  const int32_t sel_cap = (flags & FB_CACHE_SPARSE) ? split_bound(d, 1, std::max(max_sel_k, 1)) : 0;
+  // the selected-keys pass is a per-head gather or, for dense selections, a
+  // masked pass over the whole prefix: room for the larger of the two plans
+  const int32_t sel_cap =
+      (flags & FB_CACHE_SPARSE) ? std::max(split_bound(d, 1, std::max(max_sel_k, 1)), part_cap) : 0;
   const int64_t words = (max_prefix + 31) / 32;
   const int32_t chunks = (d.Nb + gamma_chunk_rows() - 1) / gamma_chunk_rows();
   float* ca = cv.take<float>(base, rows * d.D * 4);
@@ -767,13 +770,14 @@ fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
     bool bitmap_built = false;
     if (sparse) {
       // Selected keys: gathered row by row per query head, or — when the
-      // selection covers more than 1/G of the prefix, so gathering per query
-      // head would read more than the whole prefix once per KV head — a dense
-      // pass over the prefix that leaves out every key not selected.
+      // selection covers more than 1/(3G) of the prefix, where gathering per
+      // query head would read a third of the prefix bytes or more (and reads
+      // them at a fraction of the rate of the streaming kernel) — a tcgen05
+      // pass over the whole prefix that leaves out every key not selected.
       int32_t nsel = 0;
       PrefixPlan sp;
       sp.tc = false;
-      if ((int64_t)a->sel_k * (d.Hq / d.Hkv) > a->prefix_len) {
+      if ((int64_t)a->sel_k * 3 * (d.Hq / d.Hkv) > a->prefix_len) {
         sp = plan_prefix(d, a->q, a->kp, a->vp, a->prefix_len, c->sel_cap);
       }
       if (sp.tc) {
