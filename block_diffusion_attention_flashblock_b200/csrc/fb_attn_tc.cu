@@ -18,9 +18,10 @@
 //               64..127 of S; they trade their row maxima (and at the end
 //               their row sums) through shared memory and a bounded
 //               mbarrier.  Each writes its half of P = 2^(s - m), as bf16 hi
-//               and lo parts, back into the TMEM columns its S tile came from;
-//               the final O / l and L are staged in shared memory and leave
-//               as whole rows (512 contiguous bytes per warp store).
+//               and lo parts, back over the 64 TMEM columns its half of S
+//               came from; the final O / l and L are staged in shared memory
+//               and leave as whole rows (512 contiguous bytes per warp store).
+//               A sparse pass masks keys by a per-head bitmap before the max.
 // P lives in the S buffer it replaces, so S_{j+3} is only issued once PV_j
 // has completed (a completion barrier per buffer); three buffers leave two
 // softmax tiles for the chain P_j -> PV_j -> S_{j+3}.
@@ -458,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t dVs = dV + (uint64_t)((st * kTile) >> 4);
         const uint32_t pt = tmem + sb * kBN;
 #pragma unroll
-        for (int part = 0; part < 2; ++part)   // P_hi, then P_lo
+        for (int part = 0; part < 2; ++part)   // P_hi, then P_lo (keys 64h.. at 64h + 32 part + 8 (kk & 3))
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk)
             tc_mma_ts(tmem + kTmemO, pt + (kk >> 2) * 64 + part * 32 + (kk & 3) * 8,
