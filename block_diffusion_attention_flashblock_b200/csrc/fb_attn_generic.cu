@@ -554,12 +554,13 @@ static cudaError_t launch_mma(const AttnArgs& a, cudaStream_t s) {
   constexpr int base = (64 * D + 4 * 64 * D) * 2;
   const int smem =
       base + (a.sel && a.keys_per_split <= kMaxGatherKeys ? (int)((a.keys_per_split * 4 + 15) / 16 * 16) : 0);
-  static bool attr_set = false;
-  if (!attr_set) {
+  static bool attr_set[kMaxDevices] = {};   // the attribute is per device
+  bool& done = attr_set[current_device()];
+  if (!done) {
     cudaError_t e = cudaFuncSetAttribute(attn_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          base + kMaxGatherKeys * 4);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    done = true;
   }
   dim3 grid(a.rm.units * a.rm.row_tiles, a.nsplit);
   return launch_k(attn_mma_kernel<D>, grid, dim3(128), smem, s, a);

@@ -879,11 +879,12 @@ cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys
   a.excl_invert = excl_invert ? 1 : 0;
   a.stall = debug_stall() ? 1 : 0;
   if (!a.status) return cudaErrorInvalidValue;
-  static bool attr = false;
-  if (!attr) {
+  static bool attr[kMaxDevices] = {};   // the attribute is per device
+  bool& done = attr[current_device()];
+  if (!done) {
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr = true;
+    done = true;
   }
   dim3 grid(m.units * m.tiles_per_unit, nsplit);
   if (a.cluster <= 1) return launch_k(attn_tc_kernel, grid, dim3(kThreads), kSmemBytes, s, m.q, m.k, m.v, a);

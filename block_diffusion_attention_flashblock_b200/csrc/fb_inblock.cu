@@ -374,12 +374,13 @@ cudaError_t launch_inblock_small(const fb_attn_desc& d, const void* q, const voi
                       2 * (size_t)kRows * kExtStride * 4 + 4 * 8;
   const dim3 grid(d.B * d.Hkv * a.tiles_per_unit);
   // instances above the default 48 KB of dynamic shared memory opt in once
-  static bool opted[3][kMaxExt + 1] = {};
+  static bool opted[kMaxDevices][3][kMaxExt + 1] = {};   // the attribute is per device
+  const int dev = current_device();
   auto run = [&](void (*kern)(InblockArgs), int nbi) -> cudaError_t {
-    if (smem > 48 * 1024 && !opted[nbi][next]) {
+    if (smem > 48 * 1024 && !opted[dev][nbi][next]) {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
-      opted[nbi][next] = true;
+      opted[dev][nbi][next] = true;
     }
     return launch_k(kern, grid, dim3(128), smem, s, a);
   };

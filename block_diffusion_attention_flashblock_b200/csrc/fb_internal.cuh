@@ -108,6 +108,15 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
   return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
 }
 
+// Index of the current device for per-device host caches (0 when it cannot
+// be read; caches hold kMaxDevices entries).
+constexpr int kMaxDevices = 64;
+inline int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) dev = 0;
+  return dev;
+}
+
 // Host-side planning helpers (fb_api.cu).
 int num_sms();
 RowMap make_rowmap(int B, int Hq, int Hkv, int Nb, int per_head, int tile_rows);
