@@ -474,9 +474,10 @@ __global__ void __launch_bounds__(64 * (D / 64)) attn_f32_kernel(const AttnArgs 
     const int nk = (int)min((int64_t)BN, kend - key0);
     for (int j = 0; j < nk; ++j) {
       const float* kr = sK + j * D + half * DH;
-      float s = 0.f;
+      float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // 8 independent FMA chains
 #pragma unroll
-      for (int d = 0; d < DH; ++d) s = fmaf(qr[d], kr[d], s);
+      for (int d = 0; d < DH; ++d) s8[d & 7] = fmaf(qr[d], kr[d], s8[d & 7]);
+      float s = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
       if (TPR == 2) s += __shfl_xor_sync(0xffffffffu, s, 1);
       s *= a.scale_log2;
       if (key_excluded(a, ri.b, ri.h, key0 + j)) s = -CUDART_INF_F;
