@@ -54,3 +54,27 @@ def test_selection_top_k_ascending_ties_low_index():
         kth = np.sort(score[h])[::-1][36]
         assert np.all(score[h][s] >= kth)
         assert (score[h] > kth).sum() <= 37
+
+
+def test_sweep_workloads_restate_their_recipe():
+    # context sweep: the long-context layer at B = 1 from 100k to 800k tokens
+    for n in (100, 200, 400, 800):
+        s = wl.get_spec(f"dllm_ctx_{n}k")
+        assert (s.B, s.Hq, s.Hkv, s.D, s.Nb, s.steps, s.tau) == (1, 32, 8, 128, 64, 16, 16)
+        assert s.prefix0 == n * 1000 and s.m_model == ("binomial", 64, 0.1)
+    # sparse density: the selected fraction of the 32k prefix
+    for pct in (20, 30, 40):
+        s = wl.get_spec(f"sparse_32k_d{pct}")
+        assert s.sel_k == 32768 * pct // 100 and s.prefix0 == 32768 and s.tau == 8
+    # small blocks: 4 tokens, at most 4 change per step, tau 2
+    s = wl.get_spec("dllm_8k_nb4")
+    assert s.Nb == 4 and s.tau == 2 and s.m_model == ("binomial", 4, 0.15)
+    w = wl.Workload(wl.get_spec("dllm_8k_nb4", prefix0=64, blocks=2))
+    steps = list(w.schedule())
+    assert len(steps) == 16 and all(0 <= st.M <= 4 for st in steps)
+    assert steps[0].q.shape == (1, 32, 4, 128)
+
+
+def test_distinct_seeds_per_workload():
+    seeds = [s.seed for s in wl.SPECS.values()]
+    assert len(seeds) == len(set(seeds))
