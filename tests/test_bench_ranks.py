@@ -46,3 +46,18 @@ def test_max_over_ranks_single_rank_is_identity():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.max_over_ranks(2.25, 1, torch.device("cpu")) == 2.25
+
+
+def test_layer_count_puts_the_kv_caches_past_l2():
+    """bench.py steps NL layers with their own KV caches so that the caches
+    together exceed twice the L2 (at least 2, at most 8 layers)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from block_diffusion_attention_flashblock_b200 import workloads as wl
+    for name, spec in wl.SPECS.items():
+        nl = bench.n_layers(spec)
+        kv = 2 * spec.B * spec.Hkv * spec.lcap * spec.D * (4 if spec.dtype == "f32" else 2)
+        assert 2 <= nl <= 8, name
+        assert nl == 8 or nl * kv >= 2 * bench.L2_BYTES, name
+    assert bench.n_layers(wl.get_spec("dllm_8k")) == 8
+    assert bench.n_layers(wl.get_spec("dllm_64k_b4")) == 2
