@@ -1,18 +1,18 @@
 """Benchmark of the FlashBlock attention step on B200 (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload dllm_8k] [--no-e2e]
+                    [--workload dllm_64k_b4] [--extra video_1560,dllm_8k] [--no-e2e]
 
-A timed "step" is one pass of the whole hot path over one workload: the
-diffusion-LM schedule (dllm_8k: B 1, 32 query / 8 KV heads, head dim 128,
-prefix 8192 tokens growing by 32 per block, blocks of 32 tokens, 8 diffusion
-steps per block, 4 blocks, tau = 8) for each of NL attention layers, every
-layer with its own KV cache, cache state and inputs.  Every diffusion step
-runs fb_step for each layer in turn under the reuse policy, and every block
-ends with fb_kv_append.  NL is chosen so that the layers' KV caches together
-exceed twice the L2: as between the layers of a model, each layer's data has
-left L2 by the time its next step runs.  L2 is also flushed (a 1 GiB write)
-before every timed step, outside the timed interval.
+A timed "step" is one pass of the whole hot path over one workload, by default
+the long-context diffusion-LM layer (dllm_64k_b4: B 4, 32 query / 8 KV heads,
+head dim 128, prefix 65,536 tokens, blocks of 64 tokens, 16 diffusion steps,
+tau = 16), the largest workload that fits one GPU, for each of NL attention
+layers, every layer with its own KV cache, cache state and inputs.  Every
+diffusion step runs fb_step for each layer in turn under the reuse policy, and
+every block ends with fb_kv_append.  NL is chosen so that the layers' KV caches
+together exceed twice the L2: as between the layers of a model, each layer's
+data has left L2 by the time its next step runs.  L2 is also flushed (a 1 GiB
+write) before every timed step, outside the timed interval.
 
 The metric is query tokens per second: B * Nb per layer-step (one fb_step of
 one layer, all heads), over all layer-steps of the timed step.  The same
@@ -23,9 +23,16 @@ The whole step is captured once as a CUDA graph (the reuse decisions are taken
 on the host while capturing, in schedule order) and replayed between two CUDA
 events; the same calls made eagerly are reported under "eager", and "e2e"
 repeats the eager pass with every layer-step's inputs copied from pinned host
-memory and its outputs read back.  The roofline comes from graphs of one
-library call repeated over the layers (so no per-launch event overhead enters
-the duration), with launch counts and algorithmic bytes from a profiled pass.
+memory and its outputs read back.
+
+The roofline is that of the dominant kernel, timed L2-cold: the prefix
+kernel's launches bracketed by CUDA events on their stream, with L2 flushed
+before each round of calls; the in-block call (one kernel) as a graph over
+enough distinct input sets that each call's data has left L2.  Its bytes are
+the method's (K/V and Q read once, one (A, L) written; split partials and their
+merge do not count).  The warm figure (the same call repeated) is reported
+beside it.  The other workloads named by --extra are measured the same way
+and reported under "workloads".
 
 `--impl reference` times the fp64 CPU oracle on this host's cores on a
 bounded sample of the same schedule (the reference arm; there is no other
@@ -171,11 +178,29 @@ class Layers:
             d["layer"].close()
 
 
-def run_ours(args, spec, rank, world, device):
+def _call_cost(spec):
+    """Algorithmic bytes and FLOPs of one library call of each kind, by the
+    method's definition: every input read once, every output written once;
+    split-KV partials, their merge and re-reads do not count."""
+    s = spec
+    e = 4 if s.dtype == "f32" else 2
+    rows = s.B * s.Hq * s.Nb
+    P = s.prefix0
+    q = rows * s.D * e
+    part = rows * (s.D + 1) * 4                       # one fp32 (A, L)
+    kv_prefix = 2 * s.B * s.Hkv * P * s.D * e
+    kv_block = 2 * s.B * s.Hkv * s.Nb * s.D * e
+    out = rows * (s.D * e + 4)                        # O in the input dtype, LSE fp32
+    return {
+        "prefix_attention": {"bytes": kv_prefix + q + part, "flops": 4.0 * rows * P * s.D},
+        "inblock_merge": {"bytes": q + kv_block + part + out, "flops": 4.0 * rows * s.Nb * s.D},
+    }
+
+
+def measure_workload(args, spec, rank, world, device, headline):
+    """Run and time one workload; returns the fields of its JSON record."""
     from block_diffusion_attention_flashblock_b200 import fb
     torch.cuda.set_device(device)
-    fb.fb_debug_set_prefix_kernel({"auto": 0, "generic": 1, "tcgen05": 2, "tcgen05-nocluster": 3, "tcgen05-cluster": 4}[args.prefix_kernel])
-    fb.fb_debug_set_pdl(not args.no_pdl)
     nl = n_layers(spec)
     S = Layers(spec, device, nl)
     s = spec
@@ -208,10 +233,11 @@ def run_ours(args, spec, rank, world, device):
             rec.append(S.L[0]["layer"].last_recomputed())
         return rec
 
-    def timed_region(fn, steps, warmup):
+    def timed_region(fn, steps, warmup, do_flush=True):
         """Flush L2, then time fn() between two CUDA events; max over ranks."""
         for _ in range(warmup):
-            flush.zero_()
+            if do_flush:
+                flush.zero_()
             fn()
         torch.cuda.synchronize()
         if world > 1:
@@ -219,7 +245,8 @@ def run_ours(args, spec, rank, world, device):
         torch.cuda.synchronize()
         ev = []
         for _ in range(steps):
-            flush.zero_()
+            if do_flush:
+                flush.zero_()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             fn()
@@ -241,20 +268,24 @@ def run_ours(args, spec, rank, world, device):
     tau_on = s.tau if s.tau is not None else fb.FB_TAU_OFF
     ho = [torch.empty(S.L[0]["o"].shape, dtype=S.L[0]["o"].dtype, pin_memory=True) for _ in S.steps]
     hl = [torch.empty(S.L[0]["lse"].shape, dtype=torch.float32, pin_memory=True) for _ in S.steps]
-    props = torch.cuda.get_device_properties(device)
-    try:
-        smi_id = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
-    except AttributeError:
-        smi_id = str(device.index)
-    clocks = ClockSampler(smi_id)
+    clk = None
+    steps = args.steps if headline else max(3, args.steps // 2)
 
     # eager library calls
-    ms_eager = timed_region(lambda: schedule(tau_on), args.steps, args.warmup)
+    ms_eager = timed_region(lambda: schedule(tau_on), steps, args.warmup)
     # the whole schedule as one CUDA graph (the headline number)
     g_on, rec_on = graph_of(lambda: schedule(tau_on))
-    clocks.start()
-    ms_on = timed_region(g_on.replay, args.steps, args.warmup)
-    clk = clocks.stop()
+    if headline:
+        props = torch.cuda.get_device_properties(device)
+        try:
+            smi_id = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+        except AttributeError:
+            smi_id = str(device.index)
+        clocks = ClockSampler(smi_id)
+        clocks.start()
+    ms_on = timed_region(g_on.replay, steps, args.warmup)
+    if headline:
+        clk = clocks.stop()
     del g_on
     # per-kernel launch counts and algorithmic bytes (one eager pass, events per launch)
     fb.fb_profile_read(reset=True)
@@ -266,11 +297,11 @@ def run_ours(args, spec, rank, world, device):
     ms_full = None
     if not args.profile_run:
         g_full, _ = graph_of(lambda: schedule(0))
-        ms_full = timed_region(g_full.replay, args.steps, args.warmup)
+        ms_full = timed_region(g_full.replay, steps, args.warmup)
         del g_full
     e2e = None
-    if not args.no_e2e and not args.profile_run:
-        ms_e2e = timed_region(lambda: schedule(tau_on, e2e=True), args.steps, args.warmup)
+    if headline and not args.no_e2e and not args.profile_run:
+        ms_e2e = timed_region(lambda: schedule(tau_on, e2e=True), steps, args.warmup)
         h2d = nl * sum(h["q"].numel() * h["q"].element_size() + 2 * h["kin"].numel() * h["kin"].element_size()
                        for h in S.host)
         d2h = nl * (sum(x.numel() * x.element_size() for x in ho) + sum(x.numel() * x.element_size() for x in hl))
@@ -299,13 +330,12 @@ def run_ours(args, spec, rank, world, device):
 
     g_reuse, _ = graph_of(lambda: [reuse_round() for _ in range(R)])
     reuse_recomputed = S.L[0]["layer"].last_recomputed()
-    ms_reuse = timed_region(g_reuse.replay, args.steps, args.warmup)
+    ms_reuse = timed_region(g_reuse.replay, steps, args.warmup)
     del g_reuse
 
-    # Per-kind launch durations without per-launch event overhead: a graph of
-    # R rounds over the layers of one library call, L2 flushed before it.
-    st_mid = S.steps[0]
-    P = st_mid.prefix_len
+    # ---- per-kind call and kernel durations --------------------------------
+    P = S.steps[0].prefix_len
+    cost = _call_cost(s)
     parts = []
     for d in S.L:
         a = torch.empty(s.B, s.Hq, s.Nb, s.D, dtype=torch.float32, device=device)
@@ -319,74 +349,115 @@ def run_ours(args, spec, rank, world, device):
             x = d["x"][0]
             fb.fb_attn_outblock(d["layer"].desc, x["q"], d["kp"], d["vp"], P, a, l, ws)
 
-    def call_inblock():
-        for d, (a, l, ws) in zip(S.L, parts):
-            x = d["x"][0]
-            fb.fb_attn_inblock(d["layer"].desc, x["q"], x["kin"], x["vin"], d["o"], d["lse"], [a], [l])
-
     call_prefix()
+    torch.cuda.synchronize()
+    # distinct in-block input sets, enough that together they exceed twice the
+    # L2, so a pass over them finds each call's data cold
+    ib_bytes = cost["inblock_merge"]["bytes"]
+    n_sets = int(min(512, max(nl, -(-2 * L2_BYTES // ib_bytes))))
+    x0 = S.L[0]["x"][0]
+    a0, l0, _ = parts[0]
+    sets = []
+    for i in range(n_sets):
+        sets.append(dict(q=x0["q"].clone(), kin=x0["kin"].clone(), vin=x0["vin"].clone(), a=a0.clone(),
+                         l=l0.clone(), o=torch.empty_like(S.L[0]["o"]), lse=torch.empty_like(S.L[0]["lse"])))
+    desc0 = S.L[0]["layer"].desc
+
+    def call_inblock_set(z):
+        fb.fb_attn_inblock(desc0, z["q"], z["kin"], z["vin"], z["o"], z["lse"], [z["a"]], [z["l"]])
+
     per_kind = {}
-    for kind, fn in (("prefix_attention", call_prefix), ("inblock_merge", call_inblock)):
-        fb.fb_profile_read(reset=True)
-        fb.fb_profile_enable(True)
-        fn()
+    # prefix: the kernel alone, cold (events per launch from the profiling
+    # hook, L2 flushed before each round over the layers), and the whole call
+    # (kernel + merge of its split parts) warm, as a graph of repeated calls
+    fb.fb_profile_read(reset=True)
+    for r in range(R + 1):
+        flush.zero_()
         torch.cuda.synchronize()
-        fb.fb_profile_enable(False)
-        pk = fb.fb_profile_read(reset=True)
-        g, _ = graph_of(lambda: [fn() for _ in range(R)])
-        ms = timed_region(g.replay, args.steps, args.warmup)
-        del g
-        calls = R * nl
-        byts = sum(v[2] for v in pk.values()) / nl
-        nk = P if kind == "prefix_attention" else s.Nb
-        flops = 4.0 * s.B * s.Hq * s.Nb * nk * s.D   # Q K^T and P V, algorithmic
-        per_kind[kind] = {"call": "fb_attn_outblock" if kind == "prefix_attention" else
-                          "fb_attn_inblock (one cached external part; above 64-token blocks this public call runs "
-                          "the generic kernel, fb_step the tcgen05 pass)",
-                          "kernels_per_call": sum(v[0] for v in pk.values()) / nl,
-                          "own_kernels_per_call": pk[kind][0] / nl,
-                          "avg_call_us": 1e3 * ms / calls, "alg_bytes_per_call": byts, "alg_flops_per_call": flops,
-                          "achieved_GBps": byts / (ms * 1e-3 / calls) / 1e9,
-                          "achieved_TFLOPs": flops / (ms * 1e-3 / calls) / 1e12}
+        fb.fb_profile_enable(r > 0)
+        call_prefix()
+        torch.cuda.synchronize()
+    fb.fb_profile_enable(False)
+    pk = fb.fb_profile_read(reset=True)
+    n_prefix_launch = pk["prefix_attention"][0]
+    us_prefix_cold = 1e3 * pk["prefix_attention"][1] / max(1, n_prefix_launch)
+    g, _ = graph_of(lambda: [call_prefix() for _ in range(R)])
+    ms = timed_region(g.replay, steps, args.warmup)
+    del g
+    us_prefix_call_warm = 1e3 * ms / (R * nl)
+    per_kind["prefix_attention"] = {
+        "call": "fb_attn_outblock", "kernel": "attn_tc_kernel (tcgen05)" if s.dtype == "bf16" and s.D == 128
+        else "attn generic", "kernels_per_call": (pk["prefix_attention"][0] + pk["aux"][0]) / (R * nl),
+        "avg_launch_us_cold": us_prefix_cold, "avg_call_us_warm": us_prefix_call_warm,
+        "alg_bytes_per_launch": cost["prefix_attention"]["bytes"],
+        "alg_flops_per_launch": cost["prefix_attention"]["flops"],
+        "timing": f"cold: CUDA events around each of {R * nl} kernel launches, L2 flushed before each round of "
+                  f"{nl}; warm: one graph of {R * nl} calls (kernel + merge of the split parts)"}
+    # in-block: a graph over n_sets distinct input sets (cold), and a graph of
+    # the same set repeated (warm)
+    g, _ = graph_of(lambda: [call_inblock_set(z) for z in sets])
+    ms_cold = timed_region(g.replay, steps, args.warmup)
+    del g
+    g, _ = graph_of(lambda: [call_inblock_set(sets[0]) for _ in range(n_sets)])
+    ms_warm = timed_region(g.replay, steps, args.warmup)
+    del g
+    fb.fb_profile_read(reset=True)
+    fb.fb_profile_enable(True)
+    call_inblock_set(sets[0])
+    torch.cuda.synchronize()
+    fb.fb_profile_enable(False)
+    pk_ib = fb.fb_profile_read(reset=True)
+    per_kind["inblock_merge"] = {
+        "call": "fb_attn_inblock with one cached external part" + (
+            "" if s.Nb <= 64 else " (above 64-token blocks this public call runs the generic kernel; fb_step "
+                                  "runs the tcgen05 pass)"),
+        "kernels_per_call": sum(v[0] for v in pk_ib.values()),
+        "avg_launch_us_cold": 1e3 * ms_cold / n_sets, "avg_call_us_warm": 1e3 * ms_warm / n_sets,
+        "alg_bytes_per_launch": cost["inblock_merge"]["bytes"],
+        "alg_flops_per_launch": cost["inblock_merge"]["flops"],
+        "timing": f"cold: one graph over {n_sets} distinct input sets (together > 2x L2), L2 flushed before; "
+                  f"warm: one graph of {n_sets} calls on one set"}
+    del sets
     assert fb.fb_get_device_status() == fb.FB_OK
     S.close()
 
     hbm, tf, tf_sus, peak_src = _peaks()
-    # the dominant kind: its calls in the schedule x the graph-timed call duration
-    share = {k: prof[k][0] / max(1e-9, per_kind[k]["own_kernels_per_call"]) * per_kind[k]["avg_call_us"]
-             for k in per_kind}
+    ridge = tf * 1e12 / (hbm * 1e9)
+    for k, v in per_kind.items():
+        for tag in ("cold", "warm"):
+            t = v["avg_launch_us_cold"] if tag == "cold" else v["avg_call_us_warm"]
+            v[f"achieved_GBps_{tag}"] = v["alg_bytes_per_launch"] / (t * 1e-6) / 1e9
+            v[f"achieved_TFLOPs_{tag}"] = v["alg_flops_per_launch"] / (t * 1e-6) / 1e12
+    # the dominant kernel: its launches in the schedule x its cold launch duration
+    share = {k: prof[k][0] * per_kind[k]["avg_launch_us_cold"] for k in per_kind}
+    total = sum(share.values()) or 1.0
     dom = max(share, key=share.get)
     pkd = per_kind[dom]
     traffic = _ncu_traffic(dom, spec.name)
-    # bound: the tensor pipe when the call's algorithmic flop per byte exceeds
-    # the ridge of the measured peaks, else HBM
-    ridge = tf * 1e12 / (hbm * 1e9)
-    tensor = pkd["alg_flops_per_call"] / pkd["alg_bytes_per_call"] > ridge
+    tensor = pkd["alg_flops_per_launch"] / pkd["alg_bytes_per_launch"] > ridge
     roof = {"kernel": dom, "call": pkd["call"], "bound": "tensor" if tensor else "hbm",
-            "achieved": pkd["achieved_TFLOPs"] if tensor else pkd["achieved_GBps"],
+            "achieved": pkd["achieved_TFLOPs_cold"] if tensor else pkd["achieved_GBps_cold"],
             "peak": tf if tensor else hbm, "unit": "TFLOP/s" if tensor else "GB/s",
-            "frac": pkd["achieved_TFLOPs"] / tf if tensor else pkd["achieved_GBps"] / hbm,
+            "frac": pkd["achieved_TFLOPs_cold"] / tf if tensor else pkd["achieved_GBps_cold"] / hbm,
             "peak_source": f"{peak_src} " + ("bf16_tflops (burst)" if tensor else "hbm_gbs (burst)"),
-            "frac_hbm": pkd["achieved_GBps"] / hbm, "frac_tensor": pkd["achieved_TFLOPs"] / tf,
-            "traffic": traffic, "alg_bytes_per_launch": pkd["alg_bytes_per_call"],
-            "alg_flops_per_launch": pkd["alg_flops_per_call"], "avg_launch_us": pkd["avg_call_us"],
-            "timing": f"CUDA events around one graph of {R * nl} calls ({nl} layers x {R}), L2 flushed before"}
+            "frac_hbm": pkd["achieved_GBps_cold"] / hbm, "frac_tensor": pkd["achieved_TFLOPs_cold"] / tf,
+            "frac_warm": (pkd["achieved_TFLOPs_warm"] / tf if tensor else pkd["achieved_GBps_warm"] / hbm),
+            "traffic": traffic, "alg_bytes_per_launch": pkd["alg_bytes_per_launch"],
+            "alg_flops_per_launch": pkd["alg_flops_per_launch"], "avg_launch_us": pkd["avg_launch_us_cold"],
+            "share_of_kernel_time": share[dom] / total, "timing": pkd["timing"]}
     kernels = {k: {"launches_per_step": v[0], "alg_bytes_per_step": v[2]} for k, v in prof.items()}
     n_full = sum(rec_on)
     layer_steps = nsteps * nl
     step_lat = {"mean_us": 1e3 * ms_on / layer_steps}
     if ms_full is not None:
-        t_full = ms_full / layer_steps
-        step_lat["full_step_us"] = 1e3 * t_full
+        step_lat["full_step_us"] = 1e3 * ms_full / layer_steps
     step_lat["reuse_step_us"] = 1e3 * ms_reuse / (R * nl)
     if reuse_recomputed:
         step_lat["reuse_step_note"] = "the gate recomputed at least one head in the measured reuse step"
     gpu_launches = sum(v[0] for v in prof.values())
     return {
-        "metric": METRIC, "value": world * S.query_tokens / (ms_on * 1e-3), "unit": UNIT,
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_on,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": spec.dtype,
-        "data": "synthetic (seeded; shapes of the pages' diffusion-LM workload)",
+        "value": world * S.query_tokens / (ms_on * 1e-3), "ms_per_step": ms_on, "steps": steps,
+        "dtype": spec.dtype,
         "config": {"workload": _describe(spec), "layers": nl,
                    "query_tokens_per_step": S.query_tokens,
                    "prefix_kernel": args.prefix_kernel, "diffusion_steps_per_layer": nsteps,
@@ -395,15 +466,46 @@ def run_ours(args, spec, rank, world, device):
                          f"KV caches are stepped in turn, so each layer's data has left L2 when it runs",
                    "parallelism": f"replicas x{world}", "full_steps_per_layer": n_full},
         "step_latency": step_lat,
-        "timing": "one CUDA graph of the whole schedule (all layers), replayed; CUDA events around each replay",
         "eager": {"value": world * S.query_tokens / (ms_eager * 1e-3), "ms_per_step": ms_eager},
         "full_recompute": None if ms_full is None else {
             "value": world * S.query_tokens / (ms_full * 1e-3), "ms_per_step": ms_full,
             "mean_step_us": 1e3 * ms_full / layer_steps},
         "speedup_vs_full_recompute": None if ms_full is None else ms_full / ms_on,
         "e2e": e2e, "roofline": roof, "per_call": per_kind, "kernels": kernels,
-        "gpu_launches": gpu_launches * args.steps, "gpu_launches_per_step": gpu_launches, "clocks": clk,
+        "gpu_launches_per_step": gpu_launches, "clocks": clk,
     }
+
+
+def run_ours(args, spec, rank, world, device):
+    from block_diffusion_attention_flashblock_b200 import fb
+    torch.cuda.set_device(device)
+    fb.fb_debug_set_prefix_kernel({"auto": 0, "generic": 1, "tcgen05": 2, "tcgen05-nocluster": 3,
+                                   "tcgen05-cluster": 4}[args.prefix_kernel])
+    fb.fb_debug_set_pdl(not args.no_pdl)
+    r = measure_workload(args, spec, rank, world, device, headline=True)
+    out = {
+        "metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": r["dtype"],
+        "data": "synthetic (seeded; shapes of the pages' diffusion-LM and video workloads)",
+        "config": r["config"], "step_latency": r["step_latency"],
+        "timing": "one CUDA graph of the whole schedule (all layers), replayed; CUDA events around each replay",
+    }
+    for k in ("eager", "full_recompute", "speedup_vs_full_recompute", "e2e", "roofline", "per_call", "kernels",
+              "clocks"):
+        out[k] = r[k]
+    out["gpu_launches"] = r["gpu_launches_per_step"] * args.steps
+    out["gpu_launches_per_step"] = r["gpu_launches_per_step"]
+    extras = {}
+    for name in [n for n in (args.extra or "").split(",") if n and n != spec.name]:
+        e = measure_workload(args, wl.get_spec(name), rank, world, device, headline=False)
+        extras[name] = {k: e[k] for k in ("value", "ms_per_step", "steps", "dtype", "step_latency",
+                                          "speedup_vs_full_recompute", "roofline", "per_call")}
+        extras[name]["workload"] = e["config"]["workload"]
+        extras[name]["layers"] = e["config"]["layers"]
+    if extras:
+        out["workloads"] = extras
+    return out
 
 
 def kernels_only(spec, device, n):
@@ -500,7 +602,9 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="dllm_8k", choices=list(wl.SPECS))
+    ap.add_argument("--workload", default="dllm_64k_b4", choices=list(wl.SPECS))
+    ap.add_argument("--extra", default="video_1560,dllm_8k",
+                    help="comma-separated workloads also measured and reported under 'workloads' ('' for none)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-pdl", action="store_true", help="launch kernels in plain stream order")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
@@ -512,6 +616,8 @@ def main():
                     help="only the reuse-on schedule (no full-recompute, e2e or CPU legs): for ncu captures")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
+    if args.profile_run or args.kernels_only:
+        args.extra = ""
     spec = wl.get_spec(args.workload)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -25,10 +25,20 @@ bool pdl_enabled() { return g_pdl; }
 static bool g_stall = false;
 bool debug_stall() { return g_stall; }
 
+// Device address of this device's status word, looked up once per device (the
+// first launch on a device should come before any stream capture on it; a
+// cudaDeviceReset in the process invalidates the cached address).
 int* device_status_ptr() {
-  int* p = nullptr;
-  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_fb_status) != cudaSuccess) return nullptr;
-  return p;
+  static int* cache[kMaxDevices] = {};
+  static std::mutex mu;
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    int* p = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_fb_status) != cudaSuccess) return nullptr;
+    cache[dev] = p;
+  }
+  return cache[dev];
 }
 
 int num_sms() {
@@ -607,6 +617,8 @@ struct fb_cache {
   int32_t max_sel_k;
   bool valid;
   int32_t last_recomputed;
+  int64_t cached_prefix;   // prefix length and selection size the cached part was computed over
+  int32_t cached_sel_k;    // -1: dense
   float* cache_a;     // block-external (or residual) part, packed fp32
   float* cache_l;
   float* part_a;      // split partials of the prefix / residual pass
@@ -744,8 +756,15 @@ fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
       !al16(a->lse) || !al16(a->sel) || !al16(a->gamma))
     return FB_EALIGN;
 
+  // The cached part is attention over one block-external key set; a step over
+  // another set (the prefix grew, or the selection size changed) cannot reuse
+  // it, so it starts over as at a new block.
+  if (c->valid && (a->prefix_len != c->cached_prefix || (sparse ? a->sel_k : -1) != c->cached_sel_k))
+    c->valid = false;
   const bool tau_reuse = c->valid && (a->M < a->tau);
   const int BH = d.B * d.Hq;
+  c->cached_prefix = a->prefix_len;
+  c->cached_sel_k = sparse ? a->sel_k : -1;
   fb_status st;
   PartList ext;
   memset(&ext, 0, sizeof(ext));

@@ -31,6 +31,10 @@
  * - Kernels that wait on barriers bound each wait (about 2 s by default); on
  *   expiry they record FB_ETIMEOUT in a per-device status word and return
  *   without touching their outputs further.  fb_get_device_status() reads it.
+ *   The word's device address is looked up at the first launch on each
+ *   device: make one call on a device before capturing its work in a CUDA
+ *   graph.  The library is not usable after a cudaDeviceReset in the same
+ *   process (cached device addresses and function attributes go stale).
  * - Handles are not thread-safe.
  */
 #ifndef FB_H
@@ -118,7 +122,8 @@ fb_status fb_attn_outblock(const fb_attn_desc* d, const void* q, const void* kp,
  *   process exits.
  * - The first call on a device looks up the array's device address (with
  *   that device current) and caches it.  Make that first call before any
- *   stream capture.
+ *   stream capture.  The cached address does not survive a cudaDeviceReset
+ *   in the same process: do not call the library after one.
  * - All calls share the array, and it keeps the last call's contents; this
  *   call overwrites everything it reads, so it needs no clearing.  Calls whose
  *   work overlaps on the GPU (unordered streams) race on it.
@@ -220,6 +225,12 @@ typedef struct fb_step_args {
 
 /* One diffusion step of one attention layer under the reuse policy:
  *   reuse(b, h) = cache valid && M < tau && (gamma off || sim(b, h) > gamma[h]).
+ * The cache is valid from the first step after fb_cache_begin_block on, and
+ * only for the block-external key set it was computed over: a step whose
+ * prefix_len, or sparse selection size sel_k (or dense/sparse kind), differs
+ * from the last step's starts over as at a new block (full step, similarities
+ * undefined).  A caller that changes the selection's contents but not its size
+ * must call fb_cache_begin_block itself.
  * Heads that do not reuse recompute the block-external part over the prefix
  * (or the residual, for sparse steps), refresh the cache and, with the gamma
  * gate on and the cache valid, refresh sim(b, h) = cosine of the fresh and the

@@ -221,6 +221,7 @@ class FlashBlockOracle:
         self.gamma = None if gamma is None else np.asarray(gamma, dtype=np.float64)
         self.cache_A = np.zeros((B, Hq, Nb, D))
         self.cache_L = np.full((B, Hq, Nb), NEG_INF)
+        self.key_set = None
         self.begin_block()
 
     def begin_block(self):
@@ -231,6 +232,14 @@ class FlashBlockOracle:
     def step(self, q, kin, vin, kp, vp, prefix_len: int, M: int,
              tau: Optional[int], sel=None) -> StepResult:
         B, Hq = self.B, self.Hq
+        # The cached part is attention over one block-external key set J_out
+        # ("Mécanisme Central"): the prefix, or for sparse steps the prefix
+        # minus the selection.  A step over another set cannot reuse it and
+        # starts over as at a new block.
+        key_set = (prefix_len, None if sel is None else np.asarray(sel).tobytes())
+        if self.valid and key_set != self.key_set:
+            self.begin_block()
+        self.key_set = key_set
         tau_reuse = self.valid and (tau is None or M < tau)   # strict "M < tau"
         if self.gamma is None:
             head_reuse = np.full((B, Hq), tau_reuse)

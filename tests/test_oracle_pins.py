@@ -285,6 +285,36 @@ def test_tau_decisions_enumerated():
     assert o.step(z, z, z, kp, kp, 3, 0, 2).recompute     # new block forces a full step
 
 
+def test_changed_key_set_recomputes():
+    """A cached part is attention over one block-external key set: after the
+    prefix grows (without a new block) or the selection changes, the step
+    recomputes even with tau off, and equals exact full attention over the
+    new prefix plus the block (tau off would otherwise reuse the stale part)."""
+    spec, work = _tiny(steps=2)
+    kp, vp = work.prefix_kv(); kp64, vp64 = orc.to64(kp), orc.to64(vp)
+    steps = list(work.schedule())
+    o = orc.FlashBlockOracle(spec.B, spec.Hq, spec.Hkv, spec.D, spec.Nb)
+    st = steps[0]
+    q, kin, vin = orc.to64(st.q), orc.to64(st.kin), orc.to64(st.vin)
+    assert o.step(q, kin, vin, kp64, vp64, 200, 0, None).recompute
+    assert not o.step(q, kin, vin, kp64, vp64, 200, 0, None).recompute   # same set: reuse
+    r = o.step(q, kin, vin, kp64, vp64, 256, 0, None)                    # the prefix grew
+    assert r.recompute
+    A, L = orc.full_attention(q, kin, vin, kp64, vp64, 256, 1 / 8)
+    np.testing.assert_allclose(r.o, A, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(r.lse, L, rtol=1e-12)
+    # sparse: a different selection over the same prefix is a different residual set
+    sel_a = np.tile(np.arange(0, 256, 4, dtype=np.int32), (1, spec.Hq, 1))
+    sel_b = np.tile(np.arange(1, 256, 4, dtype=np.int32), (1, spec.Hq, 1))
+    o.begin_block()
+    assert o.step(q, kin, vin, kp64, vp64, 256, 0, None, sel_a).recompute
+    assert not o.step(q, kin, vin, kp64, vp64, 256, 0, None, sel_a.copy()).recompute
+    r = o.step(q, kin, vin, kp64, vp64, 256, 0, None, sel_b)
+    assert r.recompute
+    A, L = orc.full_attention(q, kin, vin, kp64, vp64, 256, 1 / 8)
+    np.testing.assert_allclose(r.o, A, rtol=1e-11, atol=1e-12)
+
+
 def test_static_queries_reuse_equals_full():
     """Queries unchanged across steps: the cached A_out is exact, so every step equals full attention."""
     spec, work = _tiny(steps=4)

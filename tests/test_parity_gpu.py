@@ -239,6 +239,11 @@ def test_kv_append_bit_exact():
 # ------------------------------------------------------------ schedules ---
 SCHEDULES = {
     "tiny_f32": dict(),
+    # the fp32 path through fb_step with reuse: tau off reuses steps 1..3; tau 8
+    # reuses every step (M = 4, 7, 5); tau 6 alternates (reuse, recompute, reuse)
+    "tiny_f32_tau_off": dict(base="tiny_f32", tau=None),
+    "tiny_f32_tau8": dict(base="tiny_f32", tau=8),
+    "tiny_f32_tau6": dict(base="tiny_f32", tau=6),
     "dllm_8k_small": dict(base="dllm_8k", prefix0=1000, blocks=2, steps=8),
     "dllm_64k_small": dict(base="dllm_64k_b4", B=2, prefix0=2000, steps=16),
     "video_small_mixed": dict(base="video_1560", Hq=6, Hkv=6, prefix0=3120, steps=5, sigma_range=(0.01, 1.0)),
@@ -264,8 +269,10 @@ def test_step_schedule(name):
     st = compare_schedule(spec)
     if name == "tau_zero":
         assert all(st["recomputed"])
-    if name == "tau_off":
+    if name in ("tau_off", "tiny_f32_tau_off", "tiny_f32_tau8"):
         assert st["recomputed"] == [True, False, False, False]
+    if name == "tiny_f32_tau6":
+        assert st["recomputed"] == [True, False, True, False]
     if name == "video_small_mixed":
         r = np.array(st["reuse"])
         assert 0 < r[2:].mean() < 1, "the mixed video case should both reuse and recompute"
@@ -293,4 +300,31 @@ def test_full_dllm_8k_all_heads():
 def test_full_size_sampled_heads(name, groups):
     """Full-size workloads; the oracle recomputes only the sampled (b, kv-head) groups."""
     spec = wl.get_spec(name)
-    compare_schedule(spec, groups=groups, check_every={"dllm_64k_b4": 5, "dllm_ctx_200k": 4}.get(name, 1))
+    compare_schedule(spec, groups=groups, check_every=1)
+
+
+@pytest.mark.parametrize("sparse", [False, True])
+def test_step_changed_prefix_recomputes(sparse):
+    """fb_step on a longer prefix without a new block (tau off, so the stale
+    cache would otherwise be reused): the step recomputes, as the oracle's, and
+    both outputs agree; then a step on the same prefix reuses again."""
+    B, Hq, Hkv, D, Nb, Lp = 1, 8, 2, 128, 32, 1200
+    q, kin, vin, kp, vp = _mk(B, Hq, Hkv, D, Nb, Lp, "bf16", seed=71)
+    sel = wl.random_selection(B, Hq, Lp - 200, 64, seed=72) if sparse else None
+    qd, kind, vind, kpd, vpd = q.cuda(), kin.cuda(), vin.cuda(), kp.cuda(), vp.cuda()
+    o = torch.empty(B, Hq, Nb, D, device="cuda")
+    lse = torch.empty(B, Hq, Nb, device="cuda")
+    layer = fb.FlashBlockLayer(qd, kind, kpd, o, max_prefix=Lp, sparse=sparse, max_sel_k=64)
+    ref = orc.FlashBlockOracle(B, Hq, Hkv, D, Nb)
+    q64, k64, v64, kp64, vp64 = (orc.to64(t) for t in (q, kin, vin, kp, vp))
+    seld = None if sel is None else sel.cuda()
+    seln = None if sel is None else sel.numpy()
+    layer.begin_block()
+    for plen, expect in ((Lp - 200, True), (Lp - 200, False), (Lp, True), (Lp, False)):
+        layer.step(qd, kind, vind, kpd, vpd, plen, 0, fb.FB_TAU_OFF, o, lse, sel=seld)
+        r = ref.step(q64, k64, v64, kp64, vp64, plen, 0, None, seln)
+        assert layer.last_recomputed() == r.recompute == expect
+        assert_o_close(o, r.o, TOL["bf16"], f"prefix {plen}")
+        assert_lse_close(lse, r.lse, TOL["bf16"], f"prefix {plen}")
+    layer.close()
+    assert fb.fb_get_device_status() == fb.FB_OK

@@ -1,9 +1,10 @@
 """fb_attn_outblock_noalloc: block-external attention for callers that cannot
 allocate device memory (their host framework owns the pool, or they may not
 allocate while serving).  Its split-KV scratch is a fixed array inside the
-library, so the test checks it against fb_attn_outblock with caller scratch on
-two calls in a row (the second call reuses whatever the first left in the
-array), and that a call needing more than the array is refused.
+library, so the test checks it against fb_attn_outblock with caller scratch,
+and against the fp64 oracle, on two calls in a row (the second call reuses
+whatever the first left in the array), and that a call needing more than the
+array is refused.
 
 This file sorts last so that a run stopping at the first failure has run every
 other test before it; it also passes on its own in a fresh process.
@@ -14,6 +15,7 @@ import torch
 
 from block_diffusion_attention_flashblock_b200 import fb
 from block_diffusion_attention_flashblock_b200 import workloads as wl
+from oracle import flashblock_oracle as orc
 
 from _gpu_common import TOL, assert_lse_close, assert_o_close
 
@@ -46,6 +48,10 @@ def test_noalloc_matches_scratch_version_twice(shape):
         assert fb.fb_get_device_status() == fb.FB_OK
         assert_o_close(a, a_ref.double().cpu().numpy(), TOL["bf16"], f"A_out, call {call}")
         assert_lse_close(l, l_ref.double().cpu().numpy(), TOL["bf16"], f"L_out, call {call}")
+        # and independently against the fp64 oracle on the same inputs
+        A, L = orc.outblock(orc.to64(q.cpu()), orc.to64(kp.cpu()), orc.to64(vp.cpu()), Lp, 1 / np.sqrt(128))
+        assert_o_close(a, A, TOL["bf16"], f"A_out vs oracle, call {call}")
+        assert_lse_close(l, L, TOL["bf16"], f"L_out vs oracle, call {call}")
 
 
 def test_noalloc_refuses_beyond_its_array():
