@@ -172,8 +172,10 @@ static int32_t split_bound(const fb_attn_desc& d, int per_head, int64_t max_keys
   plan_split((int64_t)rm.units * rm.row_tiles, std::max<int64_t>(max_keys, 1),
              generic_ctas_per_sm(d.D, d.in_dtype == FB_BF16), generic_key_tile(), &ns, &kps);
   int mode, hg, tpu, units;
-  if (!per_head && tc_tiling(d, &mode, &hg, &tpu, &units))
+  if (!per_head && tc_tiling(d, &mode, &hg, &tpu, &units)) {
     ns = std::max(ns, tc_split_cap((int64_t)units * tpu, max_keys));
+    ns = std::max(ns, pair_slot_cap(d, max_keys));
+  }
   return ns;
 }
 
@@ -231,11 +233,14 @@ static fb_status launch_pass(const fb_attn_desc& d, AttnArgs& a, float* pa, floa
 
 // Dense block-external pass over prefix rows [0, nkeys): the tcgen05 kernel
 // when the shape and strides allow it, else the generic kernel.
-static int g_prefix_kernel = 0;  // 0 auto, 1 generic only, 2 tcgen05 whenever it applies, 3 as 2 without
-                                 // clusters, 4 as 2 with the cluster reduction taken at no cost in the plan
+static int g_prefix_kernel = 0;  // 0 auto, 1 generic only, 2 tcgen05 whenever it applies, 3 the split
+                                 // tcgen05 kernel without clusters, 4 the split kernel with the cluster
+                                 // reduction taken at no cost in the plan (3 and 4 never take the paired kernel)
 
 struct PrefixPlan {
   bool tc;
+  bool pair;         // the paired stream-K kernel applies (dense passes only)
+  PairPlan pp;
   int32_t nsplit;    // CTAs along the keys
   int32_t cluster;   // > 1: the splits reduce inside one cluster
   int32_t nparts;    // parts written: 1 when reduced in-kernel, else nsplit
@@ -258,13 +263,39 @@ static PrefixPlan plan_prefix(const fb_attn_desc& d, const void* q, const void* 
   p.excl = nullptr;
   p.excl_words = 0;
   p.excl_invert = false;
+  p.pair = false;
   const int64_t min_keys = g_prefix_kernel >= 2 ? 1 : 256;
   if (g_prefix_kernel != 1 && nkeys >= min_keys && tc_make_maps(d, q, kp, vp, nkeys, d.kp_strides, &p.maps)) {
     tc_plan_split((int64_t)p.maps.units * p.maps.tiles_per_unit, nkeys, cap, g_prefix_kernel != 3, &p.nsplit,
                   &p.kps, &p.cluster, &p.nparts, g_prefix_kernel == 4 ? 0.0 : 4.0);
     p.tc = true;
+    p.pair = (g_prefix_kernel == 0 || g_prefix_kernel == 2) && pair_plan(d, nkeys, &p.pp) && p.pp.smax <= cap;
   }
   return p;
+}
+
+static double prefix_bytes(const fb_attn_desc& d, int64_t nkeys) {
+  const int es = esize(d.in_dtype);
+  return 2.0 * d.B * d.Hkv * (double)nkeys * d.D * es + (double)rows_of(d) * d.D * es +
+         (double)rows_of(d) * (d.D + 1) * 4;
+}
+
+// The paired pass (plan p.pair, no key bitmap): the final (A, L) at dst, with
+// the parts at pa / pl and the slot counts at ns as scratch.
+static fb_status launch_prefix_pair(const fb_attn_desc& d, PrefixPlan& p, int64_t nkeys, const int8_t* mask,
+                                    int mask_active, float* pa, float* pl, int32_t* ns, float* dst_a, float* dst_l,
+                                    cudaStream_t s) {
+  {
+    ProfScope prof(kProfPrefix, prefix_bytes(d, nkeys), s);
+    if (launch_attn_pair(d, p.maps, p.pp, nkeys, mask, mask_active, scale_log2(d), pa, pl, dst_a, dst_l, ns, s,
+                         false) != cudaSuccess)
+      return FB_ECUDA;
+  }
+  ProfScope prof(kProfAux, (p.pp.smax + 1.0) * rows_of(d) * (d.D + 1) * 4.0, s);
+  return launch_attn_pair(d, p.maps, p.pp, nkeys, mask, mask_active, scale_log2(d), pa, pl, dst_a, dst_l, ns, s,
+                          true) == cudaSuccess
+             ? FB_OK
+             : FB_ECUDA;
 }
 
 static fb_status launch_prefix(const fb_attn_desc& d, PrefixPlan& p, int64_t nkeys, const int8_t* mask,
@@ -276,10 +307,7 @@ static fb_status launch_prefix(const fb_attn_desc& d, PrefixPlan& p, int64_t nke
     p.gen.a.excl_words = p.excl_words;
     return launch_pass(d, p.gen.a, pa, pl, s);
   }
-  const int es = esize(d.in_dtype);
-  const double bytes = 2.0 * d.B * d.Hkv * (double)nkeys * d.D * es + (double)rows_of(d) * d.D * es +
-                       (double)rows_of(d) * (d.D + 1) * 4;
-  ProfScope prof(kProfPrefix, bytes, s);
+  ProfScope prof(kProfPrefix, prefix_bytes(d, nkeys), s);
   return launch_attn_tc(d, p.maps, nkeys, p.nsplit, p.kps, p.cluster, mask, mask_active, scale_log2(d), pa, pl, s,
                         p.excl, p.excl_words, p.excl_invert) ==
                  cudaSuccess
@@ -421,6 +449,7 @@ fb_status fb_outblock_workspace_bytes(const fb_attn_desc* d, int64_t prefix_len,
   if (st != FB_OK) return st;
   if (!bytes || prefix_len < 0 || sel_k < 0) return FB_EINVAL;
   size_t n = part_bytes(*d, std::max(split_bound(*d, 0, prefix_len), sel_k ? split_bound(*d, 1, sel_k) : 1));
+  n += align256((size_t)pair_count(*d) * 4);
   if (sel_k) n += align256((size_t)d->B * d->Hq * ((prefix_len + 31) / 32) * 4);
   *bytes = n;
   return FB_OK;
@@ -453,10 +482,12 @@ fb_status fb_attn_outblock(const fb_attn_desc* d, const void* q, const void* kp,
   const int32_t cap = std::max(split_bound(*d, 0, prefix_len), sel ? split_bound(*d, 1, sel_k) : 1);
   float* pa = reinterpret_cast<float*>(w);
   float* pl = reinterpret_cast<float*>(w + align256((size_t)cap * rows_of(*d) * d->D * 4));
+  int32_t* ns = reinterpret_cast<int32_t*>(w + part_bytes(*d, cap));
 
   // pass 1: dense prefix, or the selected keys
   if (!sel) {
     PrefixPlan p = plan_prefix(*d, q, kp, vp, prefix_len, cap);
+    if (p.pair) return launch_prefix_pair(*d, p, prefix_len, nullptr, 0, pa, pl, ns, a_out, l_out, stream);
     if (p.nparts == 1) return launch_prefix(*d, p, prefix_len, nullptr, 0, a_out, l_out, stream);
     if ((st = launch_prefix(*d, p, prefix_len, nullptr, 0, pa, pl, stream)) != FB_OK) return st;
     PartList lst;
@@ -634,6 +665,7 @@ struct fb_cache {
   float* gpart;       // gamma: per-chunk partial sums
   int32_t* counters;  // gamma: per-head arrival counters (kept at zero)
   int32_t chunks;
+  int32_t* pair_ns;   // slot counts of the paired prefix pass
 };
 
 namespace {
@@ -662,6 +694,7 @@ fb_status layout_cache(const fb_attn_desc& d, int32_t flags, int64_t max_prefix,
   float* cl = cv.take<float>(base, rows * 4);
   float* pa = cv.take<float>(base, (size_t)part_cap * rows * d.D * 4);
   float* pl = cv.take<float>(base, (size_t)part_cap * rows * 4);
+  int32_t* pn = cv.take<int32_t>(base, (size_t)pair_count(d) * 4);
   float* sa = nullptr; float* sl = nullptr; uint32_t* bm = nullptr;
   if (flags & FB_CACHE_SPARSE) {
     sa = cv.take<float>(base, (size_t)sel_cap * rows * d.D * 4);
@@ -680,6 +713,7 @@ fb_status layout_cache(const fb_attn_desc& d, int32_t flags, int64_t max_prefix,
     c->cache_a = ca; c->cache_l = cl; c->part_a = pa; c->part_l = pl; c->part_cap = part_cap;
     c->sel_a = sa; c->sel_l = sl; c->sel_cap = sel_cap; c->bitmap = bm; c->bitmap_words = words;
     c->mask = mk; c->sim = sm; c->gpart = gp; c->counters = ct; c->chunks = chunks;
+    c->pair_ns = pn;
   }
   return FB_OK;
 }
@@ -771,18 +805,27 @@ fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
 
   if (gamma) {
     PrefixPlan p = plan_prefix(d, a->q, a->kp, a->vp, a->prefix_len, c->part_cap);
-    if ((st = launch_prefix(d, p, a->prefix_len, c->mask, tau_reuse, c->part_a, c->part_l, s)) != FB_OK) return st;
+    int32_t fresh_parts = p.nparts;
+    if (p.pair) {
+      // the fresh part of every computed head, merged, in part 0
+      if ((st = launch_prefix_pair(d, p, a->prefix_len, c->mask, tau_reuse, c->part_a, c->part_l, c->pair_ns,
+                                   c->part_a, c->part_l, s)) != FB_OK)
+        return st;
+      fresh_parts = 1;
+    } else if ((st = launch_prefix(d, p, a->prefix_len, c->mask, tau_reuse, c->part_a, c->part_l, s)) != FB_OK) {
+      return st;
+    }
     GammaArgs g;
     memset(&g, 0, sizeof(g));
     g.B = d.B; g.Hq = d.Hq; g.Nb = d.Nb; g.D = d.D;
     g.fresh.ngroups = 1;
-    g.fresh.g[0] = group_of(c->part_a, c->part_l, p.nparts, d);
+    g.fresh.g[0] = group_of(c->part_a, c->part_l, fresh_parts, d);
     g.cache_a = c->cache_a; g.cache_l = c->cache_l;
     g.mask = c->mask; g.gate_active = tau_reuse; g.cache_valid = c->valid;
     g.gamma = a->gamma; g.sim = c->sim; g.partials = c->gpart; g.counters = c->counters;
     g.chunks = c->chunks; g.reuse_out = a->reuse_out; g.sim_out = a->sim_out;
     {
-      ProfScope prof(kProfAux, (p.nparts + 2.0) * rows_of(d) * (d.D + 1) * 4.0, s);
+      ProfScope prof(kProfAux, (fresh_parts + 2.0) * rows_of(d) * (d.D + 1) * 4.0, s);
       if (launch_gamma_update(g, s) != cudaSuccess) return FB_ECUDA;
     }
   } else {
@@ -835,9 +878,13 @@ fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
         p.excl = c->bitmap;
         p.excl_words = (a->prefix_len + 31) / 32;
       }
-      // the in-block kernel can take the split parts itself and write their
-      // merge into the cache, saving a merge pass
-      if (!sparse && p.nparts > 1 && inblock_small_applies(d, p.nparts)) {
+      if (!sparse && p.pair) {
+        if ((st = launch_prefix_pair(d, p, a->prefix_len, nullptr, 0, c->part_a, c->part_l, c->pair_ns, c->cache_a,
+                                     c->cache_l, s)) != FB_OK)
+          return st;
+      } else if (!sparse && p.nparts > 1 && inblock_small_applies(d, p.nparts)) {
+        // the in-block kernel can take the split parts itself and write their
+        // merge into the cache, saving a merge pass
         if ((st = launch_prefix(d, p, a->prefix_len, nullptr, 0, c->part_a, c->part_l, s)) != FB_OK) return st;
         ext.g[ext.ngroups++] = group_of(c->part_a, c->part_l, p.nparts, d);
         if (a->reuse_out && launch_fill_decision(a->reuse_out, BH, 0, s) != cudaSuccess) return FB_ECUDA;
@@ -847,8 +894,7 @@ fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
         c->valid = true;
         c->last_recomputed = 1;
         return FB_OK;
-      }
-      if (p.nparts == 1) {
+      } else if (p.nparts == 1) {
         if ((st = launch_prefix(d, p, a->prefix_len, nullptr, 0, c->cache_a, c->cache_l, s)) != FB_OK) return st;
       } else {
         if ((st = launch_prefix(d, p, a->prefix_len, nullptr, 0, c->part_a, c->part_l, s)) != FB_OK) return st;

@@ -1,0 +1,666 @@
+// Block-external attention on the fifth-generation tensor cores (sm_100a), two
+// query tiles per CTA: the FlashBlock prefix pass, A_out with L_out = log Z_out
+// over the prefix KV cache (FlashBlock summary, "Mécanisme Central"), for bf16
+// inputs, D = 128, wherever a KV head has two or more 128-row query tiles
+// (long-context diffusion-LM blocks, video frame blocks).
+//
+// Work decomposition.  The query tiles of one KV head are paired; a pair and
+// one key tile of 128 keys is one work item.  The grid is persistent (at most
+// one CTA per SM) and stream-K: CTA c takes the items [c*T/C, (c+1)*T/C) of
+// the T = pairs x key-tiles items, so every CTA gets the same number of key
+// tiles whatever the shape.  A CTA's range splits into segments, one per pair
+// it touches; each segment leaves a partial (A, L) of its pair's rows in the
+// pair's slot (the index of the CTA among those touching the pair), or the
+// final result when one CTA covers the whole pair, and a small merge kernel
+// combines the slots in log space.  With the gamma gate, pairs whose heads
+// all reuse their cache are left out of the item space on the device.
+//
+// Warp roles (320 threads):
+//   warps 0..3  softmax of query tile 0 (slot 0), one thread per query row
+//   warps 4..7  softmax of query tile 1 (slot 1)
+//   warp 8      TMA producer, no multicast: the pair's Q tiles, then K and V
+//               tiles of 128 keys into a three-stage K ring and a two-stage
+//               V ring (128-byte swizzle), K one tile ahead of V
+//   warp 9      allocates TMEM; one thread issues every tcgen05.mma
+// TMEM: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).  Softmax s
+// reads its row of S_s, writes P = 2^(s - m) over the same columns as bf16
+// hi (columns 0..63) and lo (64..127) parts, and the issuer runs
+// O_s += P_hi V + P_lo V.  The issuer orders the tensor core as
+//   S0(j) S1(j) | PV0(j) S0(j+1) PV1(j) S1(j+1) | PV0(j+1) ...
+// so while one softmax group works on its tile the tensor core runs the other
+// group's P V and next S.  S_s(j+1) overwrites P_s(j) only after PV_s(j) has
+// read it: tcgen05.mma operations issued by one thread execute in order.
+// The running max moves only when a row's max grows by more than 2^8 (O is
+// then rescaled in TMEM by its own thread; the previous P V of that slot has
+// completed, since S_s(j) completed after it).  Every mbarrier wait is
+// bounded; on expiry the CTA records FB_ETIMEOUT, drains its own copies and
+// MMAs, frees TMEM and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math_constants.h>
+
+#include <algorithm>
+
+#include "fb_internal.cuh"
+#include "fb_ptx.cuh"
+#include "fb_tc.cuh"
+
+namespace fb {
+
+namespace {
+
+using namespace tc;
+
+constexpr int kBM = 128, kBN = 128, kD = 128;
+constexpr int kThreads = 320;
+constexpr int kKSt = 3, kVSt = 2;                 // K and V ring depths
+constexpr uint32_t kHalf = 16384;                 // [128 rows][64 bf16], 128-byte swizzle
+constexpr uint32_t kTile = 2 * kHalf;             // one 128 x 128 bf16 tile
+constexpr uint32_t kOffQ = 0;                     // Q0, Q1
+constexpr uint32_t kOffK = 2 * kTile;
+constexpr uint32_t kOffV = kOffK + kKSt * kTile;
+constexpr uint32_t kOffBar = kOffV + kVSt * kTile;
+constexpr uint32_t kOffSeg = kOffBar + 256;       // segment list
+constexpr int kMaxSeg = 32;
+constexpr uint32_t kOffAct = kOffSeg + kMaxSeg * 16;   // active-pair bitmap
+constexpr int kMaxPairs = 2048;
+constexpr uint32_t kSmemSlack = 1024;
+constexpr uint32_t kSmemBytes = kOffAct + kMaxPairs / 8 + kSmemSlack;
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemO = 256;
+constexpr float kRescaleLog2 = 8.0f;
+
+enum {
+  B_QFULL = 0, B_QEMPTY = 1, B_KFULL = 2, B_KEMPTY = 5, B_VFULL = 8, B_VEMPTY = 10, B_SFULL = 12, B_PFULL = 14,
+  B_OREADY = 16, B_OFREE = 18, B_DRAIN = 20, B_STALL = 21, B_COUNT = 22
+};
+
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// max of three (one instruction on sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+}  // namespace
+
+struct PairArgs {
+  int32_t B, Hq, Hkv, G, Nb;
+  int32_t mode;            // 0: tile = hg heads x Nb queries of one KV head; 1: 128 queries of one head
+  int32_t hg, tph;         // heads per tile (mode 0); tiles per head (mode 1)
+  int32_t tiles_per_kv, pairs_per_kv, npairs;
+  int32_t nkt;             // key tiles
+  int64_t nkeys;
+  int32_t smax;            // slots per pair in the part buffer
+  float scale_log2;
+  float* part_a;           // slot s of row r at part_a + s * part_stride_a + r * D
+  float* part_l;
+  int64_t part_stride_a, part_stride_l;
+  float* dst_a;            // final (A, L) of pairs covered by one CTA (packed rows)
+  float* dst_l;
+  int32_t* nslots;         // [npairs]: CTAs that touched the pair (written by its slot-0 CTA)
+  const int8_t* mask;      // gamma: [B, Hq], 1 = head reuses (may be skipped)
+  int32_t mask_active;
+  int* status;
+  uint64_t wait_limit_ns;
+  uint32_t q_bytes;        // bytes of one Q tile (both 64-column halves)
+  int32_t stall;           // test hook: the MMA issuer first waits on a barrier nothing completes
+};
+
+namespace {
+
+struct Tile {
+  int b, kvh, h0, nheads, i0, nrows;
+  int64_t rbase;           // first packed (b, h, i) row
+};
+
+// Query tile `tl` (0 .. tiles_per_kv-1) of KV unit `u` = b * Hkv + kvh.
+__device__ __forceinline__ Tile tile_of(const PairArgs& a, int u, int tl) {
+  Tile t;
+  t.b = u / a.Hkv;
+  t.kvh = u % a.Hkv;
+  if (a.mode == 0) {
+    t.h0 = t.kvh * a.G + tl * a.hg;
+    t.nheads = min(a.hg, a.G - tl * a.hg);
+    t.i0 = 0;
+    t.nrows = t.nheads * a.Nb;
+  } else {
+    const int g = tl / a.tph, tt = tl % a.tph;
+    t.h0 = t.kvh * a.G + g;
+    t.nheads = 1;
+    t.i0 = tt * kBM;
+    t.nrows = min(kBM, a.Nb - t.i0);
+  }
+  t.rbase = ((int64_t)t.b * a.Hq + t.h0) * a.Nb + t.i0;
+  return t;
+}
+
+__device__ __forceinline__ bool pair_has_slot1(const PairArgs& a, int p) {
+  return 2 * (p % a.pairs_per_kv) + 1 < a.tiles_per_kv;
+}
+
+// A pair needs computing unless the gamma gate lets every head in it reuse.
+__device__ bool pair_active(const PairArgs& a, int p) {
+  if (!a.mask_active) return true;
+  const int u = p / a.pairs_per_kv, tl0 = 2 * (p % a.pairs_per_kv);
+  for (int k = 0; k < 2; ++k) {
+    if (tl0 + k >= a.tiles_per_kv) break;
+    const Tile t = tile_of(a, u, tl0 + k);
+    for (int h = t.h0; h < t.h0 + t.nheads; ++h)
+      if (!a.mask[t.b * a.Hq + h]) return true;
+  }
+  return false;
+}
+
+// CTA of the stream-K grid (C CTAs over T items) that holds item i.
+__device__ __forceinline__ int cta_of(int64_t i, int C, int64_t T) { return (int)(((i + 1) * C - 1) / T); }
+
+struct Seg {
+  int32_t pair, j0, j1, slot_ns;   // slot in the low 16 bits, slot count in the high 16
+};
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const PairArgs a) {
+  ptx::pdl_prologue();
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if (smem - smem_raw > (ptrdiff_t)kSmemSlack) {   // the layout would not fit: report, touch nothing
+    if (threadIdx.x == 0) atomicCAS(a.status, 0, (int)FB_EUNSUPPORTED);
+    return;
+  }
+  const uint32_t sbase = smem_addr(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffBar + B_COUNT * 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBar + B_COUNT * 8 + 4);
+  int* nseg_sh = reinterpret_cast<int*>(smem + kOffBar + B_COUNT * 8 + 8);
+  Seg* segs = reinterpret_cast<Seg*>(smem + kOffSeg);
+  uint32_t* act = reinterpret_cast<uint32_t*>(smem + kOffAct);
+  auto bar = [&](int i) { return smem_addr(bars + i); };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- the active pairs (all of them unless the gamma gate is on) ----
+  const int words = (a.npairs + 31) / 32;
+  if (a.mask_active) {
+    for (int w = threadIdx.x; w < words; w += kThreads) act[w] = 0u;
+    __syncthreads();
+    for (int p = threadIdx.x; p < a.npairs; p += kThreads)
+      if (pair_active(a, p)) atomicOr(act + (p >> 5), 1u << (p & 31));
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < B_COUNT; ++i) {
+      uint32_t cnt = 1;
+      if ((i >= B_PFULL && i < B_PFULL + 2) || (i >= B_OFREE && i < B_OFREE + 2)) cnt = 128;
+      mbar_init(bar(i), cnt);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 9) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    tc_fence_before();
+  }
+  __syncthreads();
+  // ---- this CTA's segments (thread 0) ----
+  if (threadIdx.x == 0) {
+    int nact = a.npairs;
+    if (a.mask_active) {
+      nact = 0;
+      for (int w = 0; w < words; ++w) nact += __popc(act[w]);
+    }
+    const int64_t T = (int64_t)nact * a.nkt;
+    const int C = (int)min((int64_t)min((int64_t)gridDim.x, T), (int64_t)nact * (a.smax - 1));
+    const int c = blockIdx.x;
+    int n = 0;
+    if (c < C) {
+      const int64_t i0 = (int64_t)c * T / C, i1 = (int64_t)(c + 1) * T / C;
+      int64_t ai = i0 / a.nkt;            // active index of the first pair
+      // the ai-th active pair
+      int p = (int)ai;
+      if (a.mask_active) {
+        int64_t left = ai;
+        p = -1;
+        for (int w = 0; w < words && p < 0; ++w) {
+          uint32_t bits = act[w];
+          const int cnt = __popc(bits);
+          if (left >= cnt) { left -= cnt; continue; }
+          while (left > 0) { bits &= bits - 1; --left; }
+          p = w * 32 + __ffs(bits) - 1;
+        }
+      }
+      for (int64_t it = i0; it < i1 && n < kMaxSeg && p >= 0 && p < a.npairs;) {
+        const int64_t base = ai * a.nkt;
+        const int64_t e = min(i1, base + a.nkt);
+        const int first = cta_of(base, C, T), last = cta_of(base + a.nkt - 1, C, T);
+        Seg s;
+        s.pair = p;
+        s.j0 = (int)(it - base);
+        s.j1 = (int)(e - base);
+        s.slot_ns = (c - first) | ((last - first + 1) << 16);
+        segs[n++] = s;
+        it = e;
+        ++ai;
+        // next active pair
+        ++p;
+        if (a.mask_active)
+          while (p < a.npairs && !((act[p >> 5] >> (p & 31)) & 1u)) ++p;
+      }
+    }
+    *nseg_sh = n;
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int nseg = *nseg_sh;
+  const Ctl ctl{abort_flag, a.status, a.wait_limit_ns};
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && nseg > 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQ)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmK)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmV)) : "memory");
+      int kt = 0, vt = 0;   // K and V tiles issued so far (stage = count % depth, round = count / depth)
+      int qarm = -1;
+      bool ok = true;
+      auto load_k = [&](int b, int kvh, int j) -> bool {
+        const int st = kt % kKSt, round = kt / kKSt;
+        if (kt >= kKSt && !wait_phase(bar(B_KEMPTY + st), (round - 1) & 1, ctl)) return false;
+        mbar_expect_tx(bar(B_KFULL + st), kTile);
+        const uint32_t dst = sbase + kOffK + st * kTile;
+        tma_load_4d(dst, &tmK, bar(B_KFULL + st), 0, j * kBN, kvh, b);
+        tma_load_4d(dst + kHalf, &tmK, bar(B_KFULL + st), 64, j * kBN, kvh, b);
+        ++kt;
+        return true;
+      };
+      auto load_v = [&](int b, int kvh, int j) -> bool {
+        const int st = vt % kVSt, round = vt / kVSt;
+        if (vt >= kVSt && !wait_phase(bar(B_VEMPTY + st), (round - 1) & 1, ctl)) return false;
+        mbar_expect_tx(bar(B_VFULL + st), kTile);
+        const uint32_t dst = sbase + kOffV + st * kTile;
+        tma_load_4d(dst, &tmV, bar(B_VFULL + st), 0, j * kBN, kvh, b);
+        tma_load_4d(dst + kHalf, &tmV, bar(B_VFULL + st), 64, j * kBN, kvh, b);
+        ++vt;
+        return true;
+      };
+      for (int si = 0; si < nseg && ok; ++si) {
+        const Seg sg = segs[si];
+        const int u = sg.pair / a.pairs_per_kv, tl0 = 2 * (sg.pair % a.pairs_per_kv);
+        const bool two = pair_has_slot1(a, sg.pair);
+        const Tile t0 = tile_of(a, u, tl0);
+        if (si > 0 && !(ok = wait_phase(bar(B_QEMPTY), (si - 1) & 1, ctl))) break;
+        mbar_expect_tx(bar(B_QFULL), a.q_bytes * (two ? 2u : 1u));
+        tma_load_4d(sbase + kOffQ, &tmQ, bar(B_QFULL), 0, t0.i0, t0.h0, t0.b);
+        tma_load_4d(sbase + kOffQ + kHalf, &tmQ, bar(B_QFULL), 64, t0.i0, t0.h0, t0.b);
+        if (two) {
+          const Tile t1 = tile_of(a, u, tl0 + 1);
+          tma_load_4d(sbase + kOffQ + kTile, &tmQ, bar(B_QFULL), 0, t1.i0, t1.h0, t1.b);
+          tma_load_4d(sbase + kOffQ + kTile + kHalf, &tmQ, bar(B_QFULL), 64, t1.i0, t1.h0, t1.b);
+        }
+        qarm = si;
+        for (int j = sg.j0; j < sg.j1 && ok; ++j) {
+          ok = load_k(t0.b, t0.kvh, j);
+          if (ok && j > sg.j0) ok = load_v(t0.b, t0.kvh, j - 1);
+        }
+        if (ok) ok = load_v(t0.b, t0.kvh, sg.j1 - 1);
+      }
+      // let every copy this thread started land before the CTA can exit
+      if (qarm >= 0) wait_phase(bar(B_QFULL), qarm & 1, ctl, true);
+      // (stage st was last armed in round (count - 1 - st) / depth)
+      for (int st = 0; st < kKSt; ++st)
+        if (kt > st) wait_phase(bar(B_KFULL + st), ((kt - 1 - st) / kKSt) & 1, ctl, true);
+      for (int st = 0; st < kVSt; ++st)
+        if (vt > st) wait_phase(bar(B_VFULL + st), ((vt - 1 - st) / kVSt) & 1, ctl, true);
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && nseg > 0) {
+      const uint64_t dQ0 = sw128_desc(sbase + kOffQ, 16, 1024);
+      const uint64_t dQ1 = sw128_desc(sbase + kOffQ + kTile, 16, 1024);
+      const uint64_t dK = sw128_desc(sbase + kOffK, 16, 1024);
+      const uint64_t dV = sw128_desc(sbase + kOffV, kHalf, 1024);
+      int kt = 0, vt = 0;
+      int pcnt[2] = {0, 0}, segcnt[2] = {0, 0};
+      bool ok = !a.stall || wait_phase(bar(B_STALL), 0, ctl);
+      // S_s = Q_s K^T for the K tile in stage kst
+      auto issue_s = [&](int s, int kst) {
+        const uint64_t dKs = dK + (uint64_t)((kst * kTile) >> 4);
+        const uint64_t dQs = s ? dQ1 : dQ0;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint64_t off = (uint64_t)(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4);
+          tc_mma(tmem + s * kBN, dQs + off, dKs + off, kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(B_SFULL + s));
+      };
+      // O_s += P_hi V + P_lo V for the V tile in stage vst
+      auto issue_pv = [&](int s, int vst, bool first) {
+        const uint64_t dVs = dV + (uint64_t)((vst * kTile) >> 4);
+        const uint32_t pt = tmem + s * kBN;
+#pragma unroll
+        for (int part = 0; part < 2; ++part)
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            tc_mma_ts(tmem + kTmemO + s * kBN, pt + part * 64 + kk * 8, dVs + (uint64_t)((kk * 2048) >> 4),
+                      kIdescPV, (!first || part > 0 || kk > 0) ? 1u : 0u);
+      };
+      for (int si = 0; si < nseg && ok; ++si) {
+        const Seg sg = segs[si];
+        const bool two = pair_has_slot1(a, sg.pair);
+        const int ns = two ? 2 : 1;
+        if (!(ok = wait_phase(bar(B_QFULL), si & 1, ctl))) break;
+        int kst = kt % kKSt;
+        if (!(ok = wait_phase(bar(B_KFULL + kst), (kt / kKSt) & 1, ctl))) break;
+        tc_fence_after();
+        issue_s(0, kst);
+        if (ns > 1) issue_s(1, kst);
+        tc_commit(bar(B_KEMPTY + kst));
+        ++kt;
+        if (sg.j1 - sg.j0 == 1) tc_commit(bar(B_QEMPTY));
+        for (int j = sg.j0; j < sg.j1 && ok; ++j) {
+          const int vst = vt % kVSt;
+          const bool more = j + 1 < sg.j1;
+          kst = kt % kKSt;
+#pragma unroll
+          for (int s = 0; s < 2; ++s) {
+            if (s >= ns || !ok) break;
+            ok = wait_phase(bar(B_PFULL + s), pcnt[s] & 1, ctl);
+            if (ok && j == sg.j0 && segcnt[s] > 0) ok = wait_phase(bar(B_OFREE + s), (segcnt[s] - 1) & 1, ctl);
+            if (ok && s == 0) ok = wait_phase(bar(B_VFULL + vst), (vt / kVSt) & 1, ctl);
+            if (ok && s == 0 && more) ok = wait_phase(bar(B_KFULL + kst), (kt / kKSt) & 1, ctl);
+            if (!ok) break;
+            ++pcnt[s];
+            tc_fence_after();
+            issue_pv(s, vst, j == sg.j0);
+            if (more) issue_s(s, kst);
+            if (!more) tc_commit(bar(B_OREADY + s));
+          }
+          if (!ok) break;
+          tc_commit(bar(B_VEMPTY + vst));
+          ++vt;
+          if (more) {
+            tc_commit(bar(B_KEMPTY + kst));
+            ++kt;
+            if (j + 2 == sg.j1) tc_commit(bar(B_QEMPTY));   // the segment's last S has been issued
+          }
+        }
+        ++segcnt[0];
+        if (ns > 1) ++segcnt[1];
+      }
+      // quiesce this thread's tensor-core work before TMEM is freed
+      tc_commit(bar(B_DRAIN));
+      wait_phase(bar(B_DRAIN), 0, ctl, true);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int s = warp >> 2;                 // slot: query tile 0 or 1 of the pair
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
+    const uint32_t tS = tl + s * kBN, tO = tl + kTmemO + s * kBN;
+    int scnt = 0, ocnt = 0;
+    bool ok = true;
+    auto uniform = [](bool v) { return __all_sync(0xffffffffu, v); };
+    for (int si = 0; si < nseg && ok; ++si) {
+      const Seg sg = segs[si];
+      if (s == 1 && !pair_has_slot1(a, sg.pair)) continue;
+      const int u = sg.pair / a.pairs_per_kv, tl0 = 2 * (sg.pair % a.pairs_per_kv);
+      const Tile t = tile_of(a, u, tl0 + s);
+      float m = -CUDART_INF_F, l = 0.f;
+      for (int j = sg.j0; j < sg.j1; ++j) {
+        ok = uniform(wait_phase(bar(B_SFULL + s), scnt & 1, ctl));
+        if (!ok) break;
+        ++scnt;
+        tc_fence_after();
+        float sv[128];
+        tmem_ld32(tS, sv);
+        tmem_ld32(tS + 32, sv + 32);
+        tmem_ld32(tS + 64, sv + 64);
+        tmem_ld32(tS + 96, sv + 96);
+        tmem_wait_ld();
+        const int64_t nvalid = a.nkeys - (int64_t)j * kBN;
+        if (nvalid < kBN) {   // ragged last key tile
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c >= nvalid) sv[c] = -CUDART_INF_F;
+        }
+        float mx[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) mx[e] = sv[e];
+#pragma unroll
+        for (int c = 4; c < 128; c += 8) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) mx[e] = fmax3(mx[e], sv[c + e], c + 4 + e < 128 ? sv[c + 4 + e] : mx[e]);
+        }
+        const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * a.scale_log2;
+        const bool move = tmax > m + kRescaleLog2;
+        const bool scale_o = move && m != -CUDART_INF_F;
+        const float alpha = scale_o ? fast_exp2(m - tmax) : 1.f;
+        if (__any_sync(0xffffffffu, scale_o)) {
+          // O_s holds this segment's earlier tiles: PV_s(j-1) has completed
+          // (S_s(j), issued after it, has), and PV_s(j) waits for this P
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            float o[16];
+            tmem_ld16(tO + c * 16, o);
+            tmem_wait_ld();
+            uint32_t ob[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) ob[e] = __float_as_uint(o[e] * alpha);
+            tmem_st16u(tO + c * 16, ob);
+          }
+          tmem_wait_st();
+        }
+        if (move) {
+          l *= alpha;
+          m = tmax;
+        }
+        const float nref = m == -CUDART_INF_F ? 0.f : -m;
+        float sum[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {   // 32 keys: 16 hi words at 16c, 16 lo words at 64 + 16c
+          // the hi and lo words take the registers of the two scores they replace
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = fast_exp2(fmaf(sv[32 * c + 2 * e], a.scale_log2, nref));
+            const float p1 = fast_exp2(fmaf(sv[32 * c + 2 * e + 1], a.scale_log2, nref));
+            sum[e & 3] += p0 + p1;
+            uint32_t h, lw;
+            split_pair(p0, p1, h, lw);
+            sv[32 * c + 2 * e] = __uint_as_float(h);
+            sv[32 * c + 2 * e + 1] = __uint_as_float(lw);
+          }
+          uint32_t hi[16], lo[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            hi[e] = __float_as_uint(sv[32 * c + 2 * e]);
+            lo[e] = __float_as_uint(sv[32 * c + 2 * e + 1]);
+          }
+          tmem_st16u(tS + 16 * c, hi);
+          tmem_st16u(tS + 64 + 16 * c, lo);
+        }
+        l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(B_PFULL + s));
+      }
+      if (!ok) break;
+      // ---- epilogue of the segment: O / l and L of this row ----
+      ok = uniform(wait_phase(bar(B_OREADY + s), ocnt & 1, ctl));
+      if (!ok) break;
+      ++ocnt;
+      tc_fence_after();
+      const int slot = sg.slot_ns & 0xFFFF, nsl = sg.slot_ns >> 16;
+      const bool direct = nsl == 1;
+      const int64_t r = t.rbase + row;
+      float* dA = direct ? a.dst_a : a.part_a + slot * a.part_stride_a;
+      float* dL = direct ? a.dst_l : a.part_l + slot * a.part_stride_l;
+      const bool mine = row < t.nrows;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float o[32];
+        tmem_ld32(tO + c * 32, o);
+        tmem_wait_ld();
+        if (mine) {
+          float4* d4 = reinterpret_cast<float4*>(dA + r * kD + c * 32);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            d4[e] = make_float4(o[4 * e] * inv, o[4 * e + 1] * inv, o[4 * e + 2] * inv, o[4 * e + 3] * inv);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(B_OFREE + s));   // O_s may be overwritten by the next segment
+      if (mine) dL[r] = l > 0.f ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
+      if (mine && row == 0 && s == 0 && slot == 0) a.nslots[sg.pair] = nsl;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+  }
+}
+
+// Log-space merge of the slots of every pair covered by two or more CTAs into
+// the final (A, L); one warp per packed row.  Rows of heads that reuse their
+// cache (gamma) and rows of pairs finished by one CTA are left alone.
+__global__ void __launch_bounds__(256) pair_merge_kernel(const PairArgs a) {
+  ptx::pdl_prologue();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t r = (int64_t)blockIdx.x * 8 + warp;
+  const int64_t nrows = (int64_t)a.B * a.Hq * a.Nb;
+  if (r >= nrows) return;
+  const int64_t bh = r / a.Nb;
+  if (a.mask_active && a.mask[bh]) return;
+  const int b = (int)(bh / a.Hq), h = (int)(bh % a.Hq), i = (int)(r % a.Nb);
+  const int kvh = h / a.G, g = h % a.G;
+  const int tl = a.mode == 0 ? g / a.hg : g * a.tph + i / kBM;
+  const int p = (b * a.Hkv + kvh) * a.pairs_per_kv + tl / 2;
+  const int ns = a.nslots[p];
+  if (ns <= 1 || ns > a.smax) return;   // one CTA wrote dst itself (a count outside [2, smax]: the pass failed)
+  float m = -CUDART_INF_F;
+  for (int s = 0; s < ns; ++s) m = fmaxf(m, a.part_l[s * a.part_stride_l + r]);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float wsum = 0.f;
+  for (int s = 0; s < ns; ++s) {
+    const float Ls = a.part_l[s * a.part_stride_l + r];
+    if (Ls == -CUDART_INF_F) continue;
+    const float w = __expf(Ls - m);
+    const float4 v = *reinterpret_cast<const float4*>(a.part_a + s * a.part_stride_a + r * kD + lane * 4);
+    wsum += w;
+    acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
+    acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  __syncwarp();   // every lane has read the slots before any writes (dst may be slot 0)
+  *reinterpret_cast<float4*>(a.dst_a + r * kD + lane * 4) =
+      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  if (lane == 0) a.dst_l[r] = m == -CUDART_INF_F ? -CUDART_INF_F : m + __logf(wsum);
+}
+
+// ------------------------------------------------------------------ host --
+int* device_status_ptr();
+uint64_t wait_limit_ns();
+
+// Plan of the paired pass over nkeys keys, or false where it does not apply
+// (fewer than two query tiles per KV head, too few key tiles, or more pairs
+// than one CTA can list).
+bool pair_plan(const fb_attn_desc& d, int64_t nkeys, PairPlan* p) {
+  int mode, hg, tpu, units;
+  if (nkeys <= 0 || !tc_tiling(d, &mode, &hg, &tpu, &units)) return false;
+  const int G = d.Hq / d.Hkv;
+  p->mode = mode;
+  p->hg = hg;
+  p->tph = mode == 0 ? 1 : tpu;
+  p->tiles_per_kv = mode == 0 ? tpu : G * tpu;
+  if (p->tiles_per_kv < 2) return false;
+  p->pairs_per_kv = (p->tiles_per_kv + 1) / 2;
+  p->npairs = d.B * d.Hkv * p->pairs_per_kv;
+  p->nkt = (int32_t)((nkeys + kBN - 1) / kBN);
+  if (p->nkt < 4 || p->npairs > kMaxPairs) return false;
+  const int64_t T = (int64_t)p->npairs * p->nkt;
+  p->grid = (int32_t)std::min<int64_t>(num_sms(), T);
+  // segments per CTA: at most ceil(items per CTA / key tiles) + 1
+  const int64_t per = (T + p->grid - 1) / p->grid;
+  if ((per + p->nkt - 1) / p->nkt + 1 > kMaxSeg) return false;
+  p->smax = (p->grid + p->npairs - 1) / p->npairs + 1;
+  return true;
+}
+
+// Slots the paired pass may use for a prefix of up to max_keys keys (sizes workspaces).
+int32_t pair_slot_cap(const fb_attn_desc& d, int64_t max_keys) {
+  PairPlan p;
+  if (!pair_plan(d, std::max<int64_t>(max_keys, kBN * 4), &p)) return 0;
+  return p.smax;
+}
+
+cudaError_t launch_attn_pair(const fb_attn_desc& d, const TcMaps& m, const PairPlan& pp, int64_t nkeys,
+                             const int8_t* mask, int mask_active, float scale_log2, float* pa, float* pl,
+                             float* dst_a, float* dst_l, int32_t* nslots, cudaStream_t s, bool merge_only) {
+  PairArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = d.B; a.Hq = d.Hq; a.Hkv = d.Hkv; a.G = d.Hq / d.Hkv; a.Nb = d.Nb;
+  a.mode = pp.mode; a.hg = pp.hg; a.tph = pp.tph;
+  a.tiles_per_kv = pp.tiles_per_kv; a.pairs_per_kv = pp.pairs_per_kv; a.npairs = pp.npairs;
+  a.nkt = pp.nkt; a.nkeys = nkeys; a.smax = pp.smax;
+  a.scale_log2 = scale_log2;
+  a.part_a = pa; a.part_l = pl;
+  a.part_stride_a = (int64_t)d.B * d.Hq * d.Nb * d.D;
+  a.part_stride_l = (int64_t)d.B * d.Hq * d.Nb;
+  a.dst_a = dst_a; a.dst_l = dst_l; a.nslots = nslots;
+  a.mask = mask; a.mask_active = mask_active;
+  a.status = device_status_ptr();
+  a.wait_limit_ns = wait_limit_ns();
+  a.q_bytes = 2u * 64u * 2u * (uint32_t)(pp.mode == 0 ? d.Nb * pp.hg : kBM);
+  a.stall = debug_stall() ? 1 : 0;
+  if (!a.status) return cudaErrorInvalidValue;
+  static bool attr[kMaxDevices] = {};
+  bool& done = attr[current_device()];
+  if (!done) {
+    cudaError_t e = cudaFuncSetAttribute(attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    done = true;
+  }
+  if (merge_only) {
+    const int64_t nrows = (int64_t)d.B * d.Hq * d.Nb;
+    return launch_k(pair_merge_kernel, dim3((unsigned)((nrows + 7) / 8)), dim3(256), 0, s, a);
+  }
+  return launch_k(attn_pair_kernel, dim3(pp.grid), dim3(kThreads), kSmemBytes, s, m.q, m.k, m.v, a);
+}
+
+int32_t pair_count(const fb_attn_desc& d) {
+  int mode, hg, tpu, units;
+  if (!tc_tiling(d, &mode, &hg, &tpu, &units)) return 0;
+  const int tiles_per_kv = mode == 0 ? tpu : (d.Hq / d.Hkv) * tpu;
+  if (tiles_per_kv < 2) return 0;
+  return d.B * d.Hkv * ((tiles_per_kv + 1) / 2);
+}
+
+}  // namespace fb

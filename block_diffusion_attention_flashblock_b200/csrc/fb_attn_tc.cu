@@ -43,6 +43,7 @@
 
 #include "fb_internal.cuh"
 #include "fb_ptx.cuh"
+#include "fb_tc.cuh"
 
 namespace fb {
 
@@ -71,130 +72,7 @@ enum {
   B_PVDONE = 19, B_DRAIN = 22, B_PAIR = 24, B_RECV = 28, B_STALL = 29, B_COUNT = 30
 };
 
-using ptx::globaltimer;
-using ptx::mbar_arrive;
-using ptx::mbar_expect_tx;
-using ptx::mbar_init;
-using ptx::mbar_try;
-using ptx::smem_addr;
-
-// Shared control block: first-failure flag, TMEM base.
-struct Ctl {
-  volatile int* abort;
-  int* status;
-  uint64_t limit_ns;
-};
-
-// A drain (waiting for this CTA's own copies or MMAs before it exits) is
-// bounded by at least this, whatever the configured limit, so a short test
-// limit never lets a CTA exit with its own asynchronous work in flight.
-constexpr uint64_t kDrainLimitNs = 1000000000ull;
-
-// Bounded wait for the phase of `parity` to complete.  Gives up when the limit
-// passes or (unless `draining`) another role has given up; the first to give
-// up records the error.
-__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const Ctl& c, bool draining = false) {
-  if (mbar_try(bar, parity)) return true;
-  const uint64_t limit = draining ? (c.limit_ns > kDrainLimitNs ? c.limit_ns : kDrainLimitNs) : c.limit_ns;
-  const uint64_t t0 = globaltimer();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try(bar, parity)) return true;
-    if (!draining && *c.abort) return false;
-    if (globaltimer() - t0 > limit) {
-      if (atomicExch(const_cast<int*>(c.abort), 1) == 0) atomicCAS(c.status, 0, (int)FB_ETIMEOUT);
-      return false;
-    }
-  }
-}
-
-// Wait for a phase: an inline non-blocking test first (the common case is a
-// phase that already completed), the bounded polling loop only otherwise.
-__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, const Ctl& c, bool draining = false) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  if (ok) return true;
-  return wait_bounded(bar, parity, c, draining);
-}
-
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm, uint32_t bar, int c0, int c1,
-                                            int c2, int c3) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
-      "%5}], [%6];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
-      : "memory");
-}
-
-// tcgen05 wrappers
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accum) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
-          d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
-      : "memory");
-}
-// D (TMEM) += A (TMEM, row per lane, bf16 pairs per column) x B (shared memory descriptor)
-__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accum) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(
-          d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accum)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%"
-      "18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
-      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
-      "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
-      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%"
-      "19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
-        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%"
-      "18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
-      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
-      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
-      "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
-      "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])),
-      "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
-      "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])),
-      "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
-      "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
-      "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
-      : "memory");
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+using namespace tc;
 
 // Thread-block cluster helpers (split-KV reduction through distributed shared memory).
 __device__ __forceinline__ void cluster_sync_all() {
@@ -247,41 +125,6 @@ __device__ __forceinline__ void load_o_scaled(uint32_t tl, int half, int T, floa
     for (int e = 0; e < 32; e += 4)
       put((c * 32 + e) / 4, make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv));
   }
-}
-
-// Shared-memory matrix descriptor, 128-byte swizzle (layout code 2), sm_100
-// version bit 46; lbo/sbo in bytes.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
-  return d;
-}
-
-// Instruction descriptor, kind::f16: D fp32, A/B bf16, M = 128, N = 128.
-constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
-constexpr uint32_t kIdescQK = kIdescBase;              // A, B K-major
-constexpr uint32_t kIdescPV = kIdescBase | (1u << 16);  // B (V) MN-major
-
-
-// 2^x on the MUFU unit (PTX ex2.approx; relative error about 2^-22, -inf -> 0).
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// bf16 hi/lo split of a pair by truncation, on integer and FADD pipes only:
-// hi = the upper 16 bits of x (exact remainder x - hi in fp32), lo = the upper
-// 16 bits of that remainder, so x - hi - lo < 2^-14 |x|.  Lower key in the low
-// half of each packed word.
-__device__ __forceinline__ void split_pair(float x, float y, uint32_t& hi, uint32_t& lo) {
-  const uint32_t xb = __float_as_uint(x), yb = __float_as_uint(y);
-  hi = __byte_perm(xb, yb, 0x7632);
-  const float rx = x - __uint_as_float(xb & 0xFFFF0000u), ry = y - __uint_as_float(yb & 0xFFFF0000u);
-  lo = __byte_perm(__float_as_uint(rx), __float_as_uint(ry), 0x7632);
 }
 
 }  // namespace

@@ -147,6 +147,22 @@ cudaError_t launch_attn_tc(const fb_attn_desc& d, const TcMaps& m, int64_t nkeys
                            float* pl, cudaStream_t s, const uint32_t* excl = nullptr, int64_t excl_words = 0,
                            bool excl_invert = false);
 
+// Paired tcgen05 prefix pass, persistent stream-K grid (fb_attn_pair.cu).
+struct PairPlan {
+  int32_t mode, hg, tph, tiles_per_kv, pairs_per_kv, npairs, nkt, grid, smax;
+};
+bool pair_plan(const fb_attn_desc& d, int64_t nkeys, PairPlan* p);
+int32_t pair_slot_cap(const fb_attn_desc& d, int64_t max_keys);
+int32_t pair_count(const fb_attn_desc& d);   // pairs of the paired pass (0: it never applies)
+// The pass (merge_only = false) leaves the final (A, L) of rows whose pair one
+// CTA covered at dst_a / dst_l and partial results in pp.smax parts at pa /
+// pl (npairs slot counts at nslots); the merge (merge_only = true, launched
+// after it with the same arguments) combines the partials into dst.  dst may
+// be part 0.
+cudaError_t launch_attn_pair(const fb_attn_desc& d, const TcMaps& m, const PairPlan& pp, int64_t nkeys,
+                             const int8_t* mask, int mask_active, float scale_log2, float* pa, float* pl,
+                             float* dst_a, float* dst_l, int32_t* nslots, cudaStream_t s, bool merge_only);
+
 // Small-block in-block attention + merge (fb_inblock.cu).
 bool inblock_small_applies(const fb_attn_desc& d, int next);
 cudaError_t launch_inblock_small(const fb_attn_desc& d, const void* q, const void* kin, const void* vin, int next,

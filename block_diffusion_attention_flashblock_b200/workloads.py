@@ -32,7 +32,7 @@ import torch
 
 # tensor codes of the sub-streams
 _T_PREFIX_K, _T_PREFIX_V, _T_Q, _T_K, _T_V = 0, 1, 2, 3, 4
-_T_M, _T_POS, _T_NQ, _T_NK, _T_NV, _T_SIGMA, _T_SCORE = 5, 6, 7, 8, 9, 10, 11
+_T_M, _T_POS, _T_NQ, _T_NK, _T_NV, _T_SIGMA, _T_SCORE, _T_LOCK = 5, 6, 7, 8, 9, 10, 11, 12
 
 INT32_MAX = 2**31 - 1
 
@@ -57,6 +57,8 @@ class WorkloadSpec:
     tau: Optional[int] = None                 # None: tau gate off
     gamma: Optional[float] = None             # None: gamma gate off
     sel_k: Optional[int] = None               # sparse: keys kept per query head
+    lock_rate: Optional[float] = None         # active-query subsets: share of the still-active
+                                              # positions that lock at each step (None: all active)
     seed: int = 2026_0000
     sigma_redraws: Tuple[Tuple[int, int], ...] = field(default=())
     """(block, head) pairs whose sigma is redrawn from the next sub-seed, to keep
@@ -107,6 +109,13 @@ SPECS = {
         name="dllm_8k_nb4", B=1, Hq=32, Hkv=8, D=128, prefix0=8192, Nb=4, steps=8,
         blocks=4, dtype="bf16", std=0.5, m_model=("binomial", 4, 0.15),
         pert_std=0.05, tau=2, seed=2026_0020),
+    # active-query subsets (NEXT-4): the dllm_8k layer where a quarter of the
+    # still-active block positions lock at every step (32, 24, 18, 13, 10, 8,
+    # 6, 4 active); only active positions change and are recomputed
+    "dllm_8k_lock": WorkloadSpec(
+        name="dllm_8k_lock", B=1, Hq=32, Hkv=8, D=128, prefix0=8192, Nb=32, steps=8,
+        blocks=4, dtype="bf16", std=0.5, m_model=("binomial", 32, 0.15),
+        pert_std=0.05, tau=8, lock_rate=0.25, seed=2026_0040),
     "video_1560": WorkloadSpec(
         name="video_1560", B=1, Hq=24, Hkv=24, D=128, prefix0=31200, Nb=1560,
         steps=8, blocks=1, dtype="bf16", std=1.0, m_model=("all",),
@@ -156,6 +165,7 @@ class Step:
     vin: torch.Tensor           # [B, Hkv, Nb, D]
     sel: Optional[torch.Tensor]  # int32 [B, Hq, sel_k] ascending, or None
     last_in_block: bool
+    active: Optional[torch.Tensor] = None   # int32 [B, n_active] ascending block positions, or None (all)
 
 
 class Workload:
@@ -207,10 +217,14 @@ class Workload:
             return s.Nb
         raise ValueError(kind)
 
-    def step_update(self, blk: int, step: int, q, kin, vin):
-        """Inputs of diffusion step ``step`` (>= 1) from those of step - 1."""
+    def step_update(self, blk: int, step: int, q, kin, vin, active=None):
+        """Inputs of diffusion step ``step`` (>= 1) from those of step - 1.
+        With ``active`` ([B, n] positions), only active positions change and
+        M counts updated active positions (at most n)."""
         s = self.spec
         M = self.draw_M(blk, step)
+        if active is not None:
+            M = min(M, active.shape[1])
         q = q.clone(); kin = kin.clone(); vin = vin.clone()
         if s.m_model[0] == "all":
             sig = self.head_sigmas(blk)
@@ -228,7 +242,10 @@ class Workload:
             return 0, q, kin, vin
         gp = _rng(s, _T_POS, blk, step)
         for b in range(s.B):
-            pos = np.sort(gp.choice(s.Nb, size=M, replace=False))
+            if active is None:
+                pos = np.sort(gp.choice(s.Nb, size=M, replace=False))
+            else:
+                pos = np.sort(gp.choice(active[b].numpy(), size=M, replace=False))
             idx = torch.from_numpy(pos)
             for t, code, H in ((q, _T_NQ, s.Hq), (kin, _T_NK, s.Hkv), (vin, _T_NV, s.Hkv)):
                 noise = _rng(s, code, blk, step, b).standard_normal(
@@ -256,6 +273,24 @@ class Workload:
                 out[b, h] = np.sort(order)
         return torch.from_numpy(out)
 
+    # -- active-query subsets -----------------------------------------------
+    def n_active(self, step: int) -> int:
+        """Positions still active at a block's step: all Nb at step 0, then a
+        share lock_rate of them locks at every step (at least one stays)."""
+        s = self.spec
+        return max(1, int(round(s.Nb * (1.0 - s.lock_rate) ** step)))
+
+    def lock_step(self, blk: int, step: int, active: Optional[torch.Tensor]) -> torch.Tensor:
+        """Active positions at ``step``: a seeded random subset of the previous
+        step's active positions (locking is monotone), int32 [B, n] ascending."""
+        s = self.spec
+        n = self.n_active(step)
+        if active is None:
+            return torch.arange(s.Nb, dtype=torch.int32).repeat(s.B, 1)
+        g = _rng(s, _T_LOCK, blk, step)
+        out = np.stack([np.sort(g.choice(active[b].numpy(), size=n, replace=False)) for b in range(s.B)])
+        return torch.from_numpy(out.astype(np.int32))
+
     # -- the whole schedule -------------------------------------------------
     def schedule(self) -> Iterator[Step]:
         s = self.spec
@@ -263,11 +298,14 @@ class Workload:
             plen = s.prefix0 + blk * s.Nb
             sel = self.selection(blk, plen) if s.sel_k else None
             q, kin, vin = self.block_start(blk)
+            active = None
             for st in range(s.steps):
+                if s.lock_rate is not None:
+                    active = self.lock_step(blk, st, active)
                 M = 0
                 if st > 0:
-                    M, q, kin, vin = self.step_update(blk, st, q, kin, vin)
-                yield Step(blk, st, plen, M, q, kin, vin, sel, st == s.steps - 1)
+                    M, q, kin, vin = self.step_update(blk, st, q, kin, vin, active)
+                yield Step(blk, st, plen, M, q, kin, vin, sel, st == s.steps - 1, active)
 
 
 def get_spec(name: str, **overrides) -> WorkloadSpec:

@@ -30,6 +30,10 @@ What the pages define, and how it is written here
 * Sparse attention compatibility: the keys a sparse method did not select
   are treated as the block-external set and their residual contribution is
   cached (same section, third bullet).  ``outblock_selected``.
+* Active-query subsets (SureLock page, "Principes de Fonctionnement", items 2
+  and 3): only the M_t still-unlocked positions of the block query, over the
+  cached K/V of every token; a locked position keeps its output.  Combined
+  here with the FlashBlock cache of A_out.  ``FlashBlockOracle.step(active=)``.
 
 Readings where the pages are silent (each one is listed in the design notes):
 scale = 1/sqrt(D); natural log; bidirectional attention inside the block;
@@ -228,9 +232,23 @@ class FlashBlockOracle:
         """A new block: the cache no longer describes this block's queries."""
         self.valid = False
         self.sim = np.full((self.B, self.Hq), np.nan)
+        # outputs of the previous step: the value a locked position keeps
+        self.last_o = np.full((self.B, self.Hq, self.Nb, self.D), np.nan)
+        self.last_lse = np.full((self.B, self.Hq, self.Nb), np.nan)
+        self.last_active = None
 
     def step(self, q, kin, vin, kp, vp, prefix_len: int, M: int,
-             tau: Optional[int], sel=None) -> StepResult:
+             tau: Optional[int], sel=None, active=None) -> StepResult:
+        """One diffusion step.  ``active`` ([B, n] block positions, n the
+        same for every b), if given, restricts the step to the queries that are
+        still unlocked (SureLock page, "Principes de Fonctionnement", items 2
+        and 3): only their block-external part is recomputed on a full step,
+        only they attend to the block's keys (all Nb of them, locked ones
+        included), and a locked position keeps its output of the previous
+        step.  Locking is monotone within a block.  Used without sparse
+        selection or the gamma gate."""
+        if active is not None:
+            return self._step_active(q, kin, vin, kp, vp, prefix_len, M, tau, np.asarray(active, dtype=np.int64))
         B, Hq = self.B, self.Hq
         # The cached part is attention over one block-external key set J_out
         # ("Mécanisme Central"): the prefix, or for sparse steps the prefix
@@ -273,7 +291,39 @@ class FlashBlockOracle:
         if fresh_S is not None:
             parts.insert(0, fresh_S)
         o, lse = merge(parts)
+        self.last_o, self.last_lse, self.last_active = o.copy(), lse.copy(), None
         return StepResult(o, lse, not tau_reuse, head_reuse.copy(), self.sim.copy())
+
+    def _step_active(self, q, kin, vin, kp, vp, prefix_len, M, tau, active):
+        B, Hq = self.B, self.Hq
+        assert self.gamma is None, "active-query subsets are used without the gamma gate"
+        assert active.shape[0] == B and 1 <= active.shape[1] <= self.Nb
+        if self.last_active is not None:     # monotone locking: no position comes back
+            for b in range(B):
+                assert set(active[b].tolist()) <= set(self.last_active[b].tolist()), "a locked position came back"
+        key_set = (prefix_len, None)
+        if self.valid and key_set != self.key_set:
+            self.begin_block()
+        self.key_set = key_set
+        tau_reuse = self.valid and (tau is None or M < tau)
+        o = self.last_o.copy()
+        lse = self.last_lse.copy()
+        for b in range(B):
+            rows = active[b]
+            for h in range(Hq):
+                g = kv_head(h, Hq, self.Hkv)
+                qa = q[b, h, rows]
+                if not tau_reuse:
+                    A, L = attention_part(qa, kp[b, g, :prefix_len], vp[b, g, :prefix_len], self.scale)
+                    self.cache_A[b, h, rows] = A
+                    self.cache_L[b, h, rows] = L
+                a_in, l_in = attention_part(qa, kin[b, g], vin[b, g], self.scale)
+                ob, lb = merge([(self.cache_A[b, h, rows], self.cache_L[b, h, rows]), (a_in, l_in)])
+                o[b, h, rows] = ob
+                lse[b, h, rows] = lb
+        self.valid = True
+        self.last_o, self.last_lse, self.last_active = o.copy(), lse.copy(), active.copy()
+        return StepResult(o, lse, not tau_reuse, np.full((B, Hq), tau_reuse), self.sim.copy())
 
 
 def to64(t) -> np.ndarray:

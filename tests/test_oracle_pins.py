@@ -315,6 +315,92 @@ def test_changed_key_set_recomputes():
     np.testing.assert_allclose(r.o, A, rtol=1e-11, atol=1e-12)
 
 
+# ------------------------------------------------- active-query subsets ---
+def _run_active(spec, work, tau, all_active=False):
+    kp, vp = work.prefix_kv()
+    kp64, vp64 = orc.to64(kp), orc.to64(vp)
+    o = orc.FlashBlockOracle(spec.B, spec.Hq, spec.Hkv, spec.D, spec.Nb)
+    res = []
+    for st in work.schedule():
+        if st.step == 0:
+            o.begin_block()
+        act = np.tile(np.arange(spec.Nb), (spec.B, 1)) if all_active else st.active.numpy()
+        r = o.step(orc.to64(st.q), orc.to64(st.kin), orc.to64(st.vin), kp64, vp64, st.prefix_len, st.M, tau,
+                   active=act)
+        res.append((st, r, (kp64, vp64)))
+        if st.last_in_block:
+            kp64, vp64, _ = orc.kv_append(kp64, vp64, st.prefix_len, orc.to64(st.kin), orc.to64(st.vin))
+    return res
+
+
+def _tiny_lock(**kw):
+    return _tiny(lock_rate=0.3, steps=5, **kw)
+
+
+def test_active_all_positions_is_the_dense_step():
+    """Every position active: the subset step is the dense step."""
+    spec, work = _tiny_lock(blocks=2)
+    dense, _, _ = _run(spec, work, tau=spec.tau)
+    sub = _run_active(spec, work, tau=spec.tau, all_active=True)
+    for (st, rd), (_, ra, _) in zip(dense, sub):
+        assert rd.recompute == ra.recompute
+        np.testing.assert_allclose(ra.o, rd.o, rtol=1e-13, atol=1e-14)
+        np.testing.assert_allclose(ra.lse, rd.lse, rtol=1e-13)
+
+
+def test_active_rows_of_full_steps_are_full_attention_and_locked_rows_keep_their_output():
+    """tau = 0 (every step full): each active row is exact attention over the
+    prefix and all block keys (locked tokens' keys included); each locked
+    position keeps, bit for bit, its output of the previous step."""
+    spec, work = _tiny_lock()
+    res = _run_active(spec, work, tau=0)
+    prev = None
+    for st, r, (kp64, vp64) in res:
+        assert r.recompute
+        A, L = orc.full_attention(orc.to64(st.q), orc.to64(st.kin), orc.to64(st.vin), kp64, vp64,
+                                  st.prefix_len, 1 / 8)
+        rows = st.active.numpy()[0]
+        assert 0 < len(rows) <= spec.Nb
+        np.testing.assert_allclose(r.o[:, :, rows], A[:, :, rows], rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(r.lse[:, :, rows], L[:, :, rows], rtol=1e-12)
+        locked = np.setdiff1d(np.arange(spec.Nb), rows)
+        if prev is None:
+            assert len(locked) == 0
+        else:
+            assert np.array_equal(r.o[:, :, locked], prev.o[:, :, locked])
+            assert np.array_equal(r.lse[:, :, locked], prev.lse[:, :, locked])
+        prev = r
+
+
+def test_active_reuse_rows_merge_the_block_start_cache():
+    """tau off: only step 0 computes the block-external part; an active row at
+    step s merges its step-0 cached part with fresh in-block attention."""
+    spec, work = _tiny_lock()
+    res = _run_active(spec, work, tau=None)
+    st0, _, (kp64, vp64) = res[0]
+    A0, L0 = orc.outblock(orc.to64(st0.q), kp64, vp64, st0.prefix_len, 1 / 8)
+    for st, r, _ in res:
+        assert r.recompute == (st.step == 0)
+        rows = st.active.numpy()[0]
+        Ai, Li = orc.inblock(orc.to64(st.q), orc.to64(st.kin), orc.to64(st.vin), 1 / 8)
+        A, L = orc.merge([(A0, L0), (Ai, Li)])
+        np.testing.assert_allclose(r.o[:, :, rows], A[:, :, rows], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(r.lse[:, :, rows], L[:, :, rows], rtol=1e-12)
+
+
+def test_active_sets_only_shrink():
+    spec, work = _tiny_lock()
+    steps = list(work.schedule())
+    o = orc.FlashBlockOracle(spec.B, spec.Hq, spec.Hkv, spec.D, spec.Nb)
+    kp, vp = work.prefix_kv()
+    st = steps[2]
+    o.step(orc.to64(st.q), orc.to64(st.kin), orc.to64(st.vin), orc.to64(kp), orc.to64(vp), st.prefix_len, 0, None,
+           active=steps[2].active.numpy())
+    with pytest.raises(AssertionError):   # a position locked at step 2 cannot be active again
+        o.step(orc.to64(st.q), orc.to64(st.kin), orc.to64(st.vin), orc.to64(kp), orc.to64(vp), st.prefix_len, 0,
+               None, active=steps[0].active.numpy())
+
+
 def test_static_queries_reuse_equals_full():
     """Queries unchanged across steps: the cached A_out is exact, so every step equals full attention."""
     spec, work = _tiny(steps=4)

@@ -96,15 +96,37 @@ def test_outblock_dense_tcgen05(shape, mode, prefix_kernel):
     _outblock_check(shape, seed=13)
 
 
-@pytest.mark.parametrize("which", ["generic", "tcgen05", "tcgen05-cluster"])
+PAIR_SHAPES = [
+    # (B, Hq, Hkv, D, Nb, Lp, dtype): two or more 128-row query tiles per KV head
+    (2, 32, 8, 128, 64, 3000, "bf16"),     # 2 heads x 64 queries per tile, one pair per KV head
+    (4, 32, 8, 128, 64, 4100, "bf16"),     # the long-context shape, small: CTAs span several pairs
+    (1, 16, 4, 128, 64, 777, "bf16"),      # ragged last key tile (777 = 6 * 128 + 9)
+    (1, 4, 4, 128, 200, 2000, "bf16"),     # one head per tile, ragged query tail (200 = 128 + 72)
+    (1, 6, 6, 128, 300, 1000, "bf16"),     # three tiles per head: one pair and one lone tile
+    (1, 8, 2, 128, 1560, 1700, "bf16"),    # video-like block with GQA, 52 tiles per KV head
+    (1, 2, 2, 128, 1560, 31200, "bf16"),   # a video frame block over the full 20-frame prefix
+]
+
+
+@pytest.mark.parametrize("shape", PAIR_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_outblock_dense_paired(shape, prefix_kernel):
+    """The paired stream-K tcgen05 prefix pass (two query tiles per CTA, one
+    thread per row) and the merge of its slots."""
+    prefix_kernel(fb.PREFIX_TC)
+    _outblock_check(shape, seed=17)
+
+
+@pytest.mark.parametrize("which", ["generic", "tcgen05", "tcgen05-cluster", "paired"])
 def test_outblock_rising_and_falling_scores(which, prefix_kernel):
     """Scores that grow along the prefix (KV head 0) force the running max to
     move on every key tile, so O is rescaled in place many times; scores that
     fall (KV head 1) never move it after the first tile."""
     prefix_kernel({"generic": fb.PREFIX_GENERIC, "tcgen05": fb.PREFIX_TC_NO_CLUSTER,
-                   "tcgen05-cluster": fb.PREFIX_TC_CLUSTER}[which])
-    # 8 row tiles x 64 key tiles (ragged last): several key tiles per CTA
-    B, Hq, Hkv, D, Nb, Lp = 1, 32, 8, 128, 32, 8100
+                   "tcgen05-cluster": fb.PREFIX_TC_CLUSTER, "paired": fb.PREFIX_TC}[which])
+    # 8 row tiles x 64 key tiles (ragged last): several key tiles per CTA;
+    # blocks of 64 for the paired kernel (two row tiles per KV head)
+    B, Hq, Hkv, D, Lp = 1, 32, 8, 128, 8100
+    Nb = 64 if which == "paired" else 32
     q = wl.tensor((B, Hq, Nb, D), 61, 0.5, "f32").abs().to(torch.bfloat16)
     ramp = torch.arange(Lp + 64, dtype=torch.float32) * 0.02
     sign = torch.tensor([1.0, -1.0] * (Hkv // 2)).view(1, Hkv, 1, 1)

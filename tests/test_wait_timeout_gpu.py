@@ -25,10 +25,13 @@ DEFAULT_LIMIT_NS = 2_000_000_000
 
 
 @pytest.mark.gpu
-def test_expired_wait_reports_timeout_and_the_device_recovers():
-    # dLLM-like shape: the prefix pass runs on the tcgen05 kernel (TMA + MMA
-    # barriers) and the in-block merge on the small kernel (bulk-copy barriers)
-    B, Hq, Hkv, D, Nb, Lp = 1, 8, 2, 128, 32, 2048
+@pytest.mark.parametrize("Nb", [32, 64], ids=["split-kernel", "paired-kernel"])
+def test_expired_wait_reports_timeout_and_the_device_recovers(Nb):
+    # dLLM-like shapes: the prefix pass runs on a tcgen05 kernel (TMA + MMA
+    # barriers; with blocks of 64 the KV head's 256 query rows make two tiles
+    # and the paired stream-K kernel runs) and the in-block merge on the small
+    # kernel (bulk-copy barriers)
+    B, Hq, Hkv, D, Lp = 1, 8, 2, 128, 2048
     q = wl.tensor((B, Hq, Nb, D), 41, 1.0, "bf16")
     kin = wl.tensor((B, Hkv, Nb, D), 42, 1.0, "bf16")
     vin = wl.tensor((B, Hkv, Nb, D), 43, 1.0, "bf16")
