@@ -404,6 +404,16 @@ static fb_status run_inblock(const fb_attn_desc& d, const void* q, const void* k
   if (nflat > FB_MAX_PARTS) return FB_EINVAL;
   if (cache_a) return FB_EUNSUPPORTED;   // callers only ask for the cache write where the small kernel runs
   TcMaps maps;
+  PairPlan pw;
+  if ((g_prefix_kernel == 0 || g_prefix_kernel == 2) && nflat <= FB_MAX_PARTS - 1 &&
+      tc_make_maps(d, q, kin, vin, d.Nb, d.kin_strides, &maps) && pair_plan_whole(d, d.Nb, &pw)) {
+    // large blocks: one launch of the paired kernel over the block's own keys,
+    // merged with the external parts in its epilogue
+    ProfScope prof(kProfInblock, bytes, s);
+    return launch_attn_pair_fused(d, maps, pw, d.Nb, a.scale_log2, nflat, fa, fl, o, lse, s) == cudaSuccess
+               ? FB_OK
+               : FB_ECUDA;
+  }
   if (ws_a && ws_cap >= 1 && g_prefix_kernel != 1 && d.Nb >= 128 && ext.ngroups < 8 &&
       tc_make_maps(d, q, kin, vin, d.Nb, d.kin_strides, &maps)) {
     int32_t ns, cl, np;
@@ -666,6 +676,9 @@ struct fb_cache {
   int32_t* counters;  // gamma: per-head arrival counters (kept at zero)
   int32_t chunks;
   int32_t* pair_ns;   // slot counts of the paired prefix pass
+  void* act_q;        // active subsets: compact queries [B, Hq, Nb, D]
+  float* act_a;       // active subsets: compact block-external part
+  float* act_l;
 };
 
 namespace {
@@ -701,6 +714,12 @@ fb_status layout_cache(const fb_attn_desc& d, int32_t flags, int64_t max_prefix,
     sl = cv.take<float>(base, (size_t)sel_cap * rows * 4);
     bm = cv.take<uint32_t>(base, (size_t)d.B * d.Hq * words * 4);
   }
+  void* aq = nullptr; float* aa = nullptr; float* al = nullptr;
+  if (flags & FB_CACHE_ACTIVE) {
+    aq = cv.take<uint8_t>(base, (size_t)rows * d.D * esize(d.in_dtype));
+    aa = cv.take<float>(base, (size_t)rows * d.D * 4);
+    al = cv.take<float>(base, (size_t)rows * 4);
+  }
   int8_t* mk = nullptr; float* sm = nullptr; float* gp = nullptr; int32_t* ct = nullptr;
   if (flags & FB_CACHE_GAMMA) {
     mk = cv.take<int8_t>(base, (size_t)d.B * d.Hq);
@@ -714,6 +733,7 @@ fb_status layout_cache(const fb_attn_desc& d, int32_t flags, int64_t max_prefix,
     c->sel_a = sa; c->sel_l = sl; c->sel_cap = sel_cap; c->bitmap = bm; c->bitmap_words = words;
     c->mask = mk; c->sim = sm; c->gpart = gp; c->counters = ct; c->chunks = chunks;
     c->pair_ns = pn;
+    c->act_q = aq; c->act_a = aa; c->act_l = al;
   }
   return FB_OK;
 }
@@ -725,7 +745,8 @@ fb_status fb_cache_workspace_bytes(const fb_attn_desc* d, int32_t flags, int64_t
                                    size_t* bytes) {
   fb_status st = check_desc(d);
   if (st != FB_OK) return st;
-  if (!bytes || max_prefix < 0 || max_sel_k < 0 || (flags & ~(FB_CACHE_SPARSE | FB_CACHE_GAMMA))) return FB_EINVAL;
+  if (!bytes || max_prefix < 0 || max_sel_k < 0 || (flags & ~(FB_CACHE_SPARSE | FB_CACHE_GAMMA | FB_CACHE_ACTIVE)))
+    return FB_EINVAL;
   return layout_cache(*d, flags, max_prefix, max_sel_k, nullptr, nullptr, bytes);
 }
 
@@ -786,6 +807,13 @@ fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
   if (gamma && !(c->flags & FB_CACHE_GAMMA)) return FB_ESTATE;
   if (sparse && gamma) return FB_EUNSUPPORTED;
   if (sparse && (a->sel_k < 0 || a->sel_k > a->prefix_len || a->sel_k > c->max_sel_k)) return FB_EINVAL;
+  const bool subset = a->active != nullptr;
+  if (subset) {
+    if (!(c->flags & FB_CACHE_ACTIVE)) return FB_ESTATE;
+    if (a->n_active < 1 || a->n_active > d.Nb) return FB_EINVAL;
+    if (sparse || gamma || !inblock_small_applies(d, 1)) return FB_EUNSUPPORTED;
+    if (!al16(a->active)) return FB_EALIGN;
+  }
   if (!al16(a->q) || !al16(a->kin) || !al16(a->vin) || !al16(a->kp) || !al16(a->vp) || !al16(a->o) ||
       !al16(a->lse) || !al16(a->sel) || !al16(a->gamma))
     return FB_EALIGN;
@@ -803,6 +831,55 @@ fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
   PartList ext;
   memset(&ext, 0, sizeof(ext));
 
+  if (subset) {
+    // only the active queries: on a full step their block-external part, from
+    // a compact copy of their rows, lands in their cache rows
+    if (!tau_reuse) {
+      const int32_t n = a->n_active;
+      fb_attn_desc dc = d;
+      dc.Nb = n;
+      dc.q_strides[0] = (int64_t)d.Hq * n * d.D;
+      dc.q_strides[1] = (int64_t)n * d.D;
+      dc.q_strides[2] = d.D;
+      {
+        ProfScope prof(kProfAux, 2.0 * rows_of(dc) * d.D * esize(d.in_dtype), s);
+        if (launch_gather_active_q(d, a->q, c->act_q, a->active, n, s) != cudaSuccess) return FB_ECUDA;
+      }
+      PrefixPlan p = plan_prefix(dc, c->act_q, a->kp, a->vp, a->prefix_len, c->part_cap);
+      p.pair = false;   // its slot counts are sized for the full block
+      if (p.nparts == 1) {
+        if ((st = launch_prefix(dc, p, a->prefix_len, nullptr, 0, c->act_a, c->act_l, s)) != FB_OK) return st;
+      } else {
+        if ((st = launch_prefix(dc, p, a->prefix_len, nullptr, 0, c->part_a, c->part_l, s)) != FB_OK) return st;
+        PartList lst;
+        memset(&lst, 0, sizeof(lst));
+        lst.ngroups = 1;
+        lst.g[0] = group_of(c->part_a, c->part_l, p.nparts, dc);
+        if ((st = merge_to_part(dc, lst, c->act_a, c->act_l, nullptr, 0, s)) != FB_OK) return st;
+      }
+      ProfScope prof(kProfAux, 2.0 * rows_of(dc) * (d.D + 1) * 4.0, s);
+      if (launch_scatter_active_part(d, c->act_a, c->act_l, c->cache_a, c->cache_l, a->active, n, s) != cudaSuccess)
+        return FB_ECUDA;
+    }
+    if (a->reuse_out && launch_fill_decision(a->reuse_out, BH, tau_reuse ? 1 : 0, s) != cudaSuccess)
+      return FB_ECUDA;
+    if (a->sim_out && cudaMemsetAsync(a->sim_out, 0xFF, (size_t)BH * 4, s) != cudaSuccess) return FB_ECUDA;
+    const float* ca[1] = {c->cache_a};
+    const float* cl[1] = {c->cache_l};
+    const int es = esize(d.in_dtype);
+    const double rows = (double)d.B * d.Hq * a->n_active;
+    {
+      ProfScope prof(kProfInblock, rows * d.D * es + 2.0 * d.B * d.Hkv * d.Nb * d.D * es + rows * (d.D + 1) * 4.0 +
+                                       rows * (d.D * esize(d.out_dtype) + (a->lse ? 4 : 0)),
+                     s);
+      if (launch_inblock_small(d, a->q, a->kin, a->vin, 1, ca, cl, a->o, a->lse, nullptr, nullptr, scale_log2(d), s,
+                               a->active, a->n_active) != cudaSuccess)
+        return FB_ECUDA;
+    }
+    c->valid = true;
+    c->last_recomputed = !tau_reuse;
+    return FB_OK;
+  }
   if (gamma) {
     PrefixPlan p = plan_prefix(d, a->q, a->kp, a->vp, a->prefix_len, c->part_cap);
     int32_t fresh_parts = p.nparts;

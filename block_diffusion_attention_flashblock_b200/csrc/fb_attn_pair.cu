@@ -126,6 +126,17 @@ struct PairArgs {
   uint64_t wait_limit_ns;
   uint32_t q_bytes;        // bytes of one Q tile (both 64-column halves)
   int32_t stall;           // test hook: the MMA issuer first waits on a barrier nothing completes
+  // whole-pair mode: every CTA takes whole pairs (no slots, no merge kernel)
+  // and its epilogue merges each row with `next` external parts and writes
+  // O (out dtype and strides) and LSE directly
+  int32_t whole;
+  int32_t next;
+  const float* ext_a[FB_MAX_PARTS];
+  const float* ext_l[FB_MAX_PARTS];
+  void* o;
+  int64_t o_sb, o_sh, o_st;
+  int32_t o_bf16;
+  float* lse;
 };
 
 namespace {
@@ -234,10 +245,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int w = 0; w < words; ++w) nact += __popc(act[w]);
     }
     const int64_t T = (int64_t)nact * a.nkt;
-    const int C = (int)min((int64_t)min((int64_t)gridDim.x, T), (int64_t)nact * (a.smax - 1));
+    const int C = a.whole ? min((int)gridDim.x, nact)
+                          : (int)min((int64_t)min((int64_t)gridDim.x, T), (int64_t)nact * (a.smax - 1));
     const int c = blockIdx.x;
     int n = 0;
-    if (c < C) {
+    if (a.whole) {
+      // whole pairs: active pairs c, c + C, c + 2C, ...
+      int ai = 0;
+      for (int p = 0; p < a.npairs && n < kMaxSeg; ++p) {
+        if (a.mask_active && !((act[p >> 5] >> (p & 31)) & 1u)) continue;
+        if (ai++ % C != c) continue;
+        Seg sg;
+        sg.pair = p;
+        sg.j0 = 0;
+        sg.j1 = a.nkt;
+        sg.slot_ns = 1 << 16;
+        segs[n++] = sg;
+      }
+    } else if (c < C) {
       const int64_t i0 = (int64_t)c * T / C, i1 = (int64_t)(c + 1) * T / C;
       int64_t ai = i0 / a.nkt;            // active index of the first pair
       // the ai-th active pair
@@ -515,6 +540,79 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       ++ocnt;
       tc_fence_after();
+      if (a.whole) {
+        // merge with the external parts (log space, as the standalone merge)
+        // and write this row of O and LSE
+        const bool mine = row < t.nrows;
+        const int64_t r = t.rbase + row;
+        const float Lin = l > 0.f ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
+        float mm = Lin;
+        float Lx[FB_MAX_PARTS];
+#pragma unroll
+        for (int p = 0; p < FB_MAX_PARTS - 1; ++p) {
+          Lx[p] = (p < a.next && mine) ? a.ext_l[p][r] : -CUDART_INF_F;
+          mm = fmaxf(mm, Lx[p]);
+        }
+        const bool empty = mm == -CUDART_INF_F;
+        const float win = (empty || Lin == -CUDART_INF_F) ? 0.f : __expf(Lin - mm);
+        float wx[FB_MAX_PARTS];
+        float wsum = win;
+#pragma unroll
+        for (int p = 0; p < FB_MAX_PARTS - 1; ++p) {
+          wx[p] = (empty || Lx[p] == -CUDART_INF_F) ? 0.f : __expf(Lx[p] - mm);
+          wsum += wx[p];
+        }
+        const float inv = empty ? 0.f : 1.f / wsum;
+        const float wi = l > 0.f ? win / l : 0.f;   // O in TMEM is unnormalised
+        const int h = a.mode == 0 ? t.h0 + row / a.Nb : t.h0;
+        const int i = a.mode == 0 ? row % a.Nb : t.i0 + row;
+        const int64_t obase = t.b * a.o_sb + (int64_t)h * a.o_sh + (int64_t)i * a.o_st;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld();
+          if (mine) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= wi;
+#pragma unroll
+            for (int p = 0; p < FB_MAX_PARTS - 1; ++p) {
+              if (p >= a.next || wx[p] == 0.f) continue;   // an empty part may hold anything
+              const float4* src = reinterpret_cast<const float4*>(a.ext_a[p] + r * kD + c * 32);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float4 v = src[e];
+                o[4 * e] = fmaf(wx[p], v.x, o[4 * e]);
+                o[4 * e + 1] = fmaf(wx[p], v.y, o[4 * e + 1]);
+                o[4 * e + 2] = fmaf(wx[p], v.z, o[4 * e + 2]);
+                o[4 * e + 3] = fmaf(wx[p], v.w, o[4 * e + 3]);
+              }
+            }
+            if (a.o_bf16) {
+              uint4* d4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + obase + c * 32);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                uint32_t w[4];
+#pragma unroll
+                for (int f = 0; f < 4; ++f) {
+                  const __nv_bfloat162 pr = __floats2bfloat162_rn(o[8 * e + 2 * f] * inv, o[8 * e + 2 * f + 1] * inv);
+                  w[f] = *reinterpret_cast<const uint32_t*>(&pr);
+                }
+                d4[e] = make_uint4(w[0], w[1], w[2], w[3]);
+              }
+            } else {
+              float4* d4 = reinterpret_cast<float4*>(static_cast<float*>(a.o) + obase + c * 32);
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                d4[e] = make_float4(o[4 * e] * inv, o[4 * e + 1] * inv, o[4 * e + 2] * inv, o[4 * e + 3] * inv);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(B_OFREE + s));
+        if (mine && a.lse) a.lse[r] = empty ? -CUDART_INF_F : mm + __logf(wsum);
+        continue;
+      }
       const int slot = sg.slot_ns & 0xFFFF, nsl = sg.slot_ns >> 16;
       const bool direct = nsl == 1;
       const int64_t r = t.rbase + row;
@@ -653,6 +751,59 @@ cudaError_t launch_attn_pair(const fb_attn_desc& d, const TcMaps& m, const PairP
     return launch_k(pair_merge_kernel, dim3((unsigned)((nrows + 7) / 8)), dim3(256), 0, s, a);
   }
   return launch_k(attn_pair_kernel, dim3(pp.grid), dim3(kThreads), kSmemBytes, s, m.q, m.k, m.v, a);
+}
+
+// Whole-pair fused pass over the keys of (k, v) [0, nkeys): attention of the
+// block's queries merged with `next` external parts, written to O and LSE.
+cudaError_t launch_attn_pair_fused(const fb_attn_desc& d, const TcMaps& m, const PairPlan& pp, int64_t nkeys,
+                                   float scale_log2, int32_t next, const float* const* ext_a,
+                                   const float* const* ext_l, void* o, float* lse, cudaStream_t s) {
+  PairArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = d.B; a.Hq = d.Hq; a.Hkv = d.Hkv; a.G = d.Hq / d.Hkv; a.Nb = d.Nb;
+  a.mode = pp.mode; a.hg = pp.hg; a.tph = pp.tph;
+  a.tiles_per_kv = pp.tiles_per_kv; a.pairs_per_kv = pp.pairs_per_kv; a.npairs = pp.npairs;
+  a.nkt = pp.nkt; a.nkeys = nkeys; a.smax = 1;
+  a.scale_log2 = scale_log2;
+  a.status = device_status_ptr();
+  a.wait_limit_ns = wait_limit_ns();
+  a.q_bytes = 2u * 64u * 2u * (uint32_t)(pp.mode == 0 ? d.Nb * pp.hg : kBM);
+  a.stall = debug_stall() ? 1 : 0;
+  a.whole = 1;
+  a.next = next;
+  for (int p = 0; p < next; ++p) { a.ext_a[p] = ext_a[p]; a.ext_l[p] = ext_l[p]; }
+  a.o = o; a.o_sb = d.o_strides[0]; a.o_sh = d.o_strides[1]; a.o_st = d.o_strides[2];
+  a.o_bf16 = d.out_dtype == FB_BF16;
+  a.lse = lse;
+  if (!a.status || next < 0 || next > FB_MAX_PARTS - 1) return cudaErrorInvalidValue;
+  static bool attr[kMaxDevices] = {};
+  bool& done = attr[current_device()];
+  if (!done) {
+    cudaError_t e = cudaFuncSetAttribute(attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    done = true;
+  }
+  const int grid = std::min(num_sms(), pp.npairs);
+  return launch_k(attn_pair_kernel, dim3(grid), dim3(kThreads), kSmemBytes, s, m.q, m.k, m.v, a);
+}
+
+// A whole-pair plan: as pair_plan, without the slot bookkeeping (each CTA
+// takes whole pairs; up to kMaxSeg pairs per CTA).
+bool pair_plan_whole(const fb_attn_desc& d, int64_t nkeys, PairPlan* p) {
+  int mode, hg, tpu, units;
+  if (nkeys <= 0 || !tc_tiling(d, &mode, &hg, &tpu, &units)) return false;
+  const int G = d.Hq / d.Hkv;
+  p->mode = mode;
+  p->hg = hg;
+  p->tph = mode == 0 ? 1 : tpu;
+  p->tiles_per_kv = mode == 0 ? tpu : G * tpu;
+  if (p->tiles_per_kv < 2) return false;
+  p->pairs_per_kv = (p->tiles_per_kv + 1) / 2;
+  p->npairs = d.B * d.Hkv * p->pairs_per_kv;
+  p->nkt = (int32_t)((nkeys + kBN - 1) / kBN);
+  p->grid = std::min(num_sms(), p->npairs);
+  p->smax = 1;
+  return p->npairs <= kMaxPairs && (p->npairs + p->grid - 1) / p->grid <= kMaxSeg;
 }
 
 int32_t pair_count(const fb_attn_desc& d) {

@@ -278,6 +278,78 @@ cudaError_t launch_build_bitmap(const int32_t* sel, int32_t sel_k, int32_t BH, u
   return launch_k(build_bitmap_kernel, dim3(BH), dim3(256), 0, s, sel, sel_k, bitmap, words);
 }
 
+// ---------------------------------------------------------------------------
+// Active-query subsets (SureLock page, "Principes de Fonctionnement"): the
+// query rows of the still-active block positions gathered into a compact
+// block, and a compact part scattered back to the rows of those positions.
+// One warp per row; positions outside [0, Nb) are skipped and reported as
+// FB_EINVAL in the device status word.
+// ---------------------------------------------------------------------------
+__global__ void gather_active_q_kernel(const uint8_t* q, int64_t q_sb, int64_t q_sh, int64_t q_st, uint8_t* out,
+                                       const int32_t* active, int32_t n_act, int32_t B, int32_t Hq, int32_t Nb,
+                                       int32_t row_bytes, int* status) {
+  ptx::pdl_prologue();
+  const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);   // compact (b, h, k)
+  const int lane = threadIdx.x & 31;
+  const int64_t bh = r / n_act;
+  const int k = (int)(r % n_act);
+  const int b = (int)(bh / Hq), h = (int)(bh % Hq);
+  if (b >= B) return;
+  const int i = active[(int64_t)b * n_act + k];
+  if (i < 0 || i >= Nb) {
+    if (lane == 0) atomicCAS(status, 0, (int)FB_EINVAL);
+    return;
+  }
+  const uint8_t* src = q + b * q_sb + h * q_sh + i * q_st;
+  uint8_t* dst = out + r * row_bytes;
+  for (int c = lane * 16; c < row_bytes; c += 512)
+    *reinterpret_cast<uint4*>(dst + c) = __ldg(reinterpret_cast<const uint4*>(src + c));
+}
+
+__global__ void scatter_active_part_kernel(const float* ca, const float* cl, float* a, float* l,
+                                           const int32_t* active, int32_t n_act, int32_t B, int32_t Hq, int32_t Nb,
+                                           int32_t D, int* status) {
+  ptx::pdl_prologue();
+  const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int64_t bh = r / n_act;
+  const int k = (int)(r % n_act);
+  const int b = (int)(bh / Hq);
+  if (b >= B) return;
+  const int i = active[(int64_t)b * n_act + k];
+  if (i < 0 || i >= Nb) {
+    if (lane == 0) atomicCAS(status, 0, (int)FB_EINVAL);
+    return;
+  }
+  const int64_t dst = bh * Nb + i;
+  for (int c = lane * 4; c < D; c += 128)
+    *reinterpret_cast<float4*>(a + dst * D + c) = *reinterpret_cast<const float4*>(ca + r * D + c);
+  if (lane == 0) l[dst] = cl[r];
+}
+
+int* device_status_ptr();
+
+cudaError_t launch_gather_active_q(const fb_attn_desc& d, const void* q, void* out, const int32_t* active,
+                                   int32_t n_act, cudaStream_t s) {
+  const int es = d.in_dtype == FB_BF16 ? 2 : 4;
+  int* st = device_status_ptr();
+  if (!st) return cudaErrorInvalidValue;
+  const int64_t rows = (int64_t)d.B * d.Hq * n_act;
+  return launch_k(gather_active_q_kernel, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0, s,
+                  static_cast<const uint8_t*>(q), d.q_strides[0] * es, d.q_strides[1] * es, d.q_strides[2] * es,
+                  static_cast<uint8_t*>(out), active, n_act, (int32_t)d.B, (int32_t)d.Hq, (int32_t)d.Nb,
+                  (int32_t)(d.D * es), st);
+}
+
+cudaError_t launch_scatter_active_part(const fb_attn_desc& d, const float* ca, const float* cl, float* a, float* l,
+                                       const int32_t* active, int32_t n_act, cudaStream_t s) {
+  int* st = device_status_ptr();
+  if (!st) return cudaErrorInvalidValue;
+  const int64_t rows = (int64_t)d.B * d.Hq * n_act;
+  return launch_k(scatter_active_part_kernel, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0, s, ca, cl, a, l,
+                  active, n_act, (int32_t)d.B, (int32_t)d.Hq, (int32_t)d.Nb, (int32_t)d.D, st);
+}
+
 cudaError_t launch_fill_decision(int8_t* reuse_out, int32_t n, int8_t value, cudaStream_t s) {
   return cudaMemsetAsync(reuse_out, value, (size_t)n, s);
 }

@@ -84,6 +84,8 @@ struct InblockArgs {
   int* status;
   uint64_t wait_limit_ns;
   int32_t stall;      // test hook: thread 0 first waits on a barrier nothing completes
+  const int32_t* active;  // non-null: [B, n_act] block positions of the queries to compute (the rest untouched)
+  int32_t n_act;
 };
 
 // Bounded wait on phase 0 of a load barrier; the first expiry is recorded.  A
@@ -122,24 +124,37 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int unit = blockIdx.x / a.tiles_per_unit, tile = blockIdx.x % a.tiles_per_unit;
   const int b = unit / a.Hkv, kvh = unit % a.Hkv;
-  const int rows_unit = a.G * a.Nb;
+  const int nqh = a.active ? a.n_act : a.Nb;     // queries per head computed
+  const int rows_unit = a.G * nqh;
   const int row0 = tile * kRows;
   const int nq = min(kRows, rows_unit - row0);   // rows of this CTA that exist
-  // packed row r -> (query head kvh*G + r / Nb, query r % Nb); the rows of one
-  // KV head are consecutive in the packed (b, h, i) order of parts and LSE.
-  const int64_t prow0 = ((int64_t)b * a.Hq + (int64_t)kvh * a.G) * a.Nb + row0;
+  // CTA row r -> (query head kvh*G + g, block position i) with g, k = the
+  // row's head and index among the computed queries (i = k, or the k-th
+  // active position); returns the packed (b, h, i) row of parts and LSE, or
+  // -1 for a row that does not exist or names a position outside the block.
+  auto row_at = [&](int r, int& h, int& i) -> int64_t {
+    if (r >= nq) return -1;
+    const int rr = row0 + r, g = rr / nqh, k = rr % nqh;
+    i = a.active ? a.active[(int64_t)b * a.n_act + k] : k;
+    if (i < 0 || i >= a.Nb) return -1;
+    h = kvh * a.G + g;
+    return ((int64_t)b * a.Hq + h) * a.Nb + i;
+  };
   const uint32_t bar_qk = ptx::smem_addr(bars), bar_v = bar_qk + 8, bar_e = bar_qk + 16;
 
   // ---- every load is one bulk copy per row, issued up front ----
   if (tid == 0) {
+    int nvalid = 0, hh, ii;
+    for (int r = 0; r < nq; ++r) nvalid += row_at(r, hh, ii) >= 0;
+    if (nvalid < nq) atomicCAS(a.status, 0, (int)FB_EINVAL);
     ptx::mbar_init(bar_qk, 1);
     ptx::mbar_init(bar_v, 1);
     ptx::mbar_init(bar_e, 1);
     ptx::mbar_init(bar_e + 8, 1);
     ptx::fence_mbar_init();
-    ptx::mbar_expect_tx(bar_qk, (uint32_t)(nq + a.Nb) * (kD * 2));
+    ptx::mbar_expect_tx(bar_qk, (uint32_t)(nvalid + a.Nb) * (kD * 2));
     ptx::mbar_expect_tx(bar_v, (uint32_t)a.Nb * (kD * 2));
-    ptx::mbar_expect_tx(bar_e, (uint32_t)(NX * nq) * (kD * 4));
+    ptx::mbar_expect_tx(bar_e, (uint32_t)(NX * nvalid) * (kD * 4));
   }
   // L of (part, row) = (idx / 16, idx % 16) for idx = tid, tid + 128: read
   // early, stored to shared memory after P V
@@ -147,16 +162,18 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const int idx = tid + k * 128;
-    if (idx < NX * kRows && (idx & 15) < nq) lx[k] = a.ext_l[idx >> 4][prow0 + (idx & 15)];
+    int hh, ii;
+    const int64_t pr = idx < NX * kRows ? row_at(idx & 15, hh, ii) : -1;
+    if (pr >= 0) lx[k] = a.ext_l[idx >> 4][pr];
   }
   __syncthreads();
   if (warp == 0) {
     if (lane < kRows) {
       const int r = lane;
-      if (r < nq) {
-        const int rr = row0 + r, g = rr / a.Nb, i = rr % a.Nb;
-        ptx::bulk_g2s(ptx::smem_addr(sQ + r * kRowE),
-                      a.q + b * a.q_sb + (int64_t)(kvh * a.G + g) * a.q_sh + (int64_t)i * a.q_st, kD * 2, bar_qk);
+      int h, i;
+      if (row_at(r, h, i) >= 0) {
+        ptx::bulk_g2s(ptx::smem_addr(sQ + r * kRowE), a.q + b * a.q_sb + (int64_t)h * a.q_sh + (int64_t)i * a.q_st,
+                      kD * 2, bar_qk);
       } else {
 #pragma unroll 1
         for (int c = 0; c < kD / 8; ++c) reinterpret_cast<uint4*>(sQ + r * kRowE)[c] = make_uint4(0, 0, 0, 0);
@@ -177,11 +194,13 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
     }
   } else if (NX > 0) {
     const int p = lane >> 4, r = lane & 15;
+    int hh, ii;
+    const int64_t pr = row_at(r, hh, ii);
 #pragma unroll
     for (int pp = 0; pp < NX; pp += 2)
-      if (pp + p < NX && r < nq)
-        ptx::bulk_g2s(ptx::smem_addr(sE + ((pp + p) * kRows + r) * kExtStride), a.ext_a[pp + p] + (prow0 + r) * kD,
-                      kD * 4, bar_e);
+      if (pp + p < NX && pr >= 0)
+        ptx::bulk_g2s(ptx::smem_addr(sE + ((pp + p) * kRows + r) * kExtStride), a.ext_a[pp + p] + pr * kD, kD * 4,
+                      bar_e);
   }
   __syncthreads();   // zero-filled rows
   bool ok = !(a.stall && tid == 0) || wait_loaded(bar_e + 8, a);
@@ -267,7 +286,9 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int r = (lane >> 2) + 8 * h;
-    if (r >= nq) continue;
+    int hq, iq;
+    const int64_t pr = row_at(r, hq, iq);
+    if (pr < 0) continue;
     const float Lin = lrow[h] > 0.f ? (mrow[h] + __log2f(lrow[h])) * kLn2 : -CUDART_INF_F;
     float m = Lin;
     float Lx[NXS];
@@ -306,8 +327,8 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
         *reinterpret_cast<float2*>(sO + r * kExtStride + col) = make_float2(x, y);
     }
     if (dq == 0 && (lane & 3) == 0) {
-      if (a.cache_l) a.cache_l[prow0 + r] = wext > 0.f ? m + logf(wext) : -CUDART_INF_F;
-      if (a.lse) a.lse[prow0 + r] = empty ? -CUDART_INF_F : m + logf(wsum);
+      if (a.cache_l) a.cache_l[pr] = wext > 0.f ? m + logf(wext) : -CUDART_INF_F;
+      if (a.lse) a.lse[pr] = empty ? -CUDART_INF_F : m + logf(wsum);
     }
   }
   ptx::fence_proxy_async_smem();
@@ -315,15 +336,16 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   // ---- whole-row stores: lanes 0..15 the output rows, 16..31 the cache rows (warp 0) ----
   if (ok && warp == 0) {
     const int r = lane & 15;
-    if (r < nq && lane < 16) {
-      const int rr = row0 + r, g = rr / a.Nb, i = rr % a.Nb;
-      const int64_t obase = b * a.o_sb + (int64_t)(kvh * a.G + g) * a.o_sh + (int64_t)i * a.o_st;
+    int h, i;
+    const int64_t pr = row_at(r, h, i);
+    if (pr >= 0 && lane < 16) {
+      const int64_t obase = b * a.o_sb + (int64_t)h * a.o_sh + (int64_t)i * a.o_st;
       void* dst = obf ? static_cast<void*>(static_cast<__nv_bfloat16*>(a.o) + obase)
                       : static_cast<void*>(static_cast<float*>(a.o) + obase);
       ptx::bulk_s2g(dst, ptx::smem_addr(sO + r * kExtStride), obf ? kD * 2 : kD * 4);
       ptx::bulk_commit();
-    } else if (r < nq && a.cache_a) {
-      ptx::bulk_s2g(a.cache_a + (prow0 + r) * kD, ptx::smem_addr(sC + r * kExtStride), kD * 4);
+    } else if (pr >= 0 && a.cache_a) {
+      ptx::bulk_s2g(a.cache_a + pr * kD, ptx::smem_addr(sC + r * kExtStride), kD * 4);
       ptx::bulk_commit();
     }
     ptx::bulk_wait_read();
@@ -346,11 +368,14 @@ bool inblock_small_applies(const fb_attn_desc& d, int next) {
 
 cudaError_t launch_inblock_small(const fb_attn_desc& d, const void* q, const void* kin, const void* vin, int next,
                                  const float* const* ext_a, const float* const* ext_l, void* o, float* lse,
-                                 float* cache_a, float* cache_l, float scale_log2, cudaStream_t s) {
+                                 float* cache_a, float* cache_l, float scale_log2, cudaStream_t s,
+                                 const int32_t* active, int32_t n_act) {
   InblockArgs a;
   memset(&a, 0, sizeof(a));
   a.B = d.B; a.Hq = d.Hq; a.Hkv = d.Hkv; a.G = d.Hq / d.Hkv; a.Nb = d.Nb;
-  a.tiles_per_unit = (a.G * d.Nb + kRows - 1) / kRows;
+  a.active = active;
+  a.n_act = active ? n_act : d.Nb;
+  a.tiles_per_unit = (a.G * a.n_act + kRows - 1) / kRows;
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.q_sb = d.q_strides[0]; a.q_sh = d.q_strides[1]; a.q_st = d.q_strides[2];
   a.k = static_cast<const __nv_bfloat16*>(kin);

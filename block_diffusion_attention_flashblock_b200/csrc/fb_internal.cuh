@@ -154,6 +154,12 @@ struct PairPlan {
 bool pair_plan(const fb_attn_desc& d, int64_t nkeys, PairPlan* p);
 int32_t pair_slot_cap(const fb_attn_desc& d, int64_t max_keys);
 int32_t pair_count(const fb_attn_desc& d);   // pairs of the paired pass (0: it never applies)
+bool pair_plan_whole(const fb_attn_desc& d, int64_t nkeys, PairPlan* p);
+// Whole-pair mode: each CTA takes whole pairs and merges each row with `next`
+// external parts into O (out dtype, strides) and LSE; one launch, no scratch.
+cudaError_t launch_attn_pair_fused(const fb_attn_desc& d, const TcMaps& m, const PairPlan& pp, int64_t nkeys,
+                                   float scale_log2, int32_t next, const float* const* ext_a,
+                                   const float* const* ext_l, void* o, float* lse, cudaStream_t s);
 // The pass (merge_only = false) leaves the final (A, L) of rows whose pair one
 // CTA covered at dst_a / dst_l and partial results in pp.smax parts at pa /
 // pl (npairs slot counts at nslots); the merge (merge_only = true, launched
@@ -165,9 +171,16 @@ cudaError_t launch_attn_pair(const fb_attn_desc& d, const TcMaps& m, const PairP
 
 // Small-block in-block attention + merge (fb_inblock.cu).
 bool inblock_small_applies(const fb_attn_desc& d, int next);
+// With `active` ([B, n_act] block positions) only those queries are computed
+// and only their rows of O, LSE and the cache are written.
 cudaError_t launch_inblock_small(const fb_attn_desc& d, const void* q, const void* kin, const void* vin, int next,
                                  const float* const* ext_a, const float* const* ext_l, void* o, float* lse,
-                                 float* cache_a, float* cache_l, float scale_log2, cudaStream_t s);
+                                 float* cache_a, float* cache_l, float scale_log2, cudaStream_t s,
+                                 const int32_t* active = nullptr, int32_t n_act = 0);
+cudaError_t launch_gather_active_q(const fb_attn_desc& d, const void* q, void* out, const int32_t* active,
+                                   int32_t n_act, cudaStream_t s);
+cudaError_t launch_scatter_active_part(const fb_attn_desc& d, const float* ca, const float* cl, float* a, float* l,
+                                       const int32_t* active, int32_t n_act, cudaStream_t s);
 
 struct MergeArgs {
   int32_t B, Hq, Nb, D;

@@ -26,7 +26,7 @@ FB_ESTATE, FB_ECUDA, FB_ETIMEOUT, FB_ENOSPACE = 5, 6, 7, 8
 FB_F32, FB_BF16 = 0, 1
 FB_MAX_PARTS = 8
 FB_TAU_OFF = 2**31 - 1
-FB_CACHE_SPARSE, FB_CACHE_GAMMA = 1, 2
+FB_CACHE_SPARSE, FB_CACHE_GAMMA, FB_CACHE_ACTIVE = 1, 2, 4
 
 
 class FbError(RuntimeError):
@@ -48,7 +48,8 @@ class fb_step_args(C.Structure):
                 ("kp", C.c_void_p), ("vp", C.c_void_p), ("prefix_len", C.c_int64),
                 ("M", C.c_int32), ("tau", C.c_int32), ("gamma", C.c_void_p),
                 ("sel", C.c_void_p), ("sel_k", C.c_int32), ("o", C.c_void_p),
-                ("lse", C.c_void_p), ("reuse_out", C.c_void_p), ("sim_out", C.c_void_p)]
+                ("lse", C.c_void_p), ("reuse_out", C.c_void_p), ("sim_out", C.c_void_p),
+                ("active", C.c_void_p), ("n_active", C.c_int32)]
 
 
 _P = C.c_void_p
@@ -236,8 +237,11 @@ def fb_cache_begin_block(h, stream=None):
 
 
 def fb_step(h, q, kin, vin, kp, vp, prefix_len, M, tau, o, lse=None, gamma=None, sel=None,
-            reuse_out=None, sim_out=None, stream=None):
+            reuse_out=None, sim_out=None, stream=None, active=None):
+    """active: optional device int32 [B, n_active] block positions still unlocked."""
     a = fb_step_args()
+    a.active = _ptr(active)
+    a.n_active = 0 if active is None else active.shape[-1]
     a.q, a.kin, a.vin, a.kp, a.vp = _ptr(q), _ptr(kin), _ptr(vin), _ptr(kp), _ptr(vp)
     a.prefix_len, a.M, a.tau = prefix_len, M, tau
     a.gamma, a.sel = _ptr(gamma), _sel_ptr(sel)
@@ -302,9 +306,10 @@ class FlashBlockLayer:
     """
 
     def __init__(self, q_like, kin_like, kp, o_like, max_prefix, gamma=False, sparse=False,
-                 max_sel_k=0, scale=0.0):
+                 max_sel_k=0, scale=0.0, active=False):
         self.desc = make_desc(q_like, kin_like, kp, o_like, scale)
-        self.flags = (FB_CACHE_GAMMA if gamma else 0) | (FB_CACHE_SPARSE if sparse else 0)
+        self.flags = ((FB_CACHE_GAMMA if gamma else 0) | (FB_CACHE_SPARSE if sparse else 0)
+                      | (FB_CACHE_ACTIVE if active else 0))
         nbytes = fb_cache_workspace_bytes(self.desc, self.flags, max_prefix, max_sel_k)
         self.mem = torch.empty(nbytes, dtype=torch.uint8, device=kp.device)
         self.handle = fb_cache_create(self.desc, self.flags, max_prefix, max_sel_k, self.mem)
@@ -313,9 +318,9 @@ class FlashBlockLayer:
         fb_cache_begin_block(self.handle)
 
     def step(self, q, kin, vin, kp, vp, prefix_len, M, tau, o, lse=None, gamma=None, sel=None,
-             reuse_out=None, sim_out=None):
+             reuse_out=None, sim_out=None, active=None):
         fb_step(self.handle, q, kin, vin, kp, vp, prefix_len, M, tau, o, lse, gamma, sel,
-                reuse_out, sim_out)
+                reuse_out, sim_out, active=active)
 
     def last_recomputed(self) -> bool:
         return bool(fb_cache_last_step(self.handle))

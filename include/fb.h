@@ -187,13 +187,14 @@ fb_status fb_kv_append(const fb_attn_desc* d, void* kp, void* vp,
  * itself is host memory holding sizes, pointers and the host-side validity.
  *
  * flags: FB_CACHE_SPARSE enables sparse steps (sel != NULL), FB_CACHE_GAMMA
- *   enables the gamma gate.  max_prefix / max_sel_k bound later calls.
+ *   enables the gamma gate, FB_CACHE_ACTIVE steps over active-query subsets
+ *   (active != NULL).  max_prefix / max_sel_k bound later calls.
  * fb_cache_create() zeroes its bookkeeping with cudaMemsetAsync on `stream`.
  * fb_cache_begin_block() marks the cache invalid, so the next step is full.
  * ------------------------------------------------------------------------- */
 typedef struct fb_cache* fb_cache_t;
 
-enum { FB_CACHE_SPARSE = 1, FB_CACHE_GAMMA = 2 };
+enum { FB_CACHE_SPARSE = 1, FB_CACHE_GAMMA = 2, FB_CACHE_ACTIVE = 4 };
 
 fb_status fb_cache_workspace_bytes(const fb_attn_desc* d, int32_t flags,
                                    int64_t max_prefix, int32_t max_sel_k,
@@ -221,6 +222,9 @@ typedef struct fb_step_args {
   int8_t* reuse_out;      /* output int8 [B, Hq]: 1 where the cache was used, or NULL */
   float* sim_out;         /* output fp32 [B, Hq]: similarity after the step (NaN:
                              not yet defined), or NULL */
+  const int32_t* active;  /* device int32 [B, n_active]: the block positions still
+                             active (unlocked), ascending; NULL: all Nb positions */
+  int32_t n_active;       /* 1..Nb when active != NULL */
 } fb_step_args;
 
 /* One diffusion step of one attention layer under the reuse policy:
@@ -243,6 +247,20 @@ typedef struct fb_step_args {
  *   step on a handle without FB_CACHE_SPARSE, gamma without FB_CACHE_GAMMA),
  *   FB_ECUDA. */
 fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t stream);
+
+/* Active-query subsets (SureLock page, "Principes de Fonctionnement", items 2
+ * and 3): with a->active set, only the n_active listed positions of the block
+ * query.  Their block-external part is recomputed on a full step (the cache
+ * rows of the other positions are left as they are), they attend to all Nb
+ * keys of the block (locked positions' K/V stay in K_in/V_in), and only their
+ * rows of O and LSE are written: a locked position keeps whatever the caller's
+ * O and LSE hold (its output of an earlier step).  Locking must be monotone
+ * within a block (a position locked once stays locked until
+ * fb_cache_begin_block), so every active position's cache row dates from the
+ * last full step; the library does not check this.  Requires FB_CACHE_ACTIVE,
+ * bf16 inputs, D = 128, Nb <= 64, no selection and no gamma gate
+ * (FB_EUNSUPPORTED otherwise).  A listed position outside [0, Nb) is skipped
+ * and reported as FB_EINVAL in the device status word. */
 
 /* Host-side decision of the last fb_step: *recomputed = 1 when the tau gate
  * (or an invalid cache) forced a full step. */

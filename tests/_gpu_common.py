@@ -80,24 +80,28 @@ class GpuSchedule:
         self.out_dtype = out_dtype
         self.layer = fb.FlashBlockLayer(self.q_like, self.kin_like, self.kp, self.o_like, max_prefix=s.lcap,
                                         gamma=s.gamma is not None, sparse=s.sel_k is not None,
-                                        max_sel_k=s.sel_k or 0)
+                                        max_sel_k=s.sel_k or 0, active=s.lock_rate is not None)
         self.gamma = (torch.full((s.Hq,), s.gamma, dtype=torch.float32, device="cuda")
                       if s.gamma is not None else None)
         self.tau = s.tau if s.tau is not None else fb.FB_TAU_OFF
 
     def run(self):
         s = self.spec
+        o = lse = None
         for st in self.w.schedule():
             if st.step == 0:
                 self.layer.begin_block()
             q, kin, vin = st.q.cuda(), st.kin.cuda(), st.vin.cuda()
             sel = cuda(st.sel)
-            o = torch.empty(s.B, s.Hq, s.Nb, s.D, dtype=self.out_dtype, device="cuda")
-            lse = torch.empty(s.B, s.Hq, s.Nb, dtype=torch.float32, device="cuda")
+            if st.active is None or st.step == 0:
+                o = torch.empty(s.B, s.Hq, s.Nb, s.D, dtype=self.out_dtype, device="cuda")
+                lse = torch.empty(s.B, s.Hq, s.Nb, dtype=torch.float32, device="cuda")
+            else:   # locked positions keep the previous step's rows: the same buffers, unwritten
+                o, lse = o.clone(), lse.clone()
             reuse = torch.full((s.B, s.Hq), -1, dtype=torch.int8, device="cuda")
             sim = torch.empty(s.B, s.Hq, dtype=torch.float32, device="cuda")
             self.layer.step(q, kin, vin, self.kp, self.vp, st.prefix_len, st.M, self.tau, o, lse,
-                            self.gamma, sel, reuse, sim)
+                            self.gamma, sel, reuse, sim, active=cuda(st.active))
             recomputed = self.layer.last_recomputed()
             torch.cuda.synchronize()
             yield st, o, lse, reuse.cpu(), sim.cpu(), recomputed
@@ -144,9 +148,12 @@ class OracleSchedule:
             if st.step == 0:
                 o.begin_block()
             sel = None if st.sel is None else self._slice(key, st.sel, True).numpy()
+            act = None
+            if st.active is not None:
+                act = st.active.numpy() if key is None else st.active.numpy()[key[0]:key[0] + 1]
             r = o.step(orc.to64(self._slice(key, st.q, True)), orc.to64(self._slice(key, st.kin, False)),
                        orc.to64(self._slice(key, st.vin, False)), self.kp[key], self.vp[key],
-                       st.prefix_len, st.M, s.tau, sel)
+                       st.prefix_len, st.M, s.tau, sel, act)
             out[key] = r
             if st.last_in_block:
                 self.kp[key], self.vp[key], _ = orc.kv_append(
@@ -169,8 +176,16 @@ def compare_schedule(spec, groups=None, out_dtype=torch.float32, check_every=1, 
     os_.init_prefix(kp, vp)
     stats = {"err_o": 0.0, "err_l": 0.0, "steps": 0, "recomputed": [], "sim_err": 0.0, "reuse": []}
     prev_sim = {}
+    prev_o = prev_l = None
     for st, o, lse, reuse, sim, recomputed in gs.run():
         ref = os_.step(st)
+        if st.active is not None and st.step > 0:
+            # locked positions: their rows of O and LSE were not written at all
+            for b in range(spec.B):
+                locked = np.setdiff1d(np.arange(spec.Nb), st.active[b].numpy())
+                assert torch.equal(o[b][:, locked], prev_o[b][:, locked]), f"step {st.step}: a locked row of O changed"
+                assert torch.equal(lse[b][:, locked], prev_l[b][:, locked]), f"step {st.step}: a locked LSE changed"
+        prev_o, prev_l = o, lse
         for key, r in ref.items():
             stats["recomputed"].append(recomputed)
             assert recomputed == r.recompute, f"step {st.block}.{st.step}: tau decision differs"
@@ -192,9 +207,21 @@ def compare_schedule(spec, groups=None, out_dtype=torch.float32, check_every=1, 
                 prev_sim[key] = r.sim.copy()
             assert np.array_equal(greuse, r.head_reuse), f"{what}: reuse mask differs"
             stats["reuse"].append(r.head_reuse.mean())
+            if st.active is not None:   # compare the active rows (locked rows: checked above)
+                b0 = 0 if key is None else key[0]
+                rows = st.active.numpy()[b0]
+                go, gl = go[:, :, rows], gl[:, :, rows]
+                ro, rl = r.o[:, :, rows], r.lse[:, :, rows]
+                if key is None and spec.B > 1:   # every batch element has its own positions
+                    go = torch.stack([o[b][:, st.active[b].numpy()] for b in range(spec.B)])
+                    gl = torch.stack([lse[b][:, st.active[b].numpy()] for b in range(spec.B)])
+                    ro = np.stack([r.o[b][:, st.active[b].numpy()] for b in range(spec.B)])
+                    rl = np.stack([r.lse[b][:, st.active[b].numpy()] for b in range(spec.B)])
+            else:
+                ro, rl = r.o, r.lse
             if st.step % check_every == 0 or st.step == spec.steps - 1:
-                stats["err_o"] = max(stats["err_o"], assert_o_close(go, r.o, tol, what))
-                stats["err_l"] = max(stats["err_l"], assert_lse_close(gl, r.lse, tol, what))
+                stats["err_o"] = max(stats["err_o"], assert_o_close(go, ro, tol, what))
+                stats["err_l"] = max(stats["err_l"], assert_lse_close(gl, rl, tol, what))
         stats["steps"] += 1
     gs.close()
     if report is not None:

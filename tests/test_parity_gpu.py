@@ -208,7 +208,8 @@ def _random_parts(B, Hq, Nb, D, n, seed, empty_rows=True):
 @pytest.mark.parametrize("shape", [(1, 32, 8, 128, 32, "bf16"), (1, 4, 4, 64, 32, "f32"),
                                    (1, 3, 3, 128, 150, "bf16"), (2, 8, 4, 64, 5, "bf16"),
                                    (2, 8, 2, 128, 5, "bf16"), (1, 8, 2, 128, 64, "bf16"),
-                                   (3, 4, 4, 128, 16, "bf16"), (1, 2, 1, 128, 1, "bf16")],
+                                   (3, 4, 4, 128, 16, "bf16"), (1, 2, 1, 128, 1, "bf16"),
+                                   (1, 4, 2, 128, 1560, "bf16"), (1, 3, 3, 128, 1000, "bf16")],
                          ids=lambda s: "x".join(map(str, s)))
 def test_inblock_merge(shape, nparts):
     B, Hq, Hkv, D, Nb, dt = shape
@@ -276,6 +277,11 @@ SCHEDULES = {
     "nb1_gqa": dict(base="dllm_8k", Nb=1, prefix0=300, steps=3, m_model=("uniform", 0, 1), tau=1),
     "nb4_small": dict(base="dllm_8k_nb4", prefix0=1000, blocks=2),
     "sparse_d40_small": dict(base="sparse_32k_d40", prefix0=3000, sel_k=1200, Hq=8, Hkv=2),
+    # active-query subsets: a quarter of the active positions lock per step
+    "lock_small": dict(base="dllm_8k_lock", prefix0=1000, blocks=2),
+    "lock_b2_nb64": dict(base="dllm_8k_lock", B=2, Nb=64, prefix0=700, blocks=1, steps=6, lock_rate=0.3,
+                         m_model=("binomial", 64, 0.1), tau=6),
+    "lock_tau_zero": dict(base="dllm_8k_lock", prefix0=1500, blocks=1, steps=6, tau=0),
 }
 
 
@@ -318,6 +324,7 @@ def test_full_dllm_8k_all_heads():
     ("sparse_32k_d40", [(0, 0), (0, 6)]),
     ("video_1560", [(0, 0), (0, 13), (0, 23)]),
     ("sparse_32k_k2048", [(0, 0), (0, 5)]),
+    ("dllm_8k_lock", [(0, 0), (0, 3)]),
 ])
 def test_full_size_sampled_heads(name, groups):
     """Full-size workloads; the oracle recomputes only the sampled (b, kv-head) groups."""
