@@ -532,6 +532,50 @@ fb_status fb_attn_outblock(const fb_attn_desc* d, const void* q, const void* kp,
   return merge_to_part(*d, lst, a_res, l_res, nullptr, 0, stream);
 }
 
+fb_status fb_select_workspace_bytes(const fb_attn_desc* d, int64_t prefix_len, size_t* bytes) {
+  fb_status st = check_desc(d);
+  if (st != FB_OK) return st;
+  if (!bytes || prefix_len < 0) return FB_EINVAL;
+  size_t ob = 0;
+  if ((st = fb_outblock_workspace_bytes(d, prefix_len, 0, &ob)) != FB_OK) return st;
+  *bytes = align256(ob) + align256((size_t)rows_of(*d) * d->D * 4) + align256((size_t)rows_of(*d) * 4) +
+           align256((size_t)d->B * d->Hq * prefix_len * 4);
+  return FB_OK;
+}
+
+fb_status fb_select_mass(const fb_attn_desc* d, const void* q, const void* kp, const void* vp, int64_t prefix_len,
+                         int32_t k, int32_t* sel_out, float* mass_out, void* ws, size_t ws_bytes,
+                         cudaStream_t stream) {
+  fb_status st = check_desc(d);
+  if (st != FB_OK) return st;
+  if (!q || !kp || !vp || !sel_out) return FB_EINVAL;
+  if (prefix_len < 1 || prefix_len > d->kp_capacity || k < 0 || k > prefix_len) return FB_EINVAL;
+  if (!mass_applies(*d)) return FB_EUNSUPPORTED;
+  if (!al16(q) || !al16(kp) || !al16(vp) || !al16(sel_out) || !al16(mass_out) || !al16(ws)) return FB_EALIGN;
+  size_t need = 0, ob = 0;
+  if ((st = fb_select_workspace_bytes(d, prefix_len, &need)) != FB_OK) return st;
+  if ((st = fb_outblock_workspace_bytes(d, prefix_len, 0, &ob)) != FB_OK) return st;
+  if (!ws || ws_bytes < need) return FB_ENOSPACE;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  float* A = reinterpret_cast<float*>(w + align256(ob));
+  float* L = reinterpret_cast<float*>(w + align256(ob) + align256((size_t)rows_of(*d) * d->D * 4));
+  float* mass = mass_out ? mass_out
+                         : reinterpret_cast<float*>(w + align256(ob) + align256((size_t)rows_of(*d) * d->D * 4) +
+                                                    align256((size_t)rows_of(*d) * 4));
+  // L_out of every block query over the prefix, then each key's mass, then the top k
+  if ((st = fb_attn_outblock(d, q, kp, vp, prefix_len, nullptr, 0, A, L, nullptr, nullptr, ws, ob, stream)) !=
+      FB_OK)
+    return st;
+  {
+    ProfScope prof(kProfAux, (double)d->B * d->Hkv * prefix_len * d->D * 2 + (double)rows_of(*d) * d->D * 2 +
+                                 (double)d->B * d->Hq * prefix_len * 4,
+                   stream);
+    if (launch_mass(*d, q, kp, prefix_len, L, mass, scale_log2(*d), stream) != cudaSuccess) return FB_ECUDA;
+  }
+  ProfScope prof(kProfAux, (double)d->B * d->Hq * prefix_len * 4 * 5, stream);
+  return launch_topk(mass, d->B * d->Hq, prefix_len, k, sel_out, stream) == cudaSuccess ? FB_OK : FB_ECUDA;
+}
+
 static fb_status check_parts(int32_t nparts, const float* const* a, const float* const* l, int32_t maxn) {
   if (nparts < 0 || nparts > maxn) return FB_EINVAL;
   if (nparts > 0 && (!a || !l)) return FB_EINVAL;

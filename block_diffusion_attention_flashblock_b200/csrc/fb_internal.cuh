@@ -169,6 +169,12 @@ cudaError_t launch_attn_pair(const fb_attn_desc& d, const TcMaps& m, const PairP
                              const int8_t* mask, int mask_active, float scale_log2, float* pa, float* pl,
                              float* dst_a, float* dst_l, int32_t* nslots, cudaStream_t s, bool merge_only);
 
+// Selection by attention mass (fb_select.cu).
+bool mass_applies(const fb_attn_desc& d);
+cudaError_t launch_mass(const fb_attn_desc& d, const void* q, const void* kp, int64_t nkeys, const float* l_out,
+                        float* mass, float scale_log2, cudaStream_t s);
+cudaError_t launch_topk(const float* mass, int32_t BH, int64_t n, int32_t k, int32_t* sel, cudaStream_t s);
+
 // Small-block in-block attention + merge (fb_inblock.cu).
 bool inblock_small_applies(const fb_attn_desc& d, int next);
 // With `active` ([B, n_act] block positions) only those queries are computed

@@ -61,6 +61,8 @@ _SIGS = {
                                    C.c_size_t, _P]),
     "fb_attn_outblock_noalloc": (C.c_int, [_P, _P, _P, _P, C.c_int64, _P, _P, _P]),
     "fb_attn_inblock": (C.c_int, [_P, _P, _P, _P, C.c_int32, _P, _P, _P, _P, _P]),
+    "fb_select_workspace_bytes": (C.c_int, [_P, C.c_int64, C.POINTER(C.c_size_t)]),
+    "fb_select_mass": (C.c_int, [_P, _P, _P, _P, C.c_int64, C.c_int32, _P, _P, _P, C.c_size_t, _P]),
     "fb_merge": (C.c_int, [_P, C.c_int32, _P, _P, _P, _P, _P]),
     "fb_kv_append": (C.c_int, [_P, _P, _P, C.c_int64, _P, _P, _P]),
     "fb_cache_workspace_bytes": (C.c_int, [_P, C.c_int32, C.c_int64, C.c_int32, C.POINTER(C.c_size_t)]),
@@ -195,6 +197,19 @@ def fb_attn_outblock_noalloc(desc, q, kp, vp, prefix_len, a_out, l_out, stream=N
     _check(lib().fb_attn_outblock_noalloc(C.byref(desc), _ptr(q), _ptr(kp), _ptr(vp), prefix_len,
                                           _ptr(a_out), _ptr(l_out), _stream(stream)),
            "fb_attn_outblock_noalloc")
+
+
+def fb_select_workspace_bytes(desc, prefix_len: int) -> int:
+    n = C.c_size_t(0)
+    _check(lib().fb_select_workspace_bytes(C.byref(desc), prefix_len, C.byref(n)), "fb_select_workspace_bytes")
+    return n.value
+
+
+def fb_select_mass(desc, q, kp, vp, prefix_len, k, sel_out, ws, mass_out=None, stream=None):
+    """Top-k prefix keys per (b, query head) by attention mass into sel_out [B, Hq, k]."""
+    _check(lib().fb_select_mass(C.byref(desc), _ptr(q), _ptr(kp), _ptr(vp), prefix_len, k, _ptr(sel_out),
+                                _ptr(mass_out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "fb_select_mass")
 
 
 def fb_attn_inblock(desc, q, kin, vin, o, lse=None, a_parts=(), l_parts=(), stream=None):

@@ -59,6 +59,9 @@ class WorkloadSpec:
     sel_k: Optional[int] = None               # sparse: keys kept per query head
     lock_rate: Optional[float] = None         # active-query subsets: share of the still-active
                                               # positions that lock at each step (None: all active)
+    select: str = "score"                     # sparse: "score" (seeded scores, drawn here) or "mass"
+                                              # (top-k attention mass of the block's first queries,
+                                              # computed by the caller at each block's step 0)
     seed: int = 2026_0000
     sigma_redraws: Tuple[Tuple[int, int], ...] = field(default=())
     """(block, head) pairs whose sigma is redrawn from the next sub-seed, to keep
@@ -96,6 +99,14 @@ SPECS = {
         name="dllm_64k_b4", B=4, Hq=32, Hkv=8, D=128, prefix0=65536, Nb=64,
         steps=16, blocks=1, dtype="bf16", std=0.5,
         m_model=("binomial", 64, 0.1), pert_std=0.05, tau=16, seed=2026_0002),
+    # the sparse layer with its keys chosen by attention mass (NEXT-3): the
+    # top 2048 prefix keys per head by the mass the block's first queries put
+    # on them, computed at each block's start
+    "sparse_32k_mass": WorkloadSpec(
+        name="sparse_32k_mass", B=1, Hq=32, Hkv=8, D=128, prefix0=32768,
+        Nb=32, steps=8, blocks=1, dtype="bf16", std=0.5,
+        m_model=("binomial", 32, 0.15), pert_std=0.05, tau=8, sel_k=2048, select="mass",
+        seed=2026_0080),
     # context-length sweep of the long-context shape at B = 1 (the pages'
     # latency-growth claim, 100k to 800k tokens of context)
     **{f"dllm_ctx_{n // 1000}k": WorkloadSpec(
@@ -296,7 +307,7 @@ class Workload:
         s = self.spec
         for blk in range(s.blocks):
             plen = s.prefix0 + blk * s.Nb
-            sel = self.selection(blk, plen) if s.sel_k else None
+            sel = self.selection(blk, plen) if s.sel_k and s.select == "score" else None
             q, kin, vin = self.block_start(blk)
             active = None
             for st in range(s.steps):

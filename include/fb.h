@@ -138,6 +138,32 @@ fb_status fb_attn_outblock_noalloc(const fb_attn_desc* d, const void* q, const v
                                    float* a_out, float* l_out, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Selection of the sparse keys by attention mass (summary, "Stratégies de
+ * Réutilisation Adaptatives", sparse bullet: FlashBlock caches the residual of
+ * the keys a sparse method leaves out; "Résultats Expérimentaux": SparseD at
+ * 20-40 % density).  The pages do not give the sparse method's rule; this
+ * call keeps, per (b, query head), the k prefix keys of largest
+ *     mass_j = sum_i exp(scale q_i . k_j - L_out,i)
+ * (the softmax probability over the prefix that key j receives from the
+ * block's queries, summed over them), ties to the lower index.  Call it once
+ * per block with the block's first queries and pass sel_out to that block's
+ * fb_step calls.
+ * sel_out: device int32 [B, Hq, k], written ascending.  mass_out: optional
+ *   device fp32 [B, Hq, prefix_len] that receives the masses (else they stay
+ *   in the workspace).  ws: at least fb_select_workspace_bytes() bytes.
+ * Requires bf16 inputs, D = 128, Nb in {16, 32} and (Hq / Hkv) * Nb <= 128
+ * (FB_EUNSUPPORTED otherwise).  The masses are fp32 sums in a fixed order, so
+ * a selection is the same on every run; near-tied keys at the k-th place may
+ * rank differently from an exact computation.
+ * Errors: FB_EINVAL (k outside [0, prefix_len], prefix_len < 1), FB_EALIGN,
+ *   FB_EUNSUPPORTED, FB_ENOSPACE, FB_ECUDA.
+ * ------------------------------------------------------------------------- */
+fb_status fb_select_workspace_bytes(const fb_attn_desc* d, int64_t prefix_len, size_t* bytes);
+fb_status fb_select_mass(const fb_attn_desc* d, const void* q, const void* kp, const void* vp, int64_t prefix_len,
+                         int32_t k, int32_t* sel_out, float* mass_out, void* ws, size_t ws_bytes,
+                         cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Block-internal attention fused with the log-space merge (summary,
  * "Mécanisme Central": A_in over J_in, merged with the block-external parts).
  *

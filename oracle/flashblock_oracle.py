@@ -30,6 +30,9 @@ What the pages define, and how it is written here
 * Sparse attention compatibility: the keys a sparse method did not select
   are treated as the block-external set and their residual contribution is
   cached (same section, third bullet).  ``outblock_selected``.
+* Selection of the sparse keys by attention mass (same section, sparse bullet,
+  and "Résultats Expérimentaux", SparseD bullet; the rule is a reading):
+  ``attention_mass``, ``select_top_k``.
 * Active-query subsets (SureLock page, "Principes de Fonctionnement", items 2
   and 3): only the M_t still-unlocked positions of the block query, over the
   cached K/V of every token; a locked position keeps its output.  Combined
@@ -166,6 +169,41 @@ def outblock_selected(Q, Kp, Vp, prefix_len: int, scale: float, sel, residual: b
             K = Kp[b, g, :prefix_len]; V = Vp[b, g, :prefix_len]
             A[b, h], L[b, h] = attention_part(Q[b, h], K[keep], V[keep], scale)
     return A, L
+
+
+def attention_mass(Q, Kp, prefix_len: int, scale: float):
+    """Attention mass of each prefix key per (b, query head): the sum over the
+    block's queries of the key's softmax probability over the prefix,
+        mass[b, h, j] = sum_i exp(s_ij - L_out,i),  s_ij = scale * q_i . k_j,
+    with L_out,i = log sum_j exp(s_ij) over the prefix.  Each query's
+    probabilities sum to 1, so a head's masses sum to Nb.  This is the score by
+    which the sparse selection keeps keys (the pages name a sparse method,
+    SparseD, without its rule; the top-k by mass is the reading taken).
+    Returns [B, Hq, prefix_len]."""
+    B, Hq, Nb, D = Q.shape
+    Hkv = Kp.shape[1]
+    out = np.zeros((B, Hq, prefix_len))
+    for b in range(B):
+        for h in range(Hq):
+            g = kv_head(h, Hq, Hkv)
+            s = scale * (np.asarray(Q[b, h], dtype=np.float64) @ np.asarray(Kp[b, g, :prefix_len], dtype=np.float64).T)
+            mx = s.max(axis=1, keepdims=True)
+            L = mx + np.log(np.exp(s - mx).sum(axis=1, keepdims=True))
+            out[b, h] = np.exp(s - L).sum(axis=0)
+    return out
+
+
+def select_top_k(mass, k: int):
+    """Per (b, h): the k keys of largest mass, ties to the lower index, as
+    ascending int32 positions [B, Hq, k]."""
+    B, Hq, n = mass.shape
+    k = min(k, n)
+    out = np.empty((B, Hq, k), dtype=np.int32)
+    for b in range(B):
+        for h in range(Hq):
+            order = sorted(range(n), key=lambda j: (-mass[b, h, j], j))[:k]
+            out[b, h] = np.sort(np.asarray(order, dtype=np.int64))
+    return out
 
 
 def full_attention(Q, Kin, Vin, Kp, Vp, prefix_len: int, scale: float):

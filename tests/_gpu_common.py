@@ -85,14 +85,30 @@ class GpuSchedule:
                       if s.gamma is not None else None)
         self.tau = s.tau if s.tau is not None else fb.FB_TAU_OFF
 
+    def select_mass(self, q, prefix_len):
+        """The block's selection by attention mass (fb_select_mass) and the masses."""
+        s = self.spec
+        k = min(s.sel_k, prefix_len)
+        sel = torch.empty(s.B, s.Hq, k, dtype=torch.int32, device="cuda")
+        mass = torch.empty(s.B, s.Hq, prefix_len, dtype=torch.float32, device="cuda")
+        ws = torch.empty(fb.fb_select_workspace_bytes(self.layer.desc, prefix_len), dtype=torch.uint8, device="cuda")
+        fb.fb_select_mass(self.layer.desc, q, self.kp, self.vp, prefix_len, k, sel, ws, mass_out=mass)
+        return sel, mass
+
     def run(self):
         s = self.spec
         o = lse = None
+        block_sel = None
         for st in self.w.schedule():
             if st.step == 0:
                 self.layer.begin_block()
             q, kin, vin = st.q.cuda(), st.kin.cuda(), st.vin.cuda()
             sel = cuda(st.sel)
+            if s.sel_k and s.select == "mass":
+                if st.step == 0:
+                    block_sel, self.last_mass = self.select_mass(q, st.prefix_len)
+                sel = block_sel
+                st.sel = block_sel.cpu()   # the oracle steps over the same selection
             if st.active is None or st.step == 0:
                 o = torch.empty(s.B, s.Hq, s.Nb, s.D, dtype=self.out_dtype, device="cuda")
                 lse = torch.empty(s.B, s.Hq, s.Nb, dtype=torch.float32, device="cuda")
@@ -166,6 +182,43 @@ class OracleSchedule:
         return self._slice(key, t, True)
 
 
+MASS_TOL = 2e-5   # fp32 mass vs fp64, relative to the head's largest mass
+
+
+def check_mass_selection(spec, st, gpu_mass, os_):
+    """fb_select_mass against the oracle on the sampled groups: the masses
+    within MASS_TOL; the selection equal to the oracle's top-k on every key
+    whose oracle mass lies outside MASS_TOL of the k-th largest (near-ties at
+    the boundary may rank either way in fp32), and a valid top-k on the rest."""
+    sel = st.sel.numpy()
+    for key in os_.oracles:
+        b0, b1, h0, h1 = (0, spec.B, 0, spec.Hq) if key is None else (
+            key[0], key[0] + 1, key[1] * spec.G, (key[1] + 1) * spec.G)
+        kp = os_.kp[key]
+        q64 = orc.to64(st.q[b0:b1, h0:h1])
+        M = orc.attention_mass(q64, kp, st.prefix_len, 1 / math.sqrt(spec.D))
+        gm = gpu_mass[b0:b1, h0:h1].double().cpu().numpy()
+        scale = M.max(axis=2, keepdims=True)
+        err = float(np.max(np.abs(gm - M) / scale))
+        assert err <= MASS_TOL, f"mass rel err {err:.3g}"
+        k = sel.shape[-1]
+        ref = orc.select_top_k(M, k)
+        for b in range(b1 - b0):
+            for h in range(h1 - h0):
+                g_sel = sel[b0 + b, h0 + h]
+                assert len(g_sel) == k and np.all(np.diff(g_sel) > 0), "selection not ascending and distinct"
+                if k == 0:
+                    continue
+                m = M[b, h]
+                kth = np.sort(m)[::-1][k - 1]
+                band = MASS_TOL * m.max()
+                sure_in = np.flatnonzero(m > kth + band)
+                sure_out = np.flatnonzero(m < kth - band)
+                assert np.isin(sure_in, g_sel).all(), "a key well above the k-th mass is not selected"
+                assert not np.isin(sure_out, g_sel).any(), "a key well below the k-th mass is selected"
+                assert np.isin(sure_in, ref[b, h]).all() and not np.isin(sure_out, ref[b, h]).any()
+
+
 def compare_schedule(spec, groups=None, out_dtype=torch.float32, check_every=1, report=None):
     """Run GPU and oracle side by side; assert parity on every step; return stats."""
     tol = TOL[spec.dtype]
@@ -178,6 +231,8 @@ def compare_schedule(spec, groups=None, out_dtype=torch.float32, check_every=1, 
     prev_sim = {}
     prev_o = prev_l = None
     for st, o, lse, reuse, sim, recomputed in gs.run():
+        if spec.sel_k and spec.select == "mass" and st.step == 0:
+            check_mass_selection(spec, st, gs.last_mass, os_)
         ref = os_.step(st)
         if st.active is not None and st.step > 0:
             # locked positions: their rows of O and LSE were not written at all

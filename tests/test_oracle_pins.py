@@ -401,6 +401,42 @@ def test_active_sets_only_shrink():
                None, active=steps[0].active.numpy())
 
 
+# ------------------------------------------------ selection by attention mass ---
+def test_attention_mass_sums_to_the_block_length_and_matches_brute_force():
+    """Each query's probabilities over the prefix sum to 1, so a head's masses
+    sum to Nb; on a tiny case every mass equals a 40-digit Decimal sum."""
+    g = np.random.default_rng(3)
+    Q = g.standard_normal((1, 2, 3, 4)); K = g.standard_normal((1, 1, 5, 4))
+    M = orc.attention_mass(Q, K, 5, 0.7)
+    np.testing.assert_allclose(M.sum(axis=2), 3.0, rtol=1e-14)
+    decimal.getcontext().prec = 40
+    for h in range(2):
+        for j in range(5):
+            tot = decimal.Decimal(0)
+            for i in range(3):
+                e = [(decimal.Decimal(0.7) * sum(decimal.Decimal(Q[0, h, i, d]) * decimal.Decimal(K[0, 0, jj, d])
+                                                  for d in range(4))).exp() for jj in range(5)]
+                tot += e[j] / sum(e)
+            assert abs(float(tot) - M[0, h, j]) < 1e-14
+
+
+def test_top_k_by_mass_closed_forms():
+    # zero queries: every key gets mass Nb / n, all tied -> the first k keys
+    Q = np.zeros((1, 1, 4, 8)); K = np.random.default_rng(4).standard_normal((1, 1, 10, 8))
+    M = orc.attention_mass(Q, K, 10, 0.3)
+    np.testing.assert_allclose(M, 0.4, rtol=1e-14)
+    assert orc.select_top_k(M, 3).tolist() == [[[0, 1, 2]]]
+    # a hand-worked ranking with a tie at the boundary: the lower index wins
+    m = np.array([[[0.1, 0.5, 0.3, 0.5, 0.2, 0.3]]])
+    assert orc.select_top_k(m, 3).tolist() == [[[1, 2, 3]]]
+    assert orc.select_top_k(m, 4).tolist() == [[[1, 2, 3, 5]]]
+    assert orc.select_top_k(m, 6).tolist() == [[[0, 1, 2, 3, 4, 5]]]
+    # one dominant key per head (a key equal to a scaled query) ranks first
+    K2 = np.zeros((1, 1, 6, 2)); K2[0, 0, 4] = [5.0, 0.0]
+    Q2 = np.array([[[[1.0, 0.0]]]])
+    assert orc.select_top_k(orc.attention_mass(Q2, K2, 6, 1.0), 1).tolist() == [[[4]]]
+
+
 def test_static_queries_reuse_equals_full():
     """Queries unchanged across steps: the cached A_out is exact, so every step equals full attention."""
     spec, work = _tiny(steps=4)

@@ -277,6 +277,10 @@ SCHEDULES = {
     "nb1_gqa": dict(base="dllm_8k", Nb=1, prefix0=300, steps=3, m_model=("uniform", 0, 1), tau=1),
     "nb4_small": dict(base="dllm_8k_nb4", prefix0=1000, blocks=2),
     "sparse_d40_small": dict(base="sparse_32k_d40", prefix0=3000, sel_k=1200, Hq=8, Hkv=2),
+    # the sparse keys chosen by attention mass at each block's start
+    "mass_small": dict(base="sparse_32k_mass", prefix0=4000, sel_k=256, Hq=8, Hkv=2, blocks=2),
+    "mass_nb16_b2": dict(base="sparse_32k_mass", B=2, Nb=16, prefix0=2500, sel_k=700, Hq=16, Hkv=2, steps=5,
+                         m_model=("binomial", 16, 0.15), tau=4),
     # active-query subsets: a quarter of the active positions lock per step
     "lock_small": dict(base="dllm_8k_lock", prefix0=1000, blocks=2),
     "lock_b2_nb64": dict(base="dllm_8k_lock", B=2, Nb=64, prefix0=700, blocks=1, steps=6, lock_rate=0.3,
@@ -325,6 +329,7 @@ def test_full_dllm_8k_all_heads():
     ("video_1560", [(0, 0), (0, 13), (0, 23)]),
     ("sparse_32k_k2048", [(0, 0), (0, 5)]),
     ("dllm_8k_lock", [(0, 0), (0, 3)]),
+    ("sparse_32k_mass", [(0, 0), (0, 6)]),
 ])
 def test_full_size_sampled_heads(name, groups):
     """Full-size workloads; the oracle recomputes only the sampled (b, kv-head) groups."""
@@ -357,3 +362,53 @@ def test_step_changed_prefix_recomputes(sparse):
         assert_lse_close(lse, r.lse, TOL["bf16"], f"prefix {plen}")
     layer.close()
     assert fb.fb_get_device_status() == fb.FB_OK
+
+
+@pytest.mark.parametrize("k", [0, 1, 50, 640])
+def test_select_mass_all_tied_takes_the_first_keys(k):
+    """Zero queries give every key the same mass bit for bit (each query's
+    probabilities are all 2^-log2(n)), so the top k are the first k keys."""
+    B, Hq, Hkv, D, Nb, Lp = 1, 8, 2, 128, 32, 640
+    q = torch.zeros(B, Hq, Nb, D, dtype=torch.bfloat16, device="cuda")
+    kp = wl.tensor((B, Hkv, Lp, D), 81, 1.0, "bf16").cuda()
+    vp = wl.tensor((B, Hkv, Lp, D), 82, 1.0, "bf16").cuda()
+    o = torch.empty(B, Hq, Nb, D, device="cuda")
+    desc = fb.make_desc(q, kp[:, :, :Nb], kp, o)
+    sel = torch.full((B, Hq, k), -1, dtype=torch.int32, device="cuda")
+    mass = torch.empty(B, Hq, Lp, device="cuda")
+    ws = torch.empty(fb.fb_select_workspace_bytes(desc, Lp), dtype=torch.uint8, device="cuda")
+    fb.fb_select_mass(desc, q, kp, vp, Lp, k, sel, ws, mass_out=mass)
+    assert fb.fb_get_device_status() == fb.FB_OK
+    assert torch.all(mass == mass[0, 0, 0])
+    assert abs(float(mass[0, 0, 0]) - Nb / Lp) < 1e-6 * Nb / Lp * 10
+    assert torch.equal(sel.cpu(), torch.arange(k, dtype=torch.int32).expand(B, Hq, k))
+
+
+@pytest.mark.parametrize("shape", [(1, 8, 2, 128, 32, 3000, 300), (2, 32, 8, 128, 16, 4100, 4100),
+                                   (1, 4, 4, 128, 32, 129, 7)], ids=lambda s: "x".join(map(str, s)))
+def test_select_mass_against_the_oracle(shape):
+    """fb_select_mass: masses within 2e-5 of the fp64 oracle's, and the top-k
+    equal to the oracle's outside the near-tie band at the k-th mass."""
+    from _gpu_common import MASS_TOL
+    B, Hq, Hkv, D, Nb, Lp, k = shape
+    q, kin, vin, kp, vp = _mk(B, Hq, Hkv, D, Nb, Lp, "bf16", seed=91, std=0.5)
+    qd, kpd, vpd = q.cuda(), kp.cuda(), vp.cuda()
+    o = torch.empty(B, Hq, Nb, D, device="cuda")
+    desc = fb.make_desc(qd, kin.cuda(), kpd, o)
+    sel = torch.empty(B, Hq, k, dtype=torch.int32, device="cuda")
+    mass = torch.empty(B, Hq, Lp, device="cuda")
+    ws = torch.empty(fb.fb_select_workspace_bytes(desc, Lp), dtype=torch.uint8, device="cuda")
+    fb.fb_select_mass(desc, qd, kpd, vpd, Lp, k, sel, ws, mass_out=mass)
+    assert fb.fb_get_device_status() == fb.FB_OK
+    M = orc.attention_mass(orc.to64(q), orc.to64(kp), Lp, 1 / np.sqrt(D))
+    gm = mass.double().cpu().numpy()
+    assert np.max(np.abs(gm - M) / M.max(axis=2, keepdims=True)) <= MASS_TOL
+    g_sel = sel.cpu().numpy()
+    for b in range(B):
+        for h in range(Hq):
+            m = M[b, h]
+            kth = np.sort(m)[::-1][k - 1]
+            band = MASS_TOL * m.max()
+            assert np.all(np.diff(g_sel[b, h]) > 0)
+            assert np.isin(np.flatnonzero(m > kth + band), g_sel[b, h]).all()
+            assert not np.isin(np.flatnonzero(m < kth - band), g_sel[b, h]).any()
