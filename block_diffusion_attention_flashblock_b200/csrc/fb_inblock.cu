@@ -105,6 +105,11 @@ __device__ __forceinline__ bool wait_loaded(uint32_t bar, const InblockArgs& a, 
   return true;
 }
 
+// Whether the output and cache staging rows fit in the K/V staging of NB keys.
+__host__ __device__ constexpr bool inblock_stage_aliases(int NB) {
+  return 2 * NB * kRowE * 2 >= 2 * kRows * kExtStride * 4;
+}
+
 template <int NB, int NX>
 __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a) {
   ptx::pdl_prologue();
@@ -117,9 +122,14 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   __nv_bfloat16* sV = sK + NB * kRowE;                                   // [NB][kRowE]
   float* sE = reinterpret_cast<float*>(sV + NB * kRowE);                 // [NX][16][kExtStride]
   float* sL = sE + NXS * kRows * kExtStride;                             // [NX][16]
-  float* sO = sL + NXS * kRows;                                          // [16][kExtStride] output rows
+  // Output and cache rows are staged after P V; with blocks of 32 keys or
+  // more they fit in the K/V staging, which is dead by then (a CTA barrier
+  // separates the last read of K/V from the first staged row), so more CTAs
+  // fit per SM.
+  constexpr bool kAlias = inblock_stage_aliases(NB);
+  float* sO = kAlias ? reinterpret_cast<float*>(sK) : sL + NXS * kRows;  // [16][kExtStride] output rows
   float* sC = sO + kRows * kExtStride;                                   // [16][kExtStride] cache rows
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + kRows * kExtStride);  // Q+K, V, parts, (test) stall
+  uint64_t* bars = reinterpret_cast<uint64_t*>(kAlias ? sL + NXS * kRows : sC + kRows * kExtStride);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int unit = blockIdx.x / a.tiles_per_unit, tile = blockIdx.x % a.tiles_per_unit;
@@ -396,7 +406,7 @@ cudaError_t launch_inblock_small(const fb_attn_desc& d, const void* q, const voi
   const int NB = d.Nb <= 16 ? 16 : d.Nb <= 32 ? 32 : 64;
   const int nxs = next > 0 ? next : 1;
   const size_t smem = (size_t)(kRows + 2 * NB) * kRowE * 2 + (size_t)nxs * kRows * (kExtStride + 1) * 4 +
-                      2 * (size_t)kRows * kExtStride * 4 + 4 * 8;
+                      (inblock_stage_aliases(NB) ? 0 : 2 * (size_t)kRows * kExtStride * 4) + 4 * 8;
   const dim3 grid(d.B * d.Hkv * a.tiles_per_unit);
   // instances above the default 48 KB of dynamic shared memory opt in once
   static bool opted[kMaxDevices][3][kMaxExt + 1] = {};   // the attribute is per device
