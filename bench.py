@@ -165,10 +165,19 @@ class Layers:
                      o=torch.empty(spec.B, spec.Hq, spec.Nb, spec.D, dtype=dt, device=device),
                      lse=torch.empty(spec.B, spec.Hq, spec.Nb, dtype=torch.float32, device=device),
                      x=[dict(q=st.q.to(device), kin=st.kin.to(device), vin=st.vin.to(device),
-                             sel=None if st.sel is None else st.sel.to(device)) for st in self.steps])
+                             sel=None if st.sel is None else st.sel.to(device),
+                             active=None if st.active is None else st.active.to(device)) for st in self.steps])
             d["layer"] = fb.FlashBlockLayer(d["x"][0]["q"], d["x"][0]["kin"], d["kp"], d["o"],
                                             max_prefix=spec.lcap, gamma=spec.gamma is not None,
-                                            sparse=spec.sel_k is not None, max_sel_k=spec.sel_k or 0)
+                                            sparse=spec.sel_k is not None, max_sel_k=spec.sel_k or 0,
+                                            active=spec.lock_rate is not None)
+            if spec.sel_k and spec.select == "mass":
+                # the block's selection by attention mass, made at its step 0
+                d["mass_sel"] = torch.empty(spec.B, spec.Hq, spec.sel_k, dtype=torch.int32, device=device)
+                d["mass_ws"] = torch.empty(fb.fb_select_workspace_bytes(d["layer"].desc, spec.lcap),
+                                           dtype=torch.uint8, device=device)
+                for x in d["x"]:
+                    x["sel"] = d["mass_sel"]
             self.L.append(d)
         self.host = [dict(q=st.q.pin_memory(), kin=st.kin.pin_memory(), vin=st.vin.pin_memory()) for st in self.steps]
         self.query_tokens = spec.B * spec.Nb * len(self.steps) * nl   # layer-steps x B x Nb
@@ -223,8 +232,11 @@ def measure_workload(args, spec, rank, world, device, headline):
                     x["q"].copy_(h["q"], non_blocking=True)
                     x["kin"].copy_(h["kin"], non_blocking=True)
                     x["vin"].copy_(h["vin"], non_blocking=True)
+                if st.step == 0 and "mass_sel" in d:
+                    fb.fb_select_mass(d["layer"].desc, x["q"], d["kp"], d["vp"], st.prefix_len, s.sel_k,
+                                      d["mass_sel"], d["mass_ws"])
                 d["layer"].step(x["q"], x["kin"], x["vin"], d["kp"], d["vp"], st.prefix_len, st.M, tau, d["o"],
-                                d["lse"], gamma, x["sel"])
+                                d["lse"], gamma, x["sel"], active=x["active"])
                 if st.last_in_block:
                     fb.fb_kv_append(d["layer"].desc, d["kp"], d["vp"], st.prefix_len, x["kin"], x["vin"])
                 if e2e:
@@ -319,14 +331,17 @@ def measure_workload(args, spec, rank, world, device, headline):
     for d in S.L:
         x = d["x"][0]
         d["layer"].begin_block()
+        if "mass_sel" in d:
+            fb.fb_select_mass(d["layer"].desc, x["q"], d["kp"], d["vp"], S.steps[0].prefix_len, s.sel_k,
+                              d["mass_sel"], d["mass_ws"])
         d["layer"].step(x["q"], x["kin"], x["vin"], d["kp"], d["vp"], S.steps[0].prefix_len, 0, 0, d["o"], d["lse"],
-                        gamma, x["sel"])
+                        gamma, x["sel"], active=x["active"])
 
     def reuse_round():
         for d in S.L:
             x = d["x"][1 if len(S.steps) > 1 else 0]
             d["layer"].step(x["q"], x["kin"], x["vin"], d["kp"], d["vp"], st1.prefix_len, 0, tau_on, d["o"],
-                            d["lse"], gamma, x["sel"])
+                            d["lse"], gamma, x["sel"], active=x["active"])
 
     g_reuse, _ = graph_of(lambda: [reuse_round() for _ in range(R)])
     reuse_recomputed = S.L[0]["layer"].last_recomputed()
@@ -520,11 +535,14 @@ def kernels_only(spec, device, n):
     gamma = torch.full((spec.Hq,), spec.gamma, device=device) if spec.gamma is not None else None
     st0 = S.steps[0]
     x = d["x"][0]
+    if "mass_sel" in d:
+        fb.fb_select_mass(d["layer"].desc, x["q"], d["kp"], d["vp"], st0.prefix_len, spec.sel_k, d["mass_sel"],
+                          d["mass_ws"])
     for tau in (0, fb.FB_TAU_OFF):   # every step recomputes; then every step reuses the cache
         for _ in range(n):
             flush.zero_()
             d["layer"].step(x["q"], x["kin"], x["vin"], d["kp"], d["vp"], st0.prefix_len, 0, tau, d["o"], d["lse"],
-                            gamma, x["sel"])
+                            gamma, x["sel"], active=x["active"])
     torch.cuda.synchronize()
     assert fb.fb_get_device_status() == fb.FB_OK
     S.close()
@@ -565,11 +583,17 @@ def cpu_baseline(spec, budget_s: float):
                              gamma=None if spec.gamma is None else [spec.gamma] * spec.Hq)
     t0 = time.perf_counter()
     n = 0
+    sel = None
     for st in w.schedule():
         if st.step == 0:
             o.begin_block()
+            if spec.sel_k and spec.select == "mass":
+                mass = orc.attention_mass(orc.to64(st.q), kp64, st.prefix_len, 1.0 / np.sqrt(spec.D))
+                sel = orc.select_top_k(mass, spec.sel_k)
+        if st.sel is not None:
+            sel = st.sel.numpy()
         o.step(orc.to64(st.q), orc.to64(st.kin), orc.to64(st.vin), kp64, vp64, st.prefix_len, st.M, spec.tau,
-               None if st.sel is None else st.sel.numpy())
+               sel, None if st.active is None else st.active.numpy())
         n += 1
         if st.last_in_block:
             kp64, vp64, _ = orc.kv_append(kp64, vp64, st.prefix_len, orc.to64(st.kin), orc.to64(st.vin))
