@@ -105,13 +105,17 @@ static cudaEvent_t prof_event() {
   return e;
 }
 
-// Begin/end a profiled launch on stream s (no-ops while profiling is off).
+// Begin/end a profiled launch on stream s (events: no-ops while profiling is off).
+static const char* const kProfNames[FB_PROFILE_KINDS] = {"fb block-external pass", "fb block-internal pass",
+                                                         "fb merge/gate/append"};
 ProfScope::ProfScope(int kind, double bytes, cudaStream_t s) : kind_(kind), bytes_(bytes), s_(s) {
+  nvtxRangePushA(kProfNames[kind]);
   if (!g_prof.on) return;
   start_ = prof_event();
   cudaEventRecord(start_, s_);
 }
 ProfScope::~ProfScope() {
+  nvtxRangePop();
   if (!g_prof.on || !start_) return;
   cudaEvent_t stop = prof_event();
   cudaEventRecord(stop, s_);
@@ -840,6 +844,7 @@ fb_status fb_cache_last_step(fb_cache_t c, int32_t* recomputed) {
 }
 
 fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
+  NvtxRange range("fb_step");
   if (!c || !a) return FB_EINVAL;
   const fb_attn_desc& d = c->d;
   if (!a->q || !a->kin || !a->vin || !a->kp || !a->vp || !a->o) return FB_EINVAL;

@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 #include "fb.h"
 
@@ -70,8 +71,19 @@ struct AttnArgs {
   float scale_log2;            // softmax scale * log2(e)
 };
 
+// An NVTX range for the host-side span of one API call or launch (a no-op
+// unless a profiler is attached).
+class NvtxRange {
+ public:
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 // Profiling scope: brackets one launch with events on its stream when the
-// profiling hook is on (fb_profile_enable); kinds as in fb.h.
+// profiling hook is on (fb_profile_enable), and with an NVTX range named for
+// its kind; kinds as in fb.h.
 enum { kProfPrefix = 0, kProfInblock = 1, kProfAux = 2 };
 class ProfScope {
  public:
