@@ -122,6 +122,57 @@ def test_cache_and_step_checks(L):
     assert L.fb_cache_destroy(None) == fb.FB_EINVAL
 
 
+def test_active_subset_step_checks(L):
+    """fb_step with an active-query list: the flag, the count and the list's
+    alignment are checked before any launch."""
+    d = _desc()
+    h = C.c_void_p(0)
+    n = fb.fb_cache_workspace_bytes(d, 0, 512)
+    assert L.fb_cache_create(C.byref(d), 0, 512, 0, FAKE, n, None, C.byref(h)) == fb.FB_OK
+    a = fb.fb_step_args()
+    a.q = a.kin = a.vin = a.kp = a.vp = a.o = FAKE
+    a.prefix_len, a.M, a.tau = 256, 0, 4
+    a.active, a.n_active = FAKE, 8
+    assert L.fb_step(h, C.byref(a), None) == fb.FB_ESTATE          # no FB_CACHE_ACTIVE
+    assert L.fb_cache_destroy(h) == fb.FB_OK
+    flags = fb.FB_CACHE_ACTIVE | fb.FB_CACHE_SPARSE
+    n2 = fb.fb_cache_workspace_bytes(d, flags, 512, 64)
+    assert n2 > fb.fb_cache_workspace_bytes(d, fb.FB_CACHE_SPARSE, 512, 64)   # room for the compact block
+    assert L.fb_cache_create(C.byref(d), flags, 512, 64, FAKE, n2, None, C.byref(h)) == fb.FB_OK
+    for bad in (0, 33, -1):
+        a.n_active = bad
+        assert L.fb_step(h, C.byref(a), None) == fb.FB_EINVAL
+    a.n_active = 8
+    a.active = FAKE + 4
+    assert L.fb_step(h, C.byref(a), None) == fb.FB_EALIGN
+    a.active = FAKE
+    a.sel, a.sel_k = FAKE, 16
+    assert L.fb_step(h, C.byref(a), None) == fb.FB_EUNSUPPORTED     # with a sparse selection
+    assert L.fb_cache_destroy(h) == fb.FB_OK
+
+
+def _select(L, d, plen=256, k=16, sel=FAKE, ws=FAKE, wsb=1 << 30, mass=None):
+    return L.fb_select_mass(C.byref(d), FAKE, FAKE, FAKE, plen, k, sel, mass, ws, wsb, None)
+
+
+def test_select_mass_checks(L):
+    d = _desc()
+    assert fb.fb_select_workspace_bytes(d, 512) >= fb.fb_outblock_workspace_bytes(d, 512)
+    assert _select(L, d, k=257) == fb.FB_EINVAL          # k > prefix
+    assert _select(L, d, k=-1) == fb.FB_EINVAL
+    assert _select(L, d, plen=0, k=0) == fb.FB_EINVAL
+    assert _select(L, d, plen=513) == fb.FB_EINVAL       # beyond kp_capacity
+    assert _select(L, d, sel=FAKE + 4) == fb.FB_EALIGN
+    assert _select(L, d, wsb=64) == fb.FB_ENOSPACE
+    assert _select(L, d, sel=None) == fb.FB_EINVAL
+    # the KV head's G * Nb = 4 * 64 query rows do not fit one 128-row tile
+    q = torch.empty(1, 8, 64, 128, dtype=torch.bfloat16)
+    d64 = fb.make_desc(q, torch.empty(1, 2, 64, 128, dtype=torch.bfloat16),
+                       torch.empty(1, 2, 512, 128, dtype=torch.bfloat16), q)
+    assert _select(L, d64) == fb.FB_EUNSUPPORTED
+    assert _select(L, _desc(in_dtype=fb.FB_F32, out_dtype=fb.FB_F32)) in (fb.FB_EUNSUPPORTED, fb.FB_EALIGN)
+
+
 def test_debug_hooks_validate_and_reset(L):
     assert L.fb_debug_set_prefix_kernel(5) == fb.FB_EINVAL
     assert L.fb_debug_set_prefix_kernel(-1) == fb.FB_EINVAL
