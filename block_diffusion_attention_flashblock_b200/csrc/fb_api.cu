@@ -319,6 +319,77 @@ static fb_status launch_prefix(const fb_attn_desc& d, PrefixPlan& p, int64_t nke
              : FB_ECUDA;
 }
 
+// ---- sparse selected keys over the union of each KV head's selections ----
+// Scratch of the union pass for up to umax union keys per KV head: the compact
+// K and V rows, the union's positions and sizes, and per query head a
+// membership bitmap over the union.
+struct UnionWs {
+  void* ck;
+  void* cv;
+  int32_t* upos;
+  int32_t* ucount;
+  uint32_t* memb;
+};
+static int64_t union_keys(const fb_attn_desc& d, int64_t prefix_len, int32_t sel_k) {
+  return std::min<int64_t>(prefix_len, (int64_t)(d.Hq / d.Hkv) * sel_k);
+}
+static size_t union_bytes(const fb_attn_desc& d, int64_t umax) {
+  const int64_t wu = (umax + 31) / 32;
+  return 2 * align256((size_t)d.B * d.Hkv * umax * d.D * esize(d.in_dtype)) +
+         align256((size_t)d.B * d.Hkv * umax * 4) + align256((size_t)d.B * d.Hkv * 4) +
+         align256((size_t)d.B * d.Hq * wu * 4);
+}
+static UnionWs union_carve(const fb_attn_desc& d, int64_t umax, uint8_t* base) {
+  UnionWs u;
+  const int64_t wu = (umax + 31) / 32;
+  const size_t kvb = align256((size_t)d.B * d.Hkv * umax * d.D * esize(d.in_dtype));
+  u.ck = base;
+  u.cv = base + kvb;
+  u.upos = reinterpret_cast<int32_t*>(base + 2 * kvb);
+  u.ucount = reinterpret_cast<int32_t*>(base + 2 * kvb + align256((size_t)d.B * d.Hkv * umax * 4));
+  u.memb = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(u.ucount) + align256((size_t)d.B * d.Hkv * 4));
+  (void)wu;
+  return u;
+}
+// The union pass pays off when the union's rows, read, written compact and read
+// again, are fewer bytes than one pass over the prefix.
+static bool union_applies(const fb_attn_desc& d, int64_t prefix_len, int32_t sel_k) {
+  const int64_t u = union_keys(d, prefix_len, sel_k);
+  int mode, hg, tpu, units;
+  return g_prefix_kernel != 1 && u > 0 && 3 * u < prefix_len && tc_tiling(d, &mode, &hg, &tpu, &units);
+}
+// Selected keys (membership bitmap over the prefix already built): the
+// union's rows gathered compact, then the tcgen05 pass over them that leaves
+// out, per query head, the union keys it did not select.
+static fb_status launch_selected_union(const fb_attn_desc& d, const void* q, const void* kp, const void* vp,
+                                       int64_t prefix_len, const uint32_t* bitmap, int32_t sel_k, const UnionWs& u,
+                                       int32_t cap, float* pa, float* pl, int32_t* nparts, cudaStream_t s) {
+  const int64_t umax = union_keys(d, prefix_len, sel_k);
+  const int64_t wp = (prefix_len + 31) / 32, wu = (umax + 31) / 32;
+  const int es = esize(d.in_dtype);
+  {
+    ProfScope prof(kProfAux, (double)d.B * d.Hq * wp * 4 + (double)d.B * d.Hq * wu * 4, s);
+    if (launch_union_select(d, bitmap, wp, u.upos, u.ucount, umax, u.memb, wu, s) != cudaSuccess) return FB_ECUDA;
+  }
+  {
+    ProfScope prof(kProfAux, 4.0 * d.B * d.Hkv * umax * d.D * es, s);
+    if (launch_gather_union(d, kp, vp, u.upos, u.ucount, umax, u.ck, u.cv, s) != cudaSuccess) return FB_ECUDA;
+  }
+  fb_attn_desc dc = d;
+  dc.kp_capacity = umax;
+  dc.kp_strides[0] = (int64_t)d.Hkv * umax * d.D;
+  dc.kp_strides[1] = umax * d.D;
+  dc.kp_strides[2] = d.D;
+  PrefixPlan p = plan_prefix(dc, q, u.ck, u.cv, umax, cap);
+  if (!p.tc) return FB_EUNSUPPORTED;
+  p.pair = false;
+  p.excl = u.memb;
+  p.excl_words = wu;
+  p.excl_invert = true;
+  *nparts = p.nparts;
+  return launch_prefix(dc, p, umax, nullptr, 0, pa, pl, s);
+}
+
 static PartGroup group_of(const float* a, const float* l, int32_t n, const fb_attn_desc& d) {
   PartGroup g;
   g.a = a; g.l = l; g.count = n;
@@ -465,6 +536,7 @@ fb_status fb_outblock_workspace_bytes(const fb_attn_desc* d, int64_t prefix_len,
   size_t n = part_bytes(*d, std::max(split_bound(*d, 0, prefix_len), sel_k ? split_bound(*d, 1, sel_k) : 1));
   n += align256((size_t)pair_count(*d) * 4);
   if (sel_k) n += align256((size_t)d->B * d->Hq * ((prefix_len + 31) / 32) * 4);
+  if (sel_k && union_applies(*d, prefix_len, sel_k)) n += union_bytes(*d, union_keys(*d, prefix_len, sel_k));
   *bytes = n;
   return FB_OK;
 }
@@ -510,8 +582,24 @@ fb_status fb_attn_outblock(const fb_attn_desc* d, const void* q, const void* kp,
     lst.g[0] = group_of(pa, pl, p.nparts, *d);
     return merge_to_part(*d, lst, a_out, l_out, nullptr, 0, stream);
   }
+  const bool via_union = union_applies(*d, prefix_len, sel_k);
+  if (via_union) {
+    // the union's rows once per KV head, then the pass over them
+    if (launch_build_bitmap(sel, sel_k, d->B * d->Hq, bitmap, words, stream) != cudaSuccess) return FB_ECUDA;
+    const UnionWs u = union_carve(*d, union_keys(*d, prefix_len, sel_k),
+                                  reinterpret_cast<uint8_t*>(ns) + align256((size_t)pair_count(*d) * 4));
+    int32_t np = 0;
+    if ((st = launch_selected_union(*d, q, kp, vp, prefix_len, bitmap, sel_k, u, cap, pa, pl, &np, stream)) != FB_OK)
+      return st;
+    PartList lst;
+    memset(&lst, 0, sizeof(lst));
+    lst.ngroups = 1;
+    lst.g[0] = group_of(pa, pl, np, *d);
+    if ((st = merge_to_part(*d, lst, a_out, l_out, nullptr, 0, stream)) != FB_OK) return st;
+  }
   PassPlan p = plan_pass(*d, q, kp, vp, d->kp_strides, prefix_len, sel, sel_k, cap);
-  if (p.nsplit == 1) {
+  if (via_union) {
+  } else if (p.nsplit == 1) {
     if ((st = launch_pass(*d, p.a, a_out, l_out, stream)) != FB_OK) return st;
   } else {
     if ((st = launch_pass(*d, p.a, pa, pl, stream)) != FB_OK) return st;
@@ -523,7 +611,8 @@ fb_status fb_attn_outblock(const fb_attn_desc* d, const void* q, const void* kp,
   }
   if (!sel || !a_res) return FB_OK;
   // pass 2: the residual (prefix minus the selection)
-  if (launch_build_bitmap(sel, sel_k, d->B * d->Hq, bitmap, words, stream) != cudaSuccess) return FB_ECUDA;
+  if (!via_union && launch_build_bitmap(sel, sel_k, d->B * d->Hq, bitmap, words, stream) != cudaSuccess)
+    return FB_ECUDA;
   PrefixPlan r = plan_prefix(*d, q, kp, vp, prefix_len, cap);
   r.excl = bitmap;
   r.excl_words = words;
@@ -724,6 +813,8 @@ struct fb_cache {
   int32_t* counters;  // gamma: per-head arrival counters (kept at zero)
   int32_t chunks;
   int32_t* pair_ns;   // slot counts of the paired prefix pass
+  uint8_t* union_base;  // sparse: scratch of the union pass (UnionWs)
+  int64_t union_cap;    // union keys per KV head it holds
   void* act_q;        // active subsets: compact queries [B, Hq, Nb, D]
   float* act_a;       // active subsets: compact block-external part
   float* act_l;
@@ -757,10 +848,14 @@ fb_status layout_cache(const fb_attn_desc& d, int32_t flags, int64_t max_prefix,
   float* pl = cv.take<float>(base, (size_t)part_cap * rows * 4);
   int32_t* pn = cv.take<int32_t>(base, (size_t)pair_count(d) * 4);
   float* sa = nullptr; float* sl = nullptr; uint32_t* bm = nullptr;
+  uint8_t* ub = nullptr;
+  int64_t ucap = 0;
   if (flags & FB_CACHE_SPARSE) {
     sa = cv.take<float>(base, (size_t)sel_cap * rows * d.D * 4);
     sl = cv.take<float>(base, (size_t)sel_cap * rows * 4);
     bm = cv.take<uint32_t>(base, (size_t)d.B * d.Hq * words * 4);
+    ucap = union_keys(d, max_prefix, max_sel_k);
+    ub = cv.take<uint8_t>(base, union_bytes(d, ucap));
   }
   void* aq = nullptr; float* aa = nullptr; float* al = nullptr;
   if (flags & FB_CACHE_ACTIVE) {
@@ -782,6 +877,7 @@ fb_status layout_cache(const fb_attn_desc& d, int32_t flags, int64_t max_prefix,
     c->mask = mk; c->sim = sm; c->gpart = gp; c->counters = ct; c->chunks = chunks;
     c->pair_ns = pn;
     c->act_q = aq; c->act_a = aa; c->act_l = al;
+    c->union_base = ub; c->union_cap = ucap;
   }
   return FB_OK;
 }
@@ -965,10 +1061,20 @@ fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
       int32_t nsel = 0;
       PrefixPlan sp;
       sp.tc = false;
-      if ((int64_t)a->sel_k * 3 * (d.Hq / d.Hkv) > a->prefix_len) {
+      const bool via_union = union_applies(d, a->prefix_len, a->sel_k) &&
+                             union_keys(d, a->prefix_len, a->sel_k) <= c->union_cap;
+      if (!via_union && (int64_t)a->sel_k * 3 * (d.Hq / d.Hkv) > a->prefix_len) {
         sp = plan_prefix(d, a->q, a->kp, a->vp, a->prefix_len, c->sel_cap);
       }
-      if (sp.tc) {
+      if (via_union) {
+        if (launch_build_bitmap(a->sel, a->sel_k, BH, c->bitmap, (a->prefix_len + 31) / 32, s) != cudaSuccess)
+          return FB_ECUDA;
+        bitmap_built = true;
+        const UnionWs u = union_carve(d, union_keys(d, a->prefix_len, a->sel_k), c->union_base);
+        if ((st = launch_selected_union(d, a->q, a->kp, a->vp, a->prefix_len, c->bitmap, a->sel_k, u, c->sel_cap,
+                                        c->sel_a, c->sel_l, &nsel, s)) != FB_OK)
+          return st;
+      } else if (sp.tc) {
         if (launch_build_bitmap(a->sel, a->sel_k, BH, c->bitmap, (a->prefix_len + 31) / 32, s) != cudaSuccess)
           return FB_ECUDA;
         bitmap_built = true;

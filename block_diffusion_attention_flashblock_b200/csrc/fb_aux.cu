@@ -4,6 +4,7 @@
 // Réutilisation Adaptatives").
 #include "fb_internal.cuh"
 #include "fb_ptx.cuh"
+#include <cub/block/block_scan.cuh>
 #include <math_constants.h>
 
 namespace fb {
@@ -325,6 +326,109 @@ __global__ void scatter_active_part_kernel(const float* ca, const float* cl, flo
   for (int c = lane * 4; c < D; c += 128)
     *reinterpret_cast<float4*>(a + dst * D + c) = *reinterpret_cast<const float4*>(ca + r * D + c);
   if (lane == 0) l[dst] = cl[r];
+}
+
+// ---------------------------------------------------------------------------
+// Sparse selected keys, gathered once per KV head: the union of its G query
+// heads' selections (from their membership bitmaps over the prefix), in key
+// order, and per query head a membership bitmap over that union.  The
+// tcgen05 pass then runs over the union's rows (gathered into a compact K/V
+// block) and leaves out, per query head, the union keys it did not select.
+// One CTA per (b, KV head); the union has at most `umax` keys.
+// ---------------------------------------------------------------------------
+constexpr int kUnionThreads = 1024;
+__global__ void __launch_bounds__(kUnionThreads)
+    union_select_kernel(const uint32_t* bitmap, int64_t words_p, int32_t G, int32_t Hq, int32_t Hkv, int32_t* upos,
+                        int32_t* ucount, int64_t umax, uint32_t* memb, int64_t words_u) {
+  ptx::pdl_prologue();
+  using Scan = cub::BlockScan<int64_t, kUnionThreads>;
+  __shared__ typename Scan::TempStorage tmp;
+  __shared__ int64_t s_total;
+  const int kv = blockIdx.x, b = kv / Hkv, kvh = kv % Hkv;
+  const uint32_t* hb = bitmap + ((int64_t)b * Hq + (int64_t)kvh * G) * words_p;   // G head bitmaps
+  int32_t* up = upos + (int64_t)kv * umax;
+  auto uword = [&](int64_t w) {
+    uint32_t u = 0u;
+    for (int g = 0; g < G; ++g) u |= hb[g * words_p + w];
+    return u;
+  };
+  // the union's positions, in key order
+  const int64_t chunk = (words_p + kUnionThreads - 1) / kUnionThreads;
+  const int64_t w0 = threadIdx.x * chunk, w1 = min(words_p, w0 + chunk);
+  int64_t cnt = 0;
+  for (int64_t w = w0; w < w1; ++w) cnt += __popc(uword(w));
+  int64_t base, total;
+  Scan(tmp).ExclusiveSum(cnt, base, total);
+  if (threadIdx.x == 0) s_total = total;
+  for (int64_t w = w0; w < w1; ++w) {
+    uint32_t u = uword(w);
+    while (u) {
+      const int bit = __ffs(u) - 1;
+      u &= u - 1;
+      if (base < umax) up[base] = (int32_t)(w * 32 + bit);
+      ++base;
+    }
+  }
+  __syncthreads();
+  const int64_t n = min(s_total, umax);
+  if (threadIdx.x == 0) ucount[kv] = (int32_t)n;
+  // membership of each union key in each query head's selection
+  for (int64_t i = threadIdx.x; i < (int64_t)G * words_u; i += kUnionThreads) {
+    const int g = (int)(i / words_u);
+    const int64_t cw = i % words_u;
+    uint32_t bits = 0u;
+    for (int j = 0; j < 32; ++j) {
+      const int64_t idx = cw * 32 + j;
+      if (idx >= n) break;
+      const int32_t pos = up[idx];
+      if ((hb[g * words_p + (pos >> 5)] >> (pos & 31)) & 1u) bits |= 1u << j;
+    }
+    memb[((int64_t)b * Hq + (int64_t)kvh * G + g) * words_u + cw] = bits;
+  }
+}
+
+// Rows [0, ucount) of the compact K/V block of each (b, KV head) <- the
+// prefix rows at the union's positions; rows [ucount, umax) <- zeros (their
+// keys are excluded for every head, and zeros keep P V finite).  One thread
+// per 16-byte vector of a row of K and of V.
+__global__ void gather_union_kernel(const uint8_t* kp, const uint8_t* vp, int64_t kp_sb, int64_t kp_sh,
+                                    int64_t kp_st, const int32_t* upos, const int32_t* ucount, int64_t umax,
+                                    int32_t Hkv, int32_t vec_per_row, int64_t nrows, uint8_t* ck, uint8_t* cv) {
+  ptx::pdl_prologue();
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= nrows * vec_per_row) return;
+  const int64_t r = idx / vec_per_row;   // compact row: (b * Hkv + kvh) * umax + i
+  const int c = (int)(idx % vec_per_row);
+  const int64_t kv = r / umax, i = r % umax;
+  const int64_t dst = r * vec_per_row * 16 + c * 16;
+  uint4 kx = make_uint4(0, 0, 0, 0), vx = kx;
+  if (i < ucount[kv]) {
+    const int64_t b = kv / Hkv, h = kv % Hkv;
+    const int64_t src = b * kp_sb + h * kp_sh + (int64_t)upos[r] * kp_st + c * 16;
+    kx = __ldg(reinterpret_cast<const uint4*>(kp + src));
+    vx = __ldg(reinterpret_cast<const uint4*>(vp + src));
+  }
+  *reinterpret_cast<uint4*>(ck + dst) = kx;
+  *reinterpret_cast<uint4*>(cv + dst) = vx;
+}
+
+cudaError_t launch_union_select(const fb_attn_desc& d, const uint32_t* bitmap, int64_t words_p, int32_t* upos,
+                                int32_t* ucount, int64_t umax, uint32_t* memb, int64_t words_u, cudaStream_t s) {
+  return launch_k(union_select_kernel, dim3((unsigned)(d.B * d.Hkv)), dim3(kUnionThreads), 0, s, bitmap, words_p,
+                  (int32_t)(d.Hq / d.Hkv), (int32_t)d.Hq, (int32_t)d.Hkv, upos, ucount, umax, memb, words_u);
+}
+
+cudaError_t launch_gather_union(const fb_attn_desc& d, const void* kp, const void* vp, const int32_t* upos,
+                                const int32_t* ucount, int64_t umax, void* ck, void* cv, cudaStream_t s) {
+  const int es = d.in_dtype == FB_BF16 ? 2 : 4;
+  const int vec = d.D * es / 16;
+  const int64_t rows = (int64_t)d.B * d.Hkv * umax;
+  const int threads = 256;
+  const unsigned grid = (unsigned)((rows * vec + threads - 1) / threads);
+  return launch_k(gather_union_kernel, dim3(grid), dim3(threads), 0, s, static_cast<const uint8_t*>(kp),
+                  static_cast<const uint8_t*>(vp), d.kp_strides[0] * es, d.kp_strides[1] * es, d.kp_strides[2] * es,
+                  upos, ucount, umax, (int32_t)d.Hkv, (int32_t)vec, rows, static_cast<uint8_t*>(ck),
+                  static_cast<uint8_t*>(cv));
 }
 
 int* device_status_ptr();

@@ -236,5 +236,12 @@ cudaError_t launch_kv_append(const fb_attn_desc& d, void* kp, void* vp, int64_t 
 cudaError_t launch_build_bitmap(const int32_t* sel, int32_t sel_k, int32_t BH,
                                 uint32_t* bitmap, int64_t words, cudaStream_t s);
 cudaError_t launch_fill_decision(int8_t* reuse_out, int32_t n, int8_t value, cudaStream_t s);
+// The union of each KV head's query heads' selections (positions in key order,
+// at most umax) and per query head a membership bitmap over it; then its
+// rows of K/V gathered into a compact [B, Hkv, umax, D] block.
+cudaError_t launch_union_select(const fb_attn_desc& d, const uint32_t* bitmap, int64_t words_p, int32_t* upos,
+                                int32_t* ucount, int64_t umax, uint32_t* memb, int64_t words_u, cudaStream_t s);
+cudaError_t launch_gather_union(const fb_attn_desc& d, const void* kp, const void* vp, const int32_t* upos,
+                                const int32_t* ucount, int64_t umax, void* ck, void* cv, cudaStream_t s);
 
 }  // namespace fb

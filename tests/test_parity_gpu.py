@@ -172,6 +172,7 @@ def test_outblock_empty_prefix():
 
 
 @pytest.mark.parametrize("shape", [(1, 8, 2, 128, 32, 1500, 100, "bf16"), (1, 4, 4, 64, 32, 256, 40, "f32"),
+                                   (1, 32, 8, 128, 32, 32768, 2048, "bf16"), (2, 8, 4, 128, 64, 5000, 300, "bf16"),
                                    (2, 8, 2, 128, 16, 3000, 0, "bf16"), (1, 4, 1, 128, 8, 200, 200, "bf16"),
                                    (1, 8, 2, 128, 32, 300, 300, "bf16"), (1, 4, 4, 128, 200, 2000, 700, "bf16")],
                          ids=lambda s: "x".join(map(str, s)))
