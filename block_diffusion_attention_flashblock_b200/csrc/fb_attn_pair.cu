@@ -250,17 +250,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int c = blockIdx.x;
     int n = 0;
     if (a.whole) {
-      // whole pairs: active pairs c, c + C, c + 2C, ...
-      int ai = 0;
-      for (int p = 0; p < a.npairs && n < kMaxSeg; ++p) {
-        if (a.mask_active && !((act[p >> 5] >> (p & 31)) & 1u)) continue;
-        if (ai++ % C != c) continue;
+      // whole pairs: active pairs c, c + C, c + 2C, ... (every pair is active
+      // without the gamma gate)
+      auto push = [&](int p) {
         Seg sg;
         sg.pair = p;
         sg.j0 = 0;
         sg.j1 = a.nkt;
         sg.slot_ns = 1 << 16;
         segs[n++] = sg;
+      };
+      if (!a.mask_active) {
+        for (int p = c; p < a.npairs && n < kMaxSeg; p += C) push(p);
+      } else {
+        int ai = 0;
+        for (int p = 0; p < a.npairs && n < kMaxSeg; ++p) {
+          if (!((act[p >> 5] >> (p & 31)) & 1u)) continue;
+          if (ai++ % C == c) push(p);
+        }
       }
     } else if (c < C) {
       const int64_t i0 = (int64_t)c * T / C, i1 = (int64_t)(c + 1) * T / C;
