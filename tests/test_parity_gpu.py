@@ -278,6 +278,13 @@ SCHEDULES = {
     "nb1_gqa": dict(base="dllm_8k", Nb=1, prefix0=300, steps=3, m_model=("uniform", 0, 1), tau=1),
     "nb4_small": dict(base="dllm_8k_nb4", prefix0=1000, blocks=2),
     "sparse_d40_small": dict(base="sparse_32k_d40", prefix0=3000, sel_k=1200, Hq=8, Hkv=2),
+    # gamma gates that always reuse (every similarity exceeds -1) and never
+    # reuse: from step 2 on every head is masked, or none is
+    "video_gamma_always": dict(base="video_1560", Hq=4, Hkv=4, prefix0=3120, steps=4, gamma=-1.0),
+    "video_gamma_never": dict(base="video_1560", Hq=4, Hkv=4, prefix0=3120, steps=4, gamma=1.5),
+    # the first block of a sequence: no prefix at all
+    "empty_prefix": dict(base="dllm_8k", prefix0=0, blocks=2, steps=3),
+    "empty_prefix_nb64": dict(base="dllm_64k_b4", B=1, prefix0=0, blocks=2, steps=3),
     # the sparse keys chosen by attention mass at each block's start
     "mass_small": dict(base="sparse_32k_mass", prefix0=4000, sel_k=256, Hq=8, Hkv=2, blocks=2),
     "mass_nb16_b2": dict(base="sparse_32k_mass", B=2, Nb=16, prefix0=2500, sel_k=700, Hq=16, Hkv=2, steps=5,
@@ -309,6 +316,10 @@ def test_step_schedule(name):
     if name == "video_small_mixed":
         r = np.array(st["reuse"])
         assert 0 < r[2:].mean() < 1, "the mixed video case should both reuse and recompute"
+    if name == "video_gamma_always":
+        assert np.array(st["reuse"])[2:].min() == 1.0
+    if name == "video_gamma_never":
+        assert np.array(st["reuse"]).max() == 0.0
 
 
 def test_step_bf16_output():
@@ -325,6 +336,7 @@ def test_full_dllm_8k_all_heads():
 @pytest.mark.parametrize("name, groups", [
     ("dllm_64k_b4", [(0, 0), (3, 7)]),
     ("dllm_ctx_200k", [(0, 0), (0, 7)]),
+    ("dllm_ctx_800k", [(0, 3)]),
     ("dllm_8k_nb4", [(0, 0), (0, 5)]),
     ("sparse_32k_d40", [(0, 0), (0, 6)]),
     ("video_1560", [(0, 0), (0, 13), (0, 23)]),
