@@ -183,9 +183,17 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* mass, i
     for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
     __syncthreads();
     const uint32_t prefix = s_prefix;
-    for (int64_t x = threadIdx.x; x < n; x += blockDim.x) {
-      const uint32_t v = bits[x];
-      if ((v & mask) == prefix) atomicAdd(&hist[(v >> shift) & 255u], 1);
+    // every lane takes the same trip count, so the warp can aggregate equal
+    // bins (masses share their leading bits) into one shared-memory atomic
+    const int64_t n_round = (n + blockDim.x - 1) / blockDim.x * blockDim.x;
+    for (int64_t x = threadIdx.x; x < n_round; x += blockDim.x) {
+      uint32_t bin = 256u;   // no bin
+      if (x < n) {
+        const uint32_t v = bits[x];
+        if ((v & mask) == prefix) bin = (v >> shift) & 255u;
+      }
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (bin < 256u && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
     }
     __syncthreads();
     if (threadIdx.x == 0) {
