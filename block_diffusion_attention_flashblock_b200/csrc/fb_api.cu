@@ -641,7 +641,7 @@ fb_status fb_select_mass(const fb_attn_desc* d, const void* q, const void* kp, c
                          cudaStream_t stream) {
   fb_status st = check_desc(d);
   if (st != FB_OK) return st;
-  if (!q || !kp || !vp || !sel_out) return FB_EINVAL;
+  if (!q || !kp || !vp || (!sel_out && k > 0)) return FB_EINVAL;
   if (prefix_len < 1 || prefix_len > d->kp_capacity || k < 0 || k > prefix_len) return FB_EINVAL;
   if (!mass_applies(*d)) return FB_EUNSUPPORTED;
   if (!al16(q) || !al16(kp) || !al16(vp) || !al16(sel_out) || !al16(mass_out) || !al16(ws)) return FB_EALIGN;

@@ -148,7 +148,8 @@ fb_status fb_attn_outblock_noalloc(const fb_attn_desc* d, const void* q, const v
  * block's queries, summed over them), ties to the lower index.  Call it once
  * per block with the block's first queries and pass sel_out to that block's
  * fb_step calls.
- * sel_out: device int32 [B, Hq, k], written ascending.  mass_out: optional
+ * sel_out: device int32 [B, Hq, k], written ascending (may be NULL when
+ *   k == 0).  mass_out: optional
  *   device fp32 [B, Hq, prefix_len] that receives the masses (else they stay
  *   in the workspace).  ws: at least fb_select_workspace_bytes() bytes.
  * Requires bf16 inputs, D = 128, Nb in {16, 32} and (Hq / Hkv) * Nb <= 128

@@ -164,7 +164,7 @@ def test_select_mass_checks(L):
     assert _select(L, d, plen=513) == fb.FB_EINVAL       # beyond kp_capacity
     assert _select(L, d, sel=FAKE + 4) == fb.FB_EALIGN
     assert _select(L, d, wsb=64) == fb.FB_ENOSPACE
-    assert _select(L, d, sel=None) == fb.FB_EINVAL
+    assert _select(L, d, sel=None) == fb.FB_EINVAL       # k > 0 needs somewhere to write
     # the KV head's G * Nb = 4 * 64 query rows do not fit one 128-row tile
     q = torch.empty(1, 8, 64, 128, dtype=torch.bfloat16)
     d64 = fb.make_desc(q, torch.empty(1, 2, 64, 128, dtype=torch.bfloat16),
