@@ -24,6 +24,8 @@ static bool g_pdl = true;
 bool pdl_enabled() { return g_pdl; }
 static bool g_stall = false;
 bool debug_stall() { return g_stall; }
+static bool g_inblock_bulk = false;
+bool inblock_bulk_loads() { return g_inblock_bulk; }
 
 // Device address of this device's status word, looked up once per device (the
 // first launch on a device should come before any stream capture on it; a
@@ -772,6 +774,11 @@ fb_status fb_debug_set_prefix_kernel(int32_t which) {
 
 fb_status fb_debug_set_stall(int32_t on) {
   g_stall = on != 0;
+  return FB_OK;
+}
+
+fb_status fb_debug_set_inblock_loads(int32_t bulk) {
+  g_inblock_bulk = bulk != 0;
   return FB_OK;
 }
 

@@ -86,7 +86,17 @@ struct InblockArgs {
   int32_t stall;      // test hook: thread 0 first waits on a barrier nothing completes
   const int32_t* active;  // non-null: [B, n_act] block positions of the queries to compute (the rest untouched)
   int32_t n_act;
+  int32_t bulk;           // 1: one bulk copy per row; 0: 16-byte cp.async chunks from every thread
 };
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 // Bounded wait on phase 0 of a load barrier; the first expiry is recorded.  A
 // drain (the last wait before exit after an expiry) is bounded by at least
@@ -152,7 +162,10 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   };
   const uint32_t bar_qk = ptx::smem_addr(bars), bar_v = bar_qk + 8, bar_e = bar_qk + 16;
 
-  // ---- every load is one bulk copy per row, issued up front ----
+  // ---- every load issued up front: one bulk copy per row (a.bulk), or
+  // 16-byte cp.async chunks from all 128 threads in three commit groups
+  // (Q and K_in; V_in; the parts), which keeps the SM's copy engine out of
+  // the way when a CTA needs a hundred or more rows ----
   if (tid == 0) {
     int nvalid = 0, hh, ii;
     for (int r = 0; r < nq; ++r) nvalid += row_at(r, hh, ii) >= 0;
@@ -162,9 +175,11 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
     ptx::mbar_init(bar_e, 1);
     ptx::mbar_init(bar_e + 8, 1);
     ptx::fence_mbar_init();
-    ptx::mbar_expect_tx(bar_qk, (uint32_t)(nvalid + a.Nb) * (kD * 2));
-    ptx::mbar_expect_tx(bar_v, (uint32_t)a.Nb * (kD * 2));
-    ptx::mbar_expect_tx(bar_e, (uint32_t)(NX * nvalid) * (kD * 4));
+    if (a.bulk) {
+      ptx::mbar_expect_tx(bar_qk, (uint32_t)(nvalid + a.Nb) * (kD * 2));
+      ptx::mbar_expect_tx(bar_v, (uint32_t)a.Nb * (kD * 2));
+      ptx::mbar_expect_tx(bar_e, (uint32_t)(NX * nvalid) * (kD * 4));
+    }
   }
   // L of (part, row) = (idx / 16, idx % 16) for idx = tid, tid + 128: read
   // early, stored to shared memory after P V
@@ -177,7 +192,43 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
     if (pr >= 0) lx[k] = a.ext_l[idx >> 4][pr];
   }
   __syncthreads();
-  if (warp == 0) {
+  if (!a.bulk) {
+    const __nv_bfloat16* kb = a.k + b * a.k_sb + (int64_t)kvh * a.k_sh;
+    const __nv_bfloat16* vb = a.v + b * a.k_sb + (int64_t)kvh * a.k_sh;
+    for (int c = tid; c < kRows * 16; c += 128) {   // Q rows, 16 chunks each
+      const int r = c >> 4, ch = c & 15;
+      int h, i;
+      if (row_at(r, h, i) >= 0)
+        cp_async16(ptx::smem_addr(sQ + r * kRowE + ch * 8),
+                   a.q + b * a.q_sb + (int64_t)h * a.q_sh + (int64_t)i * a.q_st + ch * 8);
+      else
+        *reinterpret_cast<uint4*>(sQ + r * kRowE + ch * 8) = make_uint4(0, 0, 0, 0);
+    }
+    for (int c = tid; c < NB * 16; c += 128) {      // K rows
+      const int r = c >> 4, ch = c & 15;
+      if (r < a.Nb)
+        cp_async16(ptx::smem_addr(sK + r * kRowE + ch * 8), kb + (int64_t)r * a.k_st + ch * 8);
+      else
+        *reinterpret_cast<uint4*>(sK + r * kRowE + ch * 8) = make_uint4(0, 0, 0, 0);
+    }
+    cp_async_commit();
+    for (int c = tid; c < NB * 16; c += 128) {      // V rows
+      const int r = c >> 4, ch = c & 15;
+      if (r < a.Nb)
+        cp_async16(ptx::smem_addr(sV + r * kRowE + ch * 8), vb + (int64_t)r * a.k_st + ch * 8);
+      else
+        *reinterpret_cast<uint4*>(sV + r * kRowE + ch * 8) = make_uint4(0, 0, 0, 0);
+    }
+    cp_async_commit();
+    for (int c = tid; c < NX * kRows * 32; c += 128) {   // the parts' rows, 32 chunks each
+      const int p = c / (kRows * 32), r = (c >> 5) % kRows, ch = c & 31;
+      int hh, ii;
+      const int64_t pr = row_at(r, hh, ii);
+      if (pr >= 0)
+        cp_async16(ptx::smem_addr(sE + (p * kRows + r) * kExtStride + ch * 4), a.ext_a[p] + pr * kD + ch * 4);
+    }
+    cp_async_commit();
+  } else if (warp == 0) {
     if (lane < kRows) {
       const int r = lane;
       int h, i;
@@ -212,9 +263,10 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
         ptx::bulk_g2s(ptx::smem_addr(sE + ((pp + p) * kRows + r) * kExtStride), a.ext_a[pp + p] + pr * kD, kD * 4,
                       bar_e);
   }
-  __syncthreads();   // zero-filled rows
+  if (!a.bulk) cp_async_wait<2>();   // this thread's Q and K chunks
+  __syncthreads();   // every thread's chunks, and the zero-filled rows
   bool ok = !(a.stall && tid == 0) || wait_loaded(bar_e + 8, a);
-  ok = wait_loaded(bar_qk, a) && ok;
+  if (a.bulk) ok = wait_loaded(bar_qk, a) && ok;
 
   // ---- S = Q K^T for the CTA's 16 rows (every warp) ----
   const int dq = warp;   // this warp's quarter of D: columns dq*32 .. dq*32+31
@@ -265,7 +317,12 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
     lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 1);
     lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 2);
   }
-  ok = wait_loaded(bar_v, a) && ok;
+  if (a.bulk) {
+    ok = wait_loaded(bar_v, a) && ok;
+  } else {
+    cp_async_wait<1>();
+    __syncthreads();
+  }
   // ---- O[:, dq*32 : dq*32+32] = P V ----
   constexpr int DT = 4;    // 8-column tiles in this warp's quarter
   float o[DT][4];
@@ -289,8 +346,11 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
 #pragma unroll
   for (int k = 0; k < 2; ++k)
     if (tid + k * 128 < NX * kRows) sL[tid + k * 128] = lx[k];
-  ok = wait_loaded(bar_e, a) && ok;
-  __syncthreads();   // sL
+  if (a.bulk)
+    ok = wait_loaded(bar_e, a) && ok;
+  else
+    cp_async_wait<0>();
+  __syncthreads();   // sL (and the parts' rows)
   // ---- merge with the external parts; rows staged for whole-row stores ----
   const bool obf = a.o_bf16 != 0;
 #pragma unroll
@@ -360,7 +420,7 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
     }
     ptx::bulk_wait_read();
   }
-  if (!ok && tid == 0) {
+  if (!ok && tid == 0 && a.bulk) {
     // a load wait expired: let every copy into shared memory land before exit
     wait_loaded(bar_qk, a, true);
     wait_loaded(bar_v, a, true);
@@ -402,6 +462,7 @@ cudaError_t launch_inblock_small(const fb_attn_desc& d, const void* q, const voi
   a.status = device_status_ptr();
   a.wait_limit_ns = wait_limit_ns();
   a.stall = debug_stall() ? 1 : 0;
+  a.bulk = inblock_bulk_loads() ? 1 : 0;
   if (!a.status) return cudaErrorInvalidValue;
   const int NB = d.Nb <= 16 ? 16 : d.Nb <= 32 ? 32 : 64;
   const int nxs = next > 0 ? next : 1;

@@ -105,6 +105,7 @@ class ProfScope {
 // memory before the kernels it depends on have completed.
 bool pdl_enabled();
 bool debug_stall();   // test hook: kernels first wait on a barrier nothing completes
+bool inblock_bulk_loads();   // tuning hook: the small in-block kernel loads by bulk copy per row
 template <class... KArgs, class... Args>
 cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
   cudaLaunchConfig_t cfg = {};

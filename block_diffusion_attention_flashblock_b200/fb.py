@@ -75,6 +75,7 @@ _SIGS = {
     "fb_get_device_status": (C.c_int, [_P, C.POINTER(C.c_int)]),
     "fb_debug_set_wait_limit_ns": (C.c_int, [C.c_uint64]),
     "fb_debug_set_pdl": (C.c_int, [C.c_int32]),
+    "fb_debug_set_inblock_loads": (C.c_int, [C.c_int32]),
     "fb_debug_set_stall": (C.c_int, [C.c_int32]),
     "fb_profile_enable": (C.c_int, [C.c_int32]),
     "fb_debug_set_prefix_kernel": (C.c_int, [C.c_int32]),
@@ -290,6 +291,10 @@ def fb_debug_set_wait_limit_ns(ns: int):
 
 def fb_debug_set_pdl(on: bool):
     _check(lib().fb_debug_set_pdl(1 if on else 0), "fb_debug_set_pdl")
+
+
+def fb_debug_set_inblock_loads(bulk: bool):
+    _check(lib().fb_debug_set_inblock_loads(1 if bulk else 0), "fb_debug_set_inblock_loads")
 
 
 def fb_debug_set_stall(on: bool):

@@ -334,6 +334,11 @@ fb_status fb_debug_set_wait_limit_ns(uint64_t ns);
  * it returns).  Off by default.  Affects only the calling process. */
 fb_status fb_debug_set_stall(int32_t on);
 
+/* Tuning hook: how the small-block in-block kernel loads its rows: 0
+ * (default) 16-byte cp.async chunks from every thread, 1 one bulk copy per
+ * row.  Affects only the calling process. */
+fb_status fb_debug_set_inblock_loads(int32_t bulk);
+
 /* Tuning hook: 1 (default) launches every kernel with programmatic dependent
  * launch allowed, so a kernel's launch overlaps the tail of the one before it
  * in the stream (each kernel waits for its predecessors before it touches
