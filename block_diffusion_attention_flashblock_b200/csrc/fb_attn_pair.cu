@@ -22,6 +22,8 @@
 //               tiles of 128 keys into a three-stage K ring and a two-stage
 //               V ring (128-byte swizzle), K one tile ahead of V
 //   warp 9      allocates TMEM; one thread issues every tcgen05.mma
+//   warps 10,11 idle (they complete the third warpgroup, whose registers
+//               go to the softmax warpgroups)
 // TMEM: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).  Softmax s
 // reads its row of S_s, writes P = 2^(s - m) over the same columns as bf16
 // hi (columns 0..63) and lo (64..127) parts, and the issuer runs
@@ -52,7 +54,14 @@ namespace {
 using namespace tc;
 
 constexpr int kBM = 128, kBN = 128, kD = 128;
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;                    // three warpgroups
+// Register split (setmaxnreg): the launch gives every thread kRegsLaunch;
+// the producer / MMA warpgroup drops to kRegsIO and the two softmax
+// warpgroups, which hold a row's 128 scores, rise to kRegsSoftmax.  The
+// shares add up to the launch's allocation exactly; the host checks the
+// kernel's launch register count before the first launch.
+constexpr int kRegsLaunch = 168, kRegsIO = 120, kRegsSoftmax = 192;
+static_assert(4 * 32 * kRegsIO + 8 * 32 * kRegsSoftmax == kThreads * kRegsLaunch, "register split");
 constexpr int kKSt = 3, kVSt = 2;                 // K and V ring depths
 constexpr uint32_t kHalf = 16384;                 // [128 rows][64 bf16], 128-byte swizzle
 constexpr uint32_t kTile = 2 * kHalf;             // one 128 x 128 bf16 tile
@@ -94,6 +103,17 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
       : "r"(taddr));
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_ld8u(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st8u(uint32_t taddr, const uint32_t* v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
 }
 
 // max of three (one instruction on sm_100)
@@ -311,6 +331,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nseg = *nseg_sh;
   const Ctl ctl{abort_flag, a.status, a.wait_limit_ns};
 
+  if (warp >= 8) {
+    // the third warpgroup: all four warps give up registers, then the
+    // producer and the MMA issuer run (warps 10 and 11 have nothing to do)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsIO));
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && nseg > 0) {
@@ -322,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       auto load_k = [&](int b, int kvh, int j) -> bool {
         const int st = kt % kKSt, round = kt / kKSt;
-        if (kt >= kKSt && !wait_phase(bar(B_KEMPTY + st), (round - 1) & 1, ctl)) return false;
+        if (kt >= kKSt && !wait_bounded_inl(bar(B_KEMPTY + st), (round - 1) & 1, ctl)) return false;
         mbar_expect_tx(bar(B_KFULL + st), kTile);
         const uint32_t dst = sbase + kOffK + st * kTile;
         tma_load_4d(dst, &tmK, bar(B_KFULL + st), 0, j * kBN, kvh, b);
@@ -332,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto load_v = [&](int b, int kvh, int j) -> bool {
         const int st = vt % kVSt, round = vt / kVSt;
-        if (vt >= kVSt && !wait_phase(bar(B_VEMPTY + st), (round - 1) & 1, ctl)) return false;
+        if (vt >= kVSt && !wait_bounded_inl(bar(B_VEMPTY + st), (round - 1) & 1, ctl)) return false;
         mbar_expect_tx(bar(B_VFULL + st), kTile);
         const uint32_t dst = sbase + kOffV + st * kTile;
         tma_load_4d(dst, &tmV, bar(B_VFULL + st), 0, j * kBN, kvh, b);
@@ -345,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int u = sg.pair / a.pairs_per_kv, tl0 = 2 * (sg.pair % a.pairs_per_kv);
         const bool two = pair_has_slot1(a, sg.pair);
         const Tile t0 = tile_of(a, u, tl0);
-        if (si > 0 && !(ok = wait_phase(bar(B_QEMPTY), (si - 1) & 1, ctl))) break;
+        if (si > 0 && !(ok = wait_bounded_inl(bar(B_QEMPTY), (si - 1) & 1, ctl))) break;
         mbar_expect_tx(bar(B_QFULL), a.q_bytes * (two ? 2u : 1u));
         tma_load_4d(sbase + kOffQ, &tmQ, bar(B_QFULL), 0, t0.i0, t0.h0, t0.b);
         tma_load_4d(sbase + kOffQ + kHalf, &tmQ, bar(B_QFULL), 64, t0.i0, t0.h0, t0.b);
@@ -362,12 +386,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) ok = load_v(t0.b, t0.kvh, sg.j1 - 1);
       }
       // let every copy this thread started land before the CTA can exit
-      if (qarm >= 0) wait_phase(bar(B_QFULL), qarm & 1, ctl, true);
+      if (qarm >= 0) wait_bounded_inl(bar(B_QFULL), qarm & 1, ctl, true);
       // (stage st was last armed in round (count - 1 - st) / depth)
       for (int st = 0; st < kKSt; ++st)
-        if (kt > st) wait_phase(bar(B_KFULL + st), ((kt - 1 - st) / kKSt) & 1, ctl, true);
+        if (kt > st) wait_bounded_inl(bar(B_KFULL + st), ((kt - 1 - st) / kKSt) & 1, ctl, true);
       for (int st = 0; st < kVSt; ++st)
-        if (vt > st) wait_phase(bar(B_VFULL + st), ((vt - 1 - st) / kVSt) & 1, ctl, true);
+        if (vt > st) wait_bounded_inl(bar(B_VFULL + st), ((vt - 1 - st) / kVSt) & 1, ctl, true);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
@@ -378,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dV = sw128_desc(sbase + kOffV, kHalf, 1024);
       int kt = 0, vt = 0;
       int pcnt[2] = {0, 0}, segcnt[2] = {0, 0};
-      bool ok = !a.stall || wait_phase(bar(B_STALL), 0, ctl);
+      bool ok = !a.stall || wait_bounded_inl(bar(B_STALL), 0, ctl);
       // S_s = Q_s K^T for the K tile in stage kst
       auto issue_s = [&](int s, int kst) {
         const uint64_t dKs = dK + (uint64_t)((kst * kTile) >> 4);
@@ -405,9 +429,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Seg sg = segs[si];
         const bool two = pair_has_slot1(a, sg.pair);
         const int ns = two ? 2 : 1;
-        if (!(ok = wait_phase(bar(B_QFULL), si & 1, ctl))) break;
+        if (!(ok = wait_bounded_inl(bar(B_QFULL), si & 1, ctl))) break;
         int kst = kt % kKSt;
-        if (!(ok = wait_phase(bar(B_KFULL + kst), (kt / kKSt) & 1, ctl))) break;
+        if (!(ok = wait_bounded_inl(bar(B_KFULL + kst), (kt / kKSt) & 1, ctl))) break;
         tc_fence_after();
         issue_s(0, kst);
         if (ns > 1) issue_s(1, kst);
@@ -421,10 +445,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
             if (s >= ns || !ok) break;
-            ok = wait_phase(bar(B_PFULL + s), pcnt[s] & 1, ctl);
-            if (ok && j == sg.j0 && segcnt[s] > 0) ok = wait_phase(bar(B_OFREE + s), (segcnt[s] - 1) & 1, ctl);
-            if (ok && s == 0) ok = wait_phase(bar(B_VFULL + vst), (vt / kVSt) & 1, ctl);
-            if (ok && s == 0 && more) ok = wait_phase(bar(B_KFULL + kst), (kt / kKSt) & 1, ctl);
+            ok = wait_bounded_inl(bar(B_PFULL + s), pcnt[s] & 1, ctl);
+            if (ok && j == sg.j0 && segcnt[s] > 0) ok = wait_bounded_inl(bar(B_OFREE + s), (segcnt[s] - 1) & 1, ctl);
+            if (ok && s == 0) ok = wait_bounded_inl(bar(B_VFULL + vst), (vt / kVSt) & 1, ctl);
+            if (ok && s == 0 && more) ok = wait_bounded_inl(bar(B_KFULL + kst), (kt / kKSt) & 1, ctl);
             if (!ok) break;
             ++pcnt[s];
             tc_fence_after();
@@ -446,10 +470,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // quiesce this thread's tensor-core work before TMEM is freed
       tc_commit(bar(B_DRAIN));
-      wait_phase(bar(B_DRAIN), 0, ctl, true);
+      wait_bounded_inl(bar(B_DRAIN), 0, ctl, true);
     }
+  }
   } else {
     // ------------------------------------------------------------ softmax
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     const int s = warp >> 2;                 // slot: query tile 0 or 1 of the pair
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
@@ -461,11 +487,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int si = 0; si < nseg && ok; ++si) {
       const Seg sg = segs[si];
       if (s == 1 && !pair_has_slot1(a, sg.pair)) continue;
-      const int u = sg.pair / a.pairs_per_kv, tl0 = 2 * (sg.pair % a.pairs_per_kv);
-      const Tile t = tile_of(a, u, tl0 + s);
       float m = -CUDART_INF_F, l = 0.f;
       for (int j = sg.j0; j < sg.j1; ++j) {
-        ok = uniform(wait_phase(bar(B_SFULL + s), scnt & 1, ctl));
+        ok = uniform(wait_bounded_inl(bar(B_SFULL + s), scnt & 1, ctl));
         if (!ok) break;
         ++scnt;
         tc_fence_after();
@@ -497,14 +521,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           // O_s holds this segment's earlier tiles: PV_s(j-1) has completed
           // (S_s(j), issued after it, has), and PV_s(j) waits for this P
 #pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
-            float o[16];
-            tmem_ld16(tO + c * 16, o);
+          for (int c = 0; c < 16; ++c) {   // 8 columns at a time: few live registers beside the scores
+            uint32_t o[8];
+            tmem_ld8u(tO + c * 8, o);
             tmem_wait_ld();
-            uint32_t ob[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) ob[e] = __float_as_uint(o[e] * alpha);
-            tmem_st16u(tO + c * 16, ob);
+            for (int e = 0; e < 8; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st8u(tO + c * 8, o);
           }
           tmem_wait_st();
         }
@@ -543,10 +566,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // ---- epilogue of the segment: O / l and L of this row ----
-      ok = uniform(wait_phase(bar(B_OREADY + s), ocnt & 1, ctl));
+      ok = uniform(wait_bounded_inl(bar(B_OREADY + s), ocnt & 1, ctl));
       if (!ok) break;
       ++ocnt;
       tc_fence_after();
+      const Tile t = tile_of(a, sg.pair / a.pairs_per_kv, 2 * (sg.pair % a.pairs_per_kv) + s);
       if (a.whole) {
         // merge with the external parts (log space, as the standalone merge)
         // and write this row of O and LSE
@@ -697,6 +721,19 @@ uint64_t wait_limit_ns();
 // Plan of the paired pass over nkeys keys, or false where it does not apply
 // (fewer than two query tiles per KV head, too few key tiles, or more pairs
 // than one CTA can list).
+// The register split of the kernel holds only if every thread is launched
+// with kRegsLaunch registers (checked once per device).
+static bool pair_regs_ok() {
+  static int cache[kMaxDevices] = {};   // 0 unknown, 1 ok, 2 not
+  int& c = cache[current_device()];
+  if (c == 0) {
+    cudaFuncAttributes fa;
+    c = (cudaFuncGetAttributes(&fa, attn_pair_kernel) == cudaSuccess && fa.numRegs == kRegsLaunch) ? 1 : 2;
+    cudaGetLastError();
+  }
+  return c == 1;
+}
+
 bool pair_plan(const fb_attn_desc& d, int64_t nkeys, PairPlan* p) {
   int mode, hg, tpu, units;
   if (nkeys <= 0 || !tc_tiling(d, &mode, &hg, &tpu, &units)) return false;
@@ -709,7 +746,7 @@ bool pair_plan(const fb_attn_desc& d, int64_t nkeys, PairPlan* p) {
   p->pairs_per_kv = (p->tiles_per_kv + 1) / 2;
   p->npairs = d.B * d.Hkv * p->pairs_per_kv;
   p->nkt = (int32_t)((nkeys + kBN - 1) / kBN);
-  if (p->nkt < 4 || p->npairs > kMaxPairs) return false;
+  if (p->nkt < 4 || p->npairs > kMaxPairs || !pair_regs_ok()) return false;
   const int64_t T = (int64_t)p->npairs * p->nkt;
   p->grid = (int32_t)std::min<int64_t>(num_sms(), T);
   // segments per CTA: at most ceil(items per CTA / key tiles) + 1
@@ -798,6 +835,7 @@ cudaError_t launch_attn_pair_fused(const fb_attn_desc& d, const TcMaps& m, const
 // takes whole pairs; up to kMaxSeg pairs per CTA).
 bool pair_plan_whole(const fb_attn_desc& d, int64_t nkeys, PairPlan* p) {
   int mode, hg, tpu, units;
+  if (!pair_regs_ok()) return false;
   if (nkeys <= 0 || !tc_tiling(d, &mode, &hg, &tpu, &units)) return false;
   const int G = d.Hq / d.Hkv;
   p->mode = mode;

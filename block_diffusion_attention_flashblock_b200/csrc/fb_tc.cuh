@@ -50,6 +50,25 @@ static __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, 
   }
 }
 
+// The same bounded wait with the polling loop inlined: for code that keeps
+// many values in registers across the wait (a call would have to save them).
+__device__ __forceinline__ bool wait_bounded_inl(uint32_t bar, uint32_t parity, const Ctl& c,
+                                                 bool draining = false) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t limit = draining ? (c.limit_ns > kDrainLimitNs ? c.limit_ns : kDrainLimitNs) : c.limit_ns;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try(bar, parity)) return true;
+    if (!draining && *c.abort) return false;
+    if (globaltimer() - t0 > limit) {
+      if (atomicExch(const_cast<int*>(c.abort), 1) == 0) atomicCAS(c.status, 0, (int)FB_ETIMEOUT);
+      return false;
+    }
+  }
+}
+
 // Wait for a phase: an inline non-blocking test first (the common case is a
 // phase that already completed), the bounded polling loop only otherwise.
 __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, const Ctl& c, bool draining = false) {
