@@ -477,6 +477,7 @@ def measure_workload(args, spec, rank, world, device, headline):
                    "query_tokens_per_step": S.query_tokens,
                    "prefix_kernel": args.prefix_kernel, "diffusion_steps_per_layer": nsteps,
                    "programmatic_dependent_launch": not args.no_pdl, "inblock_loads": args.inblock_loads,
+                   "inblock_kernel": args.inblock_kernel,
                    "l2": f"flushed (1 GiB write) before every timed step; inside it {nl} layers with their own "
                          f"KV caches are stepped in turn, so each layer's data has left L2 when it runs",
                    "parallelism": f"replicas x{world}", "full_steps_per_layer": n_full},
@@ -498,6 +499,7 @@ def run_ours(args, spec, rank, world, device):
                                    "tcgen05-cluster": 4}[args.prefix_kernel])
     fb.fb_debug_set_pdl(not args.no_pdl)
     fb.fb_debug_set_inblock_loads(args.inblock_loads == "bulk")
+    fb.fb_debug_set_inblock_kernel(1 if args.inblock_kernel == "paired" else 0)
     r = measure_workload(args, spec, rank, world, device, headline=True)
     out = {
         "metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -634,6 +636,8 @@ def main():
     ap.add_argument("--no-pdl", action="store_true", help="launch kernels in plain stream order")
     ap.add_argument("--inblock-loads", default="cpasync", choices=["cpasync", "bulk"],
                     help="how the small in-block kernel loads its rows")
+    ap.add_argument("--inblock-kernel", default="auto", choices=["auto", "paired"],
+                    help="the kernel of block-internal passes")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--prefix-kernel", default="auto", choices=["auto", "generic", "tcgen05", "tcgen05-nocluster", "tcgen05-cluster"])
     ap.add_argument("--kernels-only", type=int, default=0, metavar="N",

@@ -26,6 +26,7 @@ static bool g_stall = false;
 bool debug_stall() { return g_stall; }
 static bool g_inblock_bulk = false;
 bool inblock_bulk_loads() { return g_inblock_bulk; }
+static int g_inblock_kernel = 0;   // 0 automatic, 1 the paired tcgen05 kernel wherever it applies
 
 // Device address of this device's status word, looked up once per device (the
 // first launch on a device should come before any stream capture on it; a
@@ -471,7 +472,11 @@ static fb_status run_inblock(const fb_attn_desc& d, const void* q, const void* k
   const double bytes = (double)rows_of(d) * d.D * es + 2.0 * d.B * d.Hkv * d.Nb * d.D * es +
                        ext_parts * rows_of(d) * (d.D + 1) * 4.0 +
                        (double)rows_of(d) * (d.D * esize(d.out_dtype) + (lse ? 4 : 0));
-  if (inblock_small_applies(d, nflat)) {
+  TcMaps maps;
+  PairPlan pw;
+  const bool pair_ok = (g_prefix_kernel == 0 || g_prefix_kernel == 2) && nflat <= FB_MAX_PARTS - 1 && !cache_a &&
+                       tc_make_maps(d, q, kin, vin, d.Nb, d.kin_strides, &maps) && pair_plan_whole(d, d.Nb, &pw);
+  if (inblock_small_applies(d, nflat) && !(g_inblock_kernel == 1 && pair_ok)) {
     ProfScope prof(kProfInblock, bytes, s);
     return launch_inblock_small(d, q, kin, vin, nflat, fa, fl, o, lse, cache_a, cache_l, a.scale_log2, s) ==
                    cudaSuccess
@@ -480,10 +485,7 @@ static fb_status run_inblock(const fb_attn_desc& d, const void* q, const void* k
   }
   if (nflat > FB_MAX_PARTS) return FB_EINVAL;
   if (cache_a) return FB_EUNSUPPORTED;   // callers only ask for the cache write where the small kernel runs
-  TcMaps maps;
-  PairPlan pw;
-  if ((g_prefix_kernel == 0 || g_prefix_kernel == 2) && nflat <= FB_MAX_PARTS - 1 &&
-      tc_make_maps(d, q, kin, vin, d.Nb, d.kin_strides, &maps) && pair_plan_whole(d, d.Nb, &pw)) {
+  if (pair_ok) {
     // large blocks: one launch of the paired kernel over the block's own keys,
     // merged with the external parts in its epilogue
     ProfScope prof(kProfInblock, bytes, s);
@@ -774,6 +776,12 @@ fb_status fb_debug_set_prefix_kernel(int32_t which) {
 
 fb_status fb_debug_set_stall(int32_t on) {
   g_stall = on != 0;
+  return FB_OK;
+}
+
+fb_status fb_debug_set_inblock_kernel(int32_t which) {
+  if (which < 0 || which > 1) return FB_EINVAL;
+  g_inblock_kernel = which;
   return FB_OK;
 }
 

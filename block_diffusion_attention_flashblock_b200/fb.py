@@ -76,6 +76,7 @@ _SIGS = {
     "fb_debug_set_wait_limit_ns": (C.c_int, [C.c_uint64]),
     "fb_debug_set_pdl": (C.c_int, [C.c_int32]),
     "fb_debug_set_inblock_loads": (C.c_int, [C.c_int32]),
+    "fb_debug_set_inblock_kernel": (C.c_int, [C.c_int32]),
     "fb_debug_set_stall": (C.c_int, [C.c_int32]),
     "fb_profile_enable": (C.c_int, [C.c_int32]),
     "fb_debug_set_prefix_kernel": (C.c_int, [C.c_int32]),
@@ -291,6 +292,10 @@ def fb_debug_set_wait_limit_ns(ns: int):
 
 def fb_debug_set_pdl(on: bool):
     _check(lib().fb_debug_set_pdl(1 if on else 0), "fb_debug_set_pdl")
+
+
+def fb_debug_set_inblock_kernel(which: int):
+    _check(lib().fb_debug_set_inblock_kernel(which), "fb_debug_set_inblock_kernel")
 
 
 def fb_debug_set_inblock_loads(bulk: bool):

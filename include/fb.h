@@ -334,6 +334,13 @@ fb_status fb_debug_set_wait_limit_ns(uint64_t ns);
  * it returns).  Off by default.  Affects only the calling process. */
 fb_status fb_debug_set_stall(int32_t on);
 
+/* Tuning hook: which kernel runs block-internal passes: 0 (default)
+ * automatic (the small mma.sync kernel for blocks of up to 64 keys, the
+ * paired tcgen05 kernel above), 1 the paired tcgen05 kernel wherever it
+ * applies (two or more 128-row query tiles per KV head).  Affects only the
+ * calling process. */
+fb_status fb_debug_set_inblock_kernel(int32_t which);
+
 /* Tuning hook: how the small-block in-block kernel loads its rows: 0
  * (default) 16-byte cp.async chunks from every thread, 1 one bulk copy per
  * row.  Affects only the calling process. */
