@@ -82,8 +82,25 @@ constexpr float kRescaleLog2 = 8.0f;
 
 enum {
   B_QFULL = 0, B_QEMPTY = 1, B_KFULL = 2, B_KEMPTY = 5, B_VFULL = 8, B_VEMPTY = 10, B_SFULL = 12, B_PFULL = 14,
-  B_OREADY = 16, B_OFREE = 18, B_DRAIN = 20, B_STALL = 21, B_COUNT = 22
+  B_OREADY = 16, B_OFREE = 18, B_DRAIN = 20, B_STALL = 21, B_VCONV = 22, B_COUNT = 24
 };
+// after the barriers: abort flag, TMEM base, segment count, the V stages'
+// formats (1: converted to fp16), the converter's reduction words
+constexpr uint32_t kOffAbort = B_COUNT * 8, kOffTmem = kOffAbort + 4, kOffNseg = kOffTmem + 4,
+                   kOffVmode = kOffNseg + 4, kOffRed = kOffVmode + 4 * kVSt, kOffCtlEnd = kOffRed + 12;
+static_assert(kOffCtlEnd <= 256, "control block");
+
+// P V in fp16: A (P, in TMEM) and B (V, MN-major) fp16, D fp32, M = N = 128
+constexpr uint32_t kIdescPV16 = (1u << 4) | (1u << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+
+// fp16 pair from two floats (lo in the low half)
+__device__ __forceinline__ uint32_t f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// CTA-partial barrier of the two converter warps
+__device__ __forceinline__ void conv_sync() { asm volatile("bar.sync 1, 64;" ::: "memory"); }
 
 __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* v) {
   asm volatile(
@@ -225,9 +242,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const uint32_t sbase = smem_addr(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffBar + B_COUNT * 8);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBar + B_COUNT * 8 + 4);
-  int* nseg_sh = reinterpret_cast<int*>(smem + kOffBar + B_COUNT * 8 + 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffBar + kOffAbort);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBar + kOffTmem);
+  int* nseg_sh = reinterpret_cast<int*>(smem + kOffBar + kOffNseg);
+  volatile int* vmode = reinterpret_cast<volatile int*>(smem + kOffBar + kOffVmode);
+  volatile uint32_t* red = reinterpret_cast<volatile uint32_t*>(smem + kOffBar + kOffRed);
   Seg* segs = reinterpret_cast<Seg*>(smem + kOffSeg);
   uint32_t* act = reinterpret_cast<uint32_t*>(smem + kOffAct);
   auto bar = [&](int i) { return smem_addr(bars + i); };
@@ -414,10 +433,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_commit(bar(B_SFULL + s));
       };
-      // O_s += P_hi V + P_lo V for the V tile in stage vst
-      auto issue_pv = [&](int s, int vst, bool first) {
+      // O_s += P V for the V tile in stage vst: one pass in fp16 where the
+      // converter turned the tile into fp16, else P_hi V + P_lo V in bf16
+      auto issue_pv = [&](int s, int vst, bool first, bool f16) {
         const uint64_t dVs = dV + (uint64_t)((vst * kTile) >> 4);
         const uint32_t pt = tmem + s * kBN;
+        if (f16) {
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            tc_mma_ts(tmem + kTmemO + s * kBN, pt + kk * 8, dVs + (uint64_t)((kk * 2048) >> 4), kIdescPV16,
+                      (!first || kk > 0) ? 1u : 0u);
+          return;
+        }
 #pragma unroll
         for (int part = 0; part < 2; ++part)
 #pragma unroll
@@ -441,18 +468,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = sg.j0; j < sg.j1 && ok; ++j) {
           const int vst = vt % kVSt;
           const bool more = j + 1 < sg.j1;
+          bool vf16 = false;
           kst = kt % kKSt;
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
             if (s >= ns || !ok) break;
             ok = wait_bounded_inl(bar(B_PFULL + s), pcnt[s] & 1, ctl);
             if (ok && j == sg.j0 && segcnt[s] > 0) ok = wait_bounded_inl(bar(B_OFREE + s), (segcnt[s] - 1) & 1, ctl);
-            if (ok && s == 0) ok = wait_bounded_inl(bar(B_VFULL + vst), (vt / kVSt) & 1, ctl);
+            if (ok && s == 0) {
+              ok = wait_bounded_inl(bar(B_VCONV + vst), (vt / kVSt) & 1, ctl);
+              vf16 = vmode[vst] != 0;
+            }
             if (ok && s == 0 && more) ok = wait_bounded_inl(bar(B_KFULL + kst), (kt / kKSt) & 1, ctl);
             if (!ok) break;
             ++pcnt[s];
             tc_fence_after();
-            issue_pv(s, vst, j == sg.j0);
+            issue_pv(s, vst, j == sg.j0, vf16);
             if (more) issue_s(s, kst);
             if (!more) tc_commit(bar(B_OREADY + s));
           }
@@ -472,6 +503,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(bar(B_DRAIN));
       wait_bounded_inl(bar(B_DRAIN), 0, ctl, true);
     }
+  } else if (nseg > 0) {
+    // ------------------------------------------------------------ converter
+    // Warps 10 and 11 turn each landed V tile into fp16 in place when every
+    // value converts exactly or negligibly: the tile's largest |v| has a
+    // binary exponent in [-4, 15] (below 2^16 nothing overflows; values
+    // under fp16's 2^-14 lose at most 2^-25, under 2^-21 of the tile's
+    // largest), and publish the tile's format with the VCONV barrier.  Any
+    // other tile (huge, tiny, NaN or inf values) stays bf16 and takes the
+    // hi/lo P V.  Thread 0 alone waits on mbarriers and broadcasts the
+    // outcome, so the two warps always meet at their barrier.
+    const int ct = threadIdx.x - 320;   // 0..63
+    int vt = 0;
+    bool ok = true;
+    for (int si = 0; si < nseg && ok; ++si) {
+      const Seg sg = segs[si];
+      for (int j = sg.j0; j < sg.j1; ++j, ++vt) {
+        const int st = vt % kVSt;
+        if (ct == 0) red[2] = wait_bounded_inl(bar(B_VFULL + st), (vt / kVSt) & 1, ctl) ? 1u : 0u;
+        conv_sync();
+        ok = red[2] != 0;
+        if (!ok) break;
+        uint4* tile = reinterpret_cast<uint4*>(smem + kOffV + st * kTile);
+        uint32_t mx = 0u;
+#pragma unroll 4
+        for (int i = 0; i < 32; ++i) {
+          const uint4 v = tile[ct + 64 * i];
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) mx = max(mx, max(w[e] & 0x7FFFu, (w[e] >> 16) & 0x7FFFu));
+        }
+        mx = __reduce_max_sync(0xffffffffu, mx);
+        if (lane == 0) red[warp - 10] = mx;
+        conv_sync();
+        mx = max(red[0], red[1]);
+        const int e2 = (int)(mx >> 7) - 127;   // binary exponent of the largest |v|
+        const bool f16 = mx == 0u || (mx < 0x7F80u && e2 >= -4 && e2 <= 15);
+        if (f16) {
+#pragma unroll 4
+          for (int i = 0; i < 32; ++i) {
+            const uint4 v = tile[ct + 64 * i];
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint32_t h[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) h[e] = f16x2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
+            tile[ct + 64 * i] = make_uint4(h[0], h[1], h[2], h[3]);
+          }
+          ptx::fence_proxy_async_smem();   // the tensor core reads the tile through the async proxy
+        }
+        conv_sync();
+        if (ct == 0) {
+          vmode[st] = f16 ? 1 : 0;
+          mbar_arrive(bar(B_VCONV + st));
+        }
+      }
+    }
   }
   } else {
     // ------------------------------------------------------------ softmax
@@ -484,9 +570,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     int scnt = 0, ocnt = 0;
     bool ok = true;
     auto uniform = [](bool v) { return __all_sync(0xffffffffu, v); };
+    int vtc = 0;   // V tiles of every segment so far (slot 1 counts the lone-tile segments it skips)
     for (int si = 0; si < nseg && ok; ++si) {
       const Seg sg = segs[si];
-      if (s == 1 && !pair_has_slot1(a, sg.pair)) continue;
+      if (s == 1 && !pair_has_slot1(a, sg.pair)) {
+        vtc += sg.j1 - sg.j0;
+        continue;
+      }
       float m = -CUDART_INF_F, l = 0.f;
       for (int j = sg.j0; j < sg.j1; ++j) {
         ok = uniform(wait_bounded_inl(bar(B_SFULL + s), scnt & 1, ctl));
@@ -537,6 +627,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float nref = m == -CUDART_INF_F ? 0.f : -m;
         float sum[4] = {0.f, 0.f, 0.f, 0.f};
+        // the format of this tile's V (fp16, or bf16 for the hi/lo P V)
+        ok = uniform(wait_bounded_inl(bar(B_VCONV + vtc % kVSt), (vtc / kVSt) & 1, ctl));
+        if (!ok) break;
+        const bool vf16 = vmode[vtc % kVSt] != 0;
+        ++vtc;
+        if (vf16) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {   // 32 keys: 16 fp16 pairs at 16c
+            uint32_t hw[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float p0 = fast_exp2(fmaf(sv[32 * c + 2 * e], a.scale_log2, nref));
+              const float p1 = fast_exp2(fmaf(sv[32 * c + 2 * e + 1], a.scale_log2, nref));
+              sum[e & 3] += p0 + p1;
+              hw[e] = f16x2(p0, p1);
+            }
+            tmem_st16u(tS + 16 * c, hw);
+          }
+        } else
 #pragma unroll
         for (int c = 0; c < 4; ++c) {   // 32 keys: 16 hi words at 16c, 16 lo words at 64 + 16c
           // the hi and lo words take the registers of the two scores they replace

@@ -116,6 +116,35 @@ def test_outblock_dense_paired(shape, prefix_kernel):
     _outblock_check(shape, seed=17)
 
 
+@pytest.mark.parametrize("v_scale", [2.0 ** 17, 2.0 ** -10, 2.0 ** 12, 2.0 ** -3, "mixed"],
+                         ids=["huge", "tiny", "fp16-top", "fp16-bottom", "mixed"])
+def test_outblock_paired_v_ranges(v_scale, prefix_kernel):
+    """The paired kernel runs P V in fp16 on V tiles whose largest |v| has a
+    binary exponent in [-4, 15] and in bf16 hi/lo on any other tile; values
+    scaled out of that window (huge, tiny) take the bf16 path, values at its
+    edges the fp16 one, and a prefix whose first tiles are huge mixes both
+    within one accumulation."""
+    prefix_kernel(fb.PREFIX_TC)
+    B, Hq, Hkv, D, Nb, Lp = 1, 8, 2, 128, 64, 2000
+    q, kin, vin, kp, vp = _mk(B, Hq, Hkv, D, Nb, Lp, "bf16", seed=19)
+    vf = vp.float()
+    if v_scale == "mixed":
+        vf[:, :, :512] *= 2.0 ** 17
+    else:
+        vf *= v_scale
+    vp = vf.to(torch.bfloat16)
+    qd, kpd, vpd = q.cuda(), kp.cuda(), vp.cuda()
+    a = torch.full((B, Hq, Nb, D), float("nan"), device="cuda")
+    l = torch.full((B, Hq, Nb), float("nan"), device="cuda")
+    desc = fb.make_desc(qd, kin.cuda(), kpd, a)
+    ws = torch.empty(fb.fb_outblock_workspace_bytes(desc, Lp), dtype=torch.uint8, device="cuda")
+    fb.fb_attn_outblock(desc, qd, kpd, vpd, Lp, a, l, ws)
+    assert fb.fb_get_device_status() == fb.FB_OK
+    A, L = orc.outblock(orc.to64(q), orc.to64(kp), orc.to64(vp), Lp, 1 / np.sqrt(D))
+    assert_o_close(a, A, TOL["bf16"], "A_out")
+    assert_lse_close(l, L, TOL["bf16"], "L_out")
+
+
 @pytest.mark.parametrize("which", ["generic", "tcgen05", "tcgen05-cluster", "paired"])
 def test_outblock_rising_and_falling_scores(which, prefix_kernel):
     """Scores that grow along the prefix (KV head 0) force the running max to
