@@ -19,11 +19,11 @@
 //   warps 0..3  softmax of query tile 0 (slot 0), one thread per query row
 //   warps 4..7  softmax of query tile 1 (slot 1)
 //   warp 8      TMA producer, no multicast: the pair's Q tiles, then K and V
-//               tiles of 128 keys into a three-stage K ring and a two-stage
-//               V ring (128-byte swizzle), K one tile ahead of V
+//               tiles of 128 keys into a two-stage K ring and a three-stage
+//               V ring (128-byte swizzle)
 //   warp 9      allocates TMEM; one thread issues every tcgen05.mma
-//   warps 10,11 idle (they complete the third warpgroup, whose registers
-//               go to the softmax warpgroups)
+//   warps 10,11 convert each landed V tile to fp16 in place where that is
+//               exact (see the converter below), so P V runs in one pass
 // TMEM: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).  Softmax s
 // reads its row of S_s, writes P = 2^(s - m) over the same columns as bf16
 // hi (columns 0..63) and lo (64..127) parts, and the issuer runs
@@ -62,7 +62,7 @@ constexpr int kThreads = 384;                    // three warpgroups
 // kernel's launch register count before the first launch.
 constexpr int kRegsLaunch = 168, kRegsIO = 120, kRegsSoftmax = 192;
 static_assert(4 * 32 * kRegsIO + 8 * 32 * kRegsSoftmax == kThreads * kRegsLaunch, "register split");
-constexpr int kKSt = 3, kVSt = 2;                 // K and V ring depths
+constexpr int kKSt = 2, kVSt = 3;                 // K and V ring depths (V is converted after it lands)
 constexpr uint32_t kHalf = 16384;                 // [128 rows][64 bf16], 128-byte swizzle
 constexpr uint32_t kTile = 2 * kHalf;             // one 128 x 128 bf16 tile
 constexpr uint32_t kOffQ = 0;                     // Q0, Q1
@@ -80,9 +80,22 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 256;
 constexpr float kRescaleLog2 = 8.0f;
 
+// barrier slots, laid out from the ring depths
 enum {
-  B_QFULL = 0, B_QEMPTY = 1, B_KFULL = 2, B_KEMPTY = 5, B_VFULL = 8, B_VEMPTY = 10, B_SFULL = 12, B_PFULL = 14,
-  B_OREADY = 16, B_OFREE = 18, B_DRAIN = 20, B_STALL = 21, B_VCONV = 22, B_COUNT = 24
+  B_QFULL = 0,
+  B_QEMPTY = 1,
+  B_KFULL = 2,
+  B_KEMPTY = B_KFULL + kKSt,
+  B_VFULL = B_KEMPTY + kKSt,
+  B_VEMPTY = B_VFULL + kVSt,
+  B_VCONV = B_VEMPTY + kVSt,
+  B_SFULL = B_VCONV + kVSt,
+  B_PFULL = B_SFULL + 2,
+  B_OREADY = B_PFULL + 2,
+  B_OFREE = B_OREADY + 2,
+  B_DRAIN = B_OFREE + 2,
+  B_STALL = B_DRAIN + 1,
+  B_COUNT = B_STALL + 1
 };
 // after the barriers: abort flag, TMEM base, segment count, the V stages'
 // formats (1: converted to fp16), the converter's reduction words
@@ -400,9 +413,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         qarm = si;
         for (int j = sg.j0; j < sg.j1 && ok; ++j) {
           ok = load_k(t0.b, t0.kvh, j);
-          if (ok && j > sg.j0) ok = load_v(t0.b, t0.kvh, j - 1);
+          if (ok) ok = load_v(t0.b, t0.kvh, j);
         }
-        if (ok) ok = load_v(t0.b, t0.kvh, sg.j1 - 1);
       }
       // let every copy this thread started land before the CTA can exit
       if (qarm >= 0) wait_bounded_inl(bar(B_QFULL), qarm & 1, ctl, true);
