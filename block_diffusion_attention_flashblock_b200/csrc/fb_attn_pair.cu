@@ -15,7 +15,8 @@
 // combines the slots in log space.  With the gamma gate, pairs whose heads
 // all reuse their cache are left out of the item space on the device.
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads; the softmax warpgroups run with 192 registers a
+// thread, the other warps with 120):
 //   warps 0..3  softmax of query tile 0 (slot 0), one thread per query row
 //   warps 4..7  softmax of query tile 1 (slot 1)
 //   warp 8      TMA producer, no multicast: the pair's Q tiles, then K and V
@@ -25,9 +26,13 @@
 //   warps 10,11 convert each landed V tile to fp16 in place where that is
 //               exact (see the converter below), so P V runs in one pass
 // TMEM: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).  Softmax s
-// reads its row of S_s, writes P = 2^(s - m) over the same columns as bf16
-// hi (columns 0..63) and lo (64..127) parts, and the issuer runs
-// O_s += P_hi V + P_lo V.  The issuer orders the tensor core as
+// reads its row of S_s and writes P = 2^(s - m) over the same columns: as
+// fp16 (columns 0..63) where V_j is fp16, and the issuer runs O_s += P V in
+// one pass; else as bf16 hi (columns 0..63) and lo (64..127) parts, and the
+// issuer runs O_s += P_hi V + P_lo V.  The scaling of the scores and the row
+// sums take two lanes per instruction (f32x2), the exponentials the MUFU
+// unit; V_j's format is read before S_j lands, off the softmax's critical
+// path.  The issuer orders the tensor core as
 //   S0(j) S1(j) | PV0(j) S0(j+1) PV1(j) S1(j+1) | PV0(j+1) ...
 // so while one softmax group works on its tile the tensor core runs the other
 // group's P V and next S.  S_s(j+1) overwrites P_s(j) only after PV_s(j) has
@@ -69,7 +74,8 @@ constexpr uint32_t kOffQ = 0;                     // Q0, Q1
 constexpr uint32_t kOffK = 2 * kTile;
 constexpr uint32_t kOffV = kOffK + kKSt * kTile;
 constexpr uint32_t kOffBar = kOffV + kVSt * kTile;
-constexpr uint32_t kOffSeg = kOffBar + 256;       // segment list
+constexpr uint32_t kBarBytes = 384;               // barriers and control words
+constexpr uint32_t kOffSeg = kOffBar + kBarBytes;  // segment list
 constexpr int kMaxSeg = 32;
 constexpr uint32_t kOffAct = kOffSeg + kMaxSeg * 16;   // active-pair bitmap
 constexpr int kMaxPairs = 2048;
@@ -95,13 +101,14 @@ enum {
   B_OFREE = B_OREADY + 2,
   B_DRAIN = B_OFREE + 2,
   B_STALL = B_DRAIN + 1,
-  B_COUNT = B_STALL + 1
+  B_VRELOAD = B_STALL + 1,   // the converter fetches a tile's bf16 values again
+  B_COUNT = B_VRELOAD + 1
 };
 // after the barriers: abort flag, TMEM base, segment count, the V stages'
 // formats (1: converted to fp16), the converter's reduction words
 constexpr uint32_t kOffAbort = B_COUNT * 8, kOffTmem = kOffAbort + 4, kOffNseg = kOffTmem + 4,
                    kOffVmode = kOffNseg + 4, kOffRed = kOffVmode + 4 * kVSt, kOffCtlEnd = kOffRed + 12;
-static_assert(kOffCtlEnd <= 256, "control block");
+static_assert(kOffCtlEnd <= kBarBytes, "control block");
 
 // P V in fp16: A (P, in TMEM) and B (V, MN-major) fp16, D fp32, M = N = 128
 constexpr uint32_t kIdescPV16 = (1u << 4) | (1u << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
@@ -276,7 +283,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < B_COUNT; ++i) {
       uint32_t cnt = 1;
-      if ((i >= B_PFULL && i < B_PFULL + 2) || (i >= B_OFREE && i < B_OFREE + 2)) cnt = 128;
+      if (i >= B_PFULL && i < B_PFULL + 2) cnt = 4;   // one arrival per softmax warp
+      if (i >= B_OFREE && i < B_OFREE + 2) cnt = 128;
       mbar_init(bar(i), cnt);
     }
     *abort_flag = 0;
@@ -458,11 +466,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           return;
         }
 #pragma unroll
-        for (int part = 0; part < 2; ++part)
+        for (int hl = 0; hl < 2; ++hl)
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk)
-            tc_mma_ts(tmem + kTmemO + s * kBN, pt + part * 64 + kk * 8, dVs + (uint64_t)((kk * 2048) >> 4),
-                      kIdescPV, (!first || part > 0 || kk > 0) ? 1u : 0u);
+            tc_mma_ts(tmem + kTmemO + s * kBN, pt + hl * 64 + kk * 8, dVs + (uint64_t)((kk * 2048) >> 4),
+                      kIdescPV, (!first || hl > 0 || kk > 0) ? 1u : 0u);
       };
       for (int si = 0; si < nseg && ok; ++si) {
         const Seg sg = segs[si];
@@ -517,16 +525,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (nseg > 0) {
     // ------------------------------------------------------------ converter
-    // Warps 10 and 11 turn each landed V tile into fp16 in place when every
-    // value converts exactly or negligibly: the tile's largest |v| has a
-    // binary exponent in [-4, 15] (below 2^16 nothing overflows; values
-    // under fp16's 2^-14 lose at most 2^-25, under 2^-21 of the tile's
-    // largest), and publish the tile's format with the VCONV barrier.  Any
-    // other tile (huge, tiny, NaN or inf values) stays bf16 and takes the
-    // hi/lo P V.  Thread 0 alone waits on mbarriers and broadcasts the
+    // Warps 10 and 11 turn each landed V tile into fp16 in place, in one
+    // pass that also finds the tile's largest |v|.  The fp16 tile stands when
+    // every value converted exactly or negligibly: that largest |v| has a
+    // binary exponent in [-4, 15] (below 2^16 nothing overflows; values under
+    // fp16's 2^-14 lose at most 2^-25, under 2^-21 of the tile's largest).
+    // Any other tile (huge, tiny, NaN or inf values) is fetched again in
+    // bf16 and takes the hi/lo P V.  The tile's format goes out with the
+    // VCONV barrier.  Thread 0 alone waits on mbarriers and broadcasts the
     // outcome, so the two warps always meet at their barrier.
     const int ct = threadIdx.x - 320;   // 0..63
-    int vt = 0;
+    int vt = 0, nreload = 0;
     bool ok = true;
     for (int si = 0; si < nseg && ok; ++si) {
       const Seg sg = segs[si];
@@ -536,35 +545,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         conv_sync();
         ok = red[2] != 0;
         if (!ok) break;
+        // one pass: convert every value and track the largest |v|; a tile
+        // that did not convert exactly is fetched again in bf16 below
         uint4* tile = reinterpret_cast<uint4*>(smem + kOffV + st * kTile);
         uint32_t mx = 0u;
 #pragma unroll 4
         for (int i = 0; i < 32; ++i) {
           const uint4 v = tile[ct + 64 * i];
           const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+          uint32_t h[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) mx = max(mx, max(w[e] & 0x7FFFu, (w[e] >> 16) & 0x7FFFu));
+          for (int e = 0; e < 4; ++e) {
+            mx = max(mx, max(w[e] & 0x7FFFu, (w[e] >> 16) & 0x7FFFu));
+            h[e] = f16x2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
+          }
+          tile[ct + 64 * i] = make_uint4(h[0], h[1], h[2], h[3]);
         }
+        ptx::fence_proxy_async_smem();   // the tensor core (or a refetch) reaches the tile through the async proxy
         mx = __reduce_max_sync(0xffffffffu, mx);
         if (lane == 0) red[warp - 10] = mx;
         conv_sync();
         mx = max(red[0], red[1]);
         const int e2 = (int)(mx >> 7) - 127;   // binary exponent of the largest |v|
         const bool f16 = mx == 0u || (mx < 0x7F80u && e2 >= -4 && e2 <= 15);
-        if (f16) {
-#pragma unroll 4
-          for (int i = 0; i < 32; ++i) {
-            const uint4 v = tile[ct + 64 * i];
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            uint32_t h[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) h[e] = f16x2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
-            tile[ct + 64 * i] = make_uint4(h[0], h[1], h[2], h[3]);
-          }
-          ptx::fence_proxy_async_smem();   // the tensor core reads the tile through the async proxy
-        }
         conv_sync();
         if (ct == 0) {
+          if (!f16) {
+            const Tile tv = tile_of(a, sg.pair / a.pairs_per_kv, 2 * (sg.pair % a.pairs_per_kv));
+            const uint32_t dst = sbase + kOffV + st * kTile;
+            mbar_expect_tx(bar(B_VRELOAD), kTile);
+            tma_load_4d(dst, &tmV, bar(B_VRELOAD), 0, j * kBN, tv.kvh, tv.b);
+            tma_load_4d(dst + kHalf, &tmV, bar(B_VRELOAD), 64, j * kBN, tv.kvh, tv.b);
+            // the refetch lands whatever happens elsewhere (a draining wait)
+            wait_bounded_inl(bar(B_VRELOAD), nreload & 1, ctl, true);
+            ++nreload;
+          }
           vmode[st] = f16 ? 1 : 0;
           mbar_arrive(bar(B_VCONV + st));
         }
@@ -583,15 +598,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     auto uniform = [](bool v) { return __all_sync(0xffffffffu, v); };
     int vtc = 0;   // V tiles of every segment so far (slot 1 counts the lone-tile segments it skips)
+    bool skipped = false;
+    // the format of this tile's V (fp16, or bf16 for the hi/lo P V)
+    auto v_format = [&](bool& f16) -> bool {
+      if (!uniform(wait_bounded_inl(bar(B_VCONV + vtc % kVSt), (vtc / kVSt) & 1, ctl))) return false;
+      f16 = vmode[vtc % kVSt] != 0;
+      ++vtc;
+      return true;
+    };
     for (int si = 0; si < nseg && ok; ++si) {
       const Seg sg = segs[si];
       if (s == 1 && !pair_has_slot1(a, sg.pair)) {
         vtc += sg.j1 - sg.j0;
+        skipped = true;
         continue;
       }
       float m = -CUDART_INF_F, l = 0.f;
       for (int j = sg.j0; j < sg.j1; ++j) {
+        // V_j lands with K_j, so the format is normally known long before S_j
+        // and its wait comes first, off the chain S_j -> P_j.  A parity wait
+        // is only sound within one phase of the converter, which holds once
+        // this slot has had the tile before (S_s(j - 1) was issued after a P V
+        // that waited for the format of tile j - 2); after slot 1 skipped
+        // lone-tile segments, the first tile's format is read after S_j
+        // instead (S_j was issued after the skipped tiles' P V).
+        const bool late = skipped && j == sg.j0;
+        bool vf16 = false;
+        if (!late && !(ok = v_format(vf16))) break;
         ok = uniform(wait_bounded_inl(bar(B_SFULL + s), scnt & 1, ctl));
+        if (ok && late) ok = v_format(vf16);
+        skipped = false;
         if (!ok) break;
         ++scnt;
         tc_fence_after();
@@ -627,8 +663,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t o[8];
             tmem_ld8u(tO + c * 8, o);
             tmem_wait_ld();
+            const uint64_t al2 = pack2(alpha, alpha);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            for (int e = 0; e < 8; e += 2) {
+              float lo, hi;
+              unpack2(fmul2(pack2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), al2), lo, hi);
+              o[e] = __float_as_uint(lo);
+              o[e + 1] = __float_as_uint(hi);
+            }
             tmem_st8u(tO + c * 8, o);
           }
           tmem_wait_st();
@@ -638,21 +680,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = tmax;
         }
         const float nref = m == -CUDART_INF_F ? 0.f : -m;
-        float sum[4] = {0.f, 0.f, 0.f, 0.f};
-        // the format of this tile's V (fp16, or bf16 for the hi/lo P V)
-        ok = uniform(wait_bounded_inl(bar(B_VCONV + vtc % kVSt), (vtc / kVSt) & 1, ctl));
-        if (!ok) break;
-        const bool vf16 = vmode[vtc % kVSt] != 0;
-        ++vtc;
+        // x = s * scale - m and the row sum two lanes per instruction
+        const uint64_t sc2 = pack2(a.scale_log2, a.scale_log2), nr2 = pack2(nref, nref);
+        uint64_t acc[2] = {0ull, 0ull};   // +0.0f pairs
         if (vf16) {
 #pragma unroll
           for (int c = 0; c < 4; ++c) {   // 32 keys: 16 fp16 pairs at 16c
             uint32_t hw[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const float p0 = fast_exp2(fmaf(sv[32 * c + 2 * e], a.scale_log2, nref));
-              const float p1 = fast_exp2(fmaf(sv[32 * c + 2 * e + 1], a.scale_log2, nref));
-              sum[e & 3] += p0 + p1;
+              float x0, x1;
+              unpack2(ffma2(pack2(sv[32 * c + 2 * e], sv[32 * c + 2 * e + 1]), sc2, nr2), x0, x1);
+              const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+              acc[e & 1] = fadd2(acc[e & 1], pack2(p0, p1));
               hw[e] = f16x2(p0, p1);
             }
             tmem_st16u(tS + 16 * c, hw);
@@ -663,9 +703,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           // the hi and lo words take the registers of the two scores they replace
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = fast_exp2(fmaf(sv[32 * c + 2 * e], a.scale_log2, nref));
-            const float p1 = fast_exp2(fmaf(sv[32 * c + 2 * e + 1], a.scale_log2, nref));
-            sum[e & 3] += p0 + p1;
+            float x0, x1;
+            unpack2(ffma2(pack2(sv[32 * c + 2 * e], sv[32 * c + 2 * e + 1]), sc2, nr2), x0, x1);
+            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            acc[e & 1] = fadd2(acc[e & 1], pack2(p0, p1));
             uint32_t h, lw;
             split_pair(p0, p1, h, lw);
             sv[32 * c + 2 * e] = __uint_as_float(h);
@@ -680,10 +721,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st16u(tS + 16 * c, hi);
           tmem_st16u(tS + 64 + 16 * c, lo);
         }
-        l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
+        {
+          float s0, s1, s2, s3;
+          unpack2(acc[0], s0, s1);
+          unpack2(acc[1], s2, s3);
+          l += (s0 + s1) + (s2 + s3);
+        }
+        // P_s is in TMEM: one arrival per warp
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(B_PFULL + s));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_PFULL + s));
       }
       if (!ok) break;
       // ---- epilogue of the segment: O / l and L of this row ----
