@@ -488,18 +488,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = sg.j0; j < sg.j1 && ok; ++j) {
           const int vst = vt % kVSt;
           const bool more = j + 1 < sg.j1;
-          bool vf16 = false;
           kst = kt % kKSt;
+          // V_j's format and K_(j+1) depend only on earlier tiles and are
+          // normally ready long before P_0(j): waiting for them first keeps
+          // these waits off the chain P_s(j) -> P V(j) -> S_s(j+1)
+          if (!(ok = wait_bounded_inl(bar(B_VCONV + vst), (vt / kVSt) & 1, ctl))) break;
+          const bool vf16 = vmode[vst] != 0;
+          if (more && !(ok = wait_bounded_inl(bar(B_KFULL + kst), (kt / kKSt) & 1, ctl))) break;
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
             if (s >= ns || !ok) break;
             ok = wait_bounded_inl(bar(B_PFULL + s), pcnt[s] & 1, ctl);
             if (ok && j == sg.j0 && segcnt[s] > 0) ok = wait_bounded_inl(bar(B_OFREE + s), (segcnt[s] - 1) & 1, ctl);
-            if (ok && s == 0) {
-              ok = wait_bounded_inl(bar(B_VCONV + vst), (vt / kVSt) & 1, ctl);
-              vf16 = vmode[vst] != 0;
-            }
-            if (ok && s == 0 && more) ok = wait_bounded_inl(bar(B_KFULL + kst), (kt / kKSt) & 1, ctl);
             if (!ok) break;
             ++pcnt[s];
             tc_fence_after();
