@@ -32,10 +32,16 @@ constexpr int kD = 128;
 constexpr int kRowE = kD + 8;      // bf16 row stride of staged Q, K, V (272 bytes: conflict-free ldmatrix)
 constexpr int kExtStride = 132;    // fp32 row stride of staged parts and output rows (bank spread)
 constexpr int kMaxExt = 4;
+constexpr int kPE = 64 + 8;        // bf16 row stride of the staged P tile (144 bytes: conflict-free ldmatrix)
+// bytes of the staged P (hi and lo) and the row maxima / sums of up to four warps
+constexpr int kPBytes = 2 * kRows * kPE * 2 + 2 * 4 * kRows * 4;
 
 __device__ __forceinline__ void ldsm4(uint32_t a, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(a));
+}
+__device__ __forceinline__ void ldsm2(uint32_t a, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];\n" : "=r"(r0), "=r"(r1) : "r"(a));
 }
 __device__ __forceinline__ void ldsm4t(uint32_t a, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
@@ -132,14 +138,18 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   __nv_bfloat16* sV = sK + NB * kRowE;                                   // [NB][kRowE]
   float* sE = reinterpret_cast<float*>(sV + NB * kRowE);                 // [NX][16][kExtStride]
   float* sL = sE + NXS * kRows * kExtStride;                             // [NX][16]
+  __nv_bfloat16* sPh = reinterpret_cast<__nv_bfloat16*>(sL + NXS * kRows);  // [16][kPE] P, bf16 hi
+  __nv_bfloat16* sPl = sPh + kRows * kPE;                                   // [16][kPE] P, bf16 lo
+  float* sX = reinterpret_cast<float*>(sPl + kRows * kPE);                  // [2][4][16] row maxima, sums
+  float* sAfter = sX + 2 * 4 * kRows;
   // Output and cache rows are staged after P V; with blocks of 32 keys or
   // more they fit in the K/V staging, which is dead by then (a CTA barrier
   // separates the last read of K/V from the first staged row), so more CTAs
   // fit per SM.
   constexpr bool kAlias = inblock_stage_aliases(NB);
-  float* sO = kAlias ? reinterpret_cast<float*>(sK) : sL + NXS * kRows;  // [16][kExtStride] output rows
+  float* sO = kAlias ? reinterpret_cast<float*>(sK) : sAfter;            // [16][kExtStride] output rows
   float* sC = sO + kRows * kExtStride;                                   // [16][kExtStride] cache rows
-  uint64_t* bars = reinterpret_cast<uint64_t*>(kAlias ? sL + NXS * kRows : sC + kRows * kExtStride);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(kAlias ? sAfter : sC + kRows * kExtStride);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int unit = blockIdx.x / a.tiles_per_unit, tile = blockIdx.x % a.tiles_per_unit;
@@ -268,60 +278,103 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   bool ok = !(a.stall && tid == 0) || wait_loaded(bar_e + 8, a);
   if (a.bulk) ok = wait_loaded(bar_qk, a) && ok;
 
-  // ---- S = Q K^T for the CTA's 16 rows (every warp) ----
-  const int dq = warp;   // this warp's quarter of D: columns dq*32 .. dq*32+31
-  float s[NT][4];
+  // ---- S = Q K^T: warp w forms the key n-tiles [w NTW, (w + 1) NTW) of the
+  // CTA's 16 rows (with 16 keys, warps 0 and 1 one n-tile each) ----
+  const int dq = warp;   // this warp's quarter of D in P V: columns dq*32 .. dq*32+31
+  constexpr int NTW = NT >= 4 ? NT / 4 : 1;   // key n-tiles per S warp
+  constexpr int SW = NT / NTW;                // warps that form S
+  const bool swarp = warp < SW;
+  float s[NTW][4];
 #pragma unroll
-  for (int n = 0; n < NT; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+  for (int n = 0; n < NTW; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+  if (swarp) {
 #pragma unroll
-  for (int kk = 0; kk < kD / 16; ++kk) {
-    uint32_t qa[4];
-    ldsm4(ptx::smem_addr(sQ + (lane & 15) * kRowE + (2 * kk + (lane >> 4)) * 8), qa[0], qa[1], qa[2], qa[3]);
+    for (int kk = 0; kk < kD / 16; ++kk) {
+      uint32_t qa[4];
+      ldsm4(ptx::smem_addr(sQ + (lane & 15) * kRowE + (2 * kk + (lane >> 4)) * 8), qa[0], qa[1], qa[2], qa[3]);
 #pragma unroll
-    for (int n = 0; n < NT; n += 2) {
-      const int r = (n + (lane >> 4)) * 8 + (lane & 7), ch = 2 * kk + ((lane >> 3) & 1);
-      uint32_t b0, b1, b2, b3;
-      ldsm4(ptx::smem_addr(sK + r * kRowE + ch * 8), b0, b1, b2, b3);
-      mma16816(s[n], qa, b0, b1);
-      if (n + 1 < NT) mma16816(s[n + 1], qa, b2, b3);
+      for (int n = 0; n < NTW; n += 2) {
+        const int nt = warp * NTW + n;
+        if (NTW >= 2) {
+          const int r = (nt + (lane >> 4)) * 8 + (lane & 7), ch = 2 * kk + ((lane >> 3) & 1);
+          uint32_t b0, b1, b2, b3;
+          ldsm4(ptx::smem_addr(sK + r * kRowE + ch * 8), b0, b1, b2, b3);
+          mma16816(s[n], qa, b0, b1);
+          mma16816(s[n + 1], qa, b2, b3);
+        } else {
+          const int r = nt * 8 + (lane & 7), ch = 2 * kk + ((lane >> 3) & 1);
+          uint32_t b0, b1;
+          ldsm2(ptx::smem_addr(sK + r * kRowE + ch * 8), b0, b1);
+          mma16816(s[n], qa, b0, b1);
+        }
+      }
     }
   }
-  // ---- softmax over the block's keys (rows lane/4 and lane/4 + 8) ----
+  // ---- softmax over the block's keys (rows lane/4 and lane/4 + 8): the
+  // row maxima and sums of the S warps meet in shared memory ----
   float mrow[2] = {-CUDART_INF_F, -CUDART_INF_F};
 #pragma unroll
-  for (int n = 0; n < NT; ++n)
+  for (int n = 0; n < NTW; ++n)
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const int key = n * 8 + 2 * (lane & 3) + (e & 1);
+      const int key = (warp * NTW + n) * 8 + 2 * (lane & 3) + (e & 1);
       s[n][e] = key < a.Nb ? s[n][e] * a.scale_log2 : -CUDART_INF_F;
       mrow[e >> 1] = fmaxf(mrow[e >> 1], s[n][e]);
     }
-  float lrow[2] = {0.f, 0.f};
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     mrow[h] = fmaxf(mrow[h], __shfl_xor_sync(0xffffffffu, mrow[h], 1));
     mrow[h] = fmaxf(mrow[h], __shfl_xor_sync(0xffffffffu, mrow[h], 2));
   }
-  uint32_t ph[NT][2], pl[NT][2];
-#pragma unroll
-  for (int n = 0; n < NT; ++n) {
-    const float p0 = ex2(s[n][0] - mrow[0]), p1 = ex2(s[n][1] - mrow[0]);
-    const float p2 = ex2(s[n][2] - mrow[1]), p3 = ex2(s[n][3] - mrow[1]);
-    lrow[0] += p0 + p1;
-    lrow[1] += p2 + p3;
-    split2(p0, p1, ph[n][0], pl[n][0]);
-    split2(p2, p3, ph[n][1], pl[n][1]);
+  if (swarp && (lane & 3) == 0) {
+    sX[warp * kRows + (lane >> 2)] = mrow[0];
+    sX[warp * kRows + (lane >> 2) + 8] = mrow[1];
   }
+  __syncthreads();
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 1);
-    lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 2);
+    float m = -CUDART_INF_F;
+#pragma unroll
+    for (int w = 0; w < SW; ++w) m = fmaxf(m, sX[w * kRows + (lane >> 2) + 8 * h]);
+    mrow[h] = m;
   }
-  if (a.bulk) {
-    ok = wait_loaded(bar_v, a) && ok;
-  } else {
-    cp_async_wait<1>();
-    __syncthreads();
+  float lrow[2] = {0.f, 0.f};
+  if (swarp) {
+#pragma unroll
+    for (int n = 0; n < NTW; ++n) {
+      const float p0 = ex2(s[n][0] - mrow[0]), p1 = ex2(s[n][1] - mrow[0]);
+      const float p2 = ex2(s[n][2] - mrow[1]), p3 = ex2(s[n][3] - mrow[1]);
+      lrow[0] += p0 + p1;
+      lrow[1] += p2 + p3;
+      // P as bf16 hi + lo pairs, rows lane/4 and lane/4 + 8 of the P tile
+      const int col = (warp * NTW + n) * 8 + 2 * (lane & 3);
+      uint32_t h0, l0, h1, l1;
+      split2(p0, p1, h0, l0);
+      split2(p2, p3, h1, l1);
+      *reinterpret_cast<uint32_t*>(sPh + (lane >> 2) * kPE + col) = h0;
+      *reinterpret_cast<uint32_t*>(sPl + (lane >> 2) * kPE + col) = l0;
+      *reinterpret_cast<uint32_t*>(sPh + ((lane >> 2) + 8) * kPE + col) = h1;
+      *reinterpret_cast<uint32_t*>(sPl + ((lane >> 2) + 8) * kPE + col) = l1;
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 1);
+      lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 2);
+    }
+    if ((lane & 3) == 0) {
+      sX[(SW + warp) * kRows + (lane >> 2)] = lrow[0];
+      sX[(SW + warp) * kRows + (lane >> 2) + 8] = lrow[1];
+    }
+  }
+  if (a.bulk) ok = wait_loaded(bar_v, a) && ok;
+  else cp_async_wait<1>();
+  __syncthreads();   // V_in (every thread's chunks), P and the row sums
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float l = 0.f;
+#pragma unroll
+    for (int w = 0; w < SW; ++w) l += sX[(SW + w) * kRows + (lane >> 2) + 8 * h];
+    lrow[h] = l;
   }
   // ---- O[:, dq*32 : dq*32+32] = P V ----
   constexpr int DT = 4;    // 8-column tiles in this warp's quarter
@@ -330,8 +383,9 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   for (int d = 0; d < DT; ++d) o[d][0] = o[d][1] = o[d][2] = o[d][3] = 0.f;
 #pragma unroll
   for (int kk = 0; kk < KK; ++kk) {
-    const uint32_t ah[4] = {ph[2 * kk][0], ph[2 * kk][1], ph[2 * kk + 1][0], ph[2 * kk + 1][1]};
-    const uint32_t al[4] = {pl[2 * kk][0], pl[2 * kk][1], pl[2 * kk + 1][0], pl[2 * kk + 1][1]};
+    uint32_t ah[4], al[4];
+    ldsm4(ptx::smem_addr(sPh + (lane & 15) * kPE + (2 * kk + (lane >> 4)) * 8), ah[0], ah[1], ah[2], ah[3]);
+    ldsm4(ptx::smem_addr(sPl + (lane & 15) * kPE + (2 * kk + (lane >> 4)) * 8), al[0], al[1], al[2], al[3]);
 #pragma unroll
     for (int d = 0; d < DT; d += 2) {
       const int r = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8, ch = dq * DT + d + (lane >> 4);
@@ -466,7 +520,7 @@ cudaError_t launch_inblock_small(const fb_attn_desc& d, const void* q, const voi
   if (!a.status) return cudaErrorInvalidValue;
   const int NB = d.Nb <= 16 ? 16 : d.Nb <= 32 ? 32 : 64;
   const int nxs = next > 0 ? next : 1;
-  const size_t smem = (size_t)(kRows + 2 * NB) * kRowE * 2 + (size_t)nxs * kRows * (kExtStride + 1) * 4 +
+  const size_t smem = (size_t)(kRows + 2 * NB) * kRowE * 2 + (size_t)nxs * kRows * (kExtStride + 1) * 4 + kPBytes +
                       (inblock_stage_aliases(NB) ? 0 : 2 * (size_t)kRows * kExtStride * 4) + 4 * 8;
   const dim3 grid(d.B * d.Hkv * a.tiles_per_unit);
   // instances above the default 48 KB of dynamic shared memory opt in once
