@@ -162,9 +162,14 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   // row's head and index among the computed queries (i = k, or the k-th
   // active position); returns the packed (b, h, i) row of parts and LSE, or
   // -1 for a row that does not exist or names a position outside the block.
+  const int g0 = row0 / nqh, k0 = row0 % nqh;   // head and query index of the CTA's first row
   auto row_at = [&](int r, int& h, int& i) -> int64_t {
     if (r >= nq) return -1;
-    const int rr = row0 + r, g = rr / nqh, k = rr % nqh;
+    int g = g0, k = k0 + r;   // row0 + r = g * nqh + k (r < 16: a short walk, no division)
+    while (k >= nqh) {
+      k -= nqh;
+      ++g;
+    }
     i = a.active ? a.active[(int64_t)b * a.n_act + k] : k;
     if (i < 0 || i >= a.Nb) return -1;
     h = kvh * a.G + g;
