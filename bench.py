@@ -400,14 +400,19 @@ def measure_workload(args, spec, rank, world, device, headline):
     ms = timed_region(g.replay, steps, args.warmup)
     del g
     us_prefix_call_warm = 1e3 * ms / (R * nl)
+    G = s.Hq // s.Hkv
+    tiles_per_kv = -(-G // (128 // s.Nb)) if s.Nb <= 128 else G * -(-s.Nb // 128)
+    kname = ("attn generic" if not (s.dtype == "bf16" and s.D == 128) else
+             "attn_pair_kernel (tcgen05, two query tiles per CTA) + pair_merge_kernel" if tiles_per_kv >= 2 else
+             "attn_tc_kernel (tcgen05) + merge of its key splits")
     per_kind["prefix_attention"] = {
-        "call": "fb_attn_outblock", "kernel": "attn_tc_kernel (tcgen05)" if s.dtype == "bf16" and s.D == 128
-        else "attn generic", "kernels_per_call": (pk["prefix_attention"][0] + pk["aux"][0]) / (R * nl),
+        "call": "fb_attn_outblock", "kernel": kname,
+        "kernels_per_call": (pk["prefix_attention"][0] + pk["aux"][0]) / (R * nl),
         "avg_launch_us_cold": us_prefix_cold, "avg_call_us_warm": us_prefix_call_warm,
         "alg_bytes_per_launch": cost["prefix_attention"]["bytes"],
         "alg_flops_per_launch": cost["prefix_attention"]["flops"],
         "timing": f"cold: CUDA events around each of {R * nl} kernel launches, L2 flushed before each round of "
-                  f"{nl}; warm: one graph of {R * nl} calls (kernel + merge of the split parts)"}
+                  f"{nl}; warm: one graph of {R * nl} calls (kernel + merge of its parts)"}
     # in-block: a graph over n_sets distinct input sets (cold), and a graph of
     # the same set repeated (warm)
     g, _ = graph_of(lambda: [call_inblock_set(z) for z in sets])

@@ -260,63 +260,78 @@ __global__ void __launch_bounds__(kThreads, 1)
       nact = 0;
       for (int w = 0; w < words; ++w) nact += __popc(act[w]);
     }
-    const int64_t T = (int64_t)nact * a.nkt;
-    const int C = a.whole ? min((int)gridDim.x, nact)
-                          : (int)min((int64_t)min((int64_t)gridDim.x, T), (int64_t)nact * (a.smax - 1));
     const int c = blockIdx.x;
     int n = 0;
+    // the ai-th active pair (every pair is active without the gamma gate)
+    auto active_pair = [&](int64_t ai) -> int {
+      if (!a.mask_active) return (int)ai;
+      int64_t left = ai;
+      for (int w = 0; w < words; ++w) {
+        uint32_t bits = act[w];
+        const int cnt = __popc(bits);
+        if (left >= cnt) { left -= cnt; continue; }
+        while (left > 0) { bits &= bits - 1; --left; }
+        return w * 32 + __ffs(bits) - 1;
+      }
+      return -1;
+    };
+    auto push_whole = [&](int p) {
+      Seg sg;
+      sg.pair = p;
+      sg.j0 = 0;
+      sg.j1 = a.nkt;
+      sg.slot_ns = 1 << 16;
+      segs[n++] = sg;
+    };
     if (a.whole) {
-      // whole pairs: active pairs c, c + C, c + 2C, ... (every pair is active
-      // without the gamma gate)
-      auto push = [&](int p) {
-        Seg sg;
-        sg.pair = p;
-        sg.j0 = 0;
-        sg.j1 = a.nkt;
-        sg.slot_ns = 1 << 16;
-        segs[n++] = sg;
-      };
+      // whole pairs: active pairs c, c + C, c + 2C, ...
+      const int C = min((int)gridDim.x, nact);
       if (!a.mask_active) {
-        for (int p = c; p < a.npairs && n < kMaxSeg; p += C) push(p);
+        for (int p = c; p < a.npairs && n < kMaxSeg; p += C) push_whole(p);
       } else {
         int ai = 0;
         for (int p = 0; p < a.npairs && n < kMaxSeg; ++p) {
           if (!((act[p >> 5] >> (p & 31)) & 1u)) continue;
-          if (ai++ % C == c) push(p);
+          if (ai++ % C == c) push_whole(p);
         }
       }
-    } else if (c < C) {
-      const int64_t i0 = (int64_t)c * T / C, i1 = (int64_t)(c + 1) * T / C;
-      int64_t ai = i0 / a.nkt;            // active index of the first pair
-      // the ai-th active pair
-      int p = (int)ai;
-      if (a.mask_active) {
-        int64_t left = ai;
-        p = -1;
-        for (int w = 0; w < words && p < 0; ++w) {
-          uint32_t bits = act[w];
-          const int cnt = __popc(bits);
-          if (left >= cnt) { left -= cnt; continue; }
-          while (left > 0) { bits &= bits - 1; --left; }
-          p = w * 32 + __ffs(bits) - 1;
-        }
+    } else {
+      // Rounds of whole pairs first: with at least as many pairs as CTAs,
+      // CTA c takes active pairs c, c + G, ... in lock step with its
+      // neighbours, which hold the other query tiles of the same KV head and
+      // stream the same K/V tiles at the same time (L2 serves the second
+      // read).  The remaining pairs' key tiles are then split evenly
+      // (stream-K) over up to G CTAs, each pair over at most smax - 1 of them.
+      const int G = (int)gridDim.x;
+      const int R = nact / G;
+      for (int r = 0; r < R && n < kMaxSeg; ++r) {
+        const int p = active_pair((int64_t)r * G + c);
+        if (p >= 0) push_whole(p);
       }
-      for (int64_t it = i0; it < i1 && n < kMaxSeg && p >= 0 && p < a.npairs;) {
-        const int64_t base = ai * a.nkt;
-        const int64_t e = min(i1, base + a.nkt);
-        const int first = cta_of(base, C, T), last = cta_of(base + a.nkt - 1, C, T);
-        Seg s;
-        s.pair = p;
-        s.j0 = (int)(it - base);
-        s.j1 = (int)(e - base);
-        s.slot_ns = (c - first) | ((last - first + 1) << 16);
-        segs[n++] = s;
-        it = e;
-        ++ai;
-        // next active pair
-        ++p;
-        if (a.mask_active)
-          while (p < a.npairs && !((act[p >> 5] >> (p & 31)) & 1u)) ++p;
+      const int rem = nact - R * G;
+      const int64_t T = (int64_t)rem * a.nkt;
+      const int C = (int)min((int64_t)min((int64_t)G, T), (int64_t)rem * (a.smax - 1));
+      if (c < C) {
+        const int64_t i0 = (int64_t)c * T / C, i1 = (int64_t)(c + 1) * T / C;
+        int64_t ai = i0 / a.nkt;            // index of the first pair among the remaining ones
+        int p = active_pair((int64_t)R * G + ai);
+        for (int64_t it = i0; it < i1 && n < kMaxSeg && p >= 0 && p < a.npairs;) {
+          const int64_t base = ai * a.nkt;
+          const int64_t e = min(i1, base + a.nkt);
+          const int first = cta_of(base, C, T), last = cta_of(base + a.nkt - 1, C, T);
+          Seg sg;
+          sg.pair = p;
+          sg.j0 = (int)(it - base);
+          sg.j1 = (int)(e - base);
+          sg.slot_ns = (c - first) | ((last - first + 1) << 16);
+          segs[n++] = sg;
+          it = e;
+          ++ai;
+          // next active pair
+          ++p;
+          if (a.mask_active)
+            while (p < a.npairs && !((act[p >> 5] >> (p & 31)) & 1u)) ++p;
+        }
       }
     }
     *nseg_sh = n;
@@ -874,10 +889,17 @@ bool pair_plan(const fb_attn_desc& d, int64_t nkeys, PairPlan* p) {
   if (p->nkt < 4 || p->npairs > kMaxPairs || !pair_regs_ok()) return false;
   const int64_t T = (int64_t)p->npairs * p->nkt;
   p->grid = (int32_t)std::min<int64_t>(num_sms(), T);
-  // segments per CTA: at most ceil(items per CTA / key tiles) + 1
-  const int64_t per = (T + p->grid - 1) / p->grid;
-  if ((per + p->nkt - 1) / p->nkt + 1 > kMaxSeg) return false;
-  p->smax = (p->grid + p->npairs - 1) / p->npairs + 1;
+  // R rounds of whole pairs, then the remaining pairs' key tiles split over
+  // the grid: segments per CTA at most R + ceil(items per CTA / key tiles) + 1
+  const int64_t R = p->npairs / p->grid, rem = p->npairs - R * p->grid;
+  const int64_t per = (rem * p->nkt + p->grid - 1) / p->grid;
+  if (R + (per + p->nkt - 1) / p->nkt + 1 > kMaxSeg) return false;
+  // slots per pair: a remaining pair spans at most ceil(grid / rem) + 1 CTAs;
+  // after whole-pair rounds the split is capped (the kernel then uses fewer
+  // CTAs for the remaining pairs) to keep the part buffers small
+  constexpr int64_t kSlotCapAfterRounds = 8;
+  const int64_t span = rem > 0 ? (p->grid + rem - 1) / rem + 1 : 2;
+  p->smax = (int32_t)(R == 0 ? span : std::max<int64_t>(2, std::min(span, kSlotCapAfterRounds)));
   return true;
 }
 
