@@ -33,8 +33,9 @@ constexpr int kRowE = kD + 8;      // bf16 row stride of staged Q, K, V (272 byt
 constexpr int kExtStride = 132;    // fp32 row stride of staged parts and output rows (bank spread)
 constexpr int kMaxExt = 4;
 constexpr int kPE = 64 + 8;        // bf16 row stride of the staged P tile (144 bytes: conflict-free ldmatrix)
-// bytes of the staged P (hi and lo) and the row maxima / sums of up to four warps
-constexpr int kPBytes = 2 * kRows * kPE * 2 + 2 * 4 * kRows * 4;
+// bytes of the staged P (hi and lo), the row maxima / sums of up to four
+// warps and the CTA's row table (packed row, query and output offsets)
+constexpr int kPBytes = 2 * kRows * kPE * 2 + 2 * 4 * kRows * 4 + 3 * kRows * 8;
 
 __device__ __forceinline__ void ldsm4(uint32_t a, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
@@ -141,7 +142,10 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   __nv_bfloat16* sPh = reinterpret_cast<__nv_bfloat16*>(sL + NXS * kRows);  // [16][kPE] P, bf16 hi
   __nv_bfloat16* sPl = sPh + kRows * kPE;                                   // [16][kPE] P, bf16 lo
   float* sX = reinterpret_cast<float*>(sPl + kRows * kPE);                  // [2][4][16] row maxima, sums
-  float* sAfter = sX + 2 * 4 * kRows;
+  int64_t* sRowPr = reinterpret_cast<int64_t*>(sX + 2 * 4 * kRows);         // [16] packed (b, h, i) row or -1
+  int64_t* sRowQ = sRowPr + kRows;                                          // [16] the row's element offset in q
+  int64_t* sRowO = sRowQ + kRows;                                           // [16] the row's element offset in o
+  float* sAfter = reinterpret_cast<float*>(sRowO + kRows);
   // Output and cache rows are staged after P V; with blocks of 32 keys or
   // more they fit in the K/V staging, which is dead by then (a CTA barrier
   // separates the last read of K/V from the first staged row), so more CTAs
@@ -178,12 +182,40 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   const uint32_t bar_qk = ptx::smem_addr(bars), bar_v = bar_qk + 8, bar_e = bar_qk + 16;
 
   // ---- every load issued up front: one bulk copy per row (a.bulk), or
-  // 16-byte cp.async chunks from all 128 threads in three commit groups
-  // (Q and K_in; V_in; the parts), which keeps the SM's copy engine out of
-  // the way when a CTA needs a hundred or more rows ----
+  // 16-byte cp.async chunks from all 128 threads in two commit groups (K_in,
+  // V_in and Q; the parts), which keeps the SM's copy engine out of the way
+  // when a CTA needs a hundred or more rows.  K_in and V_in do not depend on
+  // the CTA's rows and go first ----
+  const __nv_bfloat16* kb = a.k + b * a.k_sb + (int64_t)kvh * a.k_sh;
+  const __nv_bfloat16* vb = a.v + b * a.k_sb + (int64_t)kvh * a.k_sh;
+  if (!a.bulk) {
+    for (int c = tid; c < NB * 16; c += 128) {      // K rows
+      const int r = c >> 4, ch = c & 15;
+      if (r < a.Nb)
+        cp_async16(ptx::smem_addr(sK + r * kRowE + ch * 8), kb + (int64_t)r * a.k_st + ch * 8);
+      else
+        *reinterpret_cast<uint4*>(sK + r * kRowE + ch * 8) = make_uint4(0, 0, 0, 0);
+    }
+    for (int c = tid; c < NB * 16; c += 128) {      // V rows
+      const int r = c >> 4, ch = c & 15;
+      if (r < a.Nb)
+        cp_async16(ptx::smem_addr(sV + r * kRowE + ch * 8), vb + (int64_t)r * a.k_st + ch * 8);
+      else
+        *reinterpret_cast<uint4*>(sV + r * kRowE + ch * 8) = make_uint4(0, 0, 0, 0);
+    }
+  }
+  // the CTA's row table, one thread per row
+  bool valid = false;
+  if (tid < kRows) {
+    int h = 0, i = 0;
+    const int64_t pr = row_at(tid, h, i);
+    valid = pr >= 0;
+    sRowPr[tid] = pr;
+    sRowQ[tid] = valid ? b * a.q_sb + (int64_t)h * a.q_sh + (int64_t)i * a.q_st : 0;
+    sRowO[tid] = valid ? b * a.o_sb + (int64_t)h * a.o_sh + (int64_t)i * a.o_st : 0;
+  }
+  const int nvalid = __syncthreads_count(valid);
   if (tid == 0) {
-    int nvalid = 0, hh, ii;
-    for (int r = 0; r < nq; ++r) nvalid += row_at(r, hh, ii) >= 0;
     if (nvalid < nq) atomicCAS(a.status, 0, (int)FB_EINVAL);
     ptx::mbar_init(bar_qk, 1);
     ptx::mbar_init(bar_v, 1);
@@ -202,43 +234,22 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const int idx = tid + k * 128;
-    int hh, ii;
-    const int64_t pr = idx < NX * kRows ? row_at(idx & 15, hh, ii) : -1;
+    const int64_t pr = idx < NX * kRows ? sRowPr[idx & 15] : -1;
     if (pr >= 0) lx[k] = a.ext_l[idx >> 4][pr];
   }
   __syncthreads();
   if (!a.bulk) {
-    const __nv_bfloat16* kb = a.k + b * a.k_sb + (int64_t)kvh * a.k_sh;
-    const __nv_bfloat16* vb = a.v + b * a.k_sb + (int64_t)kvh * a.k_sh;
     for (int c = tid; c < kRows * 16; c += 128) {   // Q rows, 16 chunks each
       const int r = c >> 4, ch = c & 15;
-      int h, i;
-      if (row_at(r, h, i) >= 0)
-        cp_async16(ptx::smem_addr(sQ + r * kRowE + ch * 8),
-                   a.q + b * a.q_sb + (int64_t)h * a.q_sh + (int64_t)i * a.q_st + ch * 8);
+      if (sRowPr[r] >= 0)
+        cp_async16(ptx::smem_addr(sQ + r * kRowE + ch * 8), a.q + sRowQ[r] + ch * 8);
       else
         *reinterpret_cast<uint4*>(sQ + r * kRowE + ch * 8) = make_uint4(0, 0, 0, 0);
-    }
-    for (int c = tid; c < NB * 16; c += 128) {      // K rows
-      const int r = c >> 4, ch = c & 15;
-      if (r < a.Nb)
-        cp_async16(ptx::smem_addr(sK + r * kRowE + ch * 8), kb + (int64_t)r * a.k_st + ch * 8);
-      else
-        *reinterpret_cast<uint4*>(sK + r * kRowE + ch * 8) = make_uint4(0, 0, 0, 0);
-    }
-    cp_async_commit();
-    for (int c = tid; c < NB * 16; c += 128) {      // V rows
-      const int r = c >> 4, ch = c & 15;
-      if (r < a.Nb)
-        cp_async16(ptx::smem_addr(sV + r * kRowE + ch * 8), vb + (int64_t)r * a.k_st + ch * 8);
-      else
-        *reinterpret_cast<uint4*>(sV + r * kRowE + ch * 8) = make_uint4(0, 0, 0, 0);
     }
     cp_async_commit();
     for (int c = tid; c < NX * kRows * 32; c += 128) {   // the parts' rows, 32 chunks each
       const int p = c / (kRows * 32), r = (c >> 5) % kRows, ch = c & 31;
-      int hh, ii;
-      const int64_t pr = row_at(r, hh, ii);
+      const int64_t pr = sRowPr[r];
       if (pr >= 0)
         cp_async16(ptx::smem_addr(sE + (p * kRows + r) * kExtStride + ch * 4), a.ext_a[p] + pr * kD + ch * 4);
     }
@@ -246,10 +257,8 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   } else if (warp == 0) {
     if (lane < kRows) {
       const int r = lane;
-      int h, i;
-      if (row_at(r, h, i) >= 0) {
-        ptx::bulk_g2s(ptx::smem_addr(sQ + r * kRowE), a.q + b * a.q_sb + (int64_t)h * a.q_sh + (int64_t)i * a.q_st,
-                      kD * 2, bar_qk);
+      if (sRowPr[r] >= 0) {
+        ptx::bulk_g2s(ptx::smem_addr(sQ + r * kRowE), a.q + sRowQ[r], kD * 2, bar_qk);
       } else {
 #pragma unroll 1
         for (int c = 0; c < kD / 8; ++c) reinterpret_cast<uint4*>(sQ + r * kRowE)[c] = make_uint4(0, 0, 0, 0);
@@ -258,7 +267,7 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   } else if (warp == 1 || warp == 2) {
     const bool isk = warp == 1;
     __nv_bfloat16* dst = isk ? sK : sV;
-    const __nv_bfloat16* src = (isk ? a.k : a.v) + b * a.k_sb + (int64_t)kvh * a.k_sh;
+    const __nv_bfloat16* src = isk ? kb : vb;
 #pragma unroll 1
     for (int r = lane; r < NB; r += 32) {
       if (r < a.Nb) {
@@ -270,15 +279,14 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
     }
   } else if (NX > 0) {
     const int p = lane >> 4, r = lane & 15;
-    int hh, ii;
-    const int64_t pr = row_at(r, hh, ii);
+    const int64_t pr = sRowPr[r];
 #pragma unroll
     for (int pp = 0; pp < NX; pp += 2)
       if (pp + p < NX && pr >= 0)
         ptx::bulk_g2s(ptx::smem_addr(sE + ((pp + p) * kRows + r) * kExtStride), a.ext_a[pp + p] + pr * kD, kD * 4,
                       bar_e);
   }
-  if (!a.bulk) cp_async_wait<2>();   // this thread's Q and K chunks
+  if (!a.bulk) cp_async_wait<1>();   // this thread's K, V and Q chunks
   __syncthreads();   // every thread's chunks, and the zero-filled rows
   bool ok = !(a.stall && tid == 0) || wait_loaded(bar_e + 8, a);
   if (a.bulk) ok = wait_loaded(bar_qk, a) && ok;
@@ -372,8 +380,7 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
     }
   }
   if (a.bulk) ok = wait_loaded(bar_v, a) && ok;
-  else cp_async_wait<1>();
-  __syncthreads();   // V_in (every thread's chunks), P and the row sums
+  __syncthreads();   // V_in (the bulk copies), P and the row sums
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     float l = 0.f;
@@ -415,8 +422,7 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int r = (lane >> 2) + 8 * h;
-    int hq, iq;
-    const int64_t pr = row_at(r, hq, iq);
+    const int64_t pr = sRowPr[r];
     if (pr < 0) continue;
     const float Lin = lrow[h] > 0.f ? (mrow[h] + __log2f(lrow[h])) * kLn2 : -CUDART_INF_F;
     float m = Lin;
@@ -465,10 +471,9 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   // ---- whole-row stores: lanes 0..15 the output rows, 16..31 the cache rows (warp 0) ----
   if (ok && warp == 0) {
     const int r = lane & 15;
-    int h, i;
-    const int64_t pr = row_at(r, h, i);
+    const int64_t pr = sRowPr[r];
     if (pr >= 0 && lane < 16) {
-      const int64_t obase = b * a.o_sb + (int64_t)h * a.o_sh + (int64_t)i * a.o_st;
+      const int64_t obase = sRowO[r];
       void* dst = obf ? static_cast<void*>(static_cast<__nv_bfloat16*>(a.o) + obase)
                       : static_cast<void*>(static_cast<float*>(a.o) + obase);
       ptx::bulk_s2g(dst, ptx::smem_addr(sO + r * kExtStride), obf ? kD * 2 : kD * 4);
