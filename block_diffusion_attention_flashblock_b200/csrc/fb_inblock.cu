@@ -237,7 +237,7 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
     const int64_t pr = idx < NX * kRows ? sRowPr[idx & 15] : -1;
     if (pr >= 0) lx[k] = a.ext_l[idx >> 4][pr];
   }
-  __syncthreads();
+  if (a.bulk) __syncthreads();   // the barriers' initialisation, before any bulk copy names them
   if (!a.bulk) {
     for (int c = tid; c < kRows * 16; c += 128) {   // Q rows, 16 chunks each
       const int r = c >> 4, ch = c & 15;
@@ -297,9 +297,13 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   constexpr int NTW = NT >= 4 ? NT / 4 : 1;   // key n-tiles per S warp
   constexpr int SW = NT / NTW;                // warps that form S
   const bool swarp = warp < SW;
-  float s[NTW][4];
+  // two accumulators per n-tile (even and odd k-steps) halve the chain of
+  // dependent MMAs
+  float s[NTW][4], s2[NTW][4];
 #pragma unroll
-  for (int n = 0; n < NTW; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+  for (int n = 0; n < NTW; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[n][e] = s2[n][e] = 0.f;
   if (swarp) {
 #pragma unroll
     for (int kk = 0; kk < kD / 16; ++kk) {
@@ -308,20 +312,25 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
 #pragma unroll
       for (int n = 0; n < NTW; n += 2) {
         const int nt = warp * NTW + n;
+        float(*acc)[4] = (kk & 1) ? s2 : s;
         if (NTW >= 2) {
           const int r = (nt + (lane >> 4)) * 8 + (lane & 7), ch = 2 * kk + ((lane >> 3) & 1);
           uint32_t b0, b1, b2, b3;
           ldsm4(ptx::smem_addr(sK + r * kRowE + ch * 8), b0, b1, b2, b3);
-          mma16816(s[n], qa, b0, b1);
-          mma16816(s[n + 1], qa, b2, b3);
+          mma16816(acc[n], qa, b0, b1);
+          mma16816(acc[n + 1], qa, b2, b3);
         } else {
           const int r = nt * 8 + (lane & 7), ch = 2 * kk + ((lane >> 3) & 1);
           uint32_t b0, b1;
           ldsm2(ptx::smem_addr(sK + r * kRowE + ch * 8), b0, b1);
-          mma16816(s[n], qa, b0, b1);
+          mma16816(acc[n], qa, b0, b1);
         }
       }
     }
+#pragma unroll
+    for (int n = 0; n < NTW; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[n][e] += s2[n][e];
   }
   // ---- softmax over the block's keys (rows lane/4 and lane/4 + 8): the
   // row maxima and sums of the S warps meet in shared memory ----
