@@ -361,18 +361,28 @@ static bool union_applies(const fb_attn_desc& d, int64_t prefix_len, int32_t sel
   int mode, hg, tpu, units;
   return g_prefix_kernel != 1 && u > 0 && 3 * u < prefix_len && tc_tiling(d, &mode, &hg, &tpu, &units);
 }
-// Selected keys (membership bitmap over the prefix already built): the
-// union's rows gathered compact, then the tcgen05 pass over them that leaves
-// out, per query head, the union keys it did not select.
+// Selected keys: the selections' key bitmaps (at `bitmap`) and the union of
+// each KV head's selections with every query head's membership over it —
+// from the selections in one shared-memory kernel where that fits, else the
+// bitmaps first and the union from them; then the union's rows gathered
+// compact, and the tcgen05 pass over them that leaves out, per query head,
+// the union keys it did not select.
 static fb_status launch_selected_union(const fb_attn_desc& d, const void* q, const void* kp, const void* vp,
-                                       int64_t prefix_len, const uint32_t* bitmap, int32_t sel_k, const UnionWs& u,
-                                       int32_t cap, float* pa, float* pl, int32_t* nparts, cudaStream_t s) {
+                                       int64_t prefix_len, const int32_t* sel, uint32_t* bitmap, int32_t sel_k,
+                                       const UnionWs& u, int32_t cap, float* pa, float* pl, int32_t* nparts,
+                                       cudaStream_t s) {
   const int64_t umax = union_keys(d, prefix_len, sel_k);
   const int64_t wp = (prefix_len + 31) / 32, wu = (umax + 31) / 32;
   const int es = esize(d.in_dtype);
   {
-    ProfScope prof(kProfAux, (double)d.B * d.Hq * wp * 4 + (double)d.B * d.Hq * wu * 4, s);
-    if (launch_union_select(d, bitmap, wp, u.upos, u.ucount, umax, u.memb, wu, s) != cudaSuccess) return FB_ECUDA;
+    ProfScope prof(kProfAux, (double)d.B * d.Hq * (sel_k * 4.0 + wp * 4.0 + wu * 4.0), s);
+    if (union_build_fits(d, wp, umax)) {
+      if (launch_union_build(d, sel, sel_k, bitmap, wp, u.upos, u.ucount, umax, u.memb, wu, s) != cudaSuccess)
+        return FB_ECUDA;
+    } else if (launch_build_bitmap(sel, sel_k, d.B * d.Hq, bitmap, wp, s) != cudaSuccess ||
+               launch_union_select(d, bitmap, wp, u.upos, u.ucount, umax, u.memb, wu, s) != cudaSuccess) {
+      return FB_ECUDA;
+    }
   }
   {
     ProfScope prof(kProfAux, 4.0 * d.B * d.Hkv * umax * d.D * es, s);
@@ -589,11 +599,11 @@ fb_status fb_attn_outblock(const fb_attn_desc* d, const void* q, const void* kp,
   const bool via_union = union_applies(*d, prefix_len, sel_k);
   if (via_union) {
     // the union's rows once per KV head, then the pass over them
-    if (launch_build_bitmap(sel, sel_k, d->B * d->Hq, bitmap, words, stream) != cudaSuccess) return FB_ECUDA;
     const UnionWs u = union_carve(*d, union_keys(*d, prefix_len, sel_k),
                                   reinterpret_cast<uint8_t*>(ns) + align256((size_t)pair_count(*d) * 4));
     int32_t np = 0;
-    if ((st = launch_selected_union(*d, q, kp, vp, prefix_len, bitmap, sel_k, u, cap, pa, pl, &np, stream)) != FB_OK)
+    if ((st = launch_selected_union(*d, q, kp, vp, prefix_len, sel, bitmap, sel_k, u, cap, pa, pl, &np, stream)) !=
+        FB_OK)
       return st;
     PartList lst;
     memset(&lst, 0, sizeof(lst));
@@ -1082,12 +1092,10 @@ fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
         sp = plan_prefix(d, a->q, a->kp, a->vp, a->prefix_len, c->sel_cap);
       }
       if (via_union) {
-        if (launch_build_bitmap(a->sel, a->sel_k, BH, c->bitmap, (a->prefix_len + 31) / 32, s) != cudaSuccess)
-          return FB_ECUDA;
         bitmap_built = true;
         const UnionWs u = union_carve(d, union_keys(d, a->prefix_len, a->sel_k), c->union_base);
-        if ((st = launch_selected_union(d, a->q, a->kp, a->vp, a->prefix_len, c->bitmap, a->sel_k, u, c->sel_cap,
-                                        c->sel_a, c->sel_l, &nsel, s)) != FB_OK)
+        if ((st = launch_selected_union(d, a->q, a->kp, a->vp, a->prefix_len, a->sel, c->bitmap, a->sel_k, u,
+                                        c->sel_cap, c->sel_a, c->sel_l, &nsel, s)) != FB_OK)
           return st;
       } else if (sp.tc) {
         if (launch_build_bitmap(a->sel, a->sel_k, BH, c->bitmap, (a->prefix_len + 31) / 32, s) != cudaSuccess)

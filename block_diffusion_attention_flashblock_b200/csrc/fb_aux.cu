@@ -341,9 +341,9 @@ __global__ void __launch_bounds__(kUnionThreads)
     union_select_kernel(const uint32_t* bitmap, int64_t words_p, int32_t G, int32_t Hq, int32_t Hkv, int32_t* upos,
                         int32_t* ucount, int64_t umax, uint32_t* memb, int64_t words_u) {
   ptx::pdl_prologue();
-  using Scan = cub::BlockScan<int64_t, kUnionThreads>;
+  using Scan = cub::BlockScan<int, kUnionThreads>;   // union sizes fit in 32 bits (prefix < 2^31 keys)
   __shared__ typename Scan::TempStorage tmp;
-  __shared__ int64_t s_total;
+  __shared__ int s_total;
   const int kv = blockIdx.x, b = kv / Hkv, kvh = kv % Hkv;
   const uint32_t* hb = bitmap + ((int64_t)b * Hq + (int64_t)kvh * G) * words_p;   // G head bitmaps
   int32_t* up = upos + (int64_t)kv * umax;
@@ -355,9 +355,9 @@ __global__ void __launch_bounds__(kUnionThreads)
   // the union's positions, in key order
   const int64_t chunk = (words_p + kUnionThreads - 1) / kUnionThreads;
   const int64_t w0 = threadIdx.x * chunk, w1 = min(words_p, w0 + chunk);
-  int64_t cnt = 0;
+  int cnt = 0;
   for (int64_t w = w0; w < w1; ++w) cnt += __popc(uword(w));
-  int64_t base, total;
+  int base, total;
   Scan(tmp).ExclusiveSum(cnt, base, total);
   if (threadIdx.x == 0) s_total = total;
   for (int64_t w = w0; w < w1; ++w) {
@@ -370,20 +370,104 @@ __global__ void __launch_bounds__(kUnionThreads)
     }
   }
   __syncthreads();
-  const int64_t n = min(s_total, umax);
+  const int64_t n = min((int64_t)s_total, umax);
   if (threadIdx.x == 0) ucount[kv] = (int32_t)n;
-  // membership of each union key in each query head's selection
-  for (int64_t i = threadIdx.x; i < (int64_t)G * words_u; i += kUnionThreads) {
+  // membership of each union key in each query head's selection: one warp
+  // per 32-key word, lane j testing union key 32 cw + j (coalesced reads)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int64_t i = warp; i < (int64_t)G * words_u; i += kUnionThreads / 32) {
     const int g = (int)(i / words_u);
     const int64_t cw = i % words_u;
-    uint32_t bits = 0u;
-    for (int j = 0; j < 32; ++j) {
-      const int64_t idx = cw * 32 + j;
-      if (idx >= n) break;
+    const int64_t idx = cw * 32 + lane;
+    bool in = false;
+    if (idx < n) {
       const int32_t pos = up[idx];
-      if ((hb[g * words_p + (pos >> 5)] >> (pos & 31)) & 1u) bits |= 1u << j;
+      in = (hb[g * words_p + (pos >> 5)] >> (pos & 31)) & 1u;
     }
-    memb[((int64_t)b * Hq + (int64_t)kvh * G + g) * words_u + cw] = bits;
+    const uint32_t bits = __ballot_sync(0xffffffffu, in);
+    if (lane == 0) memb[((int64_t)b * Hq + (int64_t)kvh * G + g) * words_u + cw] = bits;
+  }
+}
+
+// The same result straight from the selections, in shared memory: the G
+// query heads' key bitmaps are built there (and copied out to `bitmap` for
+// passes that need them later), then the union's positions and each head's
+// membership over the union are taken from them without a global-memory
+// round trip per bit.  One CTA per (b, KV head); the launcher checks that the
+// G bitmaps and the umax positions fit in shared memory.
+__global__ void __launch_bounds__(kUnionThreads)
+    union_build_kernel(const int32_t* sel, int32_t sel_k, uint32_t* bitmap, int32_t words_p, int32_t G, int32_t Hq,
+                       int32_t Hkv, int32_t* upos, int32_t* ucount, int32_t umax, uint32_t* memb, int32_t words_u) {
+  ptx::pdl_prologue();
+  using Scan = cub::BlockScan<int, kUnionThreads>;
+  __shared__ typename Scan::TempStorage tmp;
+  __shared__ int s_total;
+  extern __shared__ uint32_t sm_words[];
+  uint32_t* hbm = sm_words;                                     // [G][words_p] head bitmaps
+  int32_t* spos = reinterpret_cast<int32_t*>(sm_words + G * words_p);   // [umax] union positions
+  const int tid = threadIdx.x;
+  const int kv = blockIdx.x, b = kv / Hkv, kvh = kv % Hkv;
+  const int64_t bh0 = (int64_t)b * Hq + (int64_t)kvh * G;      // the first query head's (b, h) row
+  for (int i = tid; i < G * words_p; i += kUnionThreads) hbm[i] = 0u;
+  __syncthreads();
+  for (int g = 0; g < G; ++g) {
+    const int32_t* sg = sel + (bh0 + g) * sel_k;
+    // four keys in flight per thread before their atomics
+    for (int j0 = tid; j0 < sel_k; j0 += 4 * kUnionThreads) {
+      int32_t key[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j0 + u * kUnionThreads;
+        key[u] = j < sel_k ? sg[j] : -1;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (key[u] >= 0 && (key[u] >> 5) < words_p) atomicOr(hbm + g * words_p + (key[u] >> 5), 1u << (key[u] & 31));
+    }
+  }
+  __syncthreads();
+  for (int g = 0; g < G; ++g)
+    for (int w = tid; w < words_p; w += kUnionThreads) bitmap[(bh0 + g) * words_p + w] = hbm[g * words_p + w];
+  auto uword = [&](int w) {
+    uint32_t u = 0u;
+    for (int g = 0; g < G; ++g) u |= hbm[g * words_p + w];
+    return u;
+  };
+  // the union's positions, in key order
+  const int chunk = (words_p + kUnionThreads - 1) / kUnionThreads;
+  const int w0 = tid * chunk, w1 = min(words_p, w0 + chunk);
+  int cnt = 0;
+  for (int w = w0; w < w1; ++w) cnt += __popc(uword(w));
+  int base, total;
+  Scan(tmp).ExclusiveSum(cnt, base, total);
+  if (tid == 0) s_total = total;
+  int32_t* up = upos + (int64_t)kv * umax;
+  for (int w = w0; w < w1; ++w) {
+    uint32_t u = uword(w);
+    while (u) {
+      const int bit = __ffs(u) - 1;
+      u &= u - 1;
+      if (base < umax) {
+        up[base] = w * 32 + bit;
+        spos[base] = w * 32 + bit;
+      }
+      ++base;
+    }
+  }
+  __syncthreads();
+  const int n = min(s_total, umax);
+  if (tid == 0) ucount[kv] = n;
+  // membership of each union key in each query head's selection: one warp
+  // per 32-key word, lane j testing union key 32 cw + j
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int cw = warp; cw < words_u; cw += kUnionThreads / 32) {
+    const int idx = cw * 32 + lane;
+    const int32_t pos = idx < n ? spos[idx] : -1;
+    for (int g = 0; g < G; ++g) {
+      const bool in = pos >= 0 && ((hbm[g * words_p + (pos >> 5)] >> (pos & 31)) & 1u);
+      const uint32_t bits = __ballot_sync(0xffffffffu, in);
+      if (lane == 0) memb[(bh0 + g) * words_u + cw] = bits;
+    }
   }
 }
 
@@ -416,6 +500,31 @@ cudaError_t launch_union_select(const fb_attn_desc& d, const uint32_t* bitmap, i
                                 int32_t* ucount, int64_t umax, uint32_t* memb, int64_t words_u, cudaStream_t s) {
   return launch_k(union_select_kernel, dim3((unsigned)(d.B * d.Hkv)), dim3(kUnionThreads), 0, s, bitmap, words_p,
                   (int32_t)(d.Hq / d.Hkv), (int32_t)d.Hq, (int32_t)d.Hkv, upos, ucount, umax, memb, words_u);
+}
+
+static size_t union_build_smem(const fb_attn_desc& d, int64_t words_p, int64_t umax) {
+  return (size_t)(d.Hq / d.Hkv) * words_p * 4 + (size_t)umax * 4;
+}
+
+bool union_build_fits(const fb_attn_desc& d, int64_t words_p, int64_t umax) {
+  return union_build_smem(d, words_p, umax) <= 200 * 1024;
+}
+
+cudaError_t launch_union_build(const fb_attn_desc& d, const int32_t* sel, int32_t sel_k, uint32_t* bitmap,
+                               int64_t words_p, int32_t* upos, int32_t* ucount, int64_t umax, uint32_t* memb,
+                               int64_t words_u, cudaStream_t s) {
+  const size_t smem = union_build_smem(d, words_p, umax);
+  if (smem > 200 * 1024) return cudaErrorInvalidValue;
+  static size_t opted[kMaxDevices] = {};   // the attribute is per device
+  size_t& cur = opted[current_device()];
+  if (smem > cur) {   // the static scan storage counts too: opt in for any size above the last
+    cudaError_t e = cudaFuncSetAttribute(union_build_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cur = smem;
+  }
+  return launch_k(union_build_kernel, dim3((unsigned)(d.B * d.Hkv)), dim3(kUnionThreads), smem, s, sel, sel_k,
+                  bitmap, (int32_t)words_p, (int32_t)(d.Hq / d.Hkv), (int32_t)d.Hq, (int32_t)d.Hkv, upos, ucount,
+                  (int32_t)umax, memb, (int32_t)words_u);
 }
 
 cudaError_t launch_gather_union(const fb_attn_desc& d, const void* kp, const void* vp, const int32_t* upos,

@@ -242,6 +242,12 @@ cudaError_t launch_fill_decision(int8_t* reuse_out, int32_t n, int8_t value, cud
 // rows of K/V gathered into a compact [B, Hkv, umax, D] block.
 cudaError_t launch_union_select(const fb_attn_desc& d, const uint32_t* bitmap, int64_t words_p, int32_t* upos,
                                 int32_t* ucount, int64_t umax, uint32_t* memb, int64_t words_u, cudaStream_t s);
+// The selections' key bitmaps (written to `bitmap`) and the union select above
+// in one launch, in shared memory, where the G bitmaps and umax positions fit.
+bool union_build_fits(const fb_attn_desc& d, int64_t words_p, int64_t umax);
+cudaError_t launch_union_build(const fb_attn_desc& d, const int32_t* sel, int32_t sel_k, uint32_t* bitmap,
+                               int64_t words_p, int32_t* upos, int32_t* ucount, int64_t umax, uint32_t* memb,
+                               int64_t words_u, cudaStream_t s);
 cudaError_t launch_gather_union(const fb_attn_desc& d, const void* kp, const void* vp, const int32_t* upos,
                                 const int32_t* ucount, int64_t umax, void* ck, void* cv, cudaStream_t s);
 
