@@ -26,6 +26,8 @@ static bool g_stall = false;
 bool debug_stall() { return g_stall; }
 static bool g_inblock_bulk = false;
 bool inblock_bulk_loads() { return g_inblock_bulk; }
+static int g_inblock_rows = 0;
+int inblock_rows_setting() { return g_inblock_rows; }
 static int g_inblock_kernel = 0;   // 0 automatic, 1 the paired tcgen05 kernel wherever it applies
 
 // Device address of this device's status word, looked up once per device (the
@@ -797,6 +799,12 @@ fb_status fb_debug_set_inblock_kernel(int32_t which) {
 
 fb_status fb_debug_set_inblock_loads(int32_t bulk) {
   g_inblock_bulk = bulk != 0;
+  return FB_OK;
+}
+
+fb_status fb_debug_set_inblock_rows(int32_t rows) {
+  if (rows != 0 && rows != 1 && rows != 16 && rows != 32 && rows != 64) return FB_EINVAL;
+  g_inblock_rows = rows;
   return FB_OK;
 }
 

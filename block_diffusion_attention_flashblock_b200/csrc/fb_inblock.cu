@@ -501,6 +501,232 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   }
 }
 
+// ------------------------------------------------- warp-per-rows variant --
+// The same step with each warp owning 16 query rows outright: S for all the
+// block's keys, the softmax in registers (the S accumulators become the A
+// fragments of P V), P V over the whole head dimension, the merge and the
+// stores, with no exchange between warps.  A CTA of W warps takes 16 W rows
+// of one KV head, so K_in and V_in are staged once per 16 W rows (the
+// per-16-row kernel above stages them once per 16 rows); O, LSE and the
+// cache rows leave straight from registers.
+template <int NB, int NX>
+__global__ void __launch_bounds__(128) inblock_rows_kernel(const InblockArgs a) {
+  ptx::pdl_prologue();
+  constexpr int NT = NB / 8;     // key n-tiles of S
+  constexpr int KK = NB / 16;    // key k-steps of P V
+  constexpr int NXS = NX > 0 ? NX : 1;
+  const int W = blockDim.x >> 5;
+  extern __shared__ __align__(128) uint8_t sm[];
+  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(sm);   // [NB][kRowE]
+  __nv_bfloat16* sV = sK + NB * kRowE;                          // [NB][kRowE]
+  __nv_bfloat16* sQ = sV + NB * kRowE;                          // [16 W][kRowE]
+  float* sE = reinterpret_cast<float*>(sQ + W * kRows * kRowE);  // [NX][16 W][kExtStride]
+  uint64_t* sbar = reinterpret_cast<uint64_t*>(sE + NXS * W * kRows * kExtStride);
+  int* sok = reinterpret_cast<int*>(sbar + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int unit = blockIdx.x / a.tiles_per_unit, tile = blockIdx.x % a.tiles_per_unit;
+  const int b = unit / a.Hkv, kvh = unit % a.Hkv;
+  const int nqh = a.active ? a.n_act : a.Nb;     // queries per head computed
+  const int rows_unit = a.G * nqh;
+  const int wrow0 = (tile * W + warp) * kRows;   // the warp's first row among the KV head's rows
+  const bool has_rows = wrow0 < rows_unit;
+
+  // ---- K_in and V_in (every thread, 16-byte chunks; rows past the block
+  // are zero) ----
+  const __nv_bfloat16* kb = a.k + b * a.k_sb + (int64_t)kvh * a.k_sh;
+  const __nv_bfloat16* vb = a.v + b * a.k_sb + (int64_t)kvh * a.k_sh;
+  for (int c = tid; c < NB * 16; c += blockDim.x) {
+    const int r = c >> 4, ch = c & 15;
+    if (r < a.Nb) {
+      cp_async16(ptx::smem_addr(sK + r * kRowE + ch * 8), kb + (int64_t)r * a.k_st + ch * 8);
+      cp_async16(ptx::smem_addr(sV + r * kRowE + ch * 8), vb + (int64_t)r * a.k_st + ch * 8);
+    } else {
+      *reinterpret_cast<uint4*>(sK + r * kRowE + ch * 8) = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(sV + r * kRowE + ch * 8) = make_uint4(0, 0, 0, 0);
+    }
+  }
+  // ---- this warp's rows: lane r < 16 maps row wrow0 + r to its packed
+  // (b, h, i) row (or -1) and its Q and O offsets ----
+  int64_t pr = -1, qoff = 0, ooff = 0;
+  if (lane < kRows && wrow0 + lane < rows_unit) {
+    const int rr = wrow0 + lane;
+    const int g = rr / nqh, k = rr - g * nqh;
+    const int i = a.active ? a.active[(int64_t)b * a.n_act + k] : k;
+    if (i >= 0 && i < a.Nb) {
+      const int h = kvh * a.G + g;
+      pr = ((int64_t)b * a.Hq + h) * a.Nb + i;
+      qoff = b * a.q_sb + (int64_t)h * a.q_sh + (int64_t)i * a.q_st;
+      ooff = b * a.o_sb + (int64_t)h * a.o_sh + (int64_t)i * a.o_st;
+    } else {
+      atomicCAS(a.status, 0, (int)FB_EINVAL);   // an active position outside the block
+    }
+  }
+  // Q rows of the warp (16 chunks each), then the parts' rows (32 chunks)
+  __nv_bfloat16* sQw = sQ + warp * kRows * kRowE;
+#pragma unroll
+  for (int c = lane; c < kRows * 16; c += 32) {
+    const int r = c >> 4, ch = c & 15;
+    const int64_t prr = __shfl_sync(0xffffffffu, pr, r), qo = __shfl_sync(0xffffffffu, qoff, r);
+    if (prr >= 0)
+      cp_async16(ptx::smem_addr(sQw + r * kRowE + ch * 8), a.q + qo + ch * 8);
+    else
+      *reinterpret_cast<uint4*>(sQw + r * kRowE + ch * 8) = make_uint4(0, 0, 0, 0);
+  }
+  cp_async_commit();   // K_in, V_in, Q
+#pragma unroll
+  for (int p = 0; p < NX; ++p)
+#pragma unroll 4
+    for (int c = lane; c < kRows * 32; c += 32) {
+      const int r = c >> 5, ch = c & 31;
+      const int64_t prr = __shfl_sync(0xffffffffu, pr, r);
+      if (prr >= 0)
+        cp_async16(ptx::smem_addr(sE + ((p * W + warp) * kRows + r) * kExtStride + ch * 4),
+                   a.ext_a[p] + prr * kD + ch * 4);
+    }
+  cp_async_commit();   // the parts
+  // the rows of this lane's accumulators (lane/4 and lane/4 + 8) and their
+  // parts' L, read early
+  int64_t prh[2];
+  float lx[2][NXS];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    prh[h] = __shfl_sync(0xffffffffu, pr, (lane >> 2) + 8 * h);
+#pragma unroll
+    for (int p = 0; p < NXS; ++p) lx[h][p] = (p < NX && prh[h] >= 0) ? a.ext_l[p][prh[h]] : -CUDART_INF_F;
+  }
+  if (tid == 0) {
+    *sok = 1;
+    if (a.stall) {   // test hook: a wait that nothing completes runs out
+      ptx::mbar_init(ptx::smem_addr(sbar), 1);
+      ptx::fence_mbar_init();
+      if (!wait_loaded(ptx::smem_addr(sbar), a)) *sok = 0;
+    }
+  }
+  cp_async_wait<1>();   // this thread's K, V and Q chunks
+  __syncthreads();      // every thread's chunks, the zero-filled rows and the stall outcome
+  if (!*sok || !has_rows) {
+    cp_async_wait<0>();
+    return;
+  }
+
+  // ---- S = Q K^T for the warp's 16 rows and all NB keys ----
+  float s[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < kD / 16; ++kk) {
+    uint32_t qa[4];
+    ldsm4(ptx::smem_addr(sQw + (lane & 15) * kRowE + (2 * kk + (lane >> 4)) * 8), qa[0], qa[1], qa[2], qa[3]);
+#pragma unroll
+    for (int n = 0; n < NT; n += 2) {
+      const int r = (n + (lane >> 4)) * 8 + (lane & 7), ch = 2 * kk + ((lane >> 3) & 1);
+      uint32_t b0, b1, b2, b3;
+      ldsm4(ptx::smem_addr(sK + r * kRowE + ch * 8), b0, b1, b2, b3);
+      mma16816(s[n], qa, b0, b1);
+      mma16816(s[n + 1], qa, b2, b3);
+    }
+  }
+  // ---- softmax of rows lane/4 and lane/4 + 8 (a quad holds a row) ----
+  float mrow[2] = {-CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+  for (int n = 0; n < NT; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int key = n * 8 + 2 * (lane & 3) + (e & 1);
+      s[n][e] = key < a.Nb ? s[n][e] * a.scale_log2 : -CUDART_INF_F;
+      mrow[e >> 1] = fmaxf(mrow[e >> 1], s[n][e]);
+    }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    mrow[h] = fmaxf(mrow[h], __shfl_xor_sync(0xffffffffu, mrow[h], 1));
+    mrow[h] = fmaxf(mrow[h], __shfl_xor_sync(0xffffffffu, mrow[h], 2));
+  }
+  const float mref[2] = {mrow[0] == -CUDART_INF_F ? 0.f : mrow[0], mrow[1] == -CUDART_INF_F ? 0.f : mrow[1]};
+  float lrow[2] = {0.f, 0.f};
+  // P as bf16 hi + lo A fragments: k-step kk covers n-tiles 2kk and 2kk + 1
+  uint32_t ph[KK][4], pl[KK][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) {
+    const float p0 = ex2(s[n][0] - mref[0]), p1 = ex2(s[n][1] - mref[0]);
+    const float p2 = ex2(s[n][2] - mref[1]), p3 = ex2(s[n][3] - mref[1]);
+    lrow[0] += p0 + p1;
+    lrow[1] += p2 + p3;
+    const int kk = n >> 1, hf = (n & 1) * 2;
+    split2(p0, p1, ph[kk][hf], pl[kk][hf]);
+    split2(p2, p3, ph[kk][hf + 1], pl[kk][hf + 1]);
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 1);
+    lrow[h] += __shfl_xor_sync(0xffffffffu, lrow[h], 2);
+  }
+  // ---- O = P V over the whole head dimension (16 column tiles) ----
+  float o[kD / 8][4];
+#pragma unroll
+  for (int d = 0; d < kD / 8; ++d) o[d][0] = o[d][1] = o[d][2] = o[d][3] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < KK; ++kk) {
+#pragma unroll
+    for (int d = 0; d < kD / 8; d += 2) {
+      const int r = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8, ch = d + (lane >> 4);
+      uint32_t b0, b1, b2, b3;
+      ldsm4t(ptx::smem_addr(sV + r * kRowE + ch * 8), b0, b1, b2, b3);
+      mma16816(o[d], ph[kk], b0, b1);
+      mma16816(o[d + 1], ph[kk], b2, b3);
+      mma16816(o[d], pl[kk], b0, b1);
+      mma16816(o[d + 1], pl[kk], b2, b3);
+    }
+  }
+  cp_async_wait<0>();   // this lane's part chunks
+  __syncwarp();         // and the rest of the warp's
+  // ---- merge with the external parts; stores straight from registers ----
+  const bool obf = a.o_bf16 != 0;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    if (prh[h] < 0) continue;
+    const int r = (lane >> 2) + 8 * h;
+    const int64_t obase = __shfl_sync(0xffffffffu, ooff, r);
+    const float Lin = lrow[h] > 0.f ? (mrow[h] + __log2f(lrow[h])) * kLn2 : -CUDART_INF_F;
+    float m = Lin;
+#pragma unroll
+    for (int p = 0; p < NX; ++p) m = fmaxf(m, lx[h][p]);
+    const bool empty = m == -CUDART_INF_F;
+    const float w_in = (empty || Lin == -CUDART_INF_F) ? 0.f : __expf(Lin - m);
+    float wx[NXS], wext = 0.f;
+#pragma unroll
+    for (int p = 0; p < NXS; ++p) {
+      wx[p] = (p >= NX || empty || lx[h][p] == -CUDART_INF_F) ? 0.f : __expf(lx[h][p] - m);
+      wext += wx[p];
+    }
+    const float wsum = w_in + wext;
+    const float inv = empty ? 0.f : 1.f / wsum;
+    const float inv_ext = wext > 0.f ? 1.f / wext : 0.f;
+    const float win = lrow[h] > 0.f ? w_in / lrow[h] : 0.f;
+#pragma unroll
+    for (int d = 0; d < kD / 8; ++d) {
+      const int col = d * 8 + 2 * (lane & 3);
+      float ex = 0.f, ey = 0.f;   // sum of w_p A_p (a part with w = 0 may hold -inf rows)
+#pragma unroll
+      for (int p = 0; p < NX; ++p) {
+        const float2 e = *reinterpret_cast<const float2*>(sE + ((p * W + warp) * kRows + r) * kExtStride + col);
+        ex = wx[p] == 0.f ? ex : fmaf(wx[p], e.x, ex);
+        ey = wx[p] == 0.f ? ey : fmaf(wx[p], e.y, ey);
+      }
+      if (a.cache_a) *reinterpret_cast<float2*>(a.cache_a + prh[h] * kD + col) = make_float2(ex * inv_ext, ey * inv_ext);
+      const float x = (win * o[d][2 * h] + ex) * inv, y = (win * o[d][2 * h + 1] + ey) * inv;
+      if (obf)
+        *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(a.o) + obase + col) = __floats2bfloat162_rn(x, y);
+      else
+        *reinterpret_cast<float2*>(static_cast<float*>(a.o) + obase + col) = make_float2(x, y);
+    }
+    if ((lane & 3) == 0) {
+      if (a.cache_l) a.cache_l[prh[h]] = wext > 0.f ? m + logf(wext) : -CUDART_INF_F;
+      if (a.lse) a.lse[prh[h]] = empty ? -CUDART_INF_F : m + logf(wsum);
+    }
+  }
+}
+
 // ------------------------------------------------------------------ host --
 int* device_status_ptr();
 uint64_t wait_limit_ns();
@@ -539,12 +765,48 @@ cudaError_t launch_inblock_small(const fb_attn_desc& d, const void* q, const voi
   if (!a.status) return cudaErrorInvalidValue;
   const int NB = d.Nb <= 16 ? 16 : d.Nb <= 32 ? 32 : 64;
   const int nxs = next > 0 ? next : 1;
+  const int rows_unit = a.G * a.n_act;
+  const int units = d.B * d.Hkv;
+  const int dev = current_device();
+  int W = inblock_rows_setting() / kRows;   // 0: automatic; -1 below: the split-warp kernel
+  if (inblock_rows_setting() == 1) W = -1;
+  if (W == 0) {
+    // measured: 64-row CTAs win where they still fill about the whole GPU
+    // (dllm_64k_b4: 7.7 vs 8.3 us); with fewer CTAs than that the split-warp
+    // kernel's short per-warp chains win (dllm_8k 5.2 vs 6.1 us, blocks of
+    // 4: 4.9 vs 5.1 us)
+    W = (int64_t)units * ((rows_unit + 4 * kRows - 1) / (4 * kRows)) >= (num_sms() * 3) / 4 ? 4 : -1;
+  }
+  if (W > 0) {
+    a.tiles_per_unit = (rows_unit + kRows * W - 1) / (kRows * W);
+    const size_t smem_r = (size_t)(2 * NB + W * kRows) * kRowE * 2 + (size_t)nxs * W * kRows * kExtStride * 4 + 16;
+    const dim3 grid_r(units * a.tiles_per_unit);
+    static bool opted_r[kMaxDevices][3][kMaxExt + 1] = {};
+    auto run_r = [&](void (*kern)(InblockArgs), int nbi) -> cudaError_t {
+      if (smem_r > 48 * 1024 && !opted_r[dev][nbi][next]) {
+        // sized for the largest CTA this instance can get
+        const size_t most = (size_t)(2 * NB + 4 * kRows) * kRowE * 2 + (size_t)nxs * 4 * kRows * kExtStride * 4 + 16;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
+        if (e != cudaSuccess) return e;
+        opted_r[dev][nbi][next] = true;
+      }
+      return launch_k(kern, grid_r, dim3(32 * W), smem_r, s, a);
+    };
+#define FB_INR_CASE(nb, nx) \
+  if (NB == nb && next == nx) return run_r(inblock_rows_kernel<nb, nx>, nb == 16 ? 0 : nb == 32 ? 1 : 2);
+#define FB_INR_NB(nb) FB_INR_CASE(nb, 0) FB_INR_CASE(nb, 1) FB_INR_CASE(nb, 2) FB_INR_CASE(nb, 3) FB_INR_CASE(nb, 4)
+    FB_INR_NB(16)
+    FB_INR_NB(32)
+    FB_INR_NB(64)
+#undef FB_INR_NB
+#undef FB_INR_CASE
+    return cudaErrorInvalidValue;
+  }
   const size_t smem = (size_t)(kRows + 2 * NB) * kRowE * 2 + (size_t)nxs * kRows * (kExtStride + 1) * 4 + kPBytes +
                       (inblock_stage_aliases(NB) ? 0 : 2 * (size_t)kRows * kExtStride * 4) + 4 * 8;
   const dim3 grid(d.B * d.Hkv * a.tiles_per_unit);
   // instances above the default 48 KB of dynamic shared memory opt in once
   static bool opted[kMaxDevices][3][kMaxExt + 1] = {};   // the attribute is per device
-  const int dev = current_device();
   auto run = [&](void (*kern)(InblockArgs), int nbi) -> cudaError_t {
     if (smem > 48 * 1024 && !opted[dev][nbi][next]) {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -106,6 +106,7 @@ class ProfScope {
 bool pdl_enabled();
 bool debug_stall();   // test hook: kernels first wait on a barrier nothing completes
 bool inblock_bulk_loads();   // tuning hook: the small in-block kernel loads by bulk copy per row
+int inblock_rows_setting();   // tuning hook: 0 automatic, 1 the split-warp kernel, 16/32/64 rows per CTA
 template <class... KArgs, class... Args>
 cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
   cudaLaunchConfig_t cfg = {};

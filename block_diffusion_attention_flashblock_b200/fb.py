@@ -76,6 +76,7 @@ _SIGS = {
     "fb_debug_set_wait_limit_ns": (C.c_int, [C.c_uint64]),
     "fb_debug_set_pdl": (C.c_int, [C.c_int32]),
     "fb_debug_set_inblock_loads": (C.c_int, [C.c_int32]),
+    "fb_debug_set_inblock_rows": (C.c_int, [C.c_int32]),
     "fb_debug_set_inblock_kernel": (C.c_int, [C.c_int32]),
     "fb_debug_set_stall": (C.c_int, [C.c_int32]),
     "fb_profile_enable": (C.c_int, [C.c_int32]),
@@ -300,6 +301,10 @@ def fb_debug_set_inblock_kernel(which: int):
 
 def fb_debug_set_inblock_loads(bulk: bool):
     _check(lib().fb_debug_set_inblock_loads(1 if bulk else 0), "fb_debug_set_inblock_loads")
+
+
+def fb_debug_set_inblock_rows(rows: int):
+    _check(lib().fb_debug_set_inblock_rows(int(rows)), "fb_debug_set_inblock_rows")
 
 
 def fb_debug_set_stall(on: bool):

@@ -346,6 +346,13 @@ fb_status fb_debug_set_inblock_kernel(int32_t which);
  * row.  Affects only the calling process. */
 fb_status fb_debug_set_inblock_loads(int32_t bulk);
 
+/* Tuning hook: how the small-block in-block kernel (blocks of up to 64 keys)
+ * splits its work: 0 (default) automatic, 16, 32 or 64 one warp per 16 query
+ * rows with CTAs of that many rows of one KV head, 1 the split-warp kernel
+ * (CTAs of 16 rows whose four warps share S and split the head dimension).
+ * Any other value is FB_EINVAL.  Affects only the calling process. */
+fb_status fb_debug_set_inblock_rows(int32_t rows);
+
 /* Tuning hook: 1 (default) launches every kernel with programmatic dependent
  * launch allowed, so a kernel's launch overlaps the tail of the one before it
  * in the stream (each kernel waits for its predecessors before it touches

@@ -183,3 +183,7 @@ def test_debug_hooks_validate_and_reset(L):
         assert L.fb_debug_set_stall(on) == fb.FB_OK
     assert L.fb_debug_set_stall(0) == fb.FB_OK
     assert L.fb_debug_set_wait_limit_ns(2_000_000_000) == fb.FB_OK
+    for rows in (2, 8, 48, 128, -1):
+        assert L.fb_debug_set_inblock_rows(rows) == fb.FB_EINVAL
+    for rows in (1, 16, 32, 64, 0):
+        assert L.fb_debug_set_inblock_rows(rows) == fb.FB_OK

@@ -255,6 +255,32 @@ def test_inblock_merge(shape, nparts):
     assert_o_close(o, A, TOL[dt], "O"); assert_lse_close(lse, L, TOL[dt], "LSE")
 
 
+@pytest.mark.parametrize("rows", [1, 16, 32, 64])
+@pytest.mark.parametrize("nparts", [0, 1, 4])
+@pytest.mark.parametrize("shape", [(1, 32, 8, 128, 32, "bf16"), (2, 8, 2, 128, 5, "bf16"),
+                                   (1, 8, 2, 128, 64, "bf16"), (3, 4, 4, 128, 16, "bf16"),
+                                   (1, 2, 1, 128, 1, "bf16"), (2, 12, 4, 128, 50, "bf16")],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_inblock_small_variants(shape, nparts, rows):
+    # both small-block kernels (split-warp CTAs of 16 rows, and one warp per
+    # 16 rows with CTAs of 16, 32 or 64 rows), bf16 output
+    B, Hq, Hkv, D, Nb, dt = shape
+    q, kin, vin, kp, vp = _mk(B, Hq, Hkv, D, Nb, 8, dt, seed=37)
+    parts = _random_parts(B, Hq, Nb, D, nparts, seed=310)
+    o = torch.empty(B, Hq, Nb, D, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B, Hq, Nb, device="cuda")
+    desc = fb.make_desc(q.cuda(), kin.cuda(), kp.cuda(), o)
+    try:
+        fb.fb_debug_set_inblock_rows(rows)
+        fb.fb_attn_inblock(desc, q.cuda(), kin.cuda(), vin.cuda(), o, lse,
+                           [a.cuda() for a, _ in parts], [l.cuda() for _, l in parts])
+    finally:
+        fb.fb_debug_set_inblock_rows(0)
+    Ai, Li = orc.inblock(orc.to64(q), orc.to64(kin), orc.to64(vin), 1 / np.sqrt(D))
+    A, L = orc.merge([(orc.to64(a), orc.to64(l)) for a, l in parts] + [(Ai, Li)])
+    assert_o_close(o, A, TOL[dt], "O"); assert_lse_close(lse, L, TOL[dt], "LSE")
+
+
 @pytest.mark.parametrize("nparts", [1, 2, 5, 8])
 @pytest.mark.parametrize("out", ["f32", "bf16"])
 def test_merge_nway(nparts, out):
@@ -330,6 +356,18 @@ def _spec(name):
     kw = dict(SCHEDULES[name])
     base = kw.pop("base", name)
     return wl.get_spec(base, **kw)
+
+
+@pytest.mark.parametrize("rows", [1, 16, 64])
+@pytest.mark.parametrize("name", ["dllm_64k_small", "lock_b2_nb64", "nb4_small", "sparse_small"])
+def test_step_schedule_inblock_variants(name, rows):
+    # the full and reuse steps (cache rows written on full steps, active-query
+    # subsets) through each small-block in-block kernel
+    try:
+        fb.fb_debug_set_inblock_rows(rows)
+        compare_schedule(_spec(name))
+    finally:
+        fb.fb_debug_set_inblock_rows(0)
 
 
 @pytest.mark.parametrize("name", list(SCHEDULES))
