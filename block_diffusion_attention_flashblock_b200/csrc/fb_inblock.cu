@@ -1,23 +1,26 @@
 // Block-internal attention fused with the log-space merge, for small blocks
 // (FlashBlock summary, "Mécanisme Central": A_in over the block's own keys
 // J_in, then A = (e^{L_out-m} A_out + e^{L_in-m} A_in) / (...)).  This is the
-// whole reuse step of a diffusion LM, so it is built for latency:
-//   - one CTA = 16 packed query rows of one KV head (G query heads x Nb
-//     queries) and 4 warps; every warp forms S and P for the 16 rows (one
-//     m16 tile) and owns a quarter (32 columns) of the head dimension in the
-//     P V product, the merge and the stores, which keeps each warp's
-//     dependent instruction chain short;
-//   - every load (Q, K_in, V_in rows and the external parts' A rows) is one
-//     bulk copy per row, issued up front on three mbarriers (Q and K_in;
-//     V_in; the parts), so S and the softmax start while V_in and the parts
-//     are still arriving; the parts' L values are plain loads issued first;
+// whole reuse step of a diffusion LM, so it is built for latency.  Two
+// kernels, chosen by how many CTAs the step makes:
+//   - split-warp (inblock_small_kernel): one CTA = 16 packed query rows of
+//     one KV head (G query heads x Nb queries) and 4 warps; each warp forms
+//     S for a quarter of the block's keys, the row maxima and sums meet in
+//     shared memory, and each warp owns a quarter (32 columns) of the head
+//     dimension in P V, the merge and the stores, which keeps every warp's
+//     dependent instruction chain short (small steps: dllm_8k, blocks of 4);
+//   - warp-per-rows (inblock_rows_kernel): each warp owns 16 rows outright
+//     and a CTA of up to four warps shares one staging of K_in and V_in
+//     (steps large enough that 64-row CTAs still fill the GPU);
+//   - loads are 16-byte cp.async chunks from every thread, K_in and V_in
+//     first (a tuning hook switches the split-warp kernel to one bulk copy
+//     per row); the parts' L values are plain loads issued early;
 //   - S = Q K_in^T and O = P V on mma.sync m16n8k16 (bf16 in, fp32 out) with
 //     the block's keys padded to NB in {16, 32, 64}; P V uses a bf16 hi + lo
 //     split of P so the product keeps fp32-level accuracy;
 //   - the merge with NX (0..4, a template parameter) external parts reads
-//     them from shared memory; O rows (bf16 or fp32) and, on a full step, the
-//     merged external part for the cache are staged in shared memory and
-//     leave as whole-row bulk stores; LSE is written directly.
+//     them from shared memory; O (bf16 or fp32), LSE and, on a full step, the
+//     merged external part for the cache leave straight from registers.
 #include <math_constants.h>
 
 #include "fb_internal.cuh"
@@ -122,11 +125,6 @@ __device__ __forceinline__ bool wait_loaded(uint32_t bar, const InblockArgs& a, 
   return true;
 }
 
-// Whether the output and cache staging rows fit in the K/V staging of NB keys.
-__host__ __device__ constexpr bool inblock_stage_aliases(int NB) {
-  return 2 * NB * kRowE * 2 >= 2 * kRows * kExtStride * 4;
-}
-
 template <int NB, int NX>
 __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a) {
   ptx::pdl_prologue();
@@ -145,15 +143,7 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
   int64_t* sRowPr = reinterpret_cast<int64_t*>(sX + 2 * 4 * kRows);         // [16] packed (b, h, i) row or -1
   int64_t* sRowQ = sRowPr + kRows;                                          // [16] the row's element offset in q
   int64_t* sRowO = sRowQ + kRows;                                           // [16] the row's element offset in o
-  float* sAfter = reinterpret_cast<float*>(sRowO + kRows);
-  // Output and cache rows are staged after P V; with blocks of 32 keys or
-  // more they fit in the K/V staging, which is dead by then (a CTA barrier
-  // separates the last read of K/V from the first staged row), so more CTAs
-  // fit per SM.
-  constexpr bool kAlias = inblock_stage_aliases(NB);
-  float* sO = kAlias ? reinterpret_cast<float*>(sK) : sAfter;            // [16][kExtStride] output rows
-  float* sC = sO + kRows * kExtStride;                                   // [16][kExtStride] cache rows
-  uint64_t* bars = reinterpret_cast<uint64_t*>(kAlias ? sAfter : sC + kRows * kExtStride);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sRowO + kRows);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int unit = blockIdx.x / a.tiles_per_unit, tile = blockIdx.x % a.tiles_per_unit;
@@ -433,6 +423,7 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
     const int r = (lane >> 2) + 8 * h;
     const int64_t pr = sRowPr[r];
     if (pr < 0) continue;
+    const int64_t obase = sRowO[r];
     const float Lin = lrow[h] > 0.f ? (mrow[h] + __log2f(lrow[h])) * kLn2 : -CUDART_INF_F;
     float m = Lin;
     float Lx[NXS];
@@ -463,35 +454,17 @@ __global__ void __launch_bounds__(128) inblock_small_kernel(const InblockArgs a)
         ex = wx[p] == 0.f ? ex : fmaf(wx[p], e.x, ex);
         ey = wx[p] == 0.f ? ey : fmaf(wx[p], e.y, ey);
       }
-      if (a.cache_a) *reinterpret_cast<float2*>(sC + r * kExtStride + col) = make_float2(ex * inv_ext, ey * inv_ext);
+      if (a.cache_a) *reinterpret_cast<float2*>(a.cache_a + pr * kD + col) = make_float2(ex * inv_ext, ey * inv_ext);
       const float x = (win * o[d][2 * h] + ex) * inv, y = (win * o[d][2 * h + 1] + ey) * inv;
       if (obf)
-        reinterpret_cast<__nv_bfloat162*>(sO + r * kExtStride)[col >> 1] = __floats2bfloat162_rn(x, y);
+        *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(a.o) + obase + col) = __floats2bfloat162_rn(x, y);
       else
-        *reinterpret_cast<float2*>(sO + r * kExtStride + col) = make_float2(x, y);
+        *reinterpret_cast<float2*>(static_cast<float*>(a.o) + obase + col) = make_float2(x, y);
     }
     if (dq == 0 && (lane & 3) == 0) {
       if (a.cache_l) a.cache_l[pr] = wext > 0.f ? m + logf(wext) : -CUDART_INF_F;
       if (a.lse) a.lse[pr] = empty ? -CUDART_INF_F : m + logf(wsum);
     }
-  }
-  ptx::fence_proxy_async_smem();
-  __syncthreads();
-  // ---- whole-row stores: lanes 0..15 the output rows, 16..31 the cache rows (warp 0) ----
-  if (ok && warp == 0) {
-    const int r = lane & 15;
-    const int64_t pr = sRowPr[r];
-    if (pr >= 0 && lane < 16) {
-      const int64_t obase = sRowO[r];
-      void* dst = obf ? static_cast<void*>(static_cast<__nv_bfloat16*>(a.o) + obase)
-                      : static_cast<void*>(static_cast<float*>(a.o) + obase);
-      ptx::bulk_s2g(dst, ptx::smem_addr(sO + r * kExtStride), obf ? kD * 2 : kD * 4);
-      ptx::bulk_commit();
-    } else if (pr >= 0 && a.cache_a) {
-      ptx::bulk_s2g(a.cache_a + pr * kD, ptx::smem_addr(sC + r * kExtStride), kD * 4);
-      ptx::bulk_commit();
-    }
-    ptx::bulk_wait_read();
   }
   if (!ok && tid == 0 && a.bulk) {
     // a load wait expired: let every copy into shared memory land before exit
@@ -802,8 +775,7 @@ cudaError_t launch_inblock_small(const fb_attn_desc& d, const void* q, const voi
 #undef FB_INR_CASE
     return cudaErrorInvalidValue;
   }
-  const size_t smem = (size_t)(kRows + 2 * NB) * kRowE * 2 + (size_t)nxs * kRows * (kExtStride + 1) * 4 + kPBytes +
-                      (inblock_stage_aliases(NB) ? 0 : 2 * (size_t)kRows * kExtStride * 4) + 4 * 8;
+  const size_t smem = (size_t)(kRows + 2 * NB) * kRowE * 2 + (size_t)nxs * kRows * (kExtStride + 1) * 4 + kPBytes + 4 * 8;
   const dim3 grid(d.B * d.Hkv * a.tiles_per_unit);
   // instances above the default 48 KB of dynamic shared memory opt in once
   static bool opted[kMaxDevices][3][kMaxExt + 1] = {};   // the attribute is per device
