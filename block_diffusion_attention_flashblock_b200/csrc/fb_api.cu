@@ -455,7 +455,7 @@ static fb_status merge_to_out(const fb_attn_desc& d, const PartList& pl, void* o
 static fb_status run_inblock(const fb_attn_desc& d, const void* q, const void* kin, const void* vin,
                              const PartList& ext, void* o, float* lse, cudaStream_t s, float* cache_a = nullptr,
                              float* cache_l = nullptr, float* ws_a = nullptr, float* ws_l = nullptr,
-                             int32_t ws_cap = 0) {
+                             int32_t ws_cap = 0, int32_t* ws_ns = nullptr) {
   PassPlan p = plan_pass(d, q, kin, vin, d.kin_strides, d.Nb, nullptr, 0, 1);
   AttnArgs& a = p.a;
   a.nsplit = 1;
@@ -498,9 +498,19 @@ static fb_status run_inblock(const fb_attn_desc& d, const void* q, const void* k
   if (nflat > FB_MAX_PARTS) return FB_EINVAL;
   if (cache_a) return FB_EUNSUPPORTED;   // callers only ask for the cache write where the small kernel runs
   if (pair_ok) {
-    // large blocks: one launch of the paired kernel over the block's own keys,
-    // merged with the external parts in its epilogue
+    // large blocks: the paired kernel over the block's own keys, merged with
+    // the external parts in its epilogue.  When the pairs outnumber the CTAs
+    // and leave a partial last round (video frame blocks: 168 pairs on 148
+    // SMs), the remainder's key tiles are split over the grid instead and
+    // their slots merged with the external parts by the merge kernel.
+    PairPlan pp;
     ProfScope prof(kProfInblock, bytes, s);
+    if (ws_a && ws_ns && pw.npairs > pw.grid && pw.npairs % pw.grid != 0 && pair_plan(d, d.Nb, &pp) &&
+        pp.smax <= ws_cap)
+      return launch_attn_pair_split_fused(d, maps, pp, d.Nb, a.scale_log2, nflat, fa, fl, o, lse, ws_a, ws_l,
+                                          ws_ns, s) == cudaSuccess
+                 ? FB_OK
+                 : FB_ECUDA;
     return launch_attn_pair_fused(d, maps, pw, d.Nb, a.scale_log2, nflat, fa, fl, o, lse, s) == cudaSuccess
                ? FB_OK
                : FB_ECUDA;
@@ -1176,7 +1186,7 @@ fb_status fb_step(fb_cache_t c, const fb_step_args* a, cudaStream_t s) {
   // the split parts of the prefix pass are consumed by now: their slots take
   // the block-internal pass's parts
   if ((st = run_inblock(d, a->q, a->kin, a->vin, ext, a->o, a->lse, s, nullptr, nullptr, c->part_a, c->part_l,
-                        c->part_cap)) != FB_OK)
+                        c->part_cap, c->pair_ns)) != FB_OK)
     return st;
   c->valid = true;
   c->last_recomputed = !tau_reuse;

@@ -711,9 +711,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++ocnt;
       tc_fence_after();
       const Tile t = tile_of(a, sg.pair / a.pairs_per_kv, 2 * (sg.pair % a.pairs_per_kv) + s);
-      if (a.whole) {
-        // merge with the external parts (log space, as the standalone merge)
-        // and write this row of O and LSE
+      if (a.o && (sg.slot_ns >> 16) == 1) {
+        // a pair this CTA covers alone, with O requested (whole-pair mode, or
+        // a direct pair of the split mode): merge with the external parts
+        // (log space, as the standalone merge) and write this row of O and LSE
         const bool mine = row < t.nrows;
         const int64_t r = t.rbase + row;
         const float Lin = l > 0.f ? (m + log2f(l)) * kLn2 : -CUDART_INF_F;
@@ -782,6 +783,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(bar(B_OFREE + s));
         if (mine && a.lse) a.lse[r] = empty ? -CUDART_INF_F : mm + __logf(wsum);
+        if (!a.whole && mine && row == 0 && s == 0) a.nslots[sg.pair] = 1;   // the merge kernel skips the pair
         continue;
       }
       const int slot = sg.slot_ns & 0xFFFF, nsl = sg.slot_ns >> 16;
@@ -818,7 +820,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Log-space merge of the slots of every pair covered by two or more CTAs into
-// the final (A, L); one warp per packed row.  Rows of heads that reuse their
+// the final (A, L), or, when O is requested, together with the external parts
+// into O and LSE; one warp per packed row.  Rows of heads that reuse their
 // cache (gamma) and rows of pairs finished by one CTA are left alone.
 __global__ void __launch_bounds__(256) pair_merge_kernel(const PairArgs a) {
   ptx::pdl_prologue();
@@ -846,6 +849,39 @@ __global__ void __launch_bounds__(256) pair_merge_kernel(const PairArgs a) {
     wsum += w;
     acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
     acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+  }
+  if (a.o) {
+    // the split mode with O requested: fold in the external parts and write
+    // this row of O (out dtype, O strides) and LSE
+    float mx = m;
+    for (int p = 0; p < a.next; ++p) mx = fmaxf(mx, a.ext_l[p][r]);
+    const float scl = (m == -CUDART_INF_F || mx == -CUDART_INF_F) ? 0.f : __expf(m - mx);
+    acc.x *= scl; acc.y *= scl; acc.z *= scl; acc.w *= scl;
+    wsum *= scl;
+    for (int p = 0; p < a.next; ++p) {
+      const float Lx = a.ext_l[p][r];
+      if (Lx == -CUDART_INF_F) continue;   // an empty part may hold anything
+      const float w = __expf(Lx - mx);
+      const float4 v = *reinterpret_cast<const float4*>(a.ext_a[p] + r * kD + lane * 4);
+      wsum += w;
+      acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    const int64_t obase = b * a.o_sb + (int64_t)h * a.o_sh + (int64_t)i * a.o_st + lane * 4;
+    if (a.o_bf16) {
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+      uint2 w2;
+      w2.x = *reinterpret_cast<const uint32_t*>(&lo);
+      w2.y = *reinterpret_cast<const uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.o) + obase) = w2;
+    } else {
+      *reinterpret_cast<float4*>(static_cast<float*>(a.o) + obase) =
+          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    }
+    if (lane == 0 && a.lse) a.lse[r] = wsum > 0.f ? mx + __logf(wsum) : -CUDART_INF_F;
+    return;
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
   __syncwarp();   // every lane has read the slots before any writes (dst may be slot 0)
@@ -976,6 +1012,51 @@ cudaError_t launch_attn_pair_fused(const fb_attn_desc& d, const TcMaps& m, const
   }
   const int grid = std::min(num_sms(), pp.npairs);
   return launch_k(attn_pair_kernel, dim3(grid), dim3(kThreads), kSmemBytes, s, m.q, m.k, m.v, a);
+}
+
+// Split pass over the keys of (k, v) [0, nkeys) with O requested: pairs a CTA
+// covers alone are merged with the `next` external parts and written to O
+// and LSE in the kernel's epilogue; the slots of pairs split over several
+// CTAs (the stream-K remainder after the whole-pair rounds) are merged with
+// the external parts by the merge kernel.  pa/pl hold pp.smax slots, nslots
+// one count per pair.
+cudaError_t launch_attn_pair_split_fused(const fb_attn_desc& d, const TcMaps& m, const PairPlan& pp, int64_t nkeys,
+                                         float scale_log2, int32_t next, const float* const* ext_a,
+                                         const float* const* ext_l, void* o, float* lse, float* pa, float* pl,
+                                         int32_t* nslots, cudaStream_t s) {
+  PairArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = d.B; a.Hq = d.Hq; a.Hkv = d.Hkv; a.G = d.Hq / d.Hkv; a.Nb = d.Nb;
+  a.mode = pp.mode; a.hg = pp.hg; a.tph = pp.tph;
+  a.tiles_per_kv = pp.tiles_per_kv; a.pairs_per_kv = pp.pairs_per_kv; a.npairs = pp.npairs;
+  a.nkt = pp.nkt; a.nkeys = nkeys; a.smax = pp.smax;
+  a.scale_log2 = scale_log2;
+  a.part_a = pa; a.part_l = pl;
+  a.part_stride_a = (int64_t)d.B * d.Hq * d.Nb * d.D;
+  a.part_stride_l = (int64_t)d.B * d.Hq * d.Nb;
+  a.nslots = nslots;
+  a.status = device_status_ptr();
+  a.wait_limit_ns = wait_limit_ns();
+  a.q_bytes = 2u * 64u * 2u * (uint32_t)(pp.mode == 0 ? d.Nb * pp.hg : kBM);
+  a.stall = debug_stall() ? 1 : 0;
+  a.whole = 0;
+  a.next = next;
+  for (int p = 0; p < next; ++p) { a.ext_a[p] = ext_a[p]; a.ext_l[p] = ext_l[p]; }
+  a.o = o; a.o_sb = d.o_strides[0]; a.o_sh = d.o_strides[1]; a.o_st = d.o_strides[2];
+  a.o_bf16 = d.out_dtype == FB_BF16;
+  a.lse = lse;
+  if (!a.status || !o || next < 0 || next > FB_MAX_PARTS - 1) return cudaErrorInvalidValue;
+  static bool attr[kMaxDevices] = {};
+  bool& done = attr[current_device()];
+  if (!done) {
+    cudaError_t e = cudaFuncSetAttribute(attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    done = true;
+  }
+  cudaError_t e = launch_k(attn_pair_kernel, dim3(pp.grid), dim3(kThreads), kSmemBytes, s, m.q, m.k, m.v, a);
+  if (e != cudaSuccess) return e;
+  const int64_t nrows = (int64_t)d.B * d.Hq * d.Nb;
+  return launch_k(pair_merge_kernel, dim3((unsigned)((nrows + 7) / 8)), dim3(256), 0, s, a);
 }
 
 // A whole-pair plan: as pair_plan, without the slot bookkeeping (each CTA

@@ -171,6 +171,10 @@ int32_t pair_count(const fb_attn_desc& d);   // pairs of the paired pass (0: it 
 bool pair_plan_whole(const fb_attn_desc& d, int64_t nkeys, PairPlan* p);
 // Whole-pair mode: each CTA takes whole pairs and merges each row with `next`
 // external parts into O (out dtype, strides) and LSE; one launch, no scratch.
+cudaError_t launch_attn_pair_split_fused(const fb_attn_desc& d, const TcMaps& m, const PairPlan& pp, int64_t nkeys,
+                                         float scale_log2, int32_t next, const float* const* ext_a,
+                                         const float* const* ext_l, void* o, float* lse, float* pa, float* pl,
+                                         int32_t* nslots, cudaStream_t s);
 cudaError_t launch_attn_pair_fused(const fb_attn_desc& d, const TcMaps& m, const PairPlan& pp, int64_t nkeys,
                                    float scale_log2, int32_t next, const float* const* ext_a,
                                    const float* const* ext_l, void* o, float* lse, cudaStream_t s);

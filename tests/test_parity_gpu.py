@@ -327,6 +327,10 @@ SCHEDULES = {
     "dllm_64k_small": dict(base="dllm_64k_b4", B=2, prefix0=2000, steps=16),
     "video_small_mixed": dict(base="video_1560", Hq=6, Hkv=6, prefix0=3120, steps=5, sigma_range=(0.01, 1.0)),
     "video_small": dict(base="video_1560", Hq=4, Hkv=4, prefix0=3120, steps=4),
+    # more query-tile pairs (76 heads x 2) than SMs with a partial last round:
+    # the in-block pass splits the remainder's key tiles and merges their
+    # slots with the cached part in the merge kernel
+    "video_wide_split": dict(base="video_1560", Hq=76, Hkv=76, Nb=512, prefix0=1024, steps=3),
     "sparse_small": dict(base="sparse_32k_k2048", prefix0=4000, sel_k=256, Hq=8, Hkv=2),
     "tau_zero": dict(base="dllm_8k", prefix0=500, blocks=1, steps=4, tau=0),
     "tau_off": dict(base="dllm_8k", prefix0=500, blocks=1, steps=4, tau=None),
