@@ -410,19 +410,27 @@ __global__ void __launch_bounds__(kUnionThreads)
   const int64_t bh0 = (int64_t)b * Hq + (int64_t)kvh * G;      // the first query head's (b, h) row
   for (int i = tid; i < G * words_p; i += kUnionThreads) hbm[i] = 0u;
   __syncthreads();
-  for (int g = 0; g < G; ++g) {
-    const int32_t* sg = sel + (bh0 + g) * sel_k;
-    // four keys in flight per thread before their atomics
-    for (int j0 = tid; j0 < sel_k; j0 += 4 * kUnionThreads) {
-      int32_t key[4];
+  {
+    // the G heads' selections are contiguous ([B, Hq, sel_k]): eight keys in
+    // flight per thread across all of them before their atomics, so the
+    // loads cost one memory round trip rather than one per head
+    const int32_t* sg = sel + bh0 * sel_k;
+    const int total = G * sel_k;
+    for (int j0 = tid; j0 < total; j0 += 8 * kUnionThreads) {
+      int32_t key[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const int j = j0 + u * kUnionThreads;
-        key[u] = j < sel_k ? sg[j] : -1;
+        key[u] = j < total ? sg[j] : -1;
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (key[u] >= 0 && (key[u] >> 5) < words_p) atomicOr(hbm + g * words_p + (key[u] >> 5), 1u << (key[u] & 31));
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u * kUnionThreads;
+        if (key[u] >= 0 && (key[u] >> 5) < words_p) {
+          const int g = j / sel_k;
+          atomicOr(hbm + g * words_p + (key[u] >> 5), 1u << (key[u] & 31));
+        }
+      }
     }
   }
   __syncthreads();
