@@ -25,8 +25,9 @@ DEFAULT_LIMIT_NS = 2_000_000_000
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("rows", [0, 64], ids=["inblock-auto", "inblock-warp-per-rows"])
 @pytest.mark.parametrize("Nb", [32, 64], ids=["split-kernel", "paired-kernel"])
-def test_expired_wait_reports_timeout_and_the_device_recovers(Nb):
+def test_expired_wait_reports_timeout_and_the_device_recovers(Nb, rows):
     # dLLM-like shapes: the prefix pass runs on a tcgen05 kernel (TMA + MMA
     # barriers; with blocks of 64 the KV head's 256 query rows make two tiles
     # and the paired stream-K kernel runs) and the in-block merge on the small
@@ -47,6 +48,7 @@ def test_expired_wait_reports_timeout_and_the_device_recovers(Nb):
 
     assert fb.fb_get_device_status() == fb.FB_OK
     try:
+        fb.fb_debug_set_inblock_rows(rows)   # 64: the warp-per-rows small-block kernel
         fb.fb_debug_set_wait_limit_ns(1_000_000)
         fb.fb_debug_set_stall(True)
         fb.fb_attn_outblock(desc, qd, kpd, vpd, Lp, a, l, ws)
@@ -60,8 +62,11 @@ def test_expired_wait_reports_timeout_and_the_device_recovers(Nb):
     assert status == fb.FB_ETIMEOUT, fb.status_string(status)
 
     # the status word was cleared by the read, and the context still works
-    fb.fb_attn_outblock(desc, qd, kpd, vpd, Lp, a, l, ws)
-    fb.fb_attn_inblock(desc, qd, kind, vind, o, lse, [a], [l])
+    try:
+        fb.fb_attn_outblock(desc, qd, kpd, vpd, Lp, a, l, ws)
+        fb.fb_attn_inblock(desc, qd, kind, vind, o, lse, [a], [l])
+    finally:
+        fb.fb_debug_set_inblock_rows(0)
     assert fb.fb_get_device_status() == fb.FB_OK
     sc = 1.0 / np.sqrt(D)
     O, L = orc.full_attention(orc.to64(q), orc.to64(kin), orc.to64(vin), orc.to64(kp), orc.to64(vp), Lp, sc)
