@@ -657,9 +657,9 @@ __global__ void __launch_bounds__(128) inblock_rows_kernel(const InblockArgs a) 
   const bool obf = a.o_bf16 != 0;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    if (prh[h] < 0) continue;
     const int r = (lane >> 2) + 8 * h;
-    const int64_t obase = __shfl_sync(0xffffffffu, ooff, r);
+    const int64_t obase = __shfl_sync(0xffffffffu, ooff, r);   // every lane takes part in the shuffle
+    if (prh[h] < 0) continue;
     const float Lin = lrow[h] > 0.f ? (mrow[h] + __log2f(lrow[h])) * kLn2 : -CUDART_INF_F;
     float m = Lin;
 #pragma unroll
